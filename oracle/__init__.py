@@ -34,9 +34,11 @@ def _load():
         U16 = ctypes.POINTER(ctypes.c_uint16)
         I32 = ctypes.POINTER(ctypes.c_int32)
         i = ctypes.c_int
-        lib.orc_dense_ffn.argtypes = [i, i, i, D, D, D, D, D, D, D, D]
+        lib.orc_round_storage.argtypes = [ctypes.c_double, i]
+        lib.orc_round_storage.restype = ctypes.c_double
+        lib.orc_dense_ffn.argtypes = [i, i, i, D, D, D, D, i, D, D, D, D]
         lib.orc_dense_ffn.restype = None
-        lib.orc_gate_rows.argtypes = [i, I32, i, i, D, D, D]
+        lib.orc_gate_rows.argtypes = [i, I32, i, i, D, D, i, D]
         lib.orc_gate_rows.restype = None
         lib.orc_twell_encode.argtypes = [i, i, i, i, D, D, U8, U8, I32,
                                          ctypes.c_int32, I32, D]
@@ -78,27 +80,36 @@ def _pd(a):
     return _p(a, ctypes.c_double)
 
 
-def dense_ffn(x, Wg_t, Wu_t, Wd):
-    """Plain dense FFN in fp64.  Returns dict z, g, u (all [T,F]) and y [T,d]."""
+ROUND = {None: 0, "f64": 0, "bf16": 1, "f32": 2}
+
+
+def round_storage(v, dtype):
+    """Round one fp64 value to the storage dtype ('bf16', 'f32' or None)."""
+    return _load().orc_round_storage(float(v), ROUND[dtype])
+
+
+def dense_ffn(x, Wg_t, Wu_t, Wd, g_round=None):
+    """Plain dense FFN in fp64 with g rounded to its storage dtype g_round
+    (None, 'bf16' or 'f32').  Returns dict z, g, u (all [T,F]) and y [T,d]."""
     x, Wg_t, Wu_t, Wd = map(_f64, (x, Wg_t, Wu_t, Wd))
     T, d = x.shape
     F = Wg_t.shape[0]
     assert Wg_t.shape == (F, d) and Wu_t.shape == (F, d) and Wd.shape == (F, d)
     z = np.empty((T, F)); g = np.empty((T, F)); u = np.empty((T, F)); y = np.empty((T, d))
-    _load().orc_dense_ffn(T, d, F, _pd(x), _pd(Wg_t), _pd(Wu_t), _pd(Wd),
+    _load().orc_dense_ffn(T, d, F, _pd(x), _pd(Wg_t), _pd(Wu_t), _pd(Wd), ROUND[g_round],
                           _pd(z), _pd(g), _pd(u), _pd(y))
     return {"z": z, "g": g, "u": u, "y": y}
 
 
-def gate_rows(x, Wg_t, rows):
-    """g = relu(x[rows] Wg) in fp64, [len(rows), F]."""
+def gate_rows(x, Wg_t, rows, g_round=None):
+    """g = relu(x[rows] Wg) in fp64, rounded to g_round, [len(rows), F]."""
     x, Wg_t = _f64(x), _f64(Wg_t)
     rows = np.ascontiguousarray(rows, dtype=np.int32)
     d = x.shape[1]
     F = Wg_t.shape[0]
     g = np.empty((len(rows), F))
     _load().orc_gate_rows(len(rows), _p(rows, ctypes.c_int32), d, F, _pd(x),
-                          _pd(Wg_t), _pd(g))
+                          _pd(Wg_t), ROUND[g_round], _pd(g))
     return g
 
 

@@ -38,6 +38,7 @@
  *   - ReLU'(0) = 0 and sign(0) = 0; the L1 term adds lambda*sign(g) to dL/dg
  *     elementwise.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stddef.h>
 #include <string.h>
@@ -45,14 +46,37 @@
 #define ORC_API __attribute__((visibility("default")))
 
 /* ------------------------------------------------------------------------ */
+/* Storage rounding of the gate activations.  TwELL stores g in the model's  */
+/* activation dtype [SFL 2.1], so in a bf16 model g is a bf16 value; the     */
+/* oracle applies the same rounding to its exact fp64 g:                     */
+/*   mode 0  none (exact fp64)                                               */
+/*   mode 1  bf16: nearest value with 8 significant bits, ties to even       */
+/*   mode 2  fp32: the C conversion to float (round to nearest even)         */
+/* Inputs here are finite and far from the bf16/fp32 range limits.           */
+/* ------------------------------------------------------------------------ */
+ORC_API double orc_round_storage(double v, int mode)
+{
+    if (mode == 1) {
+        if (v == 0.0) return v;
+        int e;
+        double m = frexp(v, &e);          /* v = m * 2^e, 0.5 <= |m| < 1 */
+        double q = nearbyint(m * 256.0);  /* default mode: nearest, ties to even */
+        return ldexp(q, e - 8);
+    }
+    if (mode == 2) return (double)(float)v;
+    return v;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Dense FFN, the plain definition of what the sparse path computes.        */
 /* [SFL 2.2]: up projection x Wu, gate activation sigma(x Wg), down         */
 /* projection h Wd with h = sigma(x Wg) * (x Wu) elementwise.                */
-/* Any output pointer may be NULL.                                           */
+/* g is rounded to its storage dtype (g_round, see orc_round_storage); u, h  */
+/* and y stay exact.  Any output pointer may be NULL.                        */
 /* ------------------------------------------------------------------------ */
 ORC_API void orc_dense_ffn(int T, int d, int F,
                            const double* x, const double* Wg_t,
-                           const double* Wu_t, const double* Wd,
+                           const double* Wu_t, const double* Wd, int g_round,
                            double* z_out, double* g_out, double* u_out,
                            double* y_out)
 {
@@ -68,7 +92,7 @@ ORC_API void orc_dense_ffn(int T, int d, int F,
                 z += xt[i] * wg[i];
                 u += xt[i] * wu[i];
             }
-            double g = z > 0.0 ? z : 0.0;
+            double g = orc_round_storage(z > 0.0 ? z : 0.0, g_round);
             if (z_out) z_out[(size_t)t * F + j] = z;
             if (g_out) g_out[(size_t)t * F + j] = g;
             if (u_out) u_out[(size_t)t * F + j] = u;
@@ -81,9 +105,11 @@ ORC_API void orc_dense_ffn(int T, int d, int F,
     }
 }
 
-/* Gate only: g = relu(x Wg) for a subset of rows (rows[r] indexes x). */
+/* Gate only: g = relu(x Wg), rounded to storage, for a subset of rows     */
+/* (rows[r] indexes x).                                                      */
 ORC_API void orc_gate_rows(int R, const int32_t* rows, int d, int F,
-                           const double* x, const double* Wg_t, double* g_out)
+                           const double* x, const double* Wg_t, int g_round,
+                           double* g_out)
 {
     for (int r = 0; r < R; ++r) {
         const double* xt = x + (size_t)rows[r] * d;
@@ -91,7 +117,7 @@ ORC_API void orc_gate_rows(int R, const int32_t* rows, int d, int F,
             const double* wg = Wg_t + (size_t)j * d;
             double z = 0.0;
             for (int i = 0; i < d; ++i) z += xt[i] * wg[i];
-            g_out[(size_t)r * F + j] = z > 0.0 ? z : 0.0;
+            g_out[(size_t)r * F + j] = orc_round_storage(z > 0.0 ? z : 0.0, g_round);
         }
     }
 }

@@ -310,3 +310,42 @@ def test_all_inactive_gives_zero_output_and_only_zero_grads():
     dy = rng.standard_normal((4, 8))
     for a in oracle.dense_ffn_backward(x, Wg_t, Wu_t, Wd, dy, 0.1):
         assert np.all(a == 0)
+
+
+# ------------------------------------------------------------ rounding -----
+def test_storage_rounding_bf16_hand_worked_ties():
+    # bf16 keeps 8 significant bits: the spacing just above 1 is 2^-7.
+    cases = [
+        (1.0, 1.0),
+        (1.0 + 2.0 ** -8, 1.0),                        # halfway, ties to even (down)
+        (1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -6),        # halfway, ties to even (up)
+        (1.0 + 2.0 ** -8 + 2.0 ** -30, 1.0 + 2.0 ** -7),  # just above halfway
+        (-(1.0 + 2.0 ** -8 - 2.0 ** -30), -1.0),       # just below halfway, negative
+        (3.14159, 3.140625),                           # 3.140625 = 201 * 2^-6
+        (0.0, 0.0),
+        (2.0 ** -100 * 1.5, 2.0 ** -100 * 1.5),        # exactly representable
+    ]
+    for v, r in cases:
+        assert oracle.round_storage(v, "bf16") == r, v
+    assert oracle.round_storage(1.0 + 2.0 ** -30, "f32") == 1.0
+    assert oracle.round_storage(1.0 + 2.0 ** -23, "f32") == 1.0 + 2.0 ** -23
+
+
+def test_storage_rounding_matches_independent_generator_rounding():
+    from activation_sparse_transformer_tma_b200 import synth
+    v = np.random.default_rng(0).standard_normal(2000) * 10.0 ** np.random.default_rng(1).uniform(-6, 6, 2000)
+    ours = np.array([oracle.round_storage(a, "bf16") for a in v])
+    assert np.array_equal(ours, synth.round_bf16(v))
+
+
+def test_dense_ffn_rounds_only_g():
+    rng = np.random.default_rng(9)
+    x, Wg_t, Wu_t, Wd = _rand_problem(5, 16, 24, rng, bias=0.3)
+    exact = oracle.dense_ffn(x, Wg_t, Wu_t, Wd)
+    rounded = oracle.dense_ffn(x, Wg_t, Wu_t, Wd, g_round="bf16")
+    gb = np.vectorize(lambda a: oracle.round_storage(a, "bf16"))(exact["g"])
+    assert np.array_equal(rounded["g"], gb)
+    assert np.array_equal(rounded["u"], exact["u"]) and np.array_equal(rounded["z"], exact["z"])
+    assert np.allclose(rounded["y"], (gb * exact["u"]) @ Wd, rtol=1e-12, atol=1e-14)
+    g_rows = oracle.gate_rows(x, Wg_t, np.array([1, 3], np.int32), g_round="bf16")
+    assert np.array_equal(g_rows, gb[[1, 3]])
