@@ -1,0 +1,196 @@
+// abi.cu -- extern "C" entry points of libtwell.so: argument validation
+// (before any launch) and dispatch to the kernels.  The library never
+// allocates device memory and never synchronises the caller's stream.
+#include <atomic>
+#include <cstdint>
+
+#include "tw_internal.h"
+
+namespace tw {
+
+int num_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 1;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+}  // namespace tw
+
+namespace {
+
+constexpr int kTileW = 128;
+constexpr int kMaxC = 32;
+constexpr int kMaxRowD = 2048;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dtype_ok(tw_dtype t) { return t == TW_F32 || t == TW_BF16; }
+
+tw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TW_OK : TW_ERR_CUDA; }
+
+// Shared checks of a TwELL descriptor.
+tw_status check_twell(const tw_twell* g) {
+  if (!g) return TW_ERR_INVALID_ARG;
+  if (g->T < 0 || g->F <= 0 || g->C < 0 || g->spill_cap < 0 || !dtype_ok(g->dtype))
+    return TW_ERR_INVALID_ARG;
+  if (g->W != kTileW || g->F % kTileW != 0 || g->C > kMaxC) return TW_ERR_UNSUPPORTED;
+  if (g->F > 65536) return TW_ERR_UNSUPPORTED;
+  if (!g->cnt || !g->spill_ref || !g->spill_n) return TW_ERR_INVALID_ARG;
+  if (g->C > 0 && (!g->val || !g->idx)) return TW_ERR_INVALID_ARG;
+  if (g->spill_cap > 0 && (!g->spill_tk || !g->spill_val)) return TW_ERR_INVALID_ARG;
+  if ((g->val && !aligned16(g->val)) || (g->idx && !aligned16(g->idx)) ||
+      (g->spill_val && !aligned16(g->spill_val)))
+    return TW_ERR_ALIGNMENT;
+  return TW_OK;
+}
+
+tw_status check_hybrid(const tw_hybrid* h) {
+  if (!h) return TW_ERR_INVALID_ARG;
+  if (h->T < 0 || h->F <= 0 || h->C_h < 0 || h->C_h > h->F || h->backup_cap < 0 ||
+      !dtype_ok(h->dtype))
+    return TW_ERR_INVALID_ARG;
+  if (h->F > 51200) return TW_ERR_UNSUPPORTED;  // unit histograms live in shared memory
+  if ((size_t)h->T * (size_t)h->C_h + (size_t)h->backup_cap * (size_t)h->F > 0x7FFFFFFFull)
+    return TW_ERR_UNSUPPORTED;  // entry numbers are int32
+  if (!h->row_nnz || !h->row_slot || !h->n_backup) return TW_ERR_INVALID_ARG;
+  if (h->C_h > 0 && (!h->ell_g || !h->ell_idx)) return TW_ERR_INVALID_ARG;
+  if (h->backup_cap > 0 && (!h->backup_rows || !h->backup_g)) return TW_ERR_INVALID_ARG;
+  return TW_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tw_status_string(tw_status s) {
+  switch (s) {
+    case TW_OK: return "TW_OK";
+    case TW_ERR_INVALID_ARG: return "TW_ERR_INVALID_ARG";
+    case TW_ERR_UNSUPPORTED: return "TW_ERR_UNSUPPORTED";
+    case TW_ERR_ALIGNMENT: return "TW_ERR_ALIGNMENT";
+    case TW_ERR_CUDA: return "TW_ERR_CUDA";
+    case TW_ERR_SPILL_CAPACITY: return "TW_ERR_SPILL_CAPACITY";
+    case TW_ERR_BACKUP_CAPACITY: return "TW_ERR_BACKUP_CAPACITY";
+    case TW_ERR_TIMEOUT: return "TW_ERR_TIMEOUT";
+    case TW_ERR_WORKSPACE: return "TW_ERR_WORKSPACE";
+  }
+  return "TW_UNKNOWN_STATUS";
+}
+
+int32_t twell_version(void) { return 100; }
+
+tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int32_t d, int32_t F,
+                          tw_dtype dtype, const tw_twell* out, void* g_dense_dump,
+                          int32_t* dev_status, cudaStream_t stream) {
+  tw_status st = check_twell(out);
+  if (st != TW_OK) return st;
+  if (!x || !Wg_t) return TW_ERR_INVALID_ARG;
+  if (T < 0 || d <= 0 || F <= 0 || out->T != T || out->F != F || out->dtype != dtype)
+    return TW_ERR_INVALID_ARG;
+  if (d % 8 != 0) return TW_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(Wg_t) || (g_dense_dump && !aligned16(g_dense_dump)))
+    return TW_ERR_ALIGNMENT;
+  if (T == 0) return from_cuda(cudaMemsetAsync(out->spill_n, 0, sizeof(int32_t), stream));
+  if (dtype == TW_BF16) {
+    if (d < 64) return TW_ERR_UNSUPPORTED;
+    return from_cuda(tw::launch_gate_twell_tc(x, Wg_t, T, d, F, *out, g_dense_dump, dev_status,
+                                              stream));
+  }
+  return from_cuda(tw::launch_gate_twell_f32(static_cast<const float*>(x),
+                                             static_cast<const float*>(Wg_t), T, d, F, *out,
+                                             static_cast<float*>(g_dense_dump), dev_status,
+                                             stream));
+}
+
+tw_status twell_fused_updown(const void* x, const tw_twell* g, const void* Wu_t, const void* Wd,
+                             int32_t d, void* y, tw_dtype y_dtype, int32_t* dev_status,
+                             cudaStream_t stream) {
+  tw_status st = check_twell(g);
+  if (st != TW_OK) return st;
+  if (!x || !Wu_t || !Wd || !y || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
+  if (d <= 0) return TW_ERR_INVALID_ARG;
+  if (d % 8 != 0 || d > kMaxRowD) return TW_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y))
+    return TW_ERR_ALIGNMENT;
+  if (g->T == 0) return TW_OK;
+  return from_cuda(tw::launch_fused_updown(x, *g, Wu_t, Wd, d, y, y_dtype, dev_status, stream));
+}
+
+tw_status twell_to_hybrid(const tw_twell* g, const tw_hybrid* out, int32_t* dev_status,
+                          cudaStream_t stream) {
+  tw_status st = check_twell(g);
+  if (st != TW_OK) return st;
+  st = check_hybrid(out);
+  if (st != TW_OK) return st;
+  if (out->T != g->T || out->F != g->F || out->dtype != g->dtype) return TW_ERR_INVALID_ARG;
+  if (g->T == 0) return from_cuda(cudaMemsetAsync(out->n_backup, 0, sizeof(int32_t), stream));
+  return from_cuda(tw::launch_twell_to_hybrid(*g, *out, dev_status, stream));
+}
+
+tw_status hybrid_ffn_forward(const void* x, const tw_hybrid* gu, const void* Wu_t,
+                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype,
+                             int32_t* dev_status, cudaStream_t stream) {
+  tw_status st = check_hybrid(gu);
+  if (st != TW_OK) return st;
+  if (!x || !Wu_t || !Wd || !y || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
+  if ((gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
+    return TW_ERR_INVALID_ARG;
+  if (d <= 0) return TW_ERR_INVALID_ARG;
+  if (d % 8 != 0 || d > kMaxRowD) return TW_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y))
+    return TW_ERR_ALIGNMENT;
+  return from_cuda(tw::launch_hybrid_forward(x, *gu, Wu_t, Wd, d, y, y_dtype, dev_status, stream));
+}
+
+size_t hybrid_ffn_backward_workspace_size(int32_t T, int32_t d, int32_t F, int32_t C_h,
+                                          int32_t backup_cap) {
+  if (T < 0 || F <= 0 || C_h < 0 || backup_cap < 0) return 0;
+  return tw::hybrid_backward_ws_bytes(T, d, F, C_h, backup_cap);
+}
+
+tw_status hybrid_ffn_backward(const void* x, const void* dy, const tw_hybrid* gu,
+                              const void* Wg_t, const void* Wu_t, const void* Wd, int32_t d,
+                              float l1_lambda, void* dx, tw_dtype dx_dtype, float* dWg_t,
+                              float* dWu_t, float* dWd, void* ws, size_t ws_bytes,
+                              int32_t* dev_status, cudaStream_t stream) {
+  tw_status st = check_hybrid(gu);
+  if (st != TW_OK) return st;
+  if (!x || !dy || !Wg_t || !Wu_t || !Wd || !dx || !dWg_t || !dWu_t || !dWd || !ws ||
+      !dtype_ok(dx_dtype))
+    return TW_ERR_INVALID_ARG;
+  if ((gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
+    return TW_ERR_INVALID_ARG;
+  if (d <= 0) return TW_ERR_INVALID_ARG;
+  if (d % 8 != 0 || d > kMaxRowD) return TW_ERR_UNSUPPORTED;
+  const void* ptrs[] = {x, dy, Wg_t, Wu_t, Wd, dx, dWg_t, dWu_t, dWd, ws};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return TW_ERR_ALIGNMENT;
+  if (ws_bytes < tw::hybrid_backward_ws_bytes(gu->T, d, gu->F, gu->C_h, gu->backup_cap))
+    return TW_ERR_WORKSPACE;
+  return from_cuda(tw::launch_hybrid_backward(x, dy, *gu, Wg_t, Wu_t, Wd, d, l1_lambda, dx,
+                                              dx_dtype, dWg_t, dWu_t, dWd, ws, ws_bytes,
+                                              dev_status, stream));
+}
+
+tw_status dense_ffn_forward(const void* x, const void* Wg_t, const void* Wu_t,
+                            const void* Wd_dense, int32_t T, int32_t d, int32_t F, void* h_ws,
+                            void* y, int32_t* dev_status, cudaStream_t stream) {
+  if (!x || !Wg_t || !Wu_t || !Wd_dense || !h_ws || !y) return TW_ERR_INVALID_ARG;
+  if (T < 0 || d <= 0 || F <= 0) return TW_ERR_INVALID_ARG;
+  if (d % 32 != 0 || d < 64 || F % kTileW != 0) return TW_ERR_UNSUPPORTED;
+  const void* ptrs[] = {x, Wg_t, Wu_t, Wd_dense, h_ws, y};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return TW_ERR_ALIGNMENT;
+  if (T == 0) return TW_OK;
+  cudaError_t e = tw::launch_dense_gateup_tc(x, Wg_t, Wu_t, T, d, F, h_ws, dev_status, stream);
+  if (e != cudaSuccess) return TW_ERR_CUDA;
+  return from_cuda(tw::launch_dense_down_tc(h_ws, Wd_dense, T, d, F, y, dev_status, stream));
+}
+
+}  // extern "C"

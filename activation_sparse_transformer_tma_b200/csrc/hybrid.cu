@@ -1,0 +1,729 @@
+// hybrid.cu -- training-side kernels for the hybrid sparse format
+// ("Sparser, Faster, Lighter Transformer Language Models", technical summary,
+// sections 2.3 and 2.4):
+//   * TwELL -> hybrid: each token row becomes a compact ELL row (global unit
+//     indices, ascending) when it has at most C_h non-zeros, otherwise a dense
+//     backup row; backup slots follow ascending token order;
+//   * hybrid forward (dense x times dense Wu sampled on the hybrid pattern,
+//     then the sparse pattern times dense Wd);
+//   * hybrid backward with the L1 term: per-token pass for dh, du, dz and dx,
+//     then weight gradients per unit from a deterministic, token-ordered
+//     transposition of the pattern (counting sort by unit; no float atomics).
+#include "tw_common.cuh"
+#include "tw_internal.h"
+
+namespace tw {
+namespace {
+
+constexpr unsigned FULL = 0xFFFFFFFFu;
+constexpr int W = 128;
+
+template <typename T>
+TW_DEV float ld_scalar(const T* p, size_t i);
+template <>
+TW_DEV float ld_scalar<uint16_t>(const uint16_t* p, size_t i) { return bf16_to_f32(p[i]); }
+template <>
+TW_DEV float ld_scalar<float>(const float* p, size_t i) { return p[i]; }
+
+template <typename T>
+TW_DEV void st_scalar(T* p, size_t i, float v);
+template <>
+TW_DEV void st_scalar<uint16_t>(uint16_t* p, size_t i, float v) { p[i] = f32_to_bf16(v); }
+template <>
+TW_DEV void st_scalar<float>(float* p, size_t i, float v) { p[i] = v; }
+
+TW_DEV unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Row vectors of length d held by one warp: lane owns 16-byte slices.
+template <typename T>
+struct Slice;
+template <>
+struct Slice<uint16_t> {
+  static constexpr int E = 8;
+  using Raw = uint4;
+  TW_DEV static Raw load(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+  TW_DEV static Raw zero() { return make_uint4(0, 0, 0, 0); }
+  TW_DEV static void widen(const Raw& r, float (&f)[8]) {
+    f[0] = bf16_lo(r.x); f[1] = bf16_hi(r.x); f[2] = bf16_lo(r.y); f[3] = bf16_hi(r.y);
+    f[4] = bf16_lo(r.z); f[5] = bf16_hi(r.z); f[6] = bf16_lo(r.w); f[7] = bf16_hi(r.w);
+  }
+};
+template <>
+struct Slice<float> {
+  static constexpr int E = 4;
+  using Raw = float4;
+  TW_DEV static Raw load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+  TW_DEV static Raw zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  TW_DEV static void widen(const Raw& r, float (&f)[4]) { f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w; }
+};
+
+template <typename T, int NCH>
+TW_DEV void load_row(const T* row, int d, int lane, typename Slice<T>::Raw (&r)[NCH]) {
+  constexpr int SPAN = 32 * Slice<T>::E;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const int col = c * SPAN + lane * Slice<T>::E;
+    r[c] = col < d ? Slice<T>::load(row + col) : Slice<T>::zero();
+  }
+}
+
+// Warp dot product of a register-resident row with a gathered row.
+template <typename T, int NCH>
+TW_DEV float warp_dot(const typename Slice<T>::Raw (&a)[NCH], const T* row, int d, int lane) {
+  typename Slice<T>::Raw b[NCH];
+  load_row<T, NCH>(row, d, lane, b);
+  float part = 0.f;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    float af[Slice<T>::E], bf[Slice<T>::E];
+    Slice<T>::widen(a[c], af);
+    Slice<T>::widen(b[c], bf);
+#pragma unroll
+    for (int e = 0; e < Slice<T>::E; ++e) part = fmaf(af[e], bf[e], part);
+  }
+  return warp_sum(part);
+}
+
+// acc += s * row
+template <typename T, int NCH>
+TW_DEV void warp_axpy(float (&acc)[NCH][Slice<T>::E], float s, const T* row, int d, int lane) {
+  typename Slice<T>::Raw b[NCH];
+  load_row<T, NCH>(row, d, lane, b);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    float bf[Slice<T>::E];
+    Slice<T>::widen(b[c], bf);
+#pragma unroll
+    for (int e = 0; e < Slice<T>::E; ++e) acc[c][e] = fmaf(s, bf[e], acc[c][e]);
+  }
+}
+
+template <int NCH, int E>
+TW_DEV void store_row(void* out, tw_dtype dt, size_t row_off, int d, int lane,
+                      const float (&acc)[NCH][E]) {
+  constexpr int SPAN = 32 * E;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const int col = c * SPAN + lane * E;
+    if (col >= d) continue;
+    if (dt == TW_BF16) {
+      uint16_t* p = static_cast<uint16_t*>(out) + row_off + col;
+#pragma unroll
+      for (int e = 0; e < E; e += 2)
+        *reinterpret_cast<uint32_t*>(p + e) = pack_bf16x2(acc[c][e], acc[c][e + 1]);
+    } else {
+      float* p = static_cast<float*>(out) + row_off + col;
+#pragma unroll
+      for (int e = 0; e < E; e += 4)
+        *reinterpret_cast<float4*>(p + e) = make_float4(acc[c][e], acc[c][e + 1], acc[c][e + 2], acc[c][e + 3]);
+    }
+  }
+}
+
+template <typename V>
+struct HView {
+  int T, F, C_h, backup_cap;
+  const V* ell_g;
+  V* ell_u;
+  const uint16_t* ell_idx;
+  const int32_t* row_nnz;
+  const int32_t* row_slot;
+  const V* backup_g;
+  V* backup_u;
+};
+
+// Enumerates the active entries of token t in ascending unit order, 32 at a
+// time.  fn(valid, j, g, pos, is_ell, rank) receives one lane-distributed
+// chunk; pos indexes ell_* (ELL row) or backup_* (backup row); rank is the
+// entry's position among the row's non-zeros.  Rows whose backup slot was
+// dropped for lack of capacity have no entries.
+template <typename T, class Fn>
+TW_DEV void for_each_chunk(const HView<T>& h, int t, int lane, Fn&& fn) {
+  const int slot = h.row_slot[t];
+  if (slot < 0) {
+    const int nnz = h.row_nnz[t];
+    for (int s0 = 0; s0 < nnz; s0 += 32) {
+      const int s = s0 + lane;
+      const bool v = s < nnz;
+      const size_t pos = (size_t)t * h.C_h + (v ? s : 0);
+      const int j = v ? (int)h.ell_idx[pos] : 0;
+      const float g = v ? ld_scalar<T>(h.ell_g, pos) : 0.f;
+      fn(v, j, g, pos, true, s);
+    }
+  } else if (slot < h.backup_cap) {
+    int base = 0;
+    for (int c0 = 0; c0 < h.F; c0 += 32) {
+      const int j = c0 + lane;
+      const size_t pos = (size_t)slot * h.F + (j < h.F ? j : 0);
+      const float g = j < h.F ? ld_scalar<T>(h.backup_g, pos) : 0.f;
+      const bool v = g != 0.f;
+      const unsigned m = __ballot_sync(FULL, v);
+      if (m == 0u) continue;
+      fn(v, j, g, pos, false, base + __popc(m & lanemask_lt()));
+      base += __popc(m);
+    }
+  }
+}
+
+// --------------------------------------------------------- TwELL -> hybrid --
+// Warp per token: row_nnz, and the ELL row when nnz <= C_h.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    hyb_rows_kernel(int Tn, int F, int C, const uint8_t* cnt, const T* val, const uint8_t* idx,
+                    const int32_t* spill_ref, int spill_cap, const T* spill_val, int C_h,
+                    T* ell_g, uint16_t* ell_idx, int32_t* row_nnz, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  if (t >= Tn) return;
+  const int K = F / W;
+  int total = 0;
+  for (int kb = 0; kb < K; kb += 32) {
+    const int k = kb + lane;
+    total += k < K ? (int)cnt[(size_t)k * Tn + t] : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(FULL, total, o);
+  if (lane == 0) row_nnz[t] = total;
+  const size_t rbase = (size_t)t * C_h;
+  if (total > C_h) {  // backup row: its ELL slots hold (+0, 0); g is filled after the scan
+    for (int s = lane; s < C_h; s += 32) {
+      ell_g[rbase + s] = T(0);
+      ell_idx[rbase + s] = 0;
+    }
+    return;
+  }
+
+  int pos = 0;  // next ELL position of this row
+  for (int kb = 0; kb < K; kb += 32) {
+    const int k = kb + lane;
+    const int n = k < K ? (int)cnt[(size_t)k * Tn + t] : 0;
+    // exclusive prefix of counts over the 32 tiles
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - n;
+    unsigned act = __ballot_sync(FULL, n > 0);
+    while (act) {
+      const int b = __ffs(act) - 1;
+      act &= act - 1;
+      const int nk = __shfl_sync(FULL, n, b);
+      const int p0 = pos + __shfl_sync(FULL, excl, b);
+      const int kk = kb + b;
+      const size_t kt = (size_t)kk * Tn + t;
+      if (nk <= C) {
+        if (lane < nk) {
+          ell_g[rbase + p0 + lane] = val[kt * C + lane];
+          ell_idx[rbase + p0 + lane] = (uint16_t)(kk * W + idx[kt * C + lane]);
+        }
+      } else {
+        const int ref = spill_ref[kt];
+        if (ref < 0 || ref >= spill_cap) {
+          // Dropped spill entry: only the C slots are known.
+          if (lane == 0) set_status(status, kStatusSpill);
+          if (lane < C) {
+            ell_g[rbase + p0 + lane] = val[kt * C + lane];
+            ell_idx[rbase + p0 + lane] = (uint16_t)(kk * W + idx[kt * C + lane]);
+          }
+          for (int s = C + lane; s < nk; s += 32) {  // keep the row's slots defined
+            ell_g[rbase + p0 + s] = T(0);
+            ell_idx[rbase + p0 + s] = 0;
+          }
+          continue;
+        }
+        int r = 0;
+        for (int part = 0; part < W / 32; ++part) {
+          const T v = spill_val[(size_t)ref * W + part * 32 + lane];
+          const bool nz = ld_scalar<T>(&v, 0) != 0.f;
+          const unsigned m = __ballot_sync(FULL, nz);
+          if (nz) {
+            const int q = p0 + r + __popc(m & lanemask_lt());
+            ell_g[rbase + q] = v;
+            ell_idx[rbase + q] = (uint16_t)(kk * W + part * 32 + lane);
+          }
+          r += __popc(m);
+        }
+      }
+    }
+    pos += __shfl_sync(FULL, incl, 31);
+  }
+  for (int s = total + lane; s < C_h; s += 32) {
+    ell_g[rbase + s] = T(0);
+    ell_idx[rbase + s] = 0;
+  }
+}
+
+// Single-CTA exclusive scan over n int32 values.
+//  mode 0 (backup slots): flag = in[i] > thr; out[i] = flag ? slot : -1;
+//          aux[slot] = i for slot < cap; *total = number of flags.
+//  mode 1 (offsets): out[i] = exclusive prefix of in[]; out[n] = total.
+//  mode 2 (entry offsets): as mode 1, counting in[i] only for rows whose slot
+//          aux[i] is below cap (ELL rows and stored backup rows).
+constexpr int SCAN_THREADS = 1024;
+__global__ void __launch_bounds__(SCAN_THREADS)
+    scan_kernel(int mode, int n, const int32_t* in, int thr, int32_t* out, int32_t* aux, int cap,
+                int32_t* total, int32_t* status) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += SCAN_THREADS) {
+    const int i = base + tid;
+    int v = 0;
+    if (i < n) {
+      if (mode == 0) v = in[i] > thr ? 1 : 0;
+      else if (mode == 1) v = in[i];
+      else v = aux[i] < cap ? in[i] : 0;
+    }
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      int s = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, s, o);
+        if (lane >= o) s += u;
+      }
+      warp_sums[lane] = s;  // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + incl - v;
+    if (i < n) {
+      if (mode == 0) {
+        out[i] = v ? excl : -1;
+        if (v && excl < cap) aux[excl] = i;
+      } else {
+        out[i] = excl;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) carry += warp_sums[31];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (mode == 0) {
+      *total = carry;
+      if (carry > cap) set_status(status, kStatusBackup);
+    } else {
+      out[n] = carry;
+    }
+  }
+}
+
+// Warp per backup slot: dense g row from TwELL (zero fill, then scatter).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    hyb_backup_kernel(int Tn, int F, int C, const uint8_t* cnt, const T* val, const uint8_t* idx,
+                      const int32_t* spill_ref, int spill_cap, const T* spill_val,
+                      const int32_t* backup_rows, const int32_t* n_backup, int backup_cap,
+                      T* backup_g) {
+  const int lane = threadIdx.x & 31;
+  const int slot = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int nb = min(*n_backup, backup_cap);
+  if (slot >= nb) return;
+  const int t = backup_rows[slot];
+  T* row = backup_g + (size_t)slot * F;
+  for (int j = lane; j < F; j += 32) row[j] = T(0);
+  __syncwarp();
+  const int K = F / W;
+  for (int k = 0; k < K; ++k) {
+    const size_t kt = (size_t)k * Tn + t;
+    const int n = cnt[kt];
+    if (n == 0) continue;
+    if (n <= C) {
+      if (lane < n) row[k * W + idx[kt * C + lane]] = val[kt * C + lane];
+    } else {
+      const int ref = spill_ref[kt];
+      if (ref >= 0 && ref < spill_cap) {
+        for (int c = lane; c < W; c += 32) row[k * W + c] = spill_val[(size_t)ref * W + c];
+      } else if (lane < C) {
+        row[k * W + idx[kt * C + lane]] = val[kt * C + lane];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------- hybrid forward --
+template <typename T, int NCH>
+__global__ void __launch_bounds__(256)
+    hyb_forward_kernel(const HView<T> h, const T* x, const T* Wu_t, const T* Wd, int d, void* y,
+                       tw_dtype y_dtype) {
+  using S = Slice<T>;
+  const int lane = threadIdx.x & 31;
+  const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  if (t >= h.T) return;
+  typename S::Raw xr[NCH];
+  load_row<T, NCH>(x + (size_t)t * d, d, lane, xr);
+  float acc[NCH][S::E];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int e = 0; e < S::E; ++e) acc[c][e] = 0.f;
+
+  const int slot = h.row_slot[t];
+  if (slot >= 0 && slot < h.backup_cap) {
+    for (int j = lane; j < h.F; j += 32) h.backup_u[(size_t)slot * h.F + j] = T(0);
+    __syncwarp();
+  }
+  for_each_chunk<T>(h, t, lane, [&](bool v, int j, float g, size_t pos, bool is_ell, int) {
+    unsigned m = __ballot_sync(FULL, v);
+    while (m) {
+      const int s = __ffs(m) - 1;
+      m &= m - 1;
+      const int jj = __shfl_sync(FULL, j, s);
+      const float gg = __shfl_sync(FULL, g, s);
+      const unsigned long long pp = __shfl_sync(FULL, (unsigned long long)pos, s);
+      const float u = warp_dot<T, NCH>(xr, Wu_t + (size_t)jj * d, d, lane);
+      if (lane == 0) st_scalar<T>(is_ell ? h.ell_u : h.backup_u, pp, u);
+      warp_axpy<T, NCH>(acc, gg * u, Wd + (size_t)jj * d, d, lane);
+    }
+  });
+  if (slot < 0) {
+    for (int s = h.row_nnz[t] + lane; s < h.C_h; s += 32)
+      h.ell_u[(size_t)t * h.C_h + s] = T(0);
+  }
+  store_row<NCH, S::E>(y, y_dtype, (size_t)t * d, d, lane, acc);
+}
+
+// --------------------------------------------------------- hybrid backward --
+struct Payload {  // one active (t, j) entry for the weight-gradient pass
+  int32_t t;
+  float h, du, dz;
+};
+
+template <typename T, int NCH>
+__global__ void __launch_bounds__(256)
+    hyb_backward_token_kernel(const HView<T> h, const T* dy, const T* Wg_t, const T* Wu_t,
+                              const T* Wd, int d, float lam, const int32_t* e0, Payload* pay,
+                              void* dx, tw_dtype dx_dtype) {
+  using S = Slice<T>;
+  const int lane = threadIdx.x & 31;
+  const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  if (t >= h.T) return;
+  typename S::Raw dyr[NCH];
+  load_row<T, NCH>(dy + (size_t)t * d, d, lane, dyr);
+  float acc[NCH][S::E];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int e = 0; e < S::E; ++e) acc[c][e] = 0.f;
+  const int ebase = e0[t];
+  for_each_chunk<T>(h, t, lane, [&](bool v, int j, float g, size_t pos, bool is_ell, int rank) {
+    const float u = v ? ld_scalar<T>(is_ell ? h.ell_u : h.backup_u, pos) : 0.f;
+    unsigned m = __ballot_sync(FULL, v);
+    while (m) {
+      const int s = __ffs(m) - 1;
+      m &= m - 1;
+      const int jj = __shfl_sync(FULL, j, s);
+      const float gg = __shfl_sync(FULL, g, s);
+      const float uu = __shfl_sync(FULL, u, s);
+      const int rr = __shfl_sync(FULL, rank, s);
+      const float dh = warp_dot<T, NCH>(dyr, Wd + (size_t)jj * d, d, lane);
+      const float du = dh * gg;
+      const float dz = fmaf(dh, uu, lam);
+      warp_axpy<T, NCH>(acc, du, Wu_t + (size_t)jj * d, d, lane);
+      warp_axpy<T, NCH>(acc, dz, Wg_t + (size_t)jj * d, d, lane);
+      if (lane == 0) {
+        Payload p;
+        p.t = t;
+        p.h = gg * uu;
+        p.du = du;
+        p.dz = dz;
+        pay[ebase + rr] = p;
+      }
+    }
+  });
+  store_row<NCH, S::E>(dx, dx_dtype, (size_t)t * d, d, lane, acc);
+}
+
+constexpr int TB = 32;  // tokens per block of the transposition
+
+// Per (token block, unit) entry counts: cntb[b][j].
+template <typename T>
+__global__ void __launch_bounds__(256)
+    hyb_count_kernel(const HView<T> h, int32_t* cntb) {
+  extern __shared__ int32_t hist[];
+  const int b = blockIdx.x;
+  for (int j = threadIdx.x; j < h.F; j += blockDim.x) hist[j] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int tt = wid; tt < TB; tt += blockDim.x / 32) {
+    const int t = b * TB + tt;
+    if (t >= h.T) break;
+    for_each_chunk<T>(h, t, lane, [&](bool v, int j, float, size_t, bool, int) {
+      if (v) atomicAdd(&hist[j], 1);
+    });
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < h.F; j += blockDim.x) cntb[(size_t)b * h.F + j] = hist[j];
+}
+
+// Column-wise exclusive prefix over token blocks; totals per unit.
+__global__ void hyb_colscan_kernel(int nblocks, int F, int32_t* cntb, int32_t* unit_total) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= F) return;
+  int run = 0;
+  for (int b = 0; b < nblocks; ++b) {
+    const int c = cntb[(size_t)b * F + j];
+    cntb[(size_t)b * F + j] = run;
+    run += c;
+  }
+  unit_total[j] = run;
+}
+
+// Fill the unit-major list with token-major entry indices, tokens ascending.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    hyb_fill_kernel(const HView<T> h, const int32_t* cntb, const int32_t* unit_off,
+                    const int32_t* e0, int32_t* list) {
+  extern __shared__ int32_t next[];
+  const int b = blockIdx.x;
+  for (int j = threadIdx.x; j < h.F; j += blockDim.x)
+    next[j] = unit_off[j] + cntb[(size_t)b * h.F + j];
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  for (int tt = 0; tt < TB; ++tt) {
+    const int t = b * TB + tt;
+    if (t >= h.T) break;
+    const int ebase = e0[t];
+    for_each_chunk<T>(h, t, lane, [&](bool v, int j, float, size_t, bool, int rank) {
+      // the units of one row are distinct, so these increments never collide
+      if (v) list[next[j]++] = ebase + rank;
+    });
+    __syncwarp();
+  }
+}
+
+// Weight gradients of one unit per CTA, entries summed in token order.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    hyb_wgrad_kernel(int F, int d, const T* x, const T* dy, const int32_t* unit_off,
+                     const int32_t* list, const Payload* pay, float* dWg_t, float* dWu_t,
+                     float* dWd) {
+  using S = Slice<T>;
+  constexpr int E = S::E;
+  const int j = blockIdx.x;
+  const int e_begin = unit_off[j], e_end = unit_off[j + 1];
+  const int stride = blockDim.x * E;
+  for (int col = threadIdx.x * E; col < d; col += stride) {
+    float ad[E], au[E], ag[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) ad[e] = au[e] = ag[e] = 0.f;
+    for (int q = e_begin; q < e_end; ++q) {
+      const Payload p = pay[list[q]];
+      float xf[E], df[E];
+      S::widen(S::load(x + (size_t)p.t * d + col), xf);
+      S::widen(S::load(dy + (size_t)p.t * d + col), df);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        ad[e] = fmaf(p.h, df[e], ad[e]);
+        au[e] = fmaf(p.du, xf[e], au[e]);
+        ag[e] = fmaf(p.dz, xf[e], ag[e]);
+      }
+    }
+    const size_t o = (size_t)j * d + col;
+#pragma unroll
+    for (int e = 0; e < E; e += 4) {
+      *reinterpret_cast<float4*>(dWd + o + e) = make_float4(ad[e], ad[e + 1], ad[e + 2], ad[e + 3]);
+      *reinterpret_cast<float4*>(dWu_t + o + e) = make_float4(au[e], au[e + 1], au[e + 2], au[e + 3]);
+      *reinterpret_cast<float4*>(dWg_t + o + e) = make_float4(ag[e], ag[e + 1], ag[e + 2], ag[e + 3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------ workspace ----
+struct BwdWs {
+  int32_t* e0;        // [T+1]
+  Payload* pay;       // [Emax]
+  int32_t* cntb;      // [NB][F]
+  int32_t* unit_total;// [F]
+  int32_t* unit_off;  // [F+1]
+  int32_t* list;      // [Emax]
+  size_t bytes;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+BwdWs carve(void* base, int T, int F, int C_h, int backup_cap) {
+  const size_t emax = (size_t)T * C_h + (size_t)backup_cap * F;
+  const size_t nb = ((size_t)T + TB - 1) / TB;
+  BwdWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t o_e0 = take(sizeof(int32_t) * ((size_t)T + 1));
+  const size_t o_pay = take(sizeof(Payload) * (emax > 0 ? emax : 1));
+  const size_t o_cntb = take(sizeof(int32_t) * nb * F);
+  const size_t o_tot = take(sizeof(int32_t) * (size_t)F);
+  const size_t o_off = take(sizeof(int32_t) * ((size_t)F + 1));
+  const size_t o_list = take(sizeof(int32_t) * (emax > 0 ? emax : 1));
+  w.bytes = off;
+  if (base) {
+    char* p = static_cast<char*>(base);
+    w.e0 = reinterpret_cast<int32_t*>(p + o_e0);
+    w.pay = reinterpret_cast<Payload*>(p + o_pay);
+    w.cntb = reinterpret_cast<int32_t*>(p + o_cntb);
+    w.unit_total = reinterpret_cast<int32_t*>(p + o_tot);
+    w.unit_off = reinterpret_cast<int32_t*>(p + o_off);
+    w.list = reinterpret_cast<int32_t*>(p + o_list);
+  }
+  return w;
+}
+
+template <typename T>
+HView<T> view_of(const tw_hybrid& g) {
+  HView<T> h;
+  h.T = g.T;
+  h.F = g.F;
+  h.C_h = g.C_h;
+  h.backup_cap = g.backup_cap;
+  h.ell_g = static_cast<const T*>(g.ell_g);
+  h.ell_u = static_cast<T*>(g.ell_u);
+  h.ell_idx = g.ell_idx;
+  h.row_nnz = g.row_nnz;
+  h.row_slot = g.row_slot;
+  h.backup_g = static_cast<const T*>(g.backup_g);
+  h.backup_u = static_cast<T*>(g.backup_u);
+  return h;
+}
+
+unsigned warp_blocks(int n) { return (unsigned)(((size_t)n + 7) / 8); }
+
+template <typename T>
+cudaError_t to_hybrid_t(const tw_twell& g, const tw_hybrid& o, int32_t* status, cudaStream_t s) {
+  if (g.T == 0) return cudaSuccess;
+  hyb_rows_kernel<T><<<warp_blocks(g.T), 256, 0, s>>>(
+      g.T, g.F, g.C, g.cnt, static_cast<const T*>(g.val), g.idx, g.spill_ref, g.spill_cap,
+      static_cast<const T*>(g.spill_val), o.C_h, static_cast<T*>(o.ell_g), o.ell_idx, o.row_nnz,
+      status);
+  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(0, g.T, o.row_nnz, o.C_h, o.row_slot, o.backup_rows,
+                                         o.backup_cap, o.n_backup, status);
+  if (o.backup_cap > 0)
+    hyb_backup_kernel<T><<<warp_blocks(o.backup_cap), 256, 0, s>>>(
+        g.T, g.F, g.C, g.cnt, static_cast<const T*>(g.val), g.idx, g.spill_ref, g.spill_cap,
+        static_cast<const T*>(g.spill_val), o.backup_rows, o.n_backup, o.backup_cap,
+        static_cast<T*>(o.backup_g));
+  return cudaGetLastError();
+}
+
+template <typename T, int NCH>
+cudaError_t forward_t(const void* x, const tw_hybrid& gu, const void* Wu_t, const void* Wd, int d,
+                      void* y, tw_dtype y_dtype, cudaStream_t s) {
+  hyb_forward_kernel<T, NCH><<<warp_blocks(gu.T), 256, 0, s>>>(
+      view_of<T>(gu), static_cast<const T*>(x), static_cast<const T*>(Wu_t),
+      static_cast<const T*>(Wd), d, y, y_dtype);
+  return cudaGetLastError();
+}
+
+template <typename T, int NCH>
+cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const void* Wg_t,
+                       const void* Wu_t, const void* Wd, int d, float lam, void* dx,
+                       tw_dtype dx_dtype, float* dWg_t, float* dWu_t, float* dWd, void* ws,
+                       int32_t* status, cudaStream_t s) {
+  const HView<T> h = view_of<T>(gu);
+  const BwdWs w = carve(ws, gu.T, gu.F, gu.C_h, gu.backup_cap);
+  const int nb = (gu.T + TB - 1) / TB;
+  const size_t hist_bytes = sizeof(int32_t) * (size_t)gu.F;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(hyb_count_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         200 * 1024);
+    cudaFuncSetAttribute(hyb_fill_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         200 * 1024);
+    attr_set = true;
+  }
+  // entry offsets of every token (token-major order)
+  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(2, gu.T, gu.row_nnz, 0, w.e0, gu.row_slot,
+                                         gu.backup_cap, nullptr, status);
+  hyb_backward_token_kernel<T, NCH><<<warp_blocks(gu.T), 256, 0, s>>>(
+      h, static_cast<const T*>(dy), static_cast<const T*>(Wg_t), static_cast<const T*>(Wu_t),
+      static_cast<const T*>(Wd), d, lam, w.e0, w.pay, dx, dx_dtype);
+  hyb_count_kernel<T><<<nb, 256, hist_bytes, s>>>(h, w.cntb);
+  hyb_colscan_kernel<<<(gu.F + 255) / 256, 256, 0, s>>>(nb, gu.F, w.cntb, w.unit_total);
+  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.unit_total, 0, w.unit_off, nullptr, 0,
+                                         nullptr, status);
+  hyb_fill_kernel<T><<<nb, 256, hist_bytes, s>>>(h, w.cntb, w.unit_off, w.e0, w.list);
+  hyb_wgrad_kernel<T><<<gu.F, 256, 0, s>>>(gu.F, d, static_cast<const T*>(x),
+                                           static_cast<const T*>(dy), w.unit_off, w.list, w.pay,
+                                           dWg_t, dWu_t, dWd);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_twell_to_hybrid(const tw_twell& g, const tw_hybrid& out, int32_t* status,
+                                   cudaStream_t stream) {
+  return g.dtype == TW_BF16 ? to_hybrid_t<uint16_t>(g, out, status, stream)
+                            : to_hybrid_t<float>(g, out, status, stream);
+}
+
+cudaError_t launch_hybrid_forward(const void* x, const tw_hybrid& gu, const void* Wu_t,
+                                  const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                  int32_t* status, cudaStream_t stream) {
+  (void)status;
+  if (gu.T == 0) return cudaSuccess;
+  if (gu.dtype == TW_BF16) {
+    if (d <= 256) return forward_t<uint16_t, 1>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+    if (d <= 512) return forward_t<uint16_t, 2>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+    if (d <= 1024) return forward_t<uint16_t, 4>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+    return forward_t<uint16_t, 8>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+  }
+  if (d <= 128) return forward_t<float, 1>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+  if (d <= 256) return forward_t<float, 2>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+  if (d <= 512) return forward_t<float, 4>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+  if (d <= 1024) return forward_t<float, 8>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+  return forward_t<float, 16>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+}
+
+size_t hybrid_backward_ws_bytes(int T, int d, int F, int C_h, int backup_cap) {
+  (void)d;
+  return carve(nullptr, T, F, C_h, backup_cap).bytes;
+}
+
+cudaError_t launch_hybrid_backward(const void* x, const void* dy, const tw_hybrid& gu,
+                                   const void* Wg_t, const void* Wu_t, const void* Wd, int d,
+                                   float lam, void* dx, tw_dtype dx_dtype, float* dWg_t,
+                                   float* dWu_t, float* dWd, void* ws, size_t ws_bytes,
+                                   int32_t* status, cudaStream_t stream) {
+  (void)ws_bytes;
+  if (gu.T == 0) {
+    cudaMemsetAsync(dWg_t, 0, sizeof(float) * (size_t)gu.F * d, stream);
+    cudaMemsetAsync(dWu_t, 0, sizeof(float) * (size_t)gu.F * d, stream);
+    cudaMemsetAsync(dWd, 0, sizeof(float) * (size_t)gu.F * d, stream);
+    return cudaGetLastError();
+  }
+#define TW_BWD(TY, N)                                                                          \
+  return backward_t<TY, N>(x, dy, gu, Wg_t, Wu_t, Wd, d, lam, dx, dx_dtype, dWg_t, dWu_t, dWd, \
+                           ws, status, stream)
+  if (gu.dtype == TW_BF16) {
+    if (d <= 256) TW_BWD(uint16_t, 1);
+    if (d <= 512) TW_BWD(uint16_t, 2);
+    if (d <= 1024) TW_BWD(uint16_t, 4);
+    TW_BWD(uint16_t, 8);
+  }
+  if (d <= 128) TW_BWD(float, 1);
+  if (d <= 256) TW_BWD(float, 2);
+  if (d <= 512) TW_BWD(float, 4);
+  if (d <= 1024) TW_BWD(float, 8);
+  TW_BWD(float, 16);
+#undef TW_BWD
+}
+
+}  // namespace tw

@@ -1,0 +1,47 @@
+// tw_internal.h -- host-side launchers shared between the library's .cu files.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "twell.h"
+
+namespace tw {
+
+// Device properties cached per device.
+int num_sms();
+
+// Default upper bound on any single pipeline wait inside a kernel (ns).
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
+
+// tcgen05 bf16 gate GEMM with TwELL epilogue.  Shapes validated by caller.
+cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, int F,
+                                 const tw_twell& out, void* dump, int32_t* status,
+                                 cudaStream_t stream);
+// fp32 CUDA-core gate with the same TwELL packing.
+cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int d, int F,
+                                  const tw_twell& out, float* dump, int32_t* status,
+                                  cudaStream_t stream);
+// Fused up+down over TwELL.
+cudaError_t launch_fused_updown(const void* x, const tw_twell& g, const void* Wu_t,
+                                const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                int32_t* status, cudaStream_t stream);
+// Dense comparator pieces (bf16, tcgen05).
+cudaError_t launch_dense_gateup_tc(const void* x, const void* Wg_t, const void* Wu_t, int T,
+                                   int d, int F, void* h, int32_t* status, cudaStream_t stream);
+cudaError_t launch_dense_down_tc(const void* h, const void* Wd_dense, int T, int d, int F,
+                                 void* y, int32_t* status, cudaStream_t stream);
+// Hybrid (training) kernels.
+cudaError_t launch_twell_to_hybrid(const tw_twell& g, const tw_hybrid& out, int32_t* status,
+                                   cudaStream_t stream);
+cudaError_t launch_hybrid_forward(const void* x, const tw_hybrid& gu, const void* Wu_t,
+                                  const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                  int32_t* status, cudaStream_t stream);
+size_t hybrid_backward_ws_bytes(int T, int d, int F, int C_h, int backup_cap);
+cudaError_t launch_hybrid_backward(const void* x, const void* dy, const tw_hybrid& gu,
+                                   const void* Wg_t, const void* Wu_t, const void* Wd, int d,
+                                   float lam, void* dx, tw_dtype dx_dtype, float* dWg_t,
+                                   float* dWu_t, float* dWd, void* ws, size_t ws_bytes,
+                                   int32_t* status, cudaStream_t stream);
+
+}  // namespace tw

@@ -1,0 +1,391 @@
+"""Benchmark of the activation-sparse gated FFN (TwELL) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ffn_2b] [--impl ours|reference]
+
+One step = one pass of the inference hot path over one synthetic batch:
+twell_gate_gemm (tcgen05 gate GEMM + TwELL epilogue) then twell_fused_updown
+(gather up/down over the active units).  Inputs are resident in HBM; x,
+Wg, Wu, Wd total 160 MB at the 2B shape, more than the 126 MB L2, so no flush
+is done between steps.  Rank 0 prints ONE JSON line.  Under torchrun every
+rank runs an independent replica on its own GPU (weak scaling: no data-path
+collective; only the timing is max-reduced).
+
+--impl reference times the CPU oracle (single-threaded fp64 C) on a bounded
+token sample per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from activation_sparse_transformer_tma_b200 import synth  # noqa: E402
+
+METRIC = "FFN tokens/sec on 1 B200 (2B-shaped, ~99% sparse) + % HBM/tensor roofline"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="ffn_2b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip comparator/training/decode legs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        self.gpu = vis.split(",")[local_rank] if vis else str(local_rank)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- reference --
+def run_reference(args, rank):
+    """CPU oracle arm: a bounded token sample per step, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    w = synth.make_workload(args.workload)
+    dt = w["dtype"]
+    x = synth.widen(w["x"], dt)
+    Wg, Wu, Wd = (synth.widen(w[k], dt) for k in ("Wg_t", "Wu_t", "Wd"))
+
+    def one(rows):
+        g = oracle.gate_rows(x, Wg, rows)
+        enc = oracle.twell_encode(g, w["W"], w["C"])
+        return oracle.twell_ffn(x[rows], enc, Wu, Wd)
+
+    t0 = time.perf_counter()
+    one(synth.subsample_rows(w["T"], 2, seed=99))
+    per_tok = (time.perf_counter() - t0) / 2
+    total_steps = args.steps + args.warmup
+    n = int(max(1, min(256, 150.0 / max(total_steps, 1) / per_tok)))
+    for s in range(args.warmup):
+        one(synth.subsample_rows(w["T"], n, seed=1000 + s))
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        one(synth.subsample_rows(w["T"], n, seed=2000 + s))
+    el = time.perf_counter() - t0
+    v = n * args.steps / el
+    sample = (f"{n} seeded tokens of {args.workload} per step (gate + TwELL encode + sparse "
+              f"FFN, fp64), 1 thread of {os.cpu_count()} host cores")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, args),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    return {"workload": w["name"], "T": w["T"], "d": w["d"], "F": w["F"], "W": w["W"],
+            "C": w["C"], "dtype": w["dtype"], "global_batch_tokens": w["T"] * args.gpus,
+            "parallelism": f"replicas{args.gpus}", "seed": 0,
+            "l2": "inputs (x, Wg, Wu, Wd) exceed the 126 MB L2; no flush between steps"}
+
+
+# --------------------------------------------------------------------- ours --
+def src_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "activation_sparse_transformer_tma_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(profile_md, sha):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile_md)).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_b) or m_sha.group(1) != sha:
+        return None
+    return float(m_b.group(1))
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from activation_sparse_transformer_tma_b200 import twell as tw
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    w = synth.make_workload(args.workload)
+    T, d, F, C = w["T"], w["d"], w["F"], w["C"]
+    dt = torch.bfloat16 if w["dtype"] == synth.BF16 else torch.float32
+
+    def dev(a):
+        if w["dtype"] == synth.BF16:
+            return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(a).cuda()
+
+    x, Wg, Wu, Wd = (dev(w[k]) for k in ("x", "Wg_t", "Wu_t", "Wd"))
+    g = tw.Twell(T, F, C, dtype=dt, spill_cap=max(4096, (F // 128) * T // 8))
+    y = torch.empty((T, d), dtype=dt, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tw.twell_gate_gemm(x, Wg, g, None, status)
+        if ev is not None:
+            ev[1].record(stream)
+        tw.twell_fused_updown(x, g, Wu, Wd, y, status)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(K):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_gate = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    ms_fused = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    st = int(status.item())
+    if dist:
+        tt = torch.tensor([ms_total], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / K
+    value = world * T * K / (ms_total / 1e3)
+
+    # ------------------------------------------------------------- e2e leg --
+    xh = torch.empty((T, d), dtype=dt, pin_memory=True)
+    xh.copy_(x.cpu())
+    yh = torch.empty((T, d), dtype=dt, pin_memory=True)
+    E = max(3, min(K, 30))
+
+    def e2e_step():
+        x.copy_(xh, non_blocking=True)
+        tw.twell_gate_gemm(x, Wg, g, None, status)
+        tw.twell_fused_updown(x, g, Wu, Wd, y, status)
+        yh.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([ms_e2e], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    e2e = {"value": world * T * E / (ms_e2e / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+           "d2h_bytes_per_step": yh.numel() * yh.element_size()}
+
+    hbm, tf_burst, tf_sust, src = peaks()
+    flops_gate = 2.0 * T * d * F
+    tflops_gate = flops_gate / (ms_gate * 1e-3) / 1e12
+    sha = src_sha("gemm_tc.cu", "tw_common.cuh")
+    roof = {"kernel": "twell_gate_gemm (tcgen05 + TwELL epilogue)", "bound": "tensor",
+            "achieved": tflops_gate, "peak": tf_sust, "unit": "TFLOP/s",
+            "frac": tflops_gate / tf_sust,
+            "peak_source": f"{src} bf16 sustained (kernel timed inside a long loop)",
+            "frac_of_burst_peak": tflops_gate / tf_burst,
+            "traffic": profiled_traffic("gate_twell_gemm_ffn_2b.md", sha),
+            "algorithmic": f"2*T*d*F = {flops_gate:.4g} FLOP per launch"}
+
+    # fused kernel: algorithmic bytes (unique HBM) and gathered bytes, per launch
+    cnt = g.cnt.to(torch.int64)
+    nnz = int(cnt.sum().item())
+    Kt = F // 128
+    bytes_unique = (2 * T * d * 2          # x in, y out
+                    + Kt * T * (C * 3 + 1)  # TwELL read
+                    + int((cnt.sum(1) > 0).sum().item()) * 0)  # (live-unit bytes added below)
+    live_units = int(((g.cnt > 0).any(dim=1)).sum().item())  # tiles touched (coarse)
+    bytes_gathered = nnz * 2 * d * 2
+    kernels = {
+        "gate_twell_gemm": {"ms": ms_gate, "tflops": tflops_gate,
+                            "frac_sustained": tflops_gate / tf_sust,
+                            "frac_burst": tflops_gate / tf_burst},
+        "fused_updown": {"ms": ms_fused, "nnz_per_token": nnz / T,
+                         "gathered_GBps": bytes_gathered / (ms_fused * 1e-3) / 1e9,
+                         "fma_tflops": 2.0 * nnz * 2 * d / (ms_fused * 1e-3) / 1e12,
+                         "x_y_twell_GBps": bytes_unique / (ms_fused * 1e-3) / 1e9},
+        "spills_per_step": int(g.spill_n.item()),
+    }
+    _ = live_units
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded generator: Zipf(1.1) units, lognormal token skew, "
+                    "mean 29 active units per token)",
+            "config": config_of(w, args), "roofline": roof, "e2e": e2e,
+            "gpu_launches": 2 * K, "clocks": clk, "kernels": kernels,
+            "device_status": st}
+
+    if rank == 0 and not args.no_extras:
+        line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_leg(w, y)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_sparse, args):
+    """The in-library dense bf16 FFN of the same shape (tcgen05, no cuBLAS)."""
+    Wd_dense = Wd.t().contiguous()
+    h = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    yd = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        tw.dense_ffn_forward(x, Wg, Wu, Wd_dense, h, yd)
+    torch.cuda.synchronize()
+    n = max(5, min(args.steps, 100))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        tw.dense_ffn_forward(x, Wg, Wu, Wd_dense, h, yd)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    flops = 2.0 * T * d * F * 3
+    return {"ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "tflops": flops / (ms * 1e-3) / 1e12,
+            "sparse_speedup": ms / ms_sparse}
+
+
+def cpu_baseline_leg(w, y_gpu):
+    """Oracle timed on a bounded sample (rank 0); also checks the timed y rows."""
+    import oracle
+    import torch
+    rows = synth.subsample_rows(w["T"], 128, seed=5)
+    dt = w["dtype"]
+    x = synth.widen(w["x"], dt)
+    Wg, Wu, Wd = (synth.widen(w[k], dt) for k in ("Wg_t", "Wu_t", "Wd"))
+    t0 = time.perf_counter()
+    g = oracle.gate_rows(x, Wg, rows)
+    enc = oracle.twell_encode(g, w["W"], w["C"])
+    y_ref = oracle.twell_ffn(x[rows], enc, Wu, Wd)
+    el = time.perf_counter() - t0
+    yg = y_gpu[torch.as_tensor(rows, device=y_gpu.device).long()].float().cpu().numpy()
+    err = float(np.max(np.abs(yg - y_ref)) / np.sqrt(np.mean(y_ref ** 2)))
+    return {"value": len(rows) / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(rows)} seeded tokens of {w['name']}: gate + TwELL encode + sparse "
+                      f"FFN in fp64, 1 thread of {os.cpu_count()} host cores",
+            "parity_max_err_over_rms": err, "parity_tol": 1e-2}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

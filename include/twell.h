@@ -1,0 +1,216 @@
+/*
+ * twell.h -- C ABI of libtwell.so: the activation-sparse gated FFN of a
+ * ReLU-gated transformer layer on one NVIDIA B200 (sm_100a), with the
+ * activations carried in the Tile-wise ELLPACK ("TwELL") format.
+ *
+ * Method: technical summary page of "Sparser, Faster, Lighter Transformer
+ * Language Models" (arXiv 2603.23198):
+ *   section 2.1  TwELL format, built in the gate matmul's epilogue in shared
+ *                memory, g = ReLU(x Wg);
+ *   section 2.2  fused up + down projection over the non-zero activations;
+ *   section 2.3  hybrid format for training (compact ELL + dense backup rows);
+ *   section 2.4  hybrid-to-dense / dense-to-hybrid training kernels with an
+ *                L1 term on the gate activations.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * Ownership   The caller owns every buffer.  The library never allocates or
+ *             frees device memory and never keeps a pointer after the call.
+ * Pointers    All tensor pointers are DEVICE pointers, 16-byte aligned.
+ * Layouts     Row-major.  x, y, dy, dx: [T][d].  Weights: [F][d] with row j =
+ *             unit j's d-vector: Wg_t = gate_proj.weight, Wu_t = up_proj.weight,
+ *             Wd = down_proj.weight transposed ([F][d]).  The dense comparator
+ *             alone takes the down weight as down_proj.weight ([d][F]).
+ * dtypes      TW_BF16 tensors are raw bf16; TW_F32 tensors are IEEE fp32.
+ *             Arithmetic accumulates in fp32.
+ * Asynchrony  Work is enqueued on `stream` and the call returns without
+ *             synchronising.  Pass 0 for the legacy default stream.
+ * Errors      The return value reports host-side validation (checked before
+ *             any launch) and launch errors.  Conditions found on the device
+ *             (capacity exceeded, a pipeline wait that timed out) are OR-ed
+ *             into the caller's `dev_status` word as bit (1 << tw_status);
+ *             dev_status may be NULL.  The caller zeroes it and reads it after
+ *             synchronising; tw_status_string names each code.
+ * Limits      W == 128; 0 <= C <= 32; F % W == 0; d % 8 == 0; 8 <= d <= 2048
+ *             for the fused and hybrid kernels; T >= 1.  F <= 65536 (hybrid
+ *             indices are uint16).
+ */
+#ifndef TWELL_H
+#define TWELL_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define TW_API __attribute__((visibility("default")))
+#else
+#define TW_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TW_OK = 0,
+  TW_ERR_INVALID_ARG = 1,      /* null pointer, bad size, mismatched shapes   */
+  TW_ERR_UNSUPPORTED = 2,      /* valid but outside the limits above          */
+  TW_ERR_ALIGNMENT = 3,        /* a pointer is not 16-byte aligned            */
+  TW_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed        */
+  TW_ERR_SPILL_CAPACITY = 5,   /* device: more TwELL spill entries than cap   */
+  TW_ERR_BACKUP_CAPACITY = 6,  /* device: more hybrid backup rows than cap    */
+  TW_ERR_TIMEOUT = 7,          /* device: a bounded pipeline wait ran out     */
+  TW_ERR_WORKSPACE = 8         /* workspace smaller than the size query says  */
+} tw_status;
+
+typedef enum { TW_F32 = 0, TW_BF16 = 1 } tw_dtype;
+
+/*
+ * TwELL tensor for the gate activations g [T][F] (section 2.1): the F columns
+ * are cut into K = F / W tiles of width W.  For every (tile k, token t):
+ *   cnt[k][t]        number of non-zero g in columns [k*W, (k+1)*W) -- the
+ *                    true count, which may exceed C;
+ *   val[k][t][s], idx[k][t][s], s < min(cnt, C)
+ *                    the first non-zeros in ascending column order and their
+ *                    tile-local column (0..W-1); slots s >= cnt hold (+0, 0);
+ *   if cnt > C       the whole W-wide segment is copied to spill entry
+ *                    r = spill_ref[k][t]: spill_val[r][0..W-1], and
+ *                    spill_tk[r] = {t, k}.  Entries are numbered in arrival
+ *                    order (not deterministic); *spill_n receives the number
+ *                    of entries needed, which may exceed spill_cap (entries
+ *                    past the cap are dropped and TW_ERR_SPILL_CAPACITY is
+ *                    flagged).  spill_ref is written only where cnt > C.
+ * Array shapes: val [K][T][C] (dtype), idx [K][T][C] uint8, cnt [K][T] uint8,
+ * spill_ref [K][T] int32, spill_tk [spill_cap][2] int32, spill_val
+ * [spill_cap][W] (dtype), spill_n one int32.  With C == 0 val/idx may be NULL.
+ */
+typedef struct {
+  int32_t T, F, W, C;
+  tw_dtype dtype;
+  void* val;
+  uint8_t* idx;
+  uint8_t* cnt;
+  int32_t* spill_ref;
+  int32_t spill_cap;
+  int32_t* spill_tk;
+  void* spill_val;
+  int32_t* spill_n;
+} tw_twell;
+
+/*
+ * Hybrid tensor (section 2.3): every token row is either an ELL row or a
+ * dense backup row, decided by its non-zero count nnz = row_nnz[t]:
+ *   nnz <= C_h   ELL row: row_slot[t] = -1; ell_g[t][0..nnz) are its
+ *                non-zeros in ascending unit order, ell_idx the global unit
+ *                indices; slots past nnz hold (+0, 0);
+ *   nnz >  C_h   backup row: row_slot[t] = b, its slot; backup_rows[b] = t;
+ *                backup_g[b][0..F) is the dense g row.  Slots are numbered in
+ *                ascending token order.  *n_backup receives the number of
+ *                backup rows needed (rows past backup_cap are dropped and
+ *                TW_ERR_BACKUP_CAPACITY is flagged).
+ * ell_u / backup_u hold the up activation u = x Wu on the same pattern (+0
+ * elsewhere); hybrid_ffn_forward fills them and the backward reads them.
+ * Shapes: ell_g, ell_u [T][C_h] (dtype); ell_idx [T][C_h] uint16; row_nnz,
+ * row_slot [T] int32; backup_rows [backup_cap] int32; backup_g, backup_u
+ * [backup_cap][F] (dtype); n_backup one int32.
+ */
+typedef struct {
+  int32_t T, F, C_h;
+  tw_dtype dtype;
+  void* ell_g;
+  void* ell_u;
+  uint16_t* ell_idx;
+  int32_t* row_nnz;
+  int32_t* row_slot;
+  int32_t backup_cap;
+  int32_t* backup_rows;
+  void* backup_g;
+  void* backup_u;
+  int32_t* n_backup;
+} tw_hybrid;
+
+/*
+ * Gate projection with TwELL output (section 2.1): g = ReLU(x Wg), with
+ * z = x Wg accumulated in fp32 and g rounded to out->dtype, packed straight
+ * into *out by the matmul's epilogue.  x [T][d] and Wg_t [F][d] have `dtype`,
+ * which must equal out->dtype.  bf16 runs on the tcgen05 tensor cores fed by
+ * TMA; fp32 runs at full fp32 precision on the CUDA cores.  out->T, out->F
+ * must equal T, F.  g_dense_dump, if not NULL, receives the dense rounded g
+ * [T][F] (dtype) -- a test aid; pass NULL for speed.
+ */
+TW_API tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int32_t d, int32_t F,
+                          tw_dtype dtype, const tw_twell* out, void* g_dense_dump,
+                          int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Fused up + down projection over TwELL (section 2.2): for every token t and
+ * every active unit j of g (slots and spilled segments),
+ *   u = x_t . Wu_t[j]  (fp32),  h = g_tj * u,  y_t += h * Wd[j]  (fp32),
+ * and y_t is stored in y_dtype.  No dense intermediate reaches memory.
+ * x, Wu_t and Wd have g->dtype.  y [T][d].
+ */
+TW_API tw_status twell_fused_updown(const void* x, const tw_twell* g, const void* Wu_t,
+                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype,
+                             int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * TwELL -> hybrid conversion (section 2.3).  out->T, out->F equal g->T,
+ * g->F and out->dtype equals g->dtype.  Fills ell_g, ell_idx, row_nnz,
+ * row_slot, backup_rows, backup_g, n_backup.
+ */
+TW_API tw_status twell_to_hybrid(const tw_twell* g, const tw_hybrid* out, int32_t* dev_status,
+                          cudaStream_t stream);
+
+/*
+ * Training forward on the hybrid pattern (sections 2.3-2.4): u = x Wu sampled
+ * at the active positions -> gu->ell_u / gu->backup_u (rounded to gu->dtype,
+ * +0 off the pattern), then y = (g * u) Wd with fp32 accumulation and the
+ * unrounded u.  x, Wu_t, Wd have gu->dtype.  y [T][d] in y_dtype.
+ */
+TW_API tw_status hybrid_ffn_forward(const void* x, const tw_hybrid* gu, const void* Wu_t,
+                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype,
+                             int32_t* dev_status, cudaStream_t stream);
+
+/* Bytes of workspace hybrid_ffn_backward needs for these sizes. */
+TW_API size_t hybrid_ffn_backward_workspace_size(int32_t T, int32_t d, int32_t F, int32_t C_h,
+                                          int32_t backup_cap);
+
+/*
+ * Training backward on the hybrid pattern (section 2.4), for the loss
+ * L = sum(y * dy) + l1_lambda * sum(g), from the saved g and u of gu:
+ * for every active (t, j):  dh = dy_t . Wd[j];  du = dh * g;
+ * dz = dh * u + l1_lambda;  dx_t += du Wu_t[j] + dz Wg_t[j];
+ * dWd[j] += (g u) dy_t;  dWu_t[j] += du x_t;  dWg_t[j] += dz x_t.
+ * Inactive positions contribute nothing (ReLU'(0) = 0, sign(0) = 0).
+ * dx [T][d] in dx_dtype; dWg_t, dWu_t, dWd [F][d] fp32, fully overwritten.
+ * Weight gradients are summed in ascending token order (deterministic).
+ * ws: device workspace of at least hybrid_ffn_backward_workspace_size bytes.
+ */
+TW_API tw_status hybrid_ffn_backward(const void* x, const void* dy, const tw_hybrid* gu,
+                              const void* Wg_t, const void* Wu_t, const void* Wd, int32_t d,
+                              float l1_lambda, void* dx, tw_dtype dx_dtype, float* dWg_t,
+                              float* dWu_t, float* dWd, void* ws, size_t ws_bytes,
+                              int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Dense comparator (the non-sparse baseline of section 4), bf16 only, on the
+ * same tcgen05 pipeline: h = ReLU(x Wg) * (x Wu) in one GEMM over the
+ * interleaved gate/up weights, written to h_ws [T][F] bf16, then y = h Wd
+ * with Wd_dense = down_proj.weight [d][F].  y [T][d] bf16.
+ */
+TW_API tw_status dense_ffn_forward(const void* x, const void* Wg_t, const void* Wu_t,
+                            const void* Wd_dense, int32_t T, int32_t d, int32_t F, void* h_ws,
+                            void* y, int32_t* dev_status, cudaStream_t stream);
+
+/* Human-readable name of a status code. */
+TW_API const char* tw_status_string(tw_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+TW_API int32_t twell_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TWELL_H */

@@ -1,0 +1,126 @@
+"""Host-side tests of the C ABI: the library loads without a GPU, exports every
+symbol include/twell.h declares, and rejects bad arguments before any launch.
+
+Bad-argument calls pass fake (never dereferenced) device addresses: the
+library validates every argument on the host and returns before touching the
+device, so these tests run on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from activation_sparse_transformer_tma_b200 import build as tw_build
+from activation_sparse_transformer_tma_b200 import twell
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "twell.h")
+
+OK, INVALID, UNSUPPORTED, ALIGN, CUDA = 0, 1, 2, 3, 4
+FAKE = 0x10000  # 16-byte aligned, never dereferenced on the host
+
+
+@pytest.fixture(scope="module")
+def L():
+    tw_build.build()
+    return twell.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"TW_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ("twell_gate_gemm", "twell_fused_updown", "twell_to_hybrid", "hybrid_ffn_backward"):
+        assert n in names
+    assert sorted(names) == sorted(twell.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in declared_symbols():
+        assert hasattr(L, n), n
+        assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
+
+
+def test_nm_shows_only_the_abi_as_dynamic_text_symbols(L):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", twell.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    text_syms = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(declared_symbols()) <= text_syms
+
+
+def test_status_strings_and_version(L):
+    for code, name in enumerate(twell.STATUS):
+        assert L.tw_status_string(code).decode() == name
+    assert L.twell_version() >= 100
+
+
+def _tw(T=256, F=1024, W=128, C=8, dtype=twell.TW_BF16, spill_cap=64, base=FAKE):
+    return twell.TwTwellC(T, F, W, C, dtype, base, base, base, base, spill_cap, base, base, base)
+
+
+def _gate(L, tw, x=FAKE, w=FAKE, T=256, d=512, F=1024, dtype=twell.TW_BF16):
+    return L.twell_gate_gemm(x, w, T, d, F, dtype, ctypes.byref(tw), None, None, None)
+
+
+def test_gate_validation(L):
+    assert _gate(L, _tw(), x=None) == INVALID
+    assert _gate(L, _tw(), x=FAKE + 8) == ALIGN
+    assert _gate(L, _tw(W=64)) == UNSUPPORTED            # tile width must be 128
+    assert _gate(L, _tw(C=33)) == UNSUPPORTED            # capacity above the epilogue's 32
+    assert _gate(L, _tw(F=1000), F=1000) == UNSUPPORTED  # F not a multiple of W
+    assert _gate(L, _tw(T=255)) == INVALID               # out->T != T
+    assert _gate(L, _tw(), d=500) == UNSUPPORTED         # d % 8 != 0
+    assert _gate(L, _tw(), d=32) == UNSUPPORTED          # tensor-core path needs d >= 64
+    assert _gate(L, _tw(dtype=twell.TW_F32)) == INVALID  # dtype mismatch
+    assert _gate(L, _tw(C=-1)) == INVALID
+    bad = _tw()
+    bad.cnt = None
+    assert _gate(L, bad) == INVALID
+
+
+def test_fused_validation(L):
+    tw = _tw()
+    f = L.twell_fused_updown
+    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE, 4096, FAKE, twell.TW_BF16, None, None) == UNSUPPORTED
+    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE, 100, FAKE, twell.TW_BF16, None, None) == UNSUPPORTED
+    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE + 4, 512, FAKE, twell.TW_BF16, None, None) == ALIGN
+    assert f(FAKE, ctypes.byref(tw), None, FAKE, 512, FAKE, twell.TW_BF16, None, None) == INVALID
+    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE, 512, FAKE, 7, None, None) == INVALID
+
+
+def _hy(T=256, F=1024, C_h=64, cap=32, dtype=twell.TW_BF16, base=FAKE):
+    return twell.TwHybridC(T, F, C_h, dtype, base, base, base, base, base, cap, base, base, base, base)
+
+
+def test_hybrid_validation(L):
+    tw, hy = _tw(), _hy()
+    assert L.twell_to_hybrid(ctypes.byref(tw), ctypes.byref(_hy(T=128)), None, None) == INVALID
+    assert L.twell_to_hybrid(ctypes.byref(tw), ctypes.byref(_hy(C_h=2000)), None, None) == INVALID
+    assert L.twell_to_hybrid(ctypes.byref(tw), ctypes.byref(_hy(F=65536 + 128)), None, None) in (INVALID, UNSUPPORTED)
+    ws = L.hybrid_ffn_backward_workspace_size(256, 512, 1024, 64, 32)
+    assert ws > 0
+    args = [FAKE, FAKE, ctypes.byref(hy), FAKE, FAKE, FAKE, 512, 2e-5, FAKE, twell.TW_BF16,
+            FAKE, FAKE, FAKE, FAKE]
+    assert L.hybrid_ffn_backward(*args, ws - 1, None, None) == 8       # TW_ERR_WORKSPACE
+    args2 = list(args)
+    args2[0] = FAKE + 2
+    assert L.hybrid_ffn_backward(*args2, ws, None, None) == ALIGN
+
+
+def test_workspace_size_grows_with_capacity(L):
+    a = L.hybrid_ffn_backward_workspace_size(8192, 2048, 8192, 64, 64)
+    b = L.hybrid_ffn_backward_workspace_size(8192, 2048, 8192, 64, 1024)
+    assert b > a > 0
+    assert L.hybrid_ffn_backward_workspace_size(-1, 2048, 8192, 64, 64) == 0
+
+
+def test_dense_validation(L):
+    f = L.dense_ffn_forward
+    assert f(FAKE, FAKE, FAKE, FAKE, 256, 100, 1024, FAKE, FAKE, None, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 256, 512, 1000, FAKE, FAKE, None, None) == UNSUPPORTED
+    assert f(None, FAKE, FAKE, FAKE, 256, 512, 1024, FAKE, FAKE, None, None) == INVALID

@@ -1,0 +1,339 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars (written per check below):
+* TwELL values / indices / counts and the hybrid split: bit-exact against the
+  oracle's encoding of the GPU's own dumped gate tensor (spills as sets).
+* End-to-end y: max|y_gpu - y_ref| <= 1e-2 * rms(y_ref) for bf16 and
+  <= 1e-5 * rms(y_ref) for fp32, y_ref the fp64 oracle from the same inputs
+  with g rounded to its storage dtype (TwELL stores g in the model dtype), and
+  y stored in fp32 (the accumulator precision).  A bf16-stored y adds its own
+  rounding, up to 2^-9 |y| per element, which for heavy-tailed y exceeds the
+  first bar; it is checked elementwise against 1e-2 rms + 2^-8 |y_ref|.
+* Gradients: the oracle's backward conditioned on the GPU's saved hybrid g and
+  u; max|d_gpu - d_ref| <= 1e-2 * rms(d_ref) per tensor (bf16).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_sparse_transformer_tma_b200 import synth
+from activation_sparse_transformer_tma_b200 import twell as tw
+from gpu_helpers import assert_twell_matches_oracle, f64, inputs, raw, rms, widened
+
+pytestmark = pytest.mark.gpu
+
+TOL = {synth.BF16: 1e-2, synth.F32: 1e-5}
+TDT = {synth.BF16: torch.bfloat16, synth.F32: torch.float32}
+
+
+def run_forward(w, C=None, spill_cap=None, dump=True, y_dtype=torch.float32):
+    dev = inputs(w)
+    T, d, F = w["T"], w["d"], w["F"]
+    C = w["C"] if C is None else C
+    dt = TDT[w["dtype"]]
+    g = tw.Twell(T, F, C, dtype=dt, spill_cap=spill_cap)
+    gd = torch.empty((T, F), dtype=dt, device="cuda") if dump else None
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, gd, st)
+    y = torch.empty((T, d), dtype=y_dtype, device="cuda")
+    tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y, st)
+    torch.cuda.synchronize()
+    return dev, g, gd, y, st
+
+
+def check_gate_values(g_dump64, x64, wg64, rows, g_round="bf16"):
+    """Dumped g against the oracle's rounded fp64 gate: the fp32-accumulated z
+    may land on the other side of a rounding boundary (one bf16 ulp, 2^-7
+    relative) or of zero (|z| at the level of the fp32 accumulation error)."""
+    ref = oracle.gate_rows(x64, wg64, rows, g_round=g_round)
+    err = np.abs(g_dump64[rows] - ref)
+    assert np.all(err <= 2.0 ** -7 * np.abs(ref) + 1e-4), float(err.max())
+
+
+def check_y(y64, w64, rows, tol, g_round="bf16", elem_rel=0.0):
+    out = oracle.dense_ffn(w64["x"][rows], w64["Wg_t"], w64["Wu_t"], w64["Wd"], g_round=g_round)
+    ref = out["y"]
+    s = rms(ref)
+    err = np.abs(y64[rows] - ref)
+    assert np.all(err <= tol * s + elem_rel * np.abs(ref)), (float(err.max()), s)
+    return float(err.max()) / s
+
+
+SMALL = [
+    # T, d, F, C, kind, mean_active
+    (300, 320, 640, 8, "dead20", 29.0),      # ragged T and F, spills
+    (300, 320, 640, 8, "dead20", 120.0),     # spill-heavy
+    (1, 256, 1024, 8, "zipf", 29.0),         # one token
+    (129, 64, 256, 0, "dead20", 29.0),       # C = 0: every non-empty tile spills
+    (257, 2048, 1280, 32, "zipf", 40.0),     # full-width rows, largest C
+    (128, 512, 2048, 16, "uniform4", 29.0),
+]
+
+
+@pytest.mark.parametrize("T,d,F,C,kind,ma", SMALL)
+def test_bf16_gate_and_fused_small(T, d, F, C, kind, ma):
+    w = synth.make_workload(T=T, d=d, F=F, W=128, C=C, dtype=synth.BF16, kind=kind,
+                            mean_active=ma, seed=T + d)
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    w64 = widened(w)
+    g64 = f64(gd)
+    rows = np.arange(T, dtype=np.int32)
+    check_gate_values(g64, w64["x"], w64["Wg_t"], rows)
+    assert_twell_matches_oracle(g, g64)
+    check_y(f64(y), w64, rows, TOL[synth.BF16])
+
+
+def test_bf16_output_y():
+    w = synth.make_workload(T=300, d=320, F=640, W=128, C=8, dtype=synth.BF16, kind="dead20",
+                            mean_active=29.0, seed=620)
+    _, g, gd, y, st = run_forward(w, y_dtype=torch.bfloat16)
+    _, _, _, y32, _ = run_forward(w)
+    # the bf16 output is the fp32 result rounded once
+    assert torch.equal(y, y32.to(torch.bfloat16))
+    check_y(f64(y), widened(w), np.arange(300, dtype=np.int32), TOL[synth.BF16],
+            elem_rel=2.0 ** -8)
+
+
+@pytest.mark.parametrize("C", [16, 2])
+def test_fp32_tiny_config(C):
+    w = synth.make_workload("tiny_fp32")
+    dev, g, gd, y, st = run_forward(w, C=C)
+    assert int(st.item()) == 0
+    w64 = widened(w)
+    g64 = f64(gd)
+    rows = np.arange(w["T"], dtype=np.int32)
+    ref = oracle.gate_rows(w64["x"], w64["Wg_t"], rows, g_round="f32")
+    assert np.max(np.abs(g64 - ref)) <= 1e-5 * max(rms(ref), 1e-30)
+    assert_twell_matches_oracle(g, g64)
+    if C == 2:
+        assert int(g.spill_n.item()) > 0
+    check_y(f64(y), w64, rows, TOL[synth.F32], g_round="f32")
+
+
+def test_ffn_0p5b_full_size():
+    w = synth.make_workload("ffn_0p5b")
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    w64 = widened(w)
+    g64 = f64(gd)
+    assert_twell_matches_oracle(g, g64)
+    rows = synth.subsample_rows(w["T"], 192)
+    check_gate_values(g64, w64["x"], w64["Wg_t"], rows)
+    check_y(f64(y), w64, rows, TOL[synth.BF16])
+
+
+def test_ffn_2b_full_size():
+    """The bench workload, same launch configuration: TwELL compared on every
+    token (in chunks), y on a seeded sample of rows."""
+    w = synth.make_workload("ffn_2b")
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    T = w["T"]
+    for r0 in range(0, T, 2048):
+        rows = np.arange(r0, min(T, r0 + 2048))
+        assert_twell_matches_oracle(g, f64(gd[r0:r0 + len(rows)]), rows=rows)
+    w64 = widened(w)
+    rows = synth.subsample_rows(T, 96)
+    check_gate_values(f64(gd), w64["x"], w64["Wg_t"], rows)
+    check_y(f64(y), w64, rows, TOL[synth.BF16])
+
+
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_decode_sizes(T):
+    w = synth.make_workload("decode_2b", T=T)
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    w64 = widened(w)
+    assert_twell_matches_oracle(g, f64(gd))
+    check_y(f64(y), w64, np.arange(T, dtype=np.int32), TOL[synth.BF16])
+
+
+def test_fused_without_dump_matches_dump_run():
+    w = synth.make_workload(T=200, d=256, F=512, W=128, C=8, dtype=synth.BF16, kind="dead20",
+                            mean_active=29.0, seed=3)
+    _, g1, _, y1, _ = run_forward(w, dump=True)
+    _, g2, _, y2, _ = run_forward(w, dump=False)
+    assert torch.equal(g1.cnt, g2.cnt) and torch.equal(g1.val, g2.val)
+    assert torch.equal(y1, y2)
+
+
+def test_all_inactive_gives_zero():
+    # x >= 0 and every gate weight < 0: every pre-activation is negative.
+    rng = np.random.default_rng(4)
+    w = dict(T=130, d=256, F=512, W=128, C=8, dtype=synth.BF16)
+    w["x"] = synth.to_storage(np.abs(rng.standard_normal((130, 256))), synth.BF16)
+    w["Wg_t"] = synth.to_storage(-np.abs(rng.standard_normal((512, 256))) / 16 - 1e-3, synth.BF16)
+    w["Wu_t"] = synth.to_storage(rng.standard_normal((512, 256)) / 16, synth.BF16)
+    w["Wd"] = synth.to_storage(rng.standard_normal((512, 256)) / 16, synth.BF16)
+    _, g, gd, y, st = run_forward(w)
+    assert int(g.cnt.max().item()) == 0 and int(g.spill_n.item()) == 0
+    assert float(y.float().abs().max().item()) == 0.0
+
+
+def test_spill_capacity_overflow_is_flagged_not_faulted():
+    w = synth.make_workload(T=256, d=256, F=512, W=128, C=2, dtype=synth.BF16, kind="dead20",
+                            mean_active=60.0, seed=6)
+    _, g, gd, y, st = run_forward(w, spill_cap=4)
+    need = int(g.spill_n.item())
+    assert need > 4
+    assert "TW_ERR_SPILL_CAPACITY" in tw.status_bits(st)
+    # counts and slots stay exact; the stored spills are a subset of the oracle's
+    ref = oracle.twell_encode(f64(gd), 128, 2)
+    assert np.array_equal(raw(g.cnt), ref["cnt"])
+    assert need == ref["n_spill"]
+    assert torch.isfinite(y.float()).all()
+
+
+def test_oracle_encoded_twell_drives_the_fused_kernel():
+    """Consumer-side check of the format contract: TwELL built by the oracle,
+    uploaded, and consumed by the fused kernel."""
+    w = synth.make_workload(T=150, d=512, F=1024, W=128, C=4, dtype=synth.BF16, kind="dead20",
+                            mean_active=40.0, seed=7)
+    w64 = widened(w)
+    dense = oracle.dense_ffn(w64["x"], w64["Wg_t"], w64["Wu_t"], w64["Wd"])
+    g_b = synth.round_bf16(dense["g"])
+    enc = oracle.twell_encode(g_b, 128, 4)
+    assert enc["n_spill"] > 0
+    g = tw.Twell(150, 1024, 4, dtype=torch.bfloat16, spill_cap=enc["n_spill"] + 1)
+    bits = lambda a: torch.from_numpy(synth.bf16_bits(a).view(np.int16)).cuda().view(torch.bfloat16)
+    g.val.copy_(bits(enc["val"]))
+    g.idx.copy_(torch.from_numpy(enc["idx"]))
+    g.cnt.copy_(torch.from_numpy(enc["cnt"]))
+    g.spill_ref.copy_(torch.from_numpy(enc["spill_ref"]))
+    g.spill_val[:enc["n_spill"]].copy_(bits(enc["spill_val"]))
+    dev = inputs(w)
+    y = torch.empty((150, 512), dtype=torch.float32, device="cuda")
+    tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y)
+    torch.cuda.synchronize()
+    ref = oracle.twell_ffn(w64["x"], enc, w64["Wu_t"], w64["Wd"])
+    assert np.max(np.abs(f64(y) - ref)) <= 1e-4 * rms(ref)
+
+
+def test_dense_comparator():
+    w = synth.make_workload(T=300, d=512, F=1024, W=128, C=8, dtype=synth.BF16, kind="dead20",
+                            mean_active=29.0, seed=8)
+    dev = inputs(w)
+    Wd_dense = dev["Wd"].t().contiguous()
+    h = torch.empty((300, 1024), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((300, 512), dtype=torch.bfloat16, device="cuda")
+    tw.dense_ffn_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], Wd_dense, h, y)
+    torch.cuda.synchronize()
+    w64 = widened(w)
+    rows = np.arange(300, dtype=np.int32)
+    # the comparator stores h and y in bf16, as a dense bf16 FFN does
+    check_y(f64(y), w64, rows, TOL[synth.BF16], elem_rel=2.0 ** -7)
+    dense = oracle.dense_ffn(w64["x"], w64["Wg_t"], w64["Wu_t"], w64["Wd"])
+    hr = dense["g"] * dense["u"]
+    assert np.all(np.abs(f64(h) - hr) <= 2.0 ** -7 * np.abs(hr) + 1e-3 * rms(hr))
+
+
+def test_dense_comparator_2b_shape_sampled():
+    w = synth.make_workload("ffn_2b")
+    dev = inputs(w)
+    T, d, F = w["T"], w["d"], w["F"]
+    h = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    tw.dense_ffn_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"].t().contiguous(), h, y)
+    torch.cuda.synchronize()
+    rows = synth.subsample_rows(T, 48)
+    check_y(f64(y), widened(w), rows, TOL[synth.BF16], elem_rel=2.0 ** -7)
+
+
+# ----------------------------------------------------------------- hybrid ---
+def run_hybrid(w, backup_cap=None):
+    T, d, F = w["T"], w["d"], w["F"]
+    dev, g, gd, y, st = run_forward(w)
+    hy = tw.Hybrid(T, F, w["C_h"], dtype=torch.bfloat16, backup_cap=backup_cap)
+    tw.twell_to_hybrid(g, hy, st)
+    yh = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, st)
+    ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, w["C_h"], hy.backup_cap),
+                     dtype=torch.uint8, device="cuda")
+    dx = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    dW = [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+    tw.hybrid_ffn_backward(dev["x"], dev["dy"], hy, dev["Wg_t"], dev["Wu_t"], dev["Wd"],
+                           w["lam"], dx, dW[0], dW[1], dW[2], ws, st)
+    torch.cuda.synchronize()
+    return dev, g, gd, y, st, hy, yh, dx, dW
+
+
+def hybrid_to_np(hy):
+    nb = min(int(hy.n_backup.item()), hy.backup_cap)
+    return {"T": hy.T, "F": hy.F, "C_h": hy.C_h, "ell_g": f64(hy.ell_g),
+            "ell_idx": raw(hy.ell_idx).view(np.uint16), "row_nnz": raw(hy.row_nnz),
+            "row_slot": raw(hy.row_slot), "backup_rows": raw(hy.backup_rows)[:nb],
+            "backup_g": f64(hy.backup_g)[:nb], "n_backup": int(hy.n_backup.item())}
+
+
+def check_hybrid_all(w, res):
+    dev, g, gd, y, st, hy, yh, dx, dW = res
+    assert int(st.item()) == 0, tw.status_bits(st)
+    g64 = f64(gd)
+    # split: bit-exact against the oracle's split of the GPU's own gate
+    ref = oracle.hybrid_split(g64, w["C_h"])
+    got = hybrid_to_np(hy)
+    assert got["n_backup"] == ref["n_backup"]
+    for k in ("row_nnz", "row_slot", "backup_rows"):
+        assert np.array_equal(got[k], ref[k]), k
+    assert np.array_equal(got["ell_idx"], ref["ell_idx"])
+    assert np.array_equal(got["ell_g"].view(np.uint64), ref["ell_g"].view(np.uint64))
+    assert np.array_equal(got["backup_g"].view(np.uint64), ref["backup_g"].view(np.uint64))
+    # forward: u on the pattern and y, against the oracle on the GPU's pattern
+    w64 = widened(w)
+    ell_u, backup_u, y_ref = oracle.hybrid_forward(w64["x"], got, w64["Wu_t"], w64["Wd"])
+    nb = len(got["backup_g"])
+    ug = np.concatenate([f64(hy.ell_u).ravel(), f64(hy.backup_u)[:nb].ravel()])
+    ur = np.concatenate([ell_u.ravel(), backup_u.ravel()])
+    on = np.concatenate([got["ell_g"].ravel(), got["backup_g"].ravel()]) != 0
+    assert np.all(ug[~on] == 0)                       # +0 off the pattern
+    assert np.all(np.abs(ug - ur) <= 2.0 ** -8 * np.abs(ur) + 1e-3 * rms(ur[on]))
+    assert np.max(np.abs(f64(yh) - y_ref)) <= TOL[synth.BF16] * rms(y_ref)
+    # the hybrid forward y equals the inference y up to rounding
+    assert np.max(np.abs(f64(yh) - f64(y))) <= TOL[synth.BF16] * rms(y_ref)
+    # backward, conditioned on the GPU's saved g and u
+    got_u = dict(got)
+    grads = oracle.hybrid_backward(w64["x"], w64["dy"], got, f64(hy.ell_u),
+                                   f64(hy.backup_u)[:nb], w64["Wg_t"], w64["Wu_t"], w64["Wd"],
+                                   w["lam"])
+    for name, a, b in zip(("dx", "dWg_t", "dWu_t", "dWd"), (dx, dW[0], dW[1], dW[2]), grads):
+        err = np.max(np.abs(f64(a) - b))
+        assert err <= TOL[synth.BF16] * rms(b), (name, err, rms(b))
+    return got_u
+
+
+def test_hybrid_small_ragged():
+    w = synth.make_workload(T=700, d=256, F=1024, W=128, C=8, C_h=16, dtype=synth.BF16,
+                            kind="pareto", lam=2e-5, seed=9, mean_active=12.0)
+    got = check_hybrid_all(w, run_hybrid(w))
+    assert 0 < got["n_backup"] < 700
+
+
+@pytest.mark.parametrize("C_h", [0, 1024])
+def test_hybrid_extreme_caps(C_h):
+    w = synth.make_workload(T=130, d=128, F=1024, W=128, C=8, C_h=C_h, dtype=synth.BF16,
+                            kind="pareto", lam=2e-5, seed=10, mean_active=10.0)
+    got = check_hybrid_all(w, run_hybrid(w, backup_cap=130))
+    if C_h == 0:
+        assert got["n_backup"] == int((got["row_nnz"] > 0).sum())
+    else:
+        assert got["n_backup"] == 0
+
+
+def test_hybrid_backup_capacity_overflow_is_flagged():
+    w = synth.make_workload(T=256, d=128, F=512, W=128, C=8, C_h=2, dtype=synth.BF16,
+                            kind="pareto", lam=2e-5, seed=11, mean_active=10.0)
+    dev, g, gd, y, st = run_forward(w)
+    hy = tw.Hybrid(256, 512, 2, dtype=torch.bfloat16, backup_cap=3)
+    tw.twell_to_hybrid(g, hy, st)
+    torch.cuda.synchronize()
+    assert int(hy.n_backup.item()) > 3
+    assert "TW_ERR_BACKUP_CAPACITY" in tw.status_bits(st)
+
+
+def test_training_config_full_size():
+    w = synth.make_workload("train_2b")
+    res = run_hybrid(w, backup_cap=2048)
+    got = check_hybrid_all(w, res)
+    assert got["n_backup"] > 0
