@@ -108,18 +108,25 @@ tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int32_t d,
                                              stream));
 }
 
+size_t twell_fused_updown_workspace_size(int32_t T, int32_t d) {
+  if (T < 0 || d <= 0) return 0;
+  return tw::fused_ws_bytes(T, d);
+}
+
 tw_status twell_fused_updown(const void* x, const tw_twell* g, const void* Wu_t, const void* Wd,
-                             int32_t d, void* y, tw_dtype y_dtype, int32_t* dev_status,
-                             cudaStream_t stream) {
+                             int32_t d, void* y, tw_dtype y_dtype, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, cudaStream_t stream) {
   tw_status st = check_twell(g);
   if (st != TW_OK) return st;
-  if (!x || !Wu_t || !Wd || !y || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
+  if (!x || !Wu_t || !Wd || !y || !ws || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
   if (d <= 0) return TW_ERR_INVALID_ARG;
   if (d % 8 != 0 || d > kMaxRowD) return TW_ERR_UNSUPPORTED;
-  if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y))
+  if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y) || !aligned16(ws))
     return TW_ERR_ALIGNMENT;
+  if (ws_bytes < tw::fused_ws_bytes(g->T, d)) return TW_ERR_WORKSPACE;
   if (g->T == 0) return TW_OK;
-  return from_cuda(tw::launch_fused_updown(x, *g, Wu_t, Wd, d, y, y_dtype, dev_status, stream));
+  return from_cuda(
+      tw::launch_fused_updown(x, *g, Wu_t, Wd, d, y, y_dtype, ws, dev_status, stream));
 }
 
 tw_status twell_to_hybrid(const tw_twell* g, const tw_hybrid* out, int32_t* dev_status,

@@ -22,9 +22,10 @@ cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, 
 cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int d, int F,
                                   const tw_twell& out, float* dump, int32_t* status,
                                   cudaStream_t stream);
-// Fused up+down over TwELL.
+// Fused up+down over TwELL (plan + persistent gather kernel).
+size_t fused_ws_bytes(int T, int d);
 cudaError_t launch_fused_updown(const void* x, const tw_twell& g, const void* Wu_t,
-                                const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                const void* Wd, int d, void* y, tw_dtype y_dtype, void* ws,
                                 int32_t* status, cudaStream_t stream);
 // Dense comparator pieces (bf16, tcgen05).
 cudaError_t launch_dense_gateup_tc(const void* x, const void* Wg_t, const void* Wu_t, int T,

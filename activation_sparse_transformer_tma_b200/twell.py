@@ -22,7 +22,8 @@ TW_F32, TW_BF16 = 0, 1
 STATUS = ["TW_OK", "TW_ERR_INVALID_ARG", "TW_ERR_UNSUPPORTED", "TW_ERR_ALIGNMENT",
           "TW_ERR_CUDA", "TW_ERR_SPILL_CAPACITY", "TW_ERR_BACKUP_CAPACITY",
           "TW_ERR_TIMEOUT", "TW_ERR_WORKSPACE"]
-EXPORTS = ["twell_gate_gemm", "twell_fused_updown", "twell_to_hybrid", "hybrid_ffn_forward",
+EXPORTS = ["twell_gate_gemm", "twell_fused_updown_workspace_size", "twell_fused_updown",
+           "twell_to_hybrid", "hybrid_ffn_forward",
            "hybrid_ffn_backward_workspace_size", "hybrid_ffn_backward", "dense_ffn_forward",
            "tw_status_string", "twell_version"]
 
@@ -66,7 +67,10 @@ def lib():
         vp, i32, st = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int
         PT, PH = ctypes.POINTER(TwTwellC), ctypes.POINTER(TwHybridC)
         L.twell_gate_gemm.argtypes = [vp, vp, i32, i32, i32, ctypes.c_int, PT, vp, vp, vp]
-        L.twell_fused_updown.argtypes = [vp, PT, vp, vp, i32, vp, ctypes.c_int, vp, vp]
+        L.twell_fused_updown_workspace_size.argtypes = [i32, i32]
+        L.twell_fused_updown_workspace_size.restype = ctypes.c_size_t
+        L.twell_fused_updown.argtypes = [vp, PT, vp, vp, i32, vp, ctypes.c_int, vp,
+                                         ctypes.c_size_t, vp, vp]
         L.twell_to_hybrid.argtypes = [PT, PH, vp, vp]
         L.hybrid_ffn_forward.argtypes = [vp, PH, vp, vp, i32, vp, ctypes.c_int, vp, vp]
         L.hybrid_ffn_backward_workspace_size.argtypes = [i32, i32, i32, i32, i32]
@@ -175,11 +179,20 @@ def twell_gate_gemm(x, Wg_t, out: Twell, g_dense_dump=None, dev_status=None, str
         _ptr(dev_status), _stream(stream)))
 
 
-def twell_fused_updown(x, g: Twell, Wu_t, Wd, y, dev_status=None, stream=None):
+def twell_fused_updown_workspace_size(T, d):
+    return int(lib().twell_fused_updown_workspace_size(T, d))
+
+
+def fused_workspace(T, d, device="cuda"):
+    """A caller-owned workspace tensor of the size twell_fused_updown needs."""
+    return torch.empty(twell_fused_updown_workspace_size(T, d), dtype=torch.uint8, device=device)
+
+
+def twell_fused_updown(x, g: Twell, Wu_t, Wd, y, ws, dev_status=None, stream=None):
     s = g.struct()
     _check("twell_fused_updown", lib().twell_fused_updown(
-        _ptr(x), ctypes.byref(s), _ptr(Wu_t), _ptr(Wd), x.shape[1], _ptr(y), _dt(y),
-        _ptr(dev_status), _stream(stream)))
+        _ptr(x), ctypes.byref(s), _ptr(Wu_t), _ptr(Wd), x.shape[1], _ptr(y), _dt(y), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
 
 
 def twell_to_hybrid(g: Twell, out: Hybrid, dev_status=None, stream=None):

@@ -120,7 +120,7 @@ def run_reference(args, rank):
     Wg, Wu, Wd = (synth.widen(w[k], dt) for k in ("Wg_t", "Wu_t", "Wd"))
 
     def one(rows):
-        g = oracle.gate_rows(x, Wg, rows)
+        g = oracle.gate_rows(x, Wg, rows, g_round=dt)
         enc = oracle.twell_encode(g, w["W"], w["C"])
         return oracle.twell_ffn(x[rows], enc, Wu, Wd)
 
@@ -200,8 +200,10 @@ def run_ours(args, rank, world, local_rank):
 
     x, Wg, Wu, Wd = (dev(w[k]) for k in ("x", "Wg_t", "Wu_t", "Wd"))
     g = tw.Twell(T, F, C, dtype=dt, spill_cap=max(4096, (F // 128) * T // 8))
-    y = torch.empty((T, d), dtype=dt, device="cuda")
+    # y is accumulated and stored in fp32 (the residual-stream precision)
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = tw.fused_workspace(T, d)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
@@ -210,7 +212,7 @@ def run_ours(args, rank, world, local_rank):
         tw.twell_gate_gemm(x, Wg, g, None, status)
         if ev is not None:
             ev[1].record(stream)
-        tw.twell_fused_updown(x, g, Wu, Wd, y, status)
+        tw.twell_fused_updown(x, g, Wu, Wd, y, ws, status)
         if ev is not None:
             ev[2].record(stream)
 
@@ -250,13 +252,13 @@ def run_ours(args, rank, world, local_rank):
     # ------------------------------------------------------------- e2e leg --
     xh = torch.empty((T, d), dtype=dt, pin_memory=True)
     xh.copy_(x.cpu())
-    yh = torch.empty((T, d), dtype=dt, pin_memory=True)
+    yh = torch.empty((T, d), dtype=torch.float32, pin_memory=True)
     E = max(3, min(K, 30))
 
     def e2e_step():
         x.copy_(xh, non_blocking=True)
         tw.twell_gate_gemm(x, Wg, g, None, status)
-        tw.twell_fused_updown(x, g, Wu, Wd, y, status)
+        tw.twell_fused_updown(x, g, Wu, Wd, y, ws, status)
         yh.copy_(y, non_blocking=True)
 
     for _ in range(3):
@@ -364,7 +366,7 @@ def cpu_baseline_leg(w, y_gpu):
     x = synth.widen(w["x"], dt)
     Wg, Wu, Wd = (synth.widen(w[k], dt) for k in ("Wg_t", "Wu_t", "Wd"))
     t0 = time.perf_counter()
-    g = oracle.gate_rows(x, Wg, rows)
+    g = oracle.gate_rows(x, Wg, rows, g_round=dt)
     enc = oracle.twell_encode(g, w["W"], w["C"])
     y_ref = oracle.twell_ffn(x[rows], enc, Wu, Wd)
     el = time.perf_counter() - t0

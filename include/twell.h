@@ -143,16 +143,24 @@ TW_API tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int
                           tw_dtype dtype, const tw_twell* out, void* g_dense_dump,
                           int32_t* dev_status, cudaStream_t stream);
 
+/* Bytes of workspace twell_fused_updown needs for T tokens of width d. */
+TW_API size_t twell_fused_updown_workspace_size(int32_t T, int32_t d);
+
 /*
  * Fused up + down projection over TwELL (section 2.2): for every token t and
  * every active unit j of g (slots and spilled segments),
  *   u = x_t . Wu_t[j]  (fp32),  h = g_tj * u,  y_t += h * Wd[j]  (fp32),
  * and y_t is stored in y_dtype.  No dense intermediate reaches memory.
  * x, Wu_t and Wd have g->dtype.  y [T][d].
+ * ws: device workspace of at least twell_fused_updown_workspace_size(T, d)
+ * bytes (a work plan, and fp32 partial rows for tokens whose active units are
+ * split over several warps).  Its first bytes are cleared on `stream` by the
+ * call; calls that share one workspace must not overlap on the device.  y is
+ * deterministic: partial rows are summed in a fixed order.
  */
 TW_API tw_status twell_fused_updown(const void* x, const tw_twell* g, const void* Wu_t,
-                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype,
-                             int32_t* dev_status, cudaStream_t stream);
+                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
 
 /*
  * TwELL -> hybrid conversion (section 2.3).  out->T, out->F equal g->T,

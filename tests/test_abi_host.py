@@ -86,11 +86,17 @@ def test_gate_validation(L):
 def test_fused_validation(L):
     tw = _tw()
     f = L.twell_fused_updown
-    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE, 4096, FAKE, twell.TW_BF16, None, None) == UNSUPPORTED
-    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE, 100, FAKE, twell.TW_BF16, None, None) == UNSUPPORTED
-    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE + 4, 512, FAKE, twell.TW_BF16, None, None) == ALIGN
-    assert f(FAKE, ctypes.byref(tw), None, FAKE, 512, FAKE, twell.TW_BF16, None, None) == INVALID
-    assert f(FAKE, ctypes.byref(tw), FAKE, FAKE, 512, FAKE, 7, None, None) == INVALID
+    ws = L.twell_fused_updown_workspace_size(256, 512)
+    assert ws > 0
+    args = lambda d, wu=FAKE, yd=twell.TW_BF16, n=ws, w=FAKE: (
+        FAKE, ctypes.byref(tw), wu, FAKE, d, FAKE, yd, w, n, None, None)
+    assert f(*args(4096)) == UNSUPPORTED
+    assert f(*args(100)) == UNSUPPORTED
+    assert f(*args(512, wu=FAKE + 4)) == ALIGN
+    assert f(*args(512, wu=None)) == INVALID
+    assert f(*args(512, yd=7)) == INVALID
+    assert f(*args(512, n=ws - 1)) == 8        # TW_ERR_WORKSPACE
+    assert f(*args(512, w=None)) == INVALID
 
 
 def _hy(T=256, F=1024, C_h=64, cap=32, dtype=twell.TW_BF16, base=FAKE):

@@ -32,12 +32,14 @@ def run_forward(w, C=None, spill_cap=None, dump=True, y_dtype=torch.float32):
     T, d, F = w["T"], w["d"], w["F"]
     C = w["C"] if C is None else C
     dt = TDT[w["dtype"]]
+    if spill_cap is None:
+        spill_cap = (F // 128) * T  # room for every (t, k) to spill
     g = tw.Twell(T, F, C, dtype=dt, spill_cap=spill_cap)
     gd = torch.empty((T, F), dtype=dt, device="cuda") if dump else None
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, gd, st)
     y = torch.empty((T, d), dtype=y_dtype, device="cuda")
-    tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y, st)
+    tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y, tw.fused_workspace(T, d), st)
     torch.cuda.synchronize()
     return dev, g, gd, y, st
 
@@ -105,7 +107,10 @@ def test_fp32_tiny_config(C):
     g64 = f64(gd)
     rows = np.arange(w["T"], dtype=np.int32)
     ref = oracle.gate_rows(w64["x"], w64["Wg_t"], rows, g_round="f32")
-    assert np.max(np.abs(g64 - ref)) <= 1e-5 * max(rms(ref), 1e-30)
+    # fp32 recursive summation of d products: |err| <= d * 2^-24 * sum_i |x_i w_i|
+    # (plus one rounding of the result)
+    bound = w["d"] * 2.0 ** -24 * (np.abs(w64["x"]) @ np.abs(w64["Wg_t"]).T) + 2.0 ** -23 * np.abs(ref)
+    assert np.all(np.abs(g64 - ref) <= bound)
     assert_twell_matches_oracle(g, g64)
     if C == 2:
         assert int(g.spill_n.item()) > 0
@@ -205,7 +210,7 @@ def test_oracle_encoded_twell_drives_the_fused_kernel():
     g.spill_val[:enc["n_spill"]].copy_(bits(enc["spill_val"]))
     dev = inputs(w)
     y = torch.empty((150, 512), dtype=torch.float32, device="cuda")
-    tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y)
+    tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y, tw.fused_workspace(150, 512))
     torch.cuda.synchronize()
     ref = oracle.twell_ffn(w64["x"], enc, w64["Wu_t"], w64["Wd"])
     assert np.max(np.abs(f64(y) - ref)) <= 1e-4 * rms(ref)
@@ -223,10 +228,13 @@ def test_dense_comparator():
     w64 = widened(w)
     rows = np.arange(300, dtype=np.int32)
     # the comparator stores h and y in bf16, as a dense bf16 FFN does
-    check_y(f64(y), w64, rows, TOL[synth.BF16], elem_rel=2.0 ** -7)
     dense = oracle.dense_ffn(w64["x"], w64["Wg_t"], w64["Wu_t"], w64["Wd"])
     hr = dense["g"] * dense["u"]
-    assert np.all(np.abs(f64(h) - hr) <= 2.0 ** -7 * np.abs(hr) + 1e-3 * rms(hr))
+    # h is stored in bf16 (a relative error of at most 2^-9 per element, plus
+    # a flip of g near 0); y = h Wd is then stored in bf16
+    assert np.all(np.abs(f64(h) - hr) <= 2.0 ** -8 * np.abs(hr) + 1e-4 * rms(hr))
+    bound = 2.0 ** -8 * (np.abs(hr) @ np.abs(w64["Wd"])) + 2.0 ** -8 * np.abs(dense["y"])
+    assert np.all(np.abs(f64(y) - dense["y"]) <= bound + 1e-2 * rms(dense["y"]))
 
 
 def test_dense_comparator_2b_shape_sampled():
@@ -238,7 +246,11 @@ def test_dense_comparator_2b_shape_sampled():
     tw.dense_ffn_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"].t().contiguous(), h, y)
     torch.cuda.synchronize()
     rows = synth.subsample_rows(T, 48)
-    check_y(f64(y), widened(w), rows, TOL[synth.BF16], elem_rel=2.0 ** -7)
+    w64 = widened(w)
+    dense = oracle.dense_ffn(w64["x"][rows], w64["Wg_t"], w64["Wu_t"], w64["Wd"])
+    hr = dense["g"] * dense["u"]
+    bound = 2.0 ** -8 * (np.abs(hr) @ np.abs(w64["Wd"])) + 2.0 ** -8 * np.abs(dense["y"])
+    assert np.all(np.abs(f64(y)[rows] - dense["y"]) <= bound + 1e-2 * rms(dense["y"]))
 
 
 # ----------------------------------------------------------------- hybrid ---
@@ -251,7 +263,7 @@ def run_hybrid(w, backup_cap=None):
     tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, st)
     ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, w["C_h"], hy.backup_cap),
                      dtype=torch.uint8, device="cuda")
-    dx = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((T, d), dtype=torch.float32, device="cuda")  # fp32, like y
     dW = [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
     tw.hybrid_ffn_backward(dev["x"], dev["dy"], hy, dev["Wg_t"], dev["Wu_t"], dev["Wd"],
                            w["lam"], dx, dW[0], dW[1], dW[2], ws, st)
@@ -288,7 +300,13 @@ def check_hybrid_all(w, res):
     ur = np.concatenate([ell_u.ravel(), backup_u.ravel()])
     on = np.concatenate([got["ell_g"].ravel(), got["backup_g"].ravel()]) != 0
     assert np.all(ug[~on] == 0)                       # +0 off the pattern
-    assert np.all(np.abs(ug - ur) <= 2.0 ** -8 * np.abs(ur) + 1e-3 * rms(ur[on]))
+    viol = np.abs(ug - ur) - (2.0 ** -8 * np.abs(ur) + 1e-3 * rms(ur[on]))
+    if np.any(viol > 0):
+        i = int(np.argmax(viol))
+        n_ell = f64(hy.ell_u).size
+        where = (("ell", divmod(i, w["C_h"])) if i < n_ell else ("backup", divmod(i - n_ell, w["F"])))
+        raise AssertionError(f"u mismatch at {where}: gpu {ug[i]} oracle {ur[i]}, "
+                             f"{int((viol > 0).sum())} violations")
     assert np.max(np.abs(f64(yh) - y_ref)) <= TOL[synth.BF16] * rms(y_ref)
     # the hybrid forward y equals the inference y up to rounding
     assert np.max(np.abs(f64(yh) - f64(y))) <= TOL[synth.BF16] * rms(y_ref)
