@@ -530,9 +530,90 @@ cudaError_t launch_t(FusedArgs<Tin> a, tw_dtype y_dtype, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Layout of the same work plan inside a fixed scratch area of `limit` bytes:
+// the split capacity shrinks to what fits (tokens past it stay unsplit).
+// Returns false when even the unsplit plan does not fit.
+bool carve_within(void* base, int T, int d, size_t limit, FusedWs* out) {
+  const int full_cap = T / 2 + 256;
+  int lo = 0, hi = full_cap;  // largest parts_cap whose layout fits
+  auto layout = [&](int cap) {
+    FusedWs w{};
+    w.parts_cap = cap;
+    w.max_items = T + cap;
+    size_t off = 0;
+    auto take = [&](size_t b) { size_t o = off; off = al256(off + b); return o; };
+    const size_t o_hdr = take(4 * sizeof(int32_t));
+    const size_t o_done = take(sizeof(int32_t) * (size_t)T);
+    w.zero_bytes = off;
+    const size_t o_nnz = take(sizeof(int32_t) * (size_t)T);
+    const size_t o_off = take(sizeof(int32_t) * ((size_t)T + 1));
+    const size_t o_slot = take(sizeof(int32_t) * (size_t)T);
+    const size_t o_item = take(sizeof(int32_t) * (size_t)w.max_items);
+    const size_t o_part = take(sizeof(float) * (size_t)(cap > 0 ? cap : 1) * d);
+    w.bytes = off;
+    if (base) {
+      char* p = static_cast<char*>(base);
+      w.hdr = reinterpret_cast<int32_t*>(p + o_hdr);
+      w.done = reinterpret_cast<int32_t*>(p + o_done);
+      w.nnz = reinterpret_cast<int32_t*>(p + o_nnz);
+      w.item_off = reinterpret_cast<int32_t*>(p + o_off);
+      w.slot_off = reinterpret_cast<int32_t*>(p + o_slot);
+      w.item_token = reinterpret_cast<int32_t*>(p + o_item);
+      w.partial = reinterpret_cast<float*>(p + o_part);
+    }
+    return w;
+  };
+  if (layout(0).bytes > limit) return false;
+  while (lo < hi) {
+    const int mid = lo + (hi - lo + 1) / 2;
+    if (layout(mid).bytes <= limit) lo = mid;
+    else hi = mid - 1;
+  }
+  *out = layout(lo);
+  return true;
+}
+
 }  // namespace
 
 size_t fused_ws_bytes(int T, int d) { return carve(nullptr, T, d).bytes; }
+
+bool fused_plan_fits(int T, int d, size_t limit) {
+  FusedWs w;
+  return carve_within(nullptr, T, d, limit, &w);
+}
+
+cudaError_t launch_fused_updown_in_scratch(const void* x, const tw_twell& g, const void* Wu_t,
+                                           const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                           void* scratch, size_t scratch_bytes, int32_t* status,
+                                           cudaStream_t stream) {
+  FusedWs w;
+  if (!carve_within(scratch, g.T, d, scratch_bytes, &w)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(scratch, 0, w.zero_bytes, stream);
+  if (e != cudaSuccess) return e;
+  const int K = g.F / W;
+  plan_count_kernel<<<(g.T + 255) / 256, 256, 0, stream>>>(g.T, K, g.cnt, w.nnz);
+  plan_scan_kernel<<<1, kScanThreads, 0, stream>>>(g.T, w.nnz, w.parts_cap, w.max_items,
+                                                   w.slot_off, w.item_off, w.item_token, w.hdr);
+  if (g.dtype == TW_BF16) {
+    FusedArgs<uint16_t> a{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g.val),
+                          g.idx, g.cnt, g.spill_ref, static_cast<const uint16_t*>(g.spill_val),
+                          static_cast<const uint16_t*>(Wu_t), static_cast<const uint16_t*>(Wd),
+                          y, status, g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
+    if (d <= 256) return launch_t<uint16_t, 1>(a, y_dtype, stream);
+    if (d <= 512) return launch_t<uint16_t, 2>(a, y_dtype, stream);
+    if (d <= 1024) return launch_t<uint16_t, 4>(a, y_dtype, stream);
+    return launch_t<uint16_t, 8>(a, y_dtype, stream);
+  }
+  FusedArgs<float> a{static_cast<const float*>(x), static_cast<const float*>(g.val), g.idx, g.cnt,
+                     g.spill_ref, static_cast<const float*>(g.spill_val),
+                     static_cast<const float*>(Wu_t), static_cast<const float*>(Wd), y, status,
+                     g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
+  if (d <= 128) return launch_t<float, 1>(a, y_dtype, stream);
+  if (d <= 256) return launch_t<float, 2>(a, y_dtype, stream);
+  if (d <= 512) return launch_t<float, 4>(a, y_dtype, stream);
+  if (d <= 1024) return launch_t<float, 8>(a, y_dtype, stream);
+  return launch_t<float, 16>(a, y_dtype, stream);
+}
 
 cudaError_t launch_fused_updown(const void* x, const tw_twell& g, const void* Wu_t,
                                 const void* Wd, int d, void* y, tw_dtype y_dtype, void* ws,

@@ -27,6 +27,12 @@ size_t fused_ws_bytes(int T, int d);
 cudaError_t launch_fused_updown(const void* x, const tw_twell& g, const void* Wu_t,
                                 const void* Wd, int d, void* y, tw_dtype y_dtype, void* ws,
                                 int32_t* status, cudaStream_t stream);
+// The same fused path with its work plan laid out in a fixed scratch area.
+bool fused_plan_fits(int T, int d, size_t limit);
+cudaError_t launch_fused_updown_in_scratch(const void* x, const tw_twell& g, const void* Wu_t,
+                                           const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                           void* scratch, size_t scratch_bytes, int32_t* status,
+                                           cudaStream_t stream);
 // Dense comparator pieces (bf16, tcgen05).
 cudaError_t launch_dense_gateup_tc(const void* x, const void* Wg_t, const void* Wu_t, int T,
                                    int d, int F, void* h, int32_t* status, cudaStream_t stream);

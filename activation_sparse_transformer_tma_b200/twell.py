@@ -23,7 +23,7 @@ STATUS = ["TW_OK", "TW_ERR_INVALID_ARG", "TW_ERR_UNSUPPORTED", "TW_ERR_ALIGNMENT
           "TW_ERR_CUDA", "TW_ERR_SPILL_CAPACITY", "TW_ERR_BACKUP_CAPACITY",
           "TW_ERR_TIMEOUT", "TW_ERR_WORKSPACE"]
 EXPORTS = ["twell_gate_gemm", "twell_fused_updown_workspace_size", "twell_fused_updown",
-           "twell_to_hybrid", "hybrid_ffn_forward",
+           "twell_fused_updown_noalloc", "twell_to_hybrid", "hybrid_ffn_forward",
            "hybrid_ffn_backward_workspace_size", "hybrid_ffn_backward", "dense_ffn_forward",
            "tw_status_string", "twell_version"]
 
@@ -71,6 +71,8 @@ def lib():
         L.twell_fused_updown_workspace_size.restype = ctypes.c_size_t
         L.twell_fused_updown.argtypes = [vp, PT, vp, vp, i32, vp, ctypes.c_int, vp,
                                          ctypes.c_size_t, vp, vp]
+        L.twell_fused_updown_noalloc.argtypes = [vp, PT, vp, vp, i32, vp, ctypes.c_int, vp, vp]
+        L.twell_fused_updown_noalloc.restype = st
         L.twell_to_hybrid.argtypes = [PT, PH, vp, vp]
         L.hybrid_ffn_forward.argtypes = [vp, PH, vp, vp, i32, vp, ctypes.c_int, vp, vp]
         L.hybrid_ffn_backward_workspace_size.argtypes = [i32, i32, i32, i32, i32]
@@ -193,6 +195,15 @@ def twell_fused_updown(x, g: Twell, Wu_t, Wd, y, ws, dev_status=None, stream=Non
     _check("twell_fused_updown", lib().twell_fused_updown(
         _ptr(x), ctypes.byref(s), _ptr(Wu_t), _ptr(Wd), x.shape[1], _ptr(y), _dt(y), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def twell_fused_updown_noalloc(x, g: Twell, Wu_t, Wd, y, dev_status=None, stream=None):
+    """twell_fused_updown for callers that cannot allocate a workspace: the
+    library uses its own fixed device array (see include/twell.h)."""
+    s = g.struct()
+    _check("twell_fused_updown_noalloc", lib().twell_fused_updown_noalloc(
+        _ptr(x), ctypes.byref(s), _ptr(Wu_t), _ptr(Wd), x.shape[1], _ptr(y), _dt(y),
+        _ptr(dev_status), _stream(stream)))
 
 
 def twell_to_hybrid(g: Twell, out: Hybrid, dev_status=None, stream=None):

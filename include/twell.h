@@ -163,6 +163,32 @@ TW_API tw_status twell_fused_updown(const void* x, const tw_twell* g, const void
                              size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
 
 /*
+ * twell_fused_updown without a workspace argument.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- for example a plugin whose host framework forbids device
+ * allocation in its call path, or a serving process that handed all device
+ * memory to its own pool at start-up.  It computes the same y (same
+ * kernels) with its work plan in a 16 MiB array inside the library's device
+ * image, held on every GPU that loads the library until the process exits.
+ *   - No cudaMalloc or cudaFree is called; the caller passes inputs and
+ *     outputs exactly as for twell_fused_updown.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - The plan of T tokens must fit 16 MiB: T up to 800,000 always fits (the
+ *     exact bound is a little higher and depends on d); a T whose plan does
+ *     not fit returns TW_ERR_UNSUPPORTED.  When fewer heavy tokens can be split than
+ *     the workspace version would split, the rest run unsplit: y is the same
+ *     up to fp32 summation order.
+ *   - Every call shares the one array, and the call clears the part that must
+ *     start at zero.  Calls whose work overlaps on the GPU (different streams
+ *     or host threads without ordering) race on it and give wrong results.
+ */
+TW_API tw_status twell_fused_updown_noalloc(const void* x, const tw_twell* g, const void* Wu_t,
+                                            const void* Wd, int32_t d, void* y, tw_dtype y_dtype,
+                                            int32_t* dev_status, cudaStream_t stream);
+
+/*
  * TwELL -> hybrid conversion (section 2.3).  out->T, out->F equal g->T,
  * g->F and out->dtype equals g->dtype.  Fills ell_g, ell_idx, row_nnz,
  * row_slot, backup_rows, backup_g, n_backup.
