@@ -321,6 +321,8 @@ ORC_API void orc_hybrid_forward(int T, int d, int F, int C_h,
         for (int c = 0; c < d; ++c) yt[c] = 0.0;
         int slot = row_slot[t];
         int n_items = slot < 0 ? C_h : F;
+        if (slot >= 0) /* the ELL slots of a backup row are off the pattern */
+            for (int s = 0; s < C_h; ++s) ell_u[(size_t)t * C_h + s] = 0.0;
         for (int s = 0; s < n_items; ++s) {
             double gv;
             int j;

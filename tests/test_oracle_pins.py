@@ -231,6 +231,8 @@ def test_hybrid_forward_equals_dense():
             b = backup_u[hy["row_slot"][t]]
             assert np.allclose(b[on], dense["u"][t, on], rtol=1e-13, atol=1e-14)
             assert np.all(b[~on] == 0)
+            # a backup row has no ELL entries: its ELL u slots are +0
+            assert np.all(ell_u[t].view(np.uint64) == 0)
 
 
 # ---------------------------------------------------------------- backward ---
