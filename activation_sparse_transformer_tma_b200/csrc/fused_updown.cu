@@ -9,11 +9,13 @@
 // tens of times the median number of active units), so a token with more
 // than kPart active units is split into parts of kPart entries:
 //   1. plan_count_kernel   nnz_t = sum of the TwELL tile counts of token t;
-//   2. plan_scan_kernel    (one CTA) parts per token, partial-buffer slots for
-//                          split tokens (bounded by the workspace), the work
-//                          item list and its length;
+//   2. plan_scan_kernel    (one CTA) parts per token, partial-buffer rows for
+//                          split tokens (bounded by the workspace), and one
+//                          descriptor {t, first entry, end entry, partial row}
+//                          per work item;
 //   3. fused_kernel        persistent warps take work items from a ticket
-//                          counter.  An item is a whole token or one part.
+//                          counter (the next ticket is fetched while the
+//                          current item runs).
 // A split token's parts write fp32 partial rows to the workspace; the part
 // that finishes last (atomic counter per token) sums them in part order, so
 // y is deterministic.
@@ -21,10 +23,10 @@
 // Data movement.  Each warp owns a ring of shared-memory stages; lane 0
 // gathers the Wu and Wd rows of upcoming entries with 1-D bulk copies
 // (cp.async.bulk, completion on one mbarrier per stage, no multicast) while
-// the warp computes on earlier stages, so several KB per warp are in flight.
-// Every lane owns 16-byte column slices: conflict-free shared loads.  x_t
-// stays packed in registers; the bf16 dot product uses the mixed-precision
-// fma (bf16 inputs, fp32 accumulator), the axpy uses packed fp32x2 fma.
+// the warp computes on earlier stages.  Every lane owns 16-byte column
+// slices: conflict-free shared loads.  The bf16 path keeps x_t in fp32
+// registers, widens the gathered bf16 pairs with integer shift/mask (exact)
+// and accumulates with packed fp32x2 FMAs.
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -34,52 +36,68 @@ namespace {
 constexpr unsigned FULL = 0xFFFFFFFFu;
 constexpr int W = 128;            // TwELL tile width
 constexpr int kPart = 64;         // entries per part of a split token
-constexpr int kWarps = 6;         // warps per CTA of the fused kernel
-constexpr int kRingBytes = 32768; // shared-memory ring per warp
+constexpr int kWarps = 8;         // warps per CTA of the fused kernel
+constexpr int kRingBytes = 24576; // shared-memory ring per warp
 constexpr int kListCap = 64;      // entry window collected at a time
 
 // --------------------------------------------------------------- workspace --
 struct FusedWs {
   int32_t* hdr;        // [0] item ticket, [1] number of items
-  int32_t* nnz;        // [T]
-  int32_t* item_off;   // [T+1]
-  int32_t* slot_off;   // [T] first partial slot of a split token, -1 if whole
   int32_t* done;       // [T] parts finished (split tokens)
-  int32_t* item_token; // [max_items]
+  int32_t* nnz;        // [T]
+  int32_t* slot_off;   // [T] first partial row of a split token, -1 if whole
+  int4* item_desc;     // [max_items] {t, lo, hi, partial row or -1}
   float* partial;      // [parts_cap][d]
   int parts_cap, max_items;
   size_t bytes;
-  size_t zero_bytes;   // prefix (hdr .. done) cleared before every call
+  size_t zero_bytes;   // prefix (hdr, done) cleared before every call
 };
 
 size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
-FusedWs carve(void* base, int T, int d) {
+// Layout of the workspace for T tokens of width d with room for `cap`
+// partial rows; pointers are set when base is not null.
+FusedWs layout(void* base, int T, int d, int cap) {
   FusedWs w{};
-  w.parts_cap = T / 2 + 256;
-  w.max_items = T + w.parts_cap;
+  w.parts_cap = cap;
+  w.max_items = T + cap;
   size_t off = 0;
   auto take = [&](size_t b) { size_t o = off; off = al256(off + b); return o; };
   const size_t o_hdr = take(4 * sizeof(int32_t));
   const size_t o_done = take(sizeof(int32_t) * (size_t)T);
   w.zero_bytes = off;
   const size_t o_nnz = take(sizeof(int32_t) * (size_t)T);
-  const size_t o_off = take(sizeof(int32_t) * ((size_t)T + 1));
   const size_t o_slot = take(sizeof(int32_t) * (size_t)T);
-  const size_t o_item = take(sizeof(int32_t) * (size_t)w.max_items);
-  const size_t o_part = take(sizeof(float) * (size_t)w.parts_cap * d);
+  const size_t o_desc = take(sizeof(int4) * (size_t)w.max_items);
+  const size_t o_part = take(sizeof(float) * (size_t)(cap > 0 ? cap : 1) * d);
   w.bytes = off;
   if (base) {
     char* p = static_cast<char*>(base);
     w.hdr = reinterpret_cast<int32_t*>(p + o_hdr);
     w.done = reinterpret_cast<int32_t*>(p + o_done);
     w.nnz = reinterpret_cast<int32_t*>(p + o_nnz);
-    w.item_off = reinterpret_cast<int32_t*>(p + o_off);
     w.slot_off = reinterpret_cast<int32_t*>(p + o_slot);
-    w.item_token = reinterpret_cast<int32_t*>(p + o_item);
+    w.item_desc = reinterpret_cast<int4*>(p + o_desc);
     w.partial = reinterpret_cast<float*>(p + o_part);
   }
   return w;
+}
+
+FusedWs carve(void* base, int T, int d) { return layout(base, T, d, T / 2 + 256); }
+
+// The same plan inside a fixed scratch area of `limit` bytes: the split
+// capacity shrinks to what fits (tokens past it stay unsplit).  Returns false
+// when even the unsplit plan does not fit.
+bool carve_within(void* base, int T, int d, size_t limit, FusedWs* out) {
+  if (layout(nullptr, T, d, 0).bytes > limit) return false;
+  int lo = 0, hi = T / 2 + 256;  // largest capacity whose layout fits
+  while (lo < hi) {
+    const int mid = lo + (hi - lo + 1) / 2;
+    if (layout(nullptr, T, d, mid).bytes <= limit) lo = mid;
+    else hi = mid - 1;
+  }
+  *out = layout(base, T, d, lo);
+  return true;
 }
 
 // -------------------------------------------------------------------- plan --
@@ -93,8 +111,7 @@ __global__ void plan_count_kernel(int T, int K, const uint8_t* __restrict__ cnt,
 
 constexpr int kScanThreads = 1024;
 
-// Block-wide exclusive scan of one value per thread; returns the prefix and
-// writes the block total to *total.
+// Block-wide exclusive scan of one value per thread; *total gets the sum.
 TW_DEV int block_exclusive_scan(int v, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int incl = v;
@@ -121,15 +138,15 @@ TW_DEV int block_exclusive_scan(int v, int* warp_sums, int* total) {
   return excl;
 }
 
-// One CTA: parts per token, partial slots (bounded), item offsets, item list.
+// One CTA: partial rows of split tokens (in token order, within capacity),
+// then one descriptor per work item.
 __global__ void __launch_bounds__(kScanThreads)
     plan_scan_kernel(int T, const int32_t* __restrict__ nnz, int parts_cap, int max_items,
-                     int32_t* slot_off, int32_t* item_off, int32_t* item_token, int32_t* hdr) {
+                     int32_t* slot_off, int4* item_desc, int32_t* hdr) {
   __shared__ int warp_sums[32];
   __shared__ int carry_slots, carry_items;
   if (threadIdx.x == 0) carry_slots = carry_items = 0;
   __syncthreads();
-  // pass 1: partial slots of split tokens, in token order, within capacity
   for (int base = 0; base < T; base += kScanThreads) {
     const int t = base + threadIdx.x;
     const int n = t < T ? nnz[t] : 0;
@@ -140,70 +157,70 @@ __global__ void __launch_bounds__(kScanThreads)
     if (threadIdx.x == 0) carry_slots += tot;
     __syncthreads();
   }
-  // pass 2: items (a token whose split did not fit is one item)
   for (int base = 0; base < T; base += kScanThreads) {
     const int t = base + threadIdx.x;
-    int parts = 0;
+    int parts = 0, n = 0, so = -1;
     if (t < T) {
-      const int n = nnz[t];
-      parts = (slot_off[t] >= 0) ? (n + kPart - 1) / kPart : 1;
+      n = nnz[t];
+      so = slot_off[t];
+      parts = so >= 0 ? (n + kPart - 1) / kPart : 1;
     }
     int tot;
     const int ex = block_exclusive_scan(parts, warp_sums, &tot) + carry_items;
     if (t < T) {
-      item_off[t] = ex;
-      for (int p = 0; p < parts && ex + p < max_items; ++p) item_token[ex + p] = t;
+      if (so < 0) {
+        if (ex < max_items) item_desc[ex] = make_int4(t, 0, n, -1);
+      } else {
+        for (int p = 0; p < parts && ex + p < max_items; ++p)
+          item_desc[ex + p] = make_int4(t, p * kPart, min(n, (p + 1) * kPart), so + p);
+      }
     }
     if (threadIdx.x == 0) carry_items += tot;
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    item_off[T] = carry_items;
-    hdr[1] = carry_items < max_items ? carry_items : max_items;
-  }
+  if (threadIdx.x == 0) hdr[1] = carry_items < max_items ? carry_items : max_items;
 }
 
-// ----------------------------------------------------------- element types --
+// ------------------------------------------------------------- arithmetic --
+TW_DEV void ffma2(float& a0, float& a1, float x0, float x1, float y0, float y1) {
+  asm("{\n\t.reg .b64 a, x, y;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "fma.rn.f32x2 a, x, y, a;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+}
+// exact bf16 -> fp32 of both halves of a packed pair, with integer ops
+TW_DEV float lo16(uint32_t p) { return __uint_as_float(p << 16); }
+TW_DEV float hi16(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
+
 template <typename T>
 struct Elem;
 
 template <>
-struct Elem<uint16_t> {  // bf16
+struct Elem<uint16_t> {       // bf16
   static constexpr int E = 8;  // values per 16-byte slice
+  using X = float[8];          // x slice held in fp32
   TW_DEV static float scalar(uint16_t v) { return bf16_to_f32(v); }
-  // acc0 += x.lo*w.lo, acc1 += x.hi*w.hi for every bf16 pair of a slice
-  TW_DEV static void dot(const uint4& x, const uint4& w, float& a0, float& a1) {
-    dot_pair(x.x, w.x, a0, a1);
-    dot_pair(x.y, w.y, a0, a1);
-    dot_pair(x.z, w.z, a0, a1);
-    dot_pair(x.w, w.w, a0, a1);
+  TW_DEV static void load_x(const uint16_t* p, float (&x)[8]) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    x[0] = lo16(r.x); x[1] = hi16(r.x); x[2] = lo16(r.y); x[3] = hi16(r.y);
+    x[4] = lo16(r.z); x[5] = hi16(r.z); x[6] = lo16(r.w); x[7] = hi16(r.w);
   }
-  TW_DEV static void dot_pair(uint32_t xp, uint32_t wp, float& a0, float& a1) {
-    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
-        "mov.b32 {xl, xh}, %2;\n\t"
-        "mov.b32 {wl, wh}, %3;\n\t"
-        "fma.rn.f32.bf16 %0, xl, wl, %0;\n\t"
-        "fma.rn.f32.bf16 %1, xh, wh, %1;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "r"(xp), "r"(wp));
+  // four independent accumulators a[0..3] += x . w (one pair each)
+  TW_DEV static void dot(const float (&x)[8], const uint4& w, float (&a)[4]) {
+    ffma2(a[0], a[1], x[0], x[1], lo16(w.x), hi16(w.x));
+    ffma2(a[2], a[3], x[2], x[3], lo16(w.y), hi16(w.y));
+    ffma2(a[0], a[1], x[4], x[5], lo16(w.z), hi16(w.z));
+    ffma2(a[2], a[3], x[6], x[7], lo16(w.w), hi16(w.w));
   }
-  // acc[0..7] += h * w[0..7]
   TW_DEV static void axpy(float h, const uint4& w, float* acc) {
-    axpy_pair(h, w.x, acc[0], acc[1]);
-    axpy_pair(h, w.y, acc[2], acc[3]);
-    axpy_pair(h, w.z, acc[4], acc[5]);
-    axpy_pair(h, w.w, acc[6], acc[7]);
-  }
-  TW_DEV static void axpy_pair(float h, uint32_t wp, float& a0, float& a1) {
-    const float w0 = bf16_lo(wp), w1 = bf16_hi(wp);
-    asm("{\n\t.reg .b64 hh, ww, aa;\n\t"
-        "mov.b64 hh, {%2, %2};\n\t"
-        "mov.b64 ww, {%3, %4};\n\t"
-        "mov.b64 aa, {%0, %1};\n\t"
-        "fma.rn.f32x2 aa, hh, ww, aa;\n\t"
-        "mov.b64 {%0, %1}, aa;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "f"(h), "f"(w0), "f"(w1));
+    ffma2(acc[0], acc[1], h, h, lo16(w.x), hi16(w.x));
+    ffma2(acc[2], acc[3], h, h, lo16(w.y), hi16(w.y));
+    ffma2(acc[4], acc[5], h, h, lo16(w.z), hi16(w.z));
+    ffma2(acc[6], acc[7], h, h, lo16(w.w), hi16(w.w));
   }
 };
 
@@ -211,11 +228,15 @@ template <>
 struct Elem<float> {
   static constexpr int E = 4;
   TW_DEV static float scalar(float v) { return v; }
-  TW_DEV static void dot(const uint4& x, const uint4& w, float& a0, float& a1) {
-    a0 = fmaf(__uint_as_float(x.x), __uint_as_float(w.x), a0);
-    a1 = fmaf(__uint_as_float(x.y), __uint_as_float(w.y), a1);
-    a0 = fmaf(__uint_as_float(x.z), __uint_as_float(w.z), a0);
-    a1 = fmaf(__uint_as_float(x.w), __uint_as_float(w.w), a1);
+  TW_DEV static void load_x(const float* p, float (&x)[4]) {
+    const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+    x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
+  }
+  TW_DEV static void dot(const float (&x)[4], const uint4& w, float (&a)[4]) {
+    a[0] = fmaf(x[0], __uint_as_float(w.x), a[0]);
+    a[1] = fmaf(x[1], __uint_as_float(w.y), a[1]);
+    a[2] = fmaf(x[2], __uint_as_float(w.z), a[2]);
+    a[3] = fmaf(x[3], __uint_as_float(w.w), a[3]);
   }
   TW_DEV static void axpy(float h, const uint4& w, float* acc) {
     acc[0] = fmaf(h, __uint_as_float(w.x), acc[0]);
@@ -251,7 +272,7 @@ struct FusedArgs {
   int T, d, F, C, spill_cap;
   FusedWs ws;
   int stages;        // ring depth per warp
-  int stage_bytes;   // 2 rows
+  int stage_bytes;   // two rows
   unsigned long long timeout_ns;
 };
 
@@ -263,7 +284,9 @@ struct WarpSmem {
 };
 
 // Collect the entries of token t with ordinal in [lo, hi) (tile-major order,
-// ascending within a tile) into the warp's list.  Returns the number written.
+// ascending within a tile) into the warp's list; returns how many.  Each lane
+// owns one tile, so the slots of all active tiles are read in one round;
+// spilled tiles are read by the whole warp.
 template <typename Tin>
 TW_DEV int collect(const FusedArgs<Tin>& a, int t, int lo, int hi, const WarpSmem& s, int lane) {
   const int K = a.F / W;
@@ -278,49 +301,47 @@ TW_DEV int collect(const FusedArgs<Tin>& a, int t, int lo, int hi, const WarpSme
       if (lane >= o) incl += u;
     }
     const int tb = base + incl - n;  // first ordinal of tile k
-    unsigned act = __ballot_sync(FULL, n > 0 && tb < hi && tb + n > lo);
-    while (act) {
-      const int b = __ffs(act) - 1;
-      act &= act - 1;
-      const int nk = __shfl_sync(FULL, n, b);
-      const int o0 = __shfl_sync(FULL, tb, b);
-      const int kk = kb + b;
-      const size_t kt = (size_t)kk * a.T + t;
-      int ref = -1;
-      if (nk > a.C) {
-        ref = a.spill_ref[kt];
-        if (ref < 0 || ref >= a.spill_cap) {
-          // dropped spill entry (capacity, already flagged by the producer):
-          // only the C slots are known; the rest of the tile is skipped
-          if (lane == 0) set_status(a.status, kStatusSpill);
-          ref = -1;
-        }
+    const bool over = n > 0 && tb < hi && tb + n > lo;
+    const size_t kt = (size_t)k * a.T + t;
+    int ref = -1;
+    if (over && n > a.C) {
+      ref = a.spill_ref[kt];
+      if (ref < 0 || ref >= a.spill_cap) {
+        // dropped spill entry (capacity, flagged by the producer): only the
+        // C slots are known; the other entries of the tile contribute 0
+        set_status(a.status, kStatusSpill);
+        ref = -1;
       }
-      if (ref < 0) {
-        const int m = nk <= a.C ? nk : a.C;
-        for (int s0 = 0; s0 < nk; s0 += 32) {
-          const int sl = s0 + lane;
-          const int o = o0 + sl;
-          if (sl < nk && o >= lo && o < hi) {
-            // ordinals past the known slots contribute nothing (g = 0)
-            s.g[o - lo] = sl < m ? Elem<Tin>::scalar(a.val[kt * a.C + sl]) : 0.f;
-            s.j[o - lo] = sl < m ? kk * W + a.idx[kt * a.C + sl] : kk * W;
-          }
-        }
-      } else {
-        const Tin* seg = a.spill_val + (size_t)ref * W;
-        int r = 0;
+    }
+    if (over && ref < 0) {
+      const int m = n <= a.C ? n : a.C;
+      const int s0 = lo > tb ? lo - tb : 0;
+      const int s1 = hi - tb < n ? hi - tb : n;
+#pragma unroll 4
+      for (int sl = s0; sl < s1; ++sl) {
+        const int o = tb + sl - lo;
+        s.g[o] = sl < m ? Elem<Tin>::scalar(a.val[kt * a.C + sl]) : 0.f;
+        s.j[o] = sl < m ? k * W + a.idx[kt * a.C + sl] : k * W;
+      }
+    }
+    unsigned sp = __ballot_sync(FULL, ref >= 0);
+    while (sp) {
+      const int b = __ffs(sp) - 1;
+      sp &= sp - 1;
+      const int rb = __shfl_sync(FULL, ref, b);
+      const int o0 = __shfl_sync(FULL, tb, b);
+      const Tin* seg = a.spill_val + (size_t)rb * W;
+      int r = 0;
 #pragma unroll 1
-        for (int part = 0; part < W / 32; ++part) {
-          const float v = Elem<Tin>::scalar(seg[part * 32 + lane]);
-          const unsigned m = __ballot_sync(FULL, v != 0.f);
-          const int o = o0 + r + __popc(m & ((1u << lane) - 1u));
-          if (v != 0.f && o >= lo && o < hi) {
-            s.g[o - lo] = v;
-            s.j[o - lo] = kk * W + part * 32 + lane;
-          }
-          r += __popc(m);
+      for (int part = 0; part < W / 32; ++part) {
+        const float v = Elem<Tin>::scalar(seg[part * 32 + lane]);
+        const unsigned m = __ballot_sync(FULL, v != 0.f);
+        const int o = o0 + r + __popc(m & ((1u << lane) - 1u));
+        if (v != 0.f && o >= lo && o < hi) {
+          s.g[o - lo] = v;
+          s.j[o - lo] = (kb + b) * W + part * 32 + lane;
         }
+        r += __popc(m);
       }
     }
     base += __shfl_sync(FULL, incl, 31);
@@ -328,6 +349,16 @@ TW_DEV int collect(const FusedArgs<Tin>& a, int t, int lo, int hi, const WarpSme
   __syncwarp();
   const int got = (base < hi ? base : hi) - lo;
   return got > 0 ? got : 0;
+}
+
+template <typename Tin>
+TW_DEV void issue_entry(const FusedArgs<Tin>& a, const WarpSmem& s, uint32_t st, int j,
+                        uint32_t row_bytes) {
+  uint8_t* dst = s.ring + (size_t)st * a.stage_bytes;
+  fence_proxy_async_smem();
+  mbar_arrive_expect_tx(&s.bar[st], 2 * row_bytes);
+  bulk_g2s(dst, a.Wu_t + (size_t)j * a.d, row_bytes, &s.bar[st]);
+  bulk_g2s(dst + row_bytes, a.Wd + (size_t)j * a.d, row_bytes, &s.bar[st]);
 }
 
 template <typename Tin, int NCH, bool kOutBf16>
@@ -341,7 +372,6 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
   const int d = a.d;
   const uint32_t row_bytes = (uint32_t)d * sizeof(Tin);
 
-  // per-warp shared memory: barriers, entry list, ring
   const size_t per_warp = 128 + kListCap * 8 + (size_t)a.stages * a.stage_bytes;
   uint8_t* mine = smem_raw + (size_t)wid * per_warp;
   WarpSmem s;
@@ -355,27 +385,30 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
   }
   __syncwarp();
   int never = 0;
-  uint32_t issued = 0, consumed = 0;  // bulk-copy stages issued / waited, this warp
+  // Ring position of this warp, advanced incrementally (no division):
+  // cst/cph next stage to wait on and its phase parity, pst next stage to
+  // fill, inflight stages filled but not yet waited on.
+  uint32_t cst = 0, cph = 0, pst = 0, inflight = 0;
   bool failed = false;
+  const int n_items = a.ws.hdr[1];
 
-  for (;;) {
-    int item = 0;
-    if (lane == 0) item = atomicAdd(&a.ws.hdr[0], 1);
-    item = __shfl_sync(FULL, item, 0);
-    if (item >= a.ws.hdr[1]) break;
-    const int t = a.ws.item_token[item];
-    const int p = item - a.ws.item_off[t];
-    const int nnz = a.ws.nnz[t];
-    const bool split = a.ws.slot_off[t] >= 0;
-    const int lo = split ? p * kPart : 0;
-    const int hi = split ? min(nnz, lo + kPart) : nnz;
+  int ticket = 0;
+  if (lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);
+  int item = __shfl_sync(FULL, ticket, 0);
+  while (item < n_items) {
+    if (lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);  // next item, fetched early
+    const int4 desc = a.ws.item_desc[item];
+    const int t = desc.x, lo = desc.y, hi = desc.z, prow = desc.w;
 
-    uint4 xr[NCH];
+    float xf[NCH][E];
     const Tin* xt = a.x + (size_t)t * d;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int col = c * SPAN + lane * E;
-      xr[c] = col < d ? __ldg(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
+      if (col < d) L::load_x(xt + col, xf[c]);
+      else
+#pragma unroll
+        for (int e = 0; e < E; ++e) xf[c][e] = 0.f;
     }
     float acc[NCH][E];
 #pragma unroll
@@ -385,46 +418,40 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
 
     for (int w0 = lo; w0 < hi && !failed; w0 += kListCap) {
       const int n = collect(a, t, w0, min(hi, w0 + kListCap), s, lane);
-      // prologue: fill the ring
       const int pre = n < a.stages ? n : a.stages;
-      if (lane == 0) {
-        for (int e = 0; e < pre; ++e) {
-          const uint32_t st = (issued + e) % a.stages;
-          uint8_t* dst = s.ring + (size_t)st * a.stage_bytes;
-          const int j = s.j[e];
-          fence_proxy_async_smem();
-          mbar_arrive_expect_tx(&s.bar[st], 2 * row_bytes);
-          bulk_g2s(dst, a.Wu_t + (size_t)j * d, row_bytes, &s.bar[st]);
-          bulk_g2s(dst + row_bytes, a.Wd + (size_t)j * d, row_bytes, &s.bar[st]);
-        }
+      for (int e = 0; e < pre; ++e) {
+        if (lane == 0) issue_entry(a, s, pst, s.j[e], row_bytes);
+        pst = pst + 1 == (uint32_t)a.stages ? 0u : pst + 1;
+        ++inflight;
       }
-      uint32_t base_issue = issued;
-      issued += pre;
       for (int e = 0; e < n; ++e) {
-        const uint32_t seq = base_issue + e;
-        const uint32_t st = seq % a.stages;
-        const uint32_t ph = (seq / a.stages) & 1u;
-        bool ok = mbar_wait(&s.bar[st], ph, &never, a.timeout_ns);
+        const uint32_t st = cst;
+        bool ok = mbar_wait(&s.bar[st], cph, &never, a.timeout_ns);
         ok = __all_sync(FULL, ok);
         if (!ok) {
           failed = true;
           break;
         }
-        consumed = seq + 1;
+        --inflight;
+        if (++cst == (uint32_t)a.stages) {
+          cst = 0;
+          cph ^= 1u;
+        }
         const uint8_t* stage = s.ring + (size_t)st * a.stage_bytes;
         const uint4* wu = reinterpret_cast<const uint4*>(stage);
         const uint4* wd = reinterpret_cast<const uint4*>(stage + row_bytes);
-        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+        float pa[4] = {0.f, 0.f, 0.f, 0.f};
+        float pb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           const int col = c * SPAN + lane * E;
           if (col < d) {
-            const uint4 w = wu[col / E];
-            if (c & 1) L::dot(xr[c], w, p2, p3);
-            else L::dot(xr[c], w, p0, p1);
+            if (c & 1) L::dot(xf[c], wu[col / E], pb);
+            else L::dot(xf[c], wu[col / E], pa);
           }
         }
-        const float u = warp_sum((p0 + p1) + (p2 + p3));
+        const float u = warp_sum(((pa[0] + pb[0]) + (pa[1] + pb[1])) +
+                                 ((pa[2] + pb[2]) + (pa[3] + pb[3])));
         const float h = s.g[e] * u;
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
@@ -433,23 +460,19 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
         }
         __syncwarp();  // every lane is done with this stage
         const int nxt = e + a.stages;
-        if (lane == 0 && nxt < n) {
-          const int j = s.j[nxt];
-          uint8_t* dst = s.ring + (size_t)st * a.stage_bytes;
-          fence_proxy_async_smem();
-          mbar_arrive_expect_tx(&s.bar[st], 2 * row_bytes);
-          bulk_g2s(dst, a.Wu_t + (size_t)j * d, row_bytes, &s.bar[st]);
-          bulk_g2s(dst + row_bytes, a.Wd + (size_t)j * d, row_bytes, &s.bar[st]);
+        if (nxt < n) {  // refill the stage just freed (the ring was full)
+          if (lane == 0) issue_entry(a, s, pst, s.j[nxt], row_bytes);
+          pst = pst + 1 == (uint32_t)a.stages ? 0u : pst + 1;
+          ++inflight;
         }
-        if (nxt < n) ++issued;
       }
       __syncwarp();
     }
     if (failed) break;
 
     // ------------------------------------------------------------ output --
-    float* out_row = nullptr;
-    if (split) out_row = a.ws.partial + (size_t)(a.ws.slot_off[t] + p) * d;
+    const bool split = prow >= 0;
+    float* out_row = split ? a.ws.partial + (size_t)prow * d : nullptr;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int col = c * SPAN + lane * E;
@@ -476,13 +499,13 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
       // the last part to finish sums the partial rows in part order
       __threadfence();
       __syncwarp();
-      const int parts = a.ws.item_off[t + 1] - a.ws.item_off[t];
+      const int parts = (a.ws.nnz[t] + kPart - 1) / kPart;
       int prev = 0;
       if (lane == 0) prev = atomicAdd(&a.ws.done[t], 1);
       prev = __shfl_sync(FULL, prev, 0);
       if (prev == parts - 1) {
         __threadfence();
-        const float* part0 = a.ws.partial + (size_t)a.ws.slot_off[t] * d;
+        const float* part0 = a.ws.partial + (size_t)(prow - lo / kPart) * d;
         for (int col = lane * 4; col < d; col += 128) {
           float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int q = 0; q < parts; ++q) {
@@ -499,13 +522,19 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
         }
       }
     }
+    item = __shfl_sync(FULL, ticket, 0);
   }
 
   if (failed) {
     if (lane == 0) set_status(a.status, kStatusTimeout);
     // let the copies still in flight land before the CTA may exit
-    for (uint32_t q = consumed; q < issued; ++q)
-      mbar_wait(&s.bar[q % a.stages], (q / a.stages) & 1u, &never, a.timeout_ns);
+    for (uint32_t q = 0; q < inflight; ++q) {
+      mbar_wait(&s.bar[cst], cph, &never, a.timeout_ns);
+      if (++cst == (uint32_t)a.stages) {
+        cst = 0;
+        cph ^= 1u;
+      }
+    }
   }
 }
 
@@ -517,9 +546,7 @@ cudaError_t launch_t(FusedArgs<Tin> a, tw_dtype y_dtype, cudaStream_t stream) {
   if (a.stages < 2) a.stages = 2;
   const size_t per_warp = 128 + kListCap * 8 + (size_t)a.stages * a.stage_bytes;
   const size_t smem = per_warp * kWarps;
-  auto kern_bf = fused_kernel<Tin, NCH, true>;
-  auto kern_f = fused_kernel<Tin, NCH, false>;
-  auto kern = y_dtype == TW_BF16 ? kern_bf : kern_f;
+  auto kern = y_dtype == TW_BF16 ? fused_kernel<Tin, NCH, true> : fused_kernel<Tin, NCH, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -530,52 +557,46 @@ cudaError_t launch_t(FusedArgs<Tin> a, tw_dtype y_dtype, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// Layout of the same work plan inside a fixed scratch area of `limit` bytes:
-// the split capacity shrinks to what fits (tokens past it stay unsplit).
-// Returns false when even the unsplit plan does not fit.
-bool carve_within(void* base, int T, int d, size_t limit, FusedWs* out) {
-  const int full_cap = T / 2 + 256;
-  int lo = 0, hi = full_cap;  // largest parts_cap whose layout fits
-  auto layout = [&](int cap) {
-    FusedWs w{};
-    w.parts_cap = cap;
-    w.max_items = T + cap;
-    size_t off = 0;
-    auto take = [&](size_t b) { size_t o = off; off = al256(off + b); return o; };
-    const size_t o_hdr = take(4 * sizeof(int32_t));
-    const size_t o_done = take(sizeof(int32_t) * (size_t)T);
-    w.zero_bytes = off;
-    const size_t o_nnz = take(sizeof(int32_t) * (size_t)T);
-    const size_t o_off = take(sizeof(int32_t) * ((size_t)T + 1));
-    const size_t o_slot = take(sizeof(int32_t) * (size_t)T);
-    const size_t o_item = take(sizeof(int32_t) * (size_t)w.max_items);
-    const size_t o_part = take(sizeof(float) * (size_t)(cap > 0 ? cap : 1) * d);
-    w.bytes = off;
-    if (base) {
-      char* p = static_cast<char*>(base);
-      w.hdr = reinterpret_cast<int32_t*>(p + o_hdr);
-      w.done = reinterpret_cast<int32_t*>(p + o_done);
-      w.nnz = reinterpret_cast<int32_t*>(p + o_nnz);
-      w.item_off = reinterpret_cast<int32_t*>(p + o_off);
-      w.slot_off = reinterpret_cast<int32_t*>(p + o_slot);
-      w.item_token = reinterpret_cast<int32_t*>(p + o_item);
-      w.partial = reinterpret_cast<float*>(p + o_part);
-    }
-    return w;
-  };
-  if (layout(0).bytes > limit) return false;
-  while (lo < hi) {
-    const int mid = lo + (hi - lo + 1) / 2;
-    if (layout(mid).bytes <= limit) lo = mid;
-    else hi = mid - 1;
+// Plan + fused kernel on a carved workspace.
+cudaError_t run_plan_and_fused(const void* x, const tw_twell& g, const void* Wu_t, const void* Wd,
+                               int d, void* y, tw_dtype y_dtype, void* base, const FusedWs& w,
+                               int32_t* status, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(base, 0, w.zero_bytes, stream);
+  if (e != cudaSuccess) return e;
+  const int K = g.F / W;
+  plan_count_kernel<<<(g.T + 255) / 256, 256, 0, stream>>>(g.T, K, g.cnt, w.nnz);
+  plan_scan_kernel<<<1, kScanThreads, 0, stream>>>(g.T, w.nnz, w.parts_cap, w.max_items,
+                                                   w.slot_off, w.item_desc, w.hdr);
+  if (g.dtype == TW_BF16) {
+    FusedArgs<uint16_t> a{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g.val),
+                          g.idx, g.cnt, g.spill_ref, static_cast<const uint16_t*>(g.spill_val),
+                          static_cast<const uint16_t*>(Wu_t), static_cast<const uint16_t*>(Wd),
+                          y, status, g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
+    if (d <= 256) return launch_t<uint16_t, 1>(a, y_dtype, stream);
+    if (d <= 512) return launch_t<uint16_t, 2>(a, y_dtype, stream);
+    if (d <= 1024) return launch_t<uint16_t, 4>(a, y_dtype, stream);
+    return launch_t<uint16_t, 8>(a, y_dtype, stream);
   }
-  *out = layout(lo);
-  return true;
+  FusedArgs<float> a{static_cast<const float*>(x), static_cast<const float*>(g.val), g.idx, g.cnt,
+                     g.spill_ref, static_cast<const float*>(g.spill_val),
+                     static_cast<const float*>(Wu_t), static_cast<const float*>(Wd), y, status,
+                     g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
+  if (d <= 128) return launch_t<float, 1>(a, y_dtype, stream);
+  if (d <= 256) return launch_t<float, 2>(a, y_dtype, stream);
+  if (d <= 512) return launch_t<float, 4>(a, y_dtype, stream);
+  if (d <= 1024) return launch_t<float, 8>(a, y_dtype, stream);
+  return launch_t<float, 16>(a, y_dtype, stream);
 }
 
 }  // namespace
 
 size_t fused_ws_bytes(int T, int d) { return carve(nullptr, T, d).bytes; }
+
+cudaError_t launch_fused_updown(const void* x, const tw_twell& g, const void* Wu_t,
+                                const void* Wd, int d, void* y, tw_dtype y_dtype, void* ws,
+                                int32_t* status, cudaStream_t stream) {
+  return run_plan_and_fused(x, g, Wu_t, Wd, d, y, y_dtype, ws, carve(ws, g.T, d), status, stream);
+}
 
 bool fused_plan_fits(int T, int d, size_t limit) {
   FusedWs w;
@@ -588,62 +609,7 @@ cudaError_t launch_fused_updown_in_scratch(const void* x, const tw_twell& g, con
                                            cudaStream_t stream) {
   FusedWs w;
   if (!carve_within(scratch, g.T, d, scratch_bytes, &w)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(scratch, 0, w.zero_bytes, stream);
-  if (e != cudaSuccess) return e;
-  const int K = g.F / W;
-  plan_count_kernel<<<(g.T + 255) / 256, 256, 0, stream>>>(g.T, K, g.cnt, w.nnz);
-  plan_scan_kernel<<<1, kScanThreads, 0, stream>>>(g.T, w.nnz, w.parts_cap, w.max_items,
-                                                   w.slot_off, w.item_off, w.item_token, w.hdr);
-  if (g.dtype == TW_BF16) {
-    FusedArgs<uint16_t> a{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g.val),
-                          g.idx, g.cnt, g.spill_ref, static_cast<const uint16_t*>(g.spill_val),
-                          static_cast<const uint16_t*>(Wu_t), static_cast<const uint16_t*>(Wd),
-                          y, status, g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
-    if (d <= 256) return launch_t<uint16_t, 1>(a, y_dtype, stream);
-    if (d <= 512) return launch_t<uint16_t, 2>(a, y_dtype, stream);
-    if (d <= 1024) return launch_t<uint16_t, 4>(a, y_dtype, stream);
-    return launch_t<uint16_t, 8>(a, y_dtype, stream);
-  }
-  FusedArgs<float> a{static_cast<const float*>(x), static_cast<const float*>(g.val), g.idx, g.cnt,
-                     g.spill_ref, static_cast<const float*>(g.spill_val),
-                     static_cast<const float*>(Wu_t), static_cast<const float*>(Wd), y, status,
-                     g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
-  if (d <= 128) return launch_t<float, 1>(a, y_dtype, stream);
-  if (d <= 256) return launch_t<float, 2>(a, y_dtype, stream);
-  if (d <= 512) return launch_t<float, 4>(a, y_dtype, stream);
-  if (d <= 1024) return launch_t<float, 8>(a, y_dtype, stream);
-  return launch_t<float, 16>(a, y_dtype, stream);
-}
-
-cudaError_t launch_fused_updown(const void* x, const tw_twell& g, const void* Wu_t,
-                                const void* Wd, int d, void* y, tw_dtype y_dtype, void* ws,
-                                int32_t* status, cudaStream_t stream) {
-  const FusedWs w = carve(ws, g.T, d);
-  cudaError_t e = cudaMemsetAsync(ws, 0, w.zero_bytes, stream);
-  if (e != cudaSuccess) return e;
-  const int K = g.F / W;
-  plan_count_kernel<<<(g.T + 255) / 256, 256, 0, stream>>>(g.T, K, g.cnt, w.nnz);
-  plan_scan_kernel<<<1, kScanThreads, 0, stream>>>(g.T, w.nnz, w.parts_cap, w.max_items,
-                                                   w.slot_off, w.item_off, w.item_token, w.hdr);
-  if (g.dtype == TW_BF16) {
-    FusedArgs<uint16_t> a{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g.val),
-                          g.idx, g.cnt, g.spill_ref, static_cast<const uint16_t*>(g.spill_val),
-                          static_cast<const uint16_t*>(Wu_t), static_cast<const uint16_t*>(Wd),
-                          y, status, g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
-    if (d <= 256) return launch_t<uint16_t, 1>(a, y_dtype, stream);
-    if (d <= 512) return launch_t<uint16_t, 2>(a, y_dtype, stream);
-    if (d <= 1024) return launch_t<uint16_t, 4>(a, y_dtype, stream);
-    return launch_t<uint16_t, 8>(a, y_dtype, stream);
-  }
-  FusedArgs<float> a{static_cast<const float*>(x), static_cast<const float*>(g.val), g.idx, g.cnt,
-                     g.spill_ref, static_cast<const float*>(g.spill_val),
-                     static_cast<const float*>(Wu_t), static_cast<const float*>(Wd), y, status,
-                     g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
-  if (d <= 128) return launch_t<float, 1>(a, y_dtype, stream);
-  if (d <= 256) return launch_t<float, 2>(a, y_dtype, stream);
-  if (d <= 512) return launch_t<float, 4>(a, y_dtype, stream);
-  if (d <= 1024) return launch_t<float, 8>(a, y_dtype, stream);
-  return launch_t<float, 16>(a, y_dtype, stream);
+  return run_plan_and_fused(x, g, Wu_t, Wd, d, y, y_dtype, scratch, w, status, stream);
 }
 
 }  // namespace tw

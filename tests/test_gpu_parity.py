@@ -261,6 +261,7 @@ def run_hybrid(w, backup_cap=None):
     tw.twell_to_hybrid(g, hy, st)
     yh = torch.empty((T, d), dtype=torch.float32, device="cuda")
     tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, st)
+    hy.ell_u_after_forward = hy.ell_u.clone()  # diagnostics: u before the backward runs
     ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, w["C_h"], hy.backup_cap),
                      dtype=torch.uint8, device="cuda")
     dx = torch.empty((T, d), dtype=torch.float32, device="cuda")  # fp32, like y
@@ -305,8 +306,15 @@ def check_hybrid_all(w, res):
         i = int(np.argmax(viol))
         n_ell = f64(hy.ell_u).size
         where = (("ell", divmod(i, w["C_h"])) if i < n_ell else ("backup", divmod(i - n_ell, w["F"])))
-        raise AssertionError(f"u mismatch at {where}: gpu {ug[i]} oracle {ur[i]}, "
-                             f"{int((viol > 0).sum())} violations")
+        bad = np.nonzero(viol[:n_ell] > 0)[0]
+        rows_bad = np.unique(bad // w["C_h"])
+        u_fwd = f64(hy.ell_u_after_forward).ravel()
+        info = [(int(r), int(got["row_nnz"][r]), int(got["row_slot"][r])) for r in rows_bad[:8]]
+        yerr = [float(np.max(np.abs(f64(yh)[r] - y_ref[r]))) for r in rows_bad[:8]]
+        raise AssertionError(
+            f"u mismatch at {where}: gpu {ug[i]} oracle {ur[i]}, {int((viol > 0).sum())} "
+            f"violations; rows (t, nnz, slot) {info}; u right after the forward "
+            f"{u_fwd[i]}; y row errors {yerr} (rms {rms(y_ref)})")
     assert np.max(np.abs(f64(yh) - y_ref)) <= TOL[synth.BF16] * rms(y_ref)
     # the hybrid forward y equals the inference y up to rounding
     assert np.max(np.abs(f64(yh) - f64(y))) <= TOL[synth.BF16] * rms(y_ref)
