@@ -182,19 +182,11 @@ __global__ void __launch_bounds__(kScanThreads)
 }
 
 // ------------------------------------------------------------- arithmetic --
-TW_DEV void ffma2(float& a0, float& a1, float x0, float x1, float y0, float y1) {
-  asm("{\n\t.reg .b64 a, x, y;\n\t"
-      "mov.b64 a, {%0, %1};\n\t"
-      "mov.b64 x, {%2, %3};\n\t"
-      "mov.b64 y, {%4, %5};\n\t"
-      "fma.rn.f32x2 a, x, y, a;\n\t"
-      "mov.b64 {%0, %1}, a;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+// Rows are handled as 16-byte slices of E values = P pairs; all arithmetic is
+// packed fp32x2 FMA (__ffma2_rn) on float2 pairs.
+TW_DEV float2 bf16_pair(uint32_t p) {  // exact widening of two packed bf16
+  return make_float2(__uint_as_float(p << 16), __uint_as_float(p & 0xFFFF0000u));
 }
-// exact bf16 -> fp32 of both halves of a packed pair, with integer ops
-TW_DEV float lo16(uint32_t p) { return __uint_as_float(p << 16); }
-TW_DEV float hi16(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
 template <typename T>
 struct Elem;
@@ -202,47 +194,21 @@ struct Elem;
 template <>
 struct Elem<uint16_t> {       // bf16
   static constexpr int E = 8;  // values per 16-byte slice
-  using X = float[8];          // x slice held in fp32
+  static constexpr int P = 4;  // pairs per slice
   TW_DEV static float scalar(uint16_t v) { return bf16_to_f32(v); }
-  TW_DEV static void load_x(const uint16_t* p, float (&x)[8]) {
-    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
-    x[0] = lo16(r.x); x[1] = hi16(r.x); x[2] = lo16(r.y); x[3] = hi16(r.y);
-    x[4] = lo16(r.z); x[5] = hi16(r.z); x[6] = lo16(r.w); x[7] = hi16(r.w);
-  }
-  // four independent accumulators a[0..3] += x . w (one pair each)
-  TW_DEV static void dot(const float (&x)[8], const uint4& w, float (&a)[4]) {
-    ffma2(a[0], a[1], x[0], x[1], lo16(w.x), hi16(w.x));
-    ffma2(a[2], a[3], x[2], x[3], lo16(w.y), hi16(w.y));
-    ffma2(a[0], a[1], x[4], x[5], lo16(w.z), hi16(w.z));
-    ffma2(a[2], a[3], x[6], x[7], lo16(w.w), hi16(w.w));
-  }
-  TW_DEV static void axpy(float h, const uint4& w, float* acc) {
-    ffma2(acc[0], acc[1], h, h, lo16(w.x), hi16(w.x));
-    ffma2(acc[2], acc[3], h, h, lo16(w.y), hi16(w.y));
-    ffma2(acc[4], acc[5], h, h, lo16(w.z), hi16(w.z));
-    ffma2(acc[6], acc[7], h, h, lo16(w.w), hi16(w.w));
+  TW_DEV static void pairs(const uint4& r, float2 (&w)[P]) {
+    w[0] = bf16_pair(r.x); w[1] = bf16_pair(r.y); w[2] = bf16_pair(r.z); w[3] = bf16_pair(r.w);
   }
 };
 
 template <>
 struct Elem<float> {
   static constexpr int E = 4;
+  static constexpr int P = 2;
   TW_DEV static float scalar(float v) { return v; }
-  TW_DEV static void load_x(const float* p, float (&x)[4]) {
-    const float4 r = __ldg(reinterpret_cast<const float4*>(p));
-    x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
-  }
-  TW_DEV static void dot(const float (&x)[4], const uint4& w, float (&a)[4]) {
-    a[0] = fmaf(x[0], __uint_as_float(w.x), a[0]);
-    a[1] = fmaf(x[1], __uint_as_float(w.y), a[1]);
-    a[2] = fmaf(x[2], __uint_as_float(w.z), a[2]);
-    a[3] = fmaf(x[3], __uint_as_float(w.w), a[3]);
-  }
-  TW_DEV static void axpy(float h, const uint4& w, float* acc) {
-    acc[0] = fmaf(h, __uint_as_float(w.x), acc[0]);
-    acc[1] = fmaf(h, __uint_as_float(w.y), acc[1]);
-    acc[2] = fmaf(h, __uint_as_float(w.z), acc[2]);
-    acc[3] = fmaf(h, __uint_as_float(w.w), acc[3]);
+  TW_DEV static void pairs(const uint4& r, float2 (&w)[P]) {
+    w[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
+    w[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
   }
 };
 
@@ -365,6 +331,7 @@ template <typename Tin, int NCH, bool kOutBf16>
 __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<Tin> a) {
   using L = Elem<Tin>;
   constexpr int E = L::E;
+  constexpr int P = L::P;
   constexpr int SPAN = 32 * E;  // columns covered by one warp-wide 16-byte slice
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31;
@@ -400,21 +367,19 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
     const int4 desc = a.ws.item_desc[item];
     const int t = desc.x, lo = desc.y, hi = desc.z, prow = desc.w;
 
-    float xf[NCH][E];
+    float2 xf[NCH][P];
     const Tin* xt = a.x + (size_t)t * d;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int col = c * SPAN + lane * E;
-      if (col < d) L::load_x(xt + col, xf[c]);
-      else
-#pragma unroll
-        for (int e = 0; e < E; ++e) xf[c][e] = 0.f;
+      const uint4 r = col < d ? __ldg(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
+      L::pairs(r, xf[c]);
     }
-    float acc[NCH][E];
+    float2 acc[NCH][P];
 #pragma unroll
     for (int c = 0; c < NCH; ++c)
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
+      for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
 
     for (int w0 = lo; w0 < hi && !failed; w0 += kListCap) {
       const int n = collect(a, t, w0, min(hi, w0 + kListCap), s, lane);
@@ -440,23 +405,33 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
         const uint8_t* stage = s.ring + (size_t)st * a.stage_bytes;
         const uint4* wu = reinterpret_cast<const uint4*>(stage);
         const uint4* wd = reinterpret_cast<const uint4*>(stage + row_bytes);
-        float pa[4] = {0.f, 0.f, 0.f, 0.f};
-        float pb[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 pd[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           const int col = c * SPAN + lane * E;
           if (col < d) {
-            if (c & 1) L::dot(xf[c], wu[col / E], pb);
-            else L::dot(xf[c], wu[col / E], pa);
+            float2 w[P];
+            L::pairs(wu[col / E], w);
+#pragma unroll
+            for (int q = 0; q < P; ++q) pd[(c * P + q) & 3] = __ffma2_rn(xf[c][q], w[q], pd[(c * P + q) & 3]);
           }
         }
-        const float u = warp_sum(((pa[0] + pb[0]) + (pa[1] + pb[1])) +
-                                 ((pa[2] + pb[2]) + (pa[3] + pb[3])));
+        const float2 p01 = __fadd2_rn(pd[0], pd[1]);
+        const float2 p23 = __fadd2_rn(pd[2], pd[3]);
+        const float2 pp = __fadd2_rn(p01, p23);
+        const float u = warp_sum(pp.x + pp.y);
         const float h = s.g[e] * u;
+        const float2 hh = make_float2(h, h);
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           const int col = c * SPAN + lane * E;
-          if (col < d) L::axpy(h, wd[col / E], acc[c]);
+          if (col < d) {
+            float2 w[P];
+            L::pairs(wd[col / E], w);
+#pragma unroll
+            for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(hh, w[q], acc[c][q]);
+          }
         }
         __syncwarp();  // every lane is done with this stage
         const int nxt = e + a.stages;
@@ -477,22 +452,17 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
     for (int c = 0; c < NCH; ++c) {
       const int col = c * SPAN + lane * E;
       if (col >= d) continue;
-      if (split) {
+      if (split || !kOutBf16) {
+        float* dst = split ? out_row + col : static_cast<float*>(a.y) + (size_t)t * d + col;
 #pragma unroll
-        for (int q = 0; q < E / 4; ++q)
-          reinterpret_cast<float4*>(out_row + col)[q] =
-              make_float4(acc[c][4 * q], acc[c][4 * q + 1], acc[c][4 * q + 2], acc[c][4 * q + 3]);
-      } else if (kOutBf16) {
+        for (int q = 0; q < P / 2; ++q)
+          reinterpret_cast<float4*>(dst)[q] = make_float4(acc[c][2 * q].x, acc[c][2 * q].y,
+                                                          acc[c][2 * q + 1].x, acc[c][2 * q + 1].y);
+      } else {
         uint16_t* yt = static_cast<uint16_t*>(a.y) + (size_t)t * d + col;
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q)
-          reinterpret_cast<uint32_t*>(yt)[q] = pack_bf16x2(acc[c][2 * q], acc[c][2 * q + 1]);
-      } else {
-        float* yt = static_cast<float*>(a.y) + (size_t)t * d + col;
-#pragma unroll
-        for (int q = 0; q < E / 4; ++q)
-          reinterpret_cast<float4*>(yt)[q] =
-              make_float4(acc[c][4 * q], acc[c][4 * q + 1], acc[c][4 * q + 2], acc[c][4 * q + 3]);
+        for (int q = 0; q < P; ++q)
+          reinterpret_cast<uint32_t*>(yt)[q] = pack_bf16x2(acc[c][q].x, acc[c][q].y);
       }
     }
     if (split) {
