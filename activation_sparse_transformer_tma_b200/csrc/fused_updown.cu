@@ -13,20 +13,27 @@
 //                          split tokens (bounded by the workspace), and one
 //                          descriptor {t, first entry, end entry, partial row}
 //                          per work item;
-//   3. fused_kernel        persistent warps take work items from a ticket
+//   3. fused_kernel        persistent teams take work items from a ticket
 //                          counter (the next ticket is fetched while the
 //                          current item runs).
 // A split token's parts write fp32 partial rows to the workspace; the part
 // that finishes last (atomic counter per token) sums them in part order, so
 // y is deterministic.
 //
+// Teams.  An item is processed by a team of kTeam warps; warp w of the team
+// owns one contiguous range of the d columns (x_t and y_t of that range live
+// in its registers).  Per entry every warp forms its partial dot product, the
+// partials meet in shared memory behind a named barrier and are added in warp
+// order, and every warp applies h = g * u to its own columns.  Splitting the
+// columns halves the registers per warp, so twice as many warps hide the
+// gather latency.
+//
 // Data movement.  Each warp owns a ring of shared-memory stages; lane 0
-// gathers the Wu and Wd rows of upcoming entries with 1-D bulk copies
-// (cp.async.bulk, completion on one mbarrier per stage, no multicast) while
-// the warp computes on earlier stages.  Every lane owns 16-byte column
-// slices: conflict-free shared loads.  The bf16 path keeps x_t in fp32
-// registers, widens the gathered bf16 pairs with integer shift/mask (exact)
-// and accumulates with packed fp32x2 FMAs.
+// gathers its column range of the Wu and Wd rows of upcoming entries with
+// 1-D bulk copies (cp.async.bulk, completion on one mbarrier per stage, no
+// multicast) while the warp computes on earlier stages.  Every lane owns
+// 16-byte column slices: conflict-free shared loads.  bf16 pairs are widened
+// with integer shift/mask (exact) and accumulated with packed fp32x2 FMA.
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -34,11 +41,13 @@ namespace tw {
 namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
-constexpr int W = 128;            // TwELL tile width
-constexpr int kPart = 64;         // entries per part of a split token
-constexpr int kWarps = 8;         // warps per CTA of the fused kernel
-constexpr int kRingBytes = 24576; // shared-memory ring per warp
-constexpr int kListCap = 64;      // entry window collected at a time
+constexpr int W = 128;             // TwELL tile width
+constexpr int kPart = 64;          // entries per part of a split token
+constexpr int kTeam = 2;           // warps per work item
+constexpr int kTeams = 8;          // teams per CTA
+constexpr int kWarps = kTeam * kTeams;
+constexpr int kRingBytes = 12288;  // shared-memory ring per warp
+constexpr int kListCap = 64;       // entry window collected at a time
 
 // --------------------------------------------------------------- workspace --
 struct FusedWs {
@@ -222,6 +231,11 @@ TW_DEV void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t*
 TW_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Named barrier over the kTeam warps of one team (ids 1..kTeams; 0 is
+// __syncthreads).  Every warp of a team executes the same sequence of these.
+TW_DEV void team_bar(int team) {
+  asm volatile("bar.sync %0, %1;" ::"r"(team + 1), "r"(kTeam * 32) : "memory");
+}
 
 template <typename Tin>
 struct FusedArgs {
@@ -238,23 +252,27 @@ struct FusedArgs {
   int T, d, F, C, spill_cap;
   FusedWs ws;
   int stages;        // ring depth per warp
-  int stage_bytes;   // two rows
+  int slice_bytes;   // bytes of one row's column range of one warp (max over warps)
   unsigned long long timeout_ns;
 };
 
-struct WarpSmem {
-  uint64_t* bar;     // [stages]
-  float* g;          // [kListCap]
-  int32_t* j;        // [kListCap]
-  uint8_t* ring;     // [stages][stage_bytes]
+// Shared state of one team.
+struct TeamSmem {
+  float g[kListCap];
+  int32_t j[kListCap];
+  float red[2][kTeam];   // partial dot products, double-buffered by entry parity
+  int ok[2][kTeam];      // wait results, same buffering
+  int4 desc[2];          // current item, double-buffered by item parity
+  int n;                 // entries in the current window
+  int prev;              // split-token finisher broadcast
 };
 
 // Collect the entries of token t with ordinal in [lo, hi) (tile-major order,
-// ascending within a tile) into the warp's list; returns how many.  Each lane
+// ascending within a tile) into the team's list; returns how many.  Each lane
 // owns one tile, so the slots of all active tiles are read in one round;
 // spilled tiles are read by the whole warp.
 template <typename Tin>
-TW_DEV int collect(const FusedArgs<Tin>& a, int t, int lo, int hi, const WarpSmem& s, int lane) {
+TW_DEV int collect(const FusedArgs<Tin>& a, int t, int lo, int hi, TeamSmem& s, int lane) {
   const int K = a.F / W;
   int base = 0;  // ordinal of the first entry of tile kb
   for (int kb = 0; kb < K && base < hi; kb += 32) {
@@ -312,88 +330,138 @@ TW_DEV int collect(const FusedArgs<Tin>& a, int t, int lo, int hi, const WarpSme
     }
     base += __shfl_sync(FULL, incl, 31);
   }
-  __syncwarp();
   const int got = (base < hi ? base : hi) - lo;
   return got > 0 ? got : 0;
 }
 
-template <typename Tin>
-TW_DEV void issue_entry(const FusedArgs<Tin>& a, const WarpSmem& s, uint32_t st, int j,
-                        uint32_t row_bytes) {
-  uint8_t* dst = s.ring + (size_t)st * a.stage_bytes;
-  fence_proxy_async_smem();
-  mbar_arrive_expect_tx(&s.bar[st], 2 * row_bytes);
-  bulk_g2s(dst, a.Wu_t + (size_t)j * a.d, row_bytes, &s.bar[st]);
-  bulk_g2s(dst + row_bytes, a.Wd + (size_t)j * a.d, row_bytes, &s.bar[st]);
-}
-
-template <typename Tin, int NCH, bool kOutBf16>
+// NCHW: 16-byte column slices per lane for one warp of a team.
+template <typename Tin, int NCHW, bool kOutBf16>
 __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<Tin> a) {
   using L = Elem<Tin>;
   constexpr int E = L::E;
   constexpr int P = L::P;
-  constexpr int SPAN = 32 * E;  // columns covered by one warp-wide 16-byte slice
+  constexpr int SPAN = 32 * E;             // columns of one warp-wide slice
+  constexpr int COLS = NCHW * SPAN;        // columns owned by one warp
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
+  const int team = wid / kTeam;
+  const int tw = wid % kTeam;              // this warp's place in its team
   const int d = a.d;
-  const uint32_t row_bytes = (uint32_t)d * sizeof(Tin);
+  const int c0 = tw * COLS;                // first column of this warp
+  const int my_cols = d - c0 < COLS ? (d - c0 > 0 ? d - c0 : 0) : COLS;
+  const uint32_t my_bytes = (uint32_t)my_cols * sizeof(Tin);
 
-  const size_t per_warp = 128 + kListCap * 8 + (size_t)a.stages * a.stage_bytes;
-  uint8_t* mine = smem_raw + (size_t)wid * per_warp;
-  WarpSmem s;
-  s.bar = reinterpret_cast<uint64_t*>(mine);
-  s.g = reinterpret_cast<float*>(mine + 128);
-  s.j = reinterpret_cast<int32_t*>(mine + 128 + kListCap * 4);
-  s.ring = mine + 128 + kListCap * 8;
+  // shared memory: [kTeams] TeamSmem, then per warp: barriers + ring
+  TeamSmem& ts = reinterpret_cast<TeamSmem*>(smem_raw)[team];
+  const size_t team_bytes = (sizeof(TeamSmem) * kTeams + 127) & ~size_t(127);
+  const size_t per_warp = 128 + (size_t)a.stages * 2 * a.slice_bytes;
+  uint8_t* mine = smem_raw + team_bytes + (size_t)wid * per_warp;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(mine);
+  uint8_t* ring = mine + 128;
   if (lane == 0) {
-    for (int i = 0; i < a.stages; ++i) mbar_init(&s.bar[i], 1);
+    for (int i = 0; i < a.stages; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
   }
   __syncwarp();
+
   int never = 0;
-  // Ring position of this warp, advanced incrementally (no division):
-  // cst/cph next stage to wait on and its phase parity, pst next stage to
-  // fill, inflight stages filled but not yet waited on.
+  // Ring position of this warp, advanced incrementally (no division).
   uint32_t cst = 0, cph = 0, pst = 0, inflight = 0;
   bool failed = false;
   const int n_items = a.ws.hdr[1];
+  const bool leader = tw == 0;
+
+  auto issue = [&](int j) {
+    uint8_t* dst = ring + (size_t)pst * 2 * a.slice_bytes;
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&bar[pst], 2 * my_bytes);
+    bulk_g2s(dst, a.Wu_t + (size_t)j * d + c0, my_bytes, &bar[pst]);
+    bulk_g2s(dst + a.slice_bytes, a.Wd + (size_t)j * d + c0, my_bytes, &bar[pst]);
+  };
 
   int ticket = 0;
-  if (lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);
-  int item = __shfl_sync(FULL, ticket, 0);
-  while (item < n_items) {
-    if (lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);  // next item, fetched early
-    const int4 desc = a.ws.item_desc[item];
+  if (leader && lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);
+  for (uint32_t it = 0;; ++it) {
+    // The descriptor slot alternates between items: the partner reads slot
+    // it&1 after this barrier, and the leader next writes it two items later,
+    // behind barriers the partner has passed.
+    if (leader && lane == 0) {
+      const int item = ticket;
+      ts.desc[it & 1] = item < n_items ? a.ws.item_desc[item] : make_int4(-1, 0, 0, -1);
+      if (item < n_items) ticket = atomicAdd(&a.ws.hdr[0], 1);  // next, fetched early
+    }
+    team_bar(team);
+    const int4 desc = ts.desc[it & 1];
+    if (desc.x < 0) break;
     const int t = desc.x, lo = desc.y, hi = desc.z, prow = desc.w;
 
-    float2 xf[NCH][P];
+    float2 xf[NCHW][P];
+    float2 acc[NCHW][P];
     const Tin* xt = a.x + (size_t)t * d;
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = c * SPAN + lane * E;
+    for (int c = 0; c < NCHW; ++c) {
+      const int col = c0 + c * SPAN + lane * E;
       const uint4 r = col < d ? __ldg(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
       L::pairs(r, xf[c]);
-    }
-    float2 acc[NCH][P];
-#pragma unroll
-    for (int c = 0; c < NCH; ++c)
 #pragma unroll
       for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
+    }
 
     for (int w0 = lo; w0 < hi && !failed; w0 += kListCap) {
-      const int n = collect(a, t, w0, min(hi, w0 + kListCap), s, lane);
+      if (leader) {
+        const int n = collect(a, t, w0, min(hi, w0 + kListCap), ts, lane);
+        if (lane == 0) ts.n = n;
+      }
+      team_bar(team);
+      const int n = ts.n;
       const int pre = n < a.stages ? n : a.stages;
       for (int e = 0; e < pre; ++e) {
-        if (lane == 0) issue_entry(a, s, pst, s.j[e], row_bytes);
+        if (lane == 0 && my_bytes) issue(ts.j[e]);
         pst = pst + 1 == (uint32_t)a.stages ? 0u : pst + 1;
         ++inflight;
       }
       for (int e = 0; e < n; ++e) {
         const uint32_t st = cst;
-        bool ok = mbar_wait(&s.bar[st], cph, &never, a.timeout_ns);
+        bool ok = true;
+        if (my_bytes) ok = mbar_wait(&bar[st], cph, &never, a.timeout_ns);
         ok = __all_sync(FULL, ok);
-        if (!ok) {
+        const uint8_t* stage = ring + (size_t)st * 2 * a.slice_bytes;
+        const uint4* wu = reinterpret_cast<const uint4*>(stage);
+        const uint4* wd = reinterpret_cast<const uint4*>(stage + a.slice_bytes);
+        float2 pd[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        if (ok) {
+#pragma unroll
+          for (int c = 0; c < NCHW; ++c) {
+            const int lc = c * SPAN + lane * E;  // column within this warp's range
+            if (lc < my_cols) {
+              float2 w[P];
+              L::pairs(wu[lc / E], w);
+#pragma unroll
+              for (int q = 0; q < P; ++q)
+                pd[(c * P + q) & 3] = __ffma2_rn(xf[c][q], w[q], pd[(c * P + q) & 3]);
+            }
+          }
+        }
+        const float2 p01 = __fadd2_rn(pd[0], pd[1]);
+        const float2 p23 = __fadd2_rn(pd[2], pd[3]);
+        const float2 pp = __fadd2_rn(p01, p23);
+        const float part = warp_sum(pp.x + pp.y);
+        const int pb = e & 1;
+        if (lane == 0) {
+          ts.red[pb][tw] = part;
+          ts.ok[pb][tw] = ok ? 1 : 0;
+        }
+        team_bar(team);  // unconditional: every warp of the team reaches it
+        float u = 0.f;
+        bool all_ok = true;
+#pragma unroll
+        for (int q = 0; q < kTeam; ++q) {
+          u += ts.red[pb][q];
+          all_ok = all_ok && ts.ok[pb][q] != 0;
+        }
+        if (!all_ok) {  // the same decision in every warp of the team
           failed = true;
           break;
         }
@@ -402,33 +470,14 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
           cst = 0;
           cph ^= 1u;
         }
-        const uint8_t* stage = s.ring + (size_t)st * a.stage_bytes;
-        const uint4* wu = reinterpret_cast<const uint4*>(stage);
-        const uint4* wd = reinterpret_cast<const uint4*>(stage + row_bytes);
-        float2 pd[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          const int col = c * SPAN + lane * E;
-          if (col < d) {
-            float2 w[P];
-            L::pairs(wu[col / E], w);
-#pragma unroll
-            for (int q = 0; q < P; ++q) pd[(c * P + q) & 3] = __ffma2_rn(xf[c][q], w[q], pd[(c * P + q) & 3]);
-          }
-        }
-        const float2 p01 = __fadd2_rn(pd[0], pd[1]);
-        const float2 p23 = __fadd2_rn(pd[2], pd[3]);
-        const float2 pp = __fadd2_rn(p01, p23);
-        const float u = warp_sum(pp.x + pp.y);
-        const float h = s.g[e] * u;
+        const float h = ts.g[e] * u;
         const float2 hh = make_float2(h, h);
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          const int col = c * SPAN + lane * E;
-          if (col < d) {
+        for (int c = 0; c < NCHW; ++c) {
+          const int lc = c * SPAN + lane * E;
+          if (lc < my_cols) {
             float2 w[P];
-            L::pairs(wd[col / E], w);
+            L::pairs(wd[lc / E], w);
 #pragma unroll
             for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(hh, w[q], acc[c][q]);
           }
@@ -436,12 +485,12 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
         __syncwarp();  // every lane is done with this stage
         const int nxt = e + a.stages;
         if (nxt < n) {  // refill the stage just freed (the ring was full)
-          if (lane == 0) issue_entry(a, s, pst, s.j[nxt], row_bytes);
+          if (lane == 0 && my_bytes) issue(ts.j[nxt]);
           pst = pst + 1 == (uint32_t)a.stages ? 0u : pst + 1;
           ++inflight;
         }
       }
-      __syncwarp();
+      team_bar(team);  // the list may be overwritten by the next window
     }
     if (failed) break;
 
@@ -449,8 +498,8 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
     const bool split = prow >= 0;
     float* out_row = split ? a.ws.partial + (size_t)prow * d : nullptr;
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = c * SPAN + lane * E;
+    for (int c = 0; c < NCHW; ++c) {
+      const int col = c0 + c * SPAN + lane * E;
       if (col >= d) continue;
       if (split || !kOutBf16) {
         float* dst = split ? out_row + col : static_cast<float*>(a.y) + (size_t)t * d + col;
@@ -468,15 +517,14 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
     if (split) {
       // the last part to finish sums the partial rows in part order
       __threadfence();
-      __syncwarp();
+      team_bar(team);  // both halves of this part's row are written
       const int parts = (a.ws.nnz[t] + kPart - 1) / kPart;
-      int prev = 0;
-      if (lane == 0) prev = atomicAdd(&a.ws.done[t], 1);
-      prev = __shfl_sync(FULL, prev, 0);
-      if (prev == parts - 1) {
+      if (leader && lane == 0) ts.prev = atomicAdd(&a.ws.done[t], 1);
+      team_bar(team);
+      if (ts.prev == parts - 1) {
         __threadfence();
         const float* part0 = a.ws.partial + (size_t)(prow - lo / kPart) * d;
-        for (int col = lane * 4; col < d; col += 128) {
+        for (int col = c0 + lane * 4; col < c0 + my_cols; col += 128) {
           float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int q = 0; q < parts; ++q) {
             const float4 v = __ldcg(reinterpret_cast<const float4*>(part0 + (size_t)q * d + col));
@@ -492,14 +540,13 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
         }
       }
     }
-    item = __shfl_sync(FULL, ticket, 0);
   }
 
   if (failed) {
     if (lane == 0) set_status(a.status, kStatusTimeout);
     // let the copies still in flight land before the CTA may exit
     for (uint32_t q = 0; q < inflight; ++q) {
-      mbar_wait(&s.bar[cst], cph, &never, a.timeout_ns);
+      if (my_bytes) mbar_wait(&bar[cst], cph, &never, a.timeout_ns);
       if (++cst == (uint32_t)a.stages) {
         cst = 0;
         cph ^= 1u;
@@ -508,15 +555,17 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
   }
 }
 
-template <typename Tin, int NCH>
+template <typename Tin, int NCHW>
 cudaError_t launch_t(FusedArgs<Tin> a, tw_dtype y_dtype, cudaStream_t stream) {
-  a.stage_bytes = 2 * a.d * (int)sizeof(Tin);
-  a.stages = kRingBytes / a.stage_bytes;
+  constexpr int SPAN = 32 * Elem<Tin>::E;
+  a.slice_bytes = NCHW * SPAN * (int)sizeof(Tin);
+  a.stages = kRingBytes / (2 * a.slice_bytes);
   if (a.stages > 8) a.stages = 8;
   if (a.stages < 2) a.stages = 2;
-  const size_t per_warp = 128 + kListCap * 8 + (size_t)a.stages * a.stage_bytes;
-  const size_t smem = per_warp * kWarps;
-  auto kern = y_dtype == TW_BF16 ? fused_kernel<Tin, NCH, true> : fused_kernel<Tin, NCH, false>;
+  const size_t team_bytes = (sizeof(TeamSmem) * kTeams + 127) & ~size_t(127);
+  const size_t per_warp = 128 + (size_t)a.stages * 2 * a.slice_bytes;
+  const size_t smem = team_bytes + per_warp * kWarps;
+  auto kern = y_dtype == TW_BF16 ? fused_kernel<Tin, NCHW, true> : fused_kernel<Tin, NCHW, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -542,20 +591,23 @@ cudaError_t run_plan_and_fused(const void* x, const tw_twell& g, const void* Wu_
                           g.idx, g.cnt, g.spill_ref, static_cast<const uint16_t*>(g.spill_val),
                           static_cast<const uint16_t*>(Wu_t), static_cast<const uint16_t*>(Wd),
                           y, status, g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
-    if (d <= 256) return launch_t<uint16_t, 1>(a, y_dtype, stream);
-    if (d <= 512) return launch_t<uint16_t, 2>(a, y_dtype, stream);
-    if (d <= 1024) return launch_t<uint16_t, 4>(a, y_dtype, stream);
-    return launch_t<uint16_t, 8>(a, y_dtype, stream);
+    // chunks of 256 columns, split over the kTeam warps
+    const int nch = (d + 255) / 256;
+    const int per = (nch + kTeam - 1) / kTeam;
+    if (per <= 1) return launch_t<uint16_t, 1>(a, y_dtype, stream);
+    if (per <= 2) return launch_t<uint16_t, 2>(a, y_dtype, stream);
+    return launch_t<uint16_t, 4>(a, y_dtype, stream);
   }
   FusedArgs<float> a{static_cast<const float*>(x), static_cast<const float*>(g.val), g.idx, g.cnt,
                      g.spill_ref, static_cast<const float*>(g.spill_val),
                      static_cast<const float*>(Wu_t), static_cast<const float*>(Wd), y, status,
                      g.T, d, g.F, g.C, g.spill_cap, w, 0, 0, kWaitTimeoutNs};
-  if (d <= 128) return launch_t<float, 1>(a, y_dtype, stream);
-  if (d <= 256) return launch_t<float, 2>(a, y_dtype, stream);
-  if (d <= 512) return launch_t<float, 4>(a, y_dtype, stream);
-  if (d <= 1024) return launch_t<float, 8>(a, y_dtype, stream);
-  return launch_t<float, 16>(a, y_dtype, stream);
+  const int nch = (d + 127) / 128;
+  const int per = (nch + kTeam - 1) / kTeam;
+  if (per <= 1) return launch_t<float, 1>(a, y_dtype, stream);
+  if (per <= 2) return launch_t<float, 2>(a, y_dtype, stream);
+  if (per <= 4) return launch_t<float, 4>(a, y_dtype, stream);
+  return launch_t<float, 8>(a, y_dtype, stream);
 }
 
 }  // namespace
