@@ -42,7 +42,8 @@ namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
 constexpr int W = 128;             // TwELL tile width
-constexpr int kPart = 64;          // entries per part of a split token
+constexpr int kPart = 64;          // entries per part of a split token (upper bound)
+constexpr int kMinPart = 8;        // lower bound of the part size
 constexpr int kTeam = 2;           // warps per work item
 constexpr int kTeams = 8;          // teams per CTA
 constexpr int kWarps = kTeam * kTeams;
@@ -92,14 +93,14 @@ FusedWs layout(void* base, int T, int d, int cap) {
   return w;
 }
 
-FusedWs carve(void* base, int T, int d) { return layout(base, T, d, T / 2 + 256); }
+FusedWs carve(void* base, int T, int d) { return layout(base, T, d, T / 2 + 1024); }
 
 // The same plan inside a fixed scratch area of `limit` bytes: the split
 // capacity shrinks to what fits (tokens past it stay unsplit).  Returns false
 // when even the unsplit plan does not fit.
 bool carve_within(void* base, int T, int d, size_t limit, FusedWs* out) {
   if (layout(nullptr, T, d, 0).bytes > limit) return false;
-  int lo = 0, hi = T / 2 + 256;  // largest capacity whose layout fits
+  int lo = 0, hi = T / 2 + 1024;  // largest capacity whose layout fits
   while (lo < hi) {
     const int mid = lo + (hi - lo + 1) / 2;
     if (layout(nullptr, T, d, mid).bytes <= limit) lo = mid;
@@ -147,47 +148,65 @@ TW_DEV int block_exclusive_scan(int v, int* warp_sums, int* total) {
   return excl;
 }
 
-// One CTA: partial rows of split tokens (in token order, within capacity),
-// then one descriptor per work item.
+// One CTA: the part size, partial rows of split tokens (in token order,
+// within capacity), then one descriptor per work item.  The part size is
+// kPart, lowered to about two items per team when there are few entries in
+// all (small batches), but not below kMinPart; it is stored in hdr[2].
+// Each thread owns a contiguous run of tokens, so each of the three passes
+// needs a single block-wide scan.
 __global__ void __launch_bounds__(kScanThreads)
     plan_scan_kernel(int T, const int32_t* __restrict__ nnz, int parts_cap, int max_items,
-                     int32_t* slot_off, int4* item_desc, int32_t* hdr) {
+                     int n_teams, int32_t* slot_off, int4* item_desc, int32_t* hdr) {
   __shared__ int warp_sums[32];
-  __shared__ int carry_slots, carry_items;
-  if (threadIdx.x == 0) carry_slots = carry_items = 0;
+  __shared__ int part_sh;
+  const int run = (T + kScanThreads - 1) / kScanThreads;
+  const int t0 = threadIdx.x * run;
+  const int t1 = min(T, t0 + run);
+  // pass 0: total number of entries -> part size
+  int local = 0;
+  for (int t = t0; t < t1; ++t) local += nnz[t];
+  int total;
+  block_exclusive_scan(local, warp_sums, &total);
+  if (threadIdx.x == 0) {
+    const int p = total / (2 * n_teams);
+    part_sh = p < kMinPart ? kMinPart : (p > kPart ? kPart : p);
+    hdr[2] = part_sh;
+  }
   __syncthreads();
-  for (int base = 0; base < T; base += kScanThreads) {
-    const int t = base + threadIdx.x;
-    const int n = t < T ? nnz[t] : 0;
-    const int parts = n > kPart ? (n + kPart - 1) / kPart : 0;
-    int tot;
-    const int ex = block_exclusive_scan(parts, warp_sums, &tot) + carry_slots;
-    if (t < T) slot_off[t] = (parts > 0 && ex + parts <= parts_cap) ? ex : -1;
-    if (threadIdx.x == 0) carry_slots += tot;
-    __syncthreads();
+  const int part = part_sh;
+  // pass 1: partial rows of split tokens, in token order; a token whose rows
+  // would pass the capacity (and every later one) stays unsplit
+  local = 0;
+  for (int t = t0; t < t1; ++t) {
+    const int n = nnz[t];
+    local += n > part ? (n + part - 1) / part : 0;
   }
-  for (int base = 0; base < T; base += kScanThreads) {
-    const int t = base + threadIdx.x;
-    int parts = 0, n = 0, so = -1;
-    if (t < T) {
-      n = nnz[t];
-      so = slot_off[t];
-      parts = so >= 0 ? (n + kPart - 1) / kPart : 1;
-    }
-    int tot;
-    const int ex = block_exclusive_scan(parts, warp_sums, &tot) + carry_items;
-    if (t < T) {
-      if (so < 0) {
-        if (ex < max_items) item_desc[ex] = make_int4(t, 0, n, -1);
-      } else {
-        for (int p = 0; p < parts && ex + p < max_items; ++p)
-          item_desc[ex + p] = make_int4(t, p * kPart, min(n, (p + 1) * kPart), so + p);
-      }
-    }
-    if (threadIdx.x == 0) carry_items += tot;
-    __syncthreads();
+  int tot;
+  int ex = block_exclusive_scan(local, warp_sums, &tot);
+  for (int t = t0; t < t1; ++t) {
+    const int n = nnz[t];
+    const int parts = n > part ? (n + part - 1) / part : 0;
+    slot_off[t] = (parts > 0 && ex + parts <= parts_cap) ? ex : -1;
+    ex += parts;
   }
-  if (threadIdx.x == 0) hdr[1] = carry_items < max_items ? carry_items : max_items;
+  // pass 2: one descriptor per work item
+  local = 0;
+  for (int t = t0; t < t1; ++t)
+    local += slot_off[t] >= 0 ? (nnz[t] + part - 1) / part : 1;
+  ex = block_exclusive_scan(local, warp_sums, &tot);
+  for (int t = t0; t < t1; ++t) {
+    const int n = nnz[t], so = slot_off[t];
+    if (so < 0) {
+      if (ex < max_items) item_desc[ex] = make_int4(t, 0, n, -1);
+      ++ex;
+    } else {
+      const int parts = (n + part - 1) / part;
+      for (int p = 0; p < parts && ex + p < max_items; ++p)
+        item_desc[ex + p] = make_int4(t, p * part, min(n, (p + 1) * part), so + p);
+      ex += parts;
+    }
+  }
+  if (threadIdx.x == 0) hdr[1] = tot < max_items ? tot : max_items;
 }
 
 // ------------------------------------------------------------- arithmetic --
@@ -208,6 +227,23 @@ struct Elem<uint16_t> {       // bf16
   TW_DEV static void pairs(const uint4& r, float2 (&w)[P]) {
     w[0] = bf16_pair(r.x); w[1] = bf16_pair(r.y); w[2] = bf16_pair(r.z); w[3] = bf16_pair(r.w);
   }
+  // a[0..3] += x . w over one slice with the mixed-precision FMA (bf16
+  // inputs, fp32 accumulator; the bf16 product is exact in fp32).
+  TW_DEV static void dot(const uint4& x, const uint4& w, float (&a)[4]) {
+    dot_pair(x.x, w.x, a[0], a[1]);
+    dot_pair(x.y, w.y, a[2], a[3]);
+    dot_pair(x.z, w.z, a[0], a[1]);
+    dot_pair(x.w, w.w, a[2], a[3]);
+  }
+  TW_DEV static void dot_pair(uint32_t xp, uint32_t wp, float& a0, float& a1) {
+    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "mov.b32 {wl, wh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, xl, wl, %0;\n\t"
+        "fma.rn.f32.bf16 %1, xh, wh, %1;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(xp), "r"(wp));
+  }
 };
 
 template <>
@@ -218,6 +254,12 @@ struct Elem<float> {
   TW_DEV static void pairs(const uint4& r, float2 (&w)[P]) {
     w[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
     w[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
+  }
+  TW_DEV static void dot(const uint4& x, const uint4& w, float (&a)[4]) {
+    a[0] = fmaf(__uint_as_float(x.x), __uint_as_float(w.x), a[0]);
+    a[1] = fmaf(__uint_as_float(x.y), __uint_as_float(w.y), a[1]);
+    a[2] = fmaf(__uint_as_float(x.z), __uint_as_float(w.z), a[2]);
+    a[3] = fmaf(__uint_as_float(x.w), __uint_as_float(w.w), a[3]);
   }
 };
 
@@ -396,14 +438,13 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
     if (desc.x < 0) break;
     const int t = desc.x, lo = desc.y, hi = desc.z, prow = desc.w;
 
-    float2 xf[NCHW][P];
+    uint4 xr[NCHW];  // x_t slices, kept in the input format
     float2 acc[NCHW][P];
     const Tin* xt = a.x + (size_t)t * d;
 #pragma unroll
     for (int c = 0; c < NCHW; ++c) {
       const int col = c0 + c * SPAN + lane * E;
-      const uint4 r = col < d ? __ldg(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
-      L::pairs(r, xf[c]);
+      xr[c] = col < d ? __ldg(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
     }
@@ -429,37 +470,32 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
         const uint8_t* stage = ring + (size_t)st * 2 * a.slice_bytes;
         const uint4* wu = reinterpret_cast<const uint4*>(stage);
         const uint4* wd = reinterpret_cast<const uint4*>(stage + a.slice_bytes);
-        float2 pd[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
+        float pa[4] = {0.f, 0.f, 0.f, 0.f};
+        float pb[4] = {0.f, 0.f, 0.f, 0.f};
         if (ok) {
 #pragma unroll
           for (int c = 0; c < NCHW; ++c) {
             const int lc = c * SPAN + lane * E;  // column within this warp's range
             if (lc < my_cols) {
-              float2 w[P];
-              L::pairs(wu[lc / E], w);
-#pragma unroll
-              for (int q = 0; q < P; ++q)
-                pd[(c * P + q) & 3] = __ffma2_rn(xf[c][q], w[q], pd[(c * P + q) & 3]);
+              if (c & 1) L::dot(xr[c], wu[lc / E], pb);
+              else L::dot(xr[c], wu[lc / E], pa);
             }
           }
         }
-        const float2 p01 = __fadd2_rn(pd[0], pd[1]);
-        const float2 p23 = __fadd2_rn(pd[2], pd[3]);
-        const float2 pp = __fadd2_rn(p01, p23);
-        const float part = warp_sum(pp.x + pp.y);
-        const int pb = e & 1;
+        const float part = warp_sum(((pa[0] + pb[0]) + (pa[1] + pb[1])) +
+                                    ((pa[2] + pb[2]) + (pa[3] + pb[3])));
+        const int rb = e & 1;  // exchange buffer of this entry
         if (lane == 0) {
-          ts.red[pb][tw] = part;
-          ts.ok[pb][tw] = ok ? 1 : 0;
+          ts.red[rb][tw] = part;
+          ts.ok[rb][tw] = ok ? 1 : 0;
         }
         team_bar(team);  // unconditional: every warp of the team reaches it
         float u = 0.f;
         bool all_ok = true;
 #pragma unroll
         for (int q = 0; q < kTeam; ++q) {
-          u += ts.red[pb][q];
-          all_ok = all_ok && ts.ok[pb][q] != 0;
+          u += ts.red[rb][q];
+          all_ok = all_ok && ts.ok[rb][q] != 0;
         }
         if (!all_ok) {  // the same decision in every warp of the team
           failed = true;
@@ -518,12 +554,13 @@ __global__ void __launch_bounds__(32 * kWarps, 1) fused_kernel(const FusedArgs<T
       // the last part to finish sums the partial rows in part order
       __threadfence();
       team_bar(team);  // both halves of this part's row are written
-      const int parts = (a.ws.nnz[t] + kPart - 1) / kPart;
+      const int part = a.ws.hdr[2];
+      const int parts = (a.ws.nnz[t] + part - 1) / part;
       if (leader && lane == 0) ts.prev = atomicAdd(&a.ws.done[t], 1);
       team_bar(team);
       if (ts.prev == parts - 1) {
         __threadfence();
-        const float* part0 = a.ws.partial + (size_t)(prow - lo / kPart) * d;
+        const float* part0 = a.ws.partial + (size_t)(prow - lo / part) * d;
         for (int col = c0 + lane * 4; col < c0 + my_cols; col += 128) {
           float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int q = 0; q < parts; ++q) {
@@ -585,7 +622,8 @@ cudaError_t run_plan_and_fused(const void* x, const tw_twell& g, const void* Wu_
   const int K = g.F / W;
   plan_count_kernel<<<(g.T + 255) / 256, 256, 0, stream>>>(g.T, K, g.cnt, w.nnz);
   plan_scan_kernel<<<1, kScanThreads, 0, stream>>>(g.T, w.nnz, w.parts_cap, w.max_items,
-                                                   w.slot_off, w.item_desc, w.hdr);
+                                                   num_sms() * kTeams, w.slot_off, w.item_desc,
+                                                   w.hdr);
   if (g.dtype == TW_BF16) {
     FusedArgs<uint16_t> a{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(g.val),
                           g.idx, g.cnt, g.spill_ref, static_cast<const uint16_t*>(g.spill_val),

@@ -283,56 +283,150 @@ def run_ours(args, rank, world, local_rank):
            "d2h_bytes_per_step": yh.numel() * yh.element_size()}
 
     hbm, tf_burst, tf_sust, src = peaks()
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    fp32_peak = n_sm * 128 * 2 * sm_max_mhz() * 1e6 / 1e12  # TFLOP/s, FMA = 2 FLOP
     flops_gate = 2.0 * T * d * F
     tflops_gate = flops_gate / (ms_gate * 1e-3) / 1e12
-    sha = src_sha("gemm_tc.cu", "tw_common.cuh")
-    roof = {"kernel": "twell_gate_gemm (tcgen05 + TwELL epilogue)", "bound": "tensor",
-            "achieved": tflops_gate, "peak": tf_sust, "unit": "TFLOP/s",
-            "frac": tflops_gate / tf_sust,
-            "peak_source": f"{src} bf16 sustained (kernel timed inside a long loop)",
-            "frac_of_burst_peak": tflops_gate / tf_burst,
-            "traffic": profiled_traffic("gate_twell_gemm_ffn_2b.md", sha),
-            "algorithmic": f"2*T*d*F = {flops_gate:.4g} FLOP per launch"}
-
-    # fused kernel: algorithmic bytes (unique HBM) and gathered bytes, per launch
-    cnt = g.cnt.to(torch.int64)
-    nnz = int(cnt.sum().item())
+    nnz = int(g.cnt.to(torch.int64).sum().item())
+    flops_fused = 2.0 * 2 * d * nnz          # one dot and one axpy of length d per entry
+    tflops_fused = flops_fused / (ms_fused * 1e-3) / 1e12
     Kt = F // 128
-    bytes_unique = (2 * T * d * 2          # x in, y out
-                    + Kt * T * (C * 3 + 1)  # TwELL read
-                    + int((cnt.sum(1) > 0).sum().item()) * 0)  # (live-unit bytes added below)
-    live_units = int(((g.cnt > 0).any(dim=1)).sum().item())  # tiles touched (coarse)
-    bytes_gathered = nnz * 2 * d * 2
-    kernels = {
-        "gate_twell_gemm": {"ms": ms_gate, "tflops": tflops_gate,
-                            "frac_sustained": tflops_gate / tf_sust,
-                            "frac_burst": tflops_gate / tf_burst},
-        "fused_updown": {"ms": ms_fused, "nnz_per_token": nnz / T,
-                         "gathered_GBps": bytes_gathered / (ms_fused * 1e-3) / 1e9,
-                         "fma_tflops": 2.0 * nnz * 2 * d / (ms_fused * 1e-3) / 1e12,
-                         "x_y_twell_GBps": bytes_unique / (ms_fused * 1e-3) / 1e9},
-        "spills_per_step": int(g.spill_n.item()),
-    }
-    _ = live_units
+    unique_bytes = 2 * T * d + 4 * T * d + Kt * T * (3 * C + 1)  # x, fp32 y, TwELL
+    roof_gate = {"kernel": "twell_gate_gemm (tcgen05 + TwELL epilogue)", "bound": "tensor",
+                 "achieved": tflops_gate, "peak": tf_sust, "unit": "TFLOP/s",
+                 "frac": tflops_gate / tf_sust,
+                 "peak_source": f"{src} bf16 sustained (kernel timed inside a long loop)",
+                 "frac_of_burst_peak": tflops_gate / tf_burst,
+                 "traffic": profiled_traffic("gate_twell_gemm_ffn_2b.md",
+                                             src_sha("gemm_tc.cu", "tw_common.cuh")),
+                 "algorithmic": f"2*T*d*F = {flops_gate:.4g} FLOP per launch"}
+    roof_fused = {"kernel": "twell_fused_updown (gather dot + axpy on CUDA cores)", "bound": "alu",
+                  "achieved": tflops_fused, "peak": fp32_peak, "unit": "TFLOP/s",
+                  "frac": tflops_fused / fp32_peak,
+                  "peak_source": f"derived: {n_sm} SMs x 128 fp32 FMA lanes x 2 x {sm_max_mhz():.0f} MHz",
+                  "traffic": profiled_traffic("fused_updown_ffn_2b.md",
+                                              src_sha("fused_updown.cu", "tw_common.cuh")),
+                  "algorithmic": f"4*d*nnz = {flops_fused:.4g} FLOP per launch (nnz = {nnz})",
+                  "gathered_GBps": nnz * 4 * d / (ms_fused * 1e-3) / 1e9,
+                  "unique_hbm_GBps": unique_bytes / (ms_fused * 1e-3) / 1e9,
+                  "unique_hbm_frac": unique_bytes / (ms_fused * 1e-3) / 1e9 / hbm}
+    dominant = roof_fused if ms_fused >= ms_gate else roof_gate
+    kernels = {"gate_twell_gemm": {"ms": ms_gate, **roof_gate},
+               "fused_updown": {"ms": ms_fused, "nnz_per_token": nnz / T, **roof_fused},
+               "spills_per_step": int(g.spill_n.item())}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
             "data": "synthetic (seeded generator: Zipf(1.1) units, lognormal token skew, "
                     "mean 29 active units per token)",
-            "config": config_of(w, args), "roofline": roof, "e2e": e2e,
-            "gpu_launches": 2 * K, "clocks": clk, "kernels": kernels,
+            "config": config_of(w, args), "roofline": dominant, "e2e": e2e,
+            "gpu_launches": KERNELS_PER_STEP * K, "clocks": clk, "kernels": kernels,
             "device_status": st}
 
-    if rank == 0 and not args.no_extras:
-        line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_leg(w, y)
+    if rank == 0 and not args.no_extras:
+        line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
+        del x, Wg, Wu, Wd, g, y, ws, xh, yh
+        torch.cuda.empty_cache()
+        line["decode"] = decode_leg(torch, tw, hbm)
+        line["training"] = training_leg(torch, tw)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# kernels of one inference step: gate GEMM; plan count, plan scan, fused kernel
+KERNELS_PER_STEP = 4
+
+
+def sm_max_mhz():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["sm_max_mhz"])
+    except Exception:
+        return 1965.0
+
+
+def decode_leg(torch, tw, hbm):
+    """Small batches (T = 1, 8, 64) of the 2B shape with a cold L2 (a 512 MB
+    buffer is rewritten between iterations): the gate streams Wg from HBM."""
+    flush = torch.empty(128 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    out = {}
+    for T in (1, 8, 64):
+        w = synth.make_workload("decode_2b", T=T)
+        d, F, C = w["d"], w["F"], w["C"]
+        dev = {k: torch.from_numpy(w[k].view(np.int16)).cuda().view(torch.bfloat16)
+               for k in ("x", "Wg_t", "Wu_t", "Wd")}
+        g = tw.Twell(T, F, C, dtype=torch.bfloat16, spill_cap=4096)
+        y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+        ws = tw.fused_workspace(T, d)
+        tg, tf = [], []
+        for it in range(25):
+            flush.fill_(float(it))
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record()
+            tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g)
+            e[1].record()
+            tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y, ws)
+            e[2].record()
+            torch.cuda.synchronize()
+            if it >= 5:
+                tg.append(e[0].elapsed_time(e[1]))
+                tf.append(e[1].elapsed_time(e[2]))
+        nnz = int(g.cnt.to(torch.int64).sum().item())
+        mg, mf = float(np.median(tg)), float(np.median(tf))
+        gate_gbs = F * d * 2 / (mg * 1e-3) / 1e9
+        rows = nnz * 2 * d * 2  # Wu and Wd rows gathered (an upper bound on unique bytes)
+        out[f"T{T}"] = {"gate_us": mg * 1e3, "fused_us": mf * 1e3, "tokens_per_s": T / ((mg + mf) * 1e-3),
+                        "gate_hbm_GBps": gate_gbs, "gate_hbm_frac": gate_gbs / hbm,
+                        "fused_gathered_GBps": rows / (mf * 1e-3) / 1e9, "nnz": nnz}
+    del flush
+    return out
+
+
+def training_leg(torch, tw):
+    """One training step of the hybrid path at the train_2b shape: gate GEMM ->
+    TwELL -> hybrid, hybrid forward, hybrid backward (with the L1 term)."""
+    w = synth.make_workload("train_2b")
+    T, d, F, C, C_h = w["T"], w["d"], w["F"], w["C"], w["C_h"]
+    dev = {k: torch.from_numpy(w[k].view(np.int16)).cuda().view(torch.bfloat16)
+           for k in ("x", "Wg_t", "Wu_t", "Wd", "dy")}
+    cap = T // 4
+    g = tw.Twell(T, F, C, dtype=torch.bfloat16, spill_cap=(F // 128) * T // 8)
+    hy = tw.Hybrid(T, F, C_h, dtype=torch.bfloat16, backup_cap=cap)
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    dW = [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+    ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, C_h, cap), dtype=torch.uint8,
+                     device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    names = ["gate_twell_gemm", "twell_to_hybrid", "hybrid_ffn_forward", "hybrid_ffn_backward"]
+    times = {n: [] for n in names}
+    for it in range(8):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e[0].record()
+        tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, None, st)
+        e[1].record()
+        tw.twell_to_hybrid(g, hy, st)
+        e[2].record()
+        tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], y, st)
+        e[3].record()
+        tw.hybrid_ffn_backward(dev["x"], dev["dy"], hy, dev["Wg_t"], dev["Wu_t"], dev["Wd"],
+                               w["lam"], dx, dW[0], dW[1], dW[2], ws, st)
+        e[4].record()
+        torch.cuda.synchronize()
+        if it >= 3:
+            for i, n in enumerate(names):
+                times[n].append(e[i].elapsed_time(e[i + 1]))
+    ms = {n: float(np.median(v)) for n, v in times.items()}
+    step = sum(ms.values())
+    return {"workload": "train_2b", "T": T, "d": d, "F": F, "C": C, "C_h": C_h,
+            "ms": ms, "ms_per_step": step, "tokens_per_s": T / (step * 1e-3),
+            "n_backup": int(hy.n_backup.item()), "backup_cap": cap, "device_status": int(st.item())}
 
 
 def dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_sparse, args):
