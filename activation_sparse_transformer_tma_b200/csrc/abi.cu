@@ -29,6 +29,13 @@ constexpr int kTileW = 128;
 constexpr int kMaxC = 32;
 constexpr int kMaxRowD = 2048;
 
+// Row width d: a multiple of 8, at most 2048 for bf16 rows and 1024 for fp32
+// rows (one warp's column range of up to three weight rows, double-buffered,
+// for sixteen warps must fit the shared memory of one SM).
+bool row_d_ok(int d, tw_dtype t) {
+  return d % 8 == 0 && d <= (t == TW_BF16 ? kMaxRowD : kMaxRowD / 2);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool dtype_ok(tw_dtype t) { return t == TW_F32 || t == TW_BF16; }
 
@@ -120,7 +127,7 @@ tw_status twell_fused_updown(const void* x, const tw_twell* g, const void* Wu_t,
   if (st != TW_OK) return st;
   if (!x || !Wu_t || !Wd || !y || !ws || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
   if (d <= 0) return TW_ERR_INVALID_ARG;
-  if (d % 8 != 0 || d > kMaxRowD) return TW_ERR_UNSUPPORTED;
+  if (!row_d_ok(d, g->dtype)) return TW_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y) || !aligned16(ws))
     return TW_ERR_ALIGNMENT;
   if (ws_bytes < tw::fused_ws_bytes(g->T, d)) return TW_ERR_WORKSPACE;
@@ -140,19 +147,26 @@ tw_status twell_to_hybrid(const tw_twell* g, const tw_hybrid* out, int32_t* dev_
   return from_cuda(tw::launch_twell_to_hybrid(*g, *out, dev_status, stream));
 }
 
+size_t hybrid_ffn_forward_workspace_size(int32_t T, int32_t d) {
+  if (T < 0 || d <= 0) return 0;
+  return tw::hybrid_forward_ws_bytes(T, d);
+}
+
 tw_status hybrid_ffn_forward(const void* x, const tw_hybrid* gu, const void* Wu_t,
-                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype,
-                             int32_t* dev_status, cudaStream_t stream) {
+                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
   tw_status st = check_hybrid(gu);
   if (st != TW_OK) return st;
-  if (!x || !Wu_t || !Wd || !y || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
+  if (!x || !Wu_t || !Wd || !y || !ws || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
   if ((gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
     return TW_ERR_INVALID_ARG;
   if (d <= 0) return TW_ERR_INVALID_ARG;
-  if (d % 8 != 0 || d > kMaxRowD) return TW_ERR_UNSUPPORTED;
-  if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y))
+  if (!row_d_ok(d, gu->dtype)) return TW_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y) || !aligned16(ws))
     return TW_ERR_ALIGNMENT;
-  return from_cuda(tw::launch_hybrid_forward(x, *gu, Wu_t, Wd, d, y, y_dtype, dev_status, stream));
+  if (ws_bytes < tw::hybrid_forward_ws_bytes(gu->T, d)) return TW_ERR_WORKSPACE;
+  return from_cuda(
+      tw::launch_hybrid_forward(x, *gu, Wu_t, Wd, d, y, y_dtype, ws, dev_status, stream));
 }
 
 size_t hybrid_ffn_backward_workspace_size(int32_t T, int32_t d, int32_t F, int32_t C_h,
@@ -174,7 +188,7 @@ tw_status hybrid_ffn_backward(const void* x, const void* dy, const tw_hybrid* gu
   if ((gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
     return TW_ERR_INVALID_ARG;
   if (d <= 0) return TW_ERR_INVALID_ARG;
-  if (d % 8 != 0 || d > kMaxRowD) return TW_ERR_UNSUPPORTED;
+  if (!row_d_ok(d, gu->dtype)) return TW_ERR_UNSUPPORTED;
   const void* ptrs[] = {x, dy, Wg_t, Wu_t, Wd, dx, dWg_t, dWu_t, dWd, ws};
   for (const void* p : ptrs)
     if (!aligned16(p)) return TW_ERR_ALIGNMENT;

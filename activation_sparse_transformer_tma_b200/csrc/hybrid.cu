@@ -61,69 +61,6 @@ struct Slice<float> {
   TW_DEV static void widen(const Raw& r, float (&f)[4]) { f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w; }
 };
 
-template <typename T, int NCH>
-TW_DEV void load_row(const T* row, int d, int lane, typename Slice<T>::Raw (&r)[NCH]) {
-  constexpr int SPAN = 32 * Slice<T>::E;
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = c * SPAN + lane * Slice<T>::E;
-    r[c] = col < d ? Slice<T>::load(row + col) : Slice<T>::zero();
-  }
-}
-
-// Warp dot product of a register-resident row with a gathered row.
-template <typename T, int NCH>
-TW_DEV float warp_dot(const typename Slice<T>::Raw (&a)[NCH], const T* row, int d, int lane) {
-  typename Slice<T>::Raw b[NCH];
-  load_row<T, NCH>(row, d, lane, b);
-  float part = 0.f;
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    float af[Slice<T>::E], bf[Slice<T>::E];
-    Slice<T>::widen(a[c], af);
-    Slice<T>::widen(b[c], bf);
-#pragma unroll
-    for (int e = 0; e < Slice<T>::E; ++e) part = fmaf(af[e], bf[e], part);
-  }
-  return warp_sum(part);
-}
-
-// acc += s * row
-template <typename T, int NCH>
-TW_DEV void warp_axpy(float (&acc)[NCH][Slice<T>::E], float s, const T* row, int d, int lane) {
-  typename Slice<T>::Raw b[NCH];
-  load_row<T, NCH>(row, d, lane, b);
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    float bf[Slice<T>::E];
-    Slice<T>::widen(b[c], bf);
-#pragma unroll
-    for (int e = 0; e < Slice<T>::E; ++e) acc[c][e] = fmaf(s, bf[e], acc[c][e]);
-  }
-}
-
-template <int NCH, int E>
-TW_DEV void store_row(void* out, tw_dtype dt, size_t row_off, int d, int lane,
-                      const float (&acc)[NCH][E]) {
-  constexpr int SPAN = 32 * E;
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = c * SPAN + lane * E;
-    if (col >= d) continue;
-    if (dt == TW_BF16) {
-      uint16_t* p = static_cast<uint16_t*>(out) + row_off + col;
-#pragma unroll
-      for (int e = 0; e < E; e += 2)
-        *reinterpret_cast<uint32_t*>(p + e) = pack_bf16x2(acc[c][e], acc[c][e + 1]);
-    } else {
-      float* p = static_cast<float*>(out) + row_off + col;
-#pragma unroll
-      for (int e = 0; e < E; e += 4)
-        *reinterpret_cast<float4*>(p + e) = make_float4(acc[c][e], acc[c][e + 1], acc[c][e + 2], acc[c][e + 3]);
-    }
-  }
-}
-
 template <typename V>
 struct HView {
   int T, F, C_h, backup_cap;
@@ -356,98 +293,11 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// ---------------------------------------------------------- hybrid forward --
-template <typename T, int NCH>
-__global__ void __launch_bounds__(256)
-    hyb_forward_kernel(const HView<T> h, const T* x, const T* Wu_t, const T* Wd, int d, void* y,
-                       tw_dtype y_dtype) {
-  using S = Slice<T>;
-  const int lane = threadIdx.x & 31;
-  const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
-  if (t >= h.T) return;
-  typename S::Raw xr[NCH];
-  load_row<T, NCH>(x + (size_t)t * d, d, lane, xr);
-  float acc[NCH][S::E];
-#pragma unroll
-  for (int c = 0; c < NCH; ++c)
-#pragma unroll
-    for (int e = 0; e < S::E; ++e) acc[c][e] = 0.f;
-
-  const int slot = h.row_slot[t];
-  if (slot >= 0 && slot < h.backup_cap) {
-    for (int j = lane; j < h.F; j += 32) h.backup_u[(size_t)slot * h.F + j] = T(0);
-    __syncwarp();
-  }
-  for_each_chunk<T>(h, t, lane, [&](bool v, int j, float g, size_t pos, bool is_ell, int) {
-    unsigned m = __ballot_sync(FULL, v);
-    while (m) {
-      const int s = __ffs(m) - 1;
-      m &= m - 1;
-      const int jj = __shfl_sync(FULL, j, s);
-      const float gg = __shfl_sync(FULL, g, s);
-      const unsigned long long pp = __shfl_sync(FULL, (unsigned long long)pos, s);
-      const float u = warp_dot<T, NCH>(xr, Wu_t + (size_t)jj * d, d, lane);
-      if (lane == 0) st_scalar<T>(is_ell ? h.ell_u : h.backup_u, pp, u);
-      warp_axpy<T, NCH>(acc, gg * u, Wd + (size_t)jj * d, d, lane);
-    }
-  });
-  if (slot < 0) {
-    for (int s = h.row_nnz[t] + lane; s < h.C_h; s += 32)
-      h.ell_u[(size_t)t * h.C_h + s] = T(0);
-  }
-  store_row<NCH, S::E>(y, y_dtype, (size_t)t * d, d, lane, acc);
-}
-
-// --------------------------------------------------------- hybrid backward --
-struct Payload {  // one active (t, j) entry for the weight-gradient pass
-  int32_t t;
-  float h, du, dz;
-};
-
-template <typename T, int NCH>
-__global__ void __launch_bounds__(256)
-    hyb_backward_token_kernel(const HView<T> h, const T* dy, const T* Wg_t, const T* Wu_t,
-                              const T* Wd, int d, float lam, const int32_t* e0, Payload* pay,
-                              void* dx, tw_dtype dx_dtype) {
-  using S = Slice<T>;
-  const int lane = threadIdx.x & 31;
-  const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
-  if (t >= h.T) return;
-  typename S::Raw dyr[NCH];
-  load_row<T, NCH>(dy + (size_t)t * d, d, lane, dyr);
-  float acc[NCH][S::E];
-#pragma unroll
-  for (int c = 0; c < NCH; ++c)
-#pragma unroll
-    for (int e = 0; e < S::E; ++e) acc[c][e] = 0.f;
-  const int ebase = e0[t];
-  for_each_chunk<T>(h, t, lane, [&](bool v, int j, float g, size_t pos, bool is_ell, int rank) {
-    const float u = v ? ld_scalar<T>(is_ell ? h.ell_u : h.backup_u, pos) : 0.f;
-    unsigned m = __ballot_sync(FULL, v);
-    while (m) {
-      const int s = __ffs(m) - 1;
-      m &= m - 1;
-      const int jj = __shfl_sync(FULL, j, s);
-      const float gg = __shfl_sync(FULL, g, s);
-      const float uu = __shfl_sync(FULL, u, s);
-      const int rr = __shfl_sync(FULL, rank, s);
-      const float dh = warp_dot<T, NCH>(dyr, Wd + (size_t)jj * d, d, lane);
-      const float du = dh * gg;
-      const float dz = fmaf(dh, uu, lam);
-      warp_axpy<T, NCH>(acc, du, Wu_t + (size_t)jj * d, d, lane);
-      warp_axpy<T, NCH>(acc, dz, Wg_t + (size_t)jj * d, d, lane);
-      if (lane == 0) {
-        Payload p;
-        p.t = t;
-        p.h = gg * uu;
-        p.du = du;
-        p.dz = dz;
-        pay[ebase + rr] = p;
-      }
-    }
-  });
-  store_row<NCH, S::E>(dx, dx_dtype, (size_t)t * d, d, lane, acc);
-}
+// ------------------------------------------------ hybrid forward/backward --
+// The per-token passes of the hybrid forward (u on the pattern, y) and of the
+// backward (dh, du, dz, dx and the per-entry record) run on the gather engine
+// (fused_updown.cu), which splits heavy rows and streams the weight rows
+// through shared memory.  The weight gradients below use its records.
 
 constexpr int TB = 32;  // tokens per block of the transposition
 
@@ -546,7 +396,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------ workspace ----
-struct BwdWs {
+struct BwdWs {  // the gather engine's own workspace follows these arrays
   int32_t* e0;        // [T+1]
   Payload* pay;       // [Emax]
   int32_t* cntb;      // [NB][F]
@@ -623,22 +473,14 @@ cudaError_t to_hybrid_t(const tw_twell& g, const tw_hybrid& o, int32_t* status, 
   return cudaGetLastError();
 }
 
-template <typename T, int NCH>
-cudaError_t forward_t(const void* x, const tw_hybrid& gu, const void* Wu_t, const void* Wd, int d,
-                      void* y, tw_dtype y_dtype, cudaStream_t s) {
-  hyb_forward_kernel<T, NCH><<<warp_blocks(gu.T), 256, 0, s>>>(
-      view_of<T>(gu), static_cast<const T*>(x), static_cast<const T*>(Wu_t),
-      static_cast<const T*>(Wd), d, y, y_dtype);
-  return cudaGetLastError();
-}
-
-template <typename T, int NCH>
+template <typename T>
 cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const void* Wg_t,
                        const void* Wu_t, const void* Wd, int d, float lam, void* dx,
                        tw_dtype dx_dtype, float* dWg_t, float* dWu_t, float* dWd, void* ws,
                        int32_t* status, cudaStream_t s) {
   const HView<T> h = view_of<T>(gu);
   const BwdWs w = carve(ws, gu.T, gu.F, gu.C_h, gu.backup_cap);
+  void* engine_ws = static_cast<char*>(ws) + w.bytes;
   const int nb = (gu.T + TB - 1) / TB;
   const size_t hist_bytes = sizeof(int32_t) * (size_t)gu.F;
   static bool attr_set = false;
@@ -652,9 +494,11 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
   // entry offsets of every token (token-major order)
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(2, gu.T, gu.row_nnz, 0, w.e0, gu.row_slot,
                                          gu.backup_cap, nullptr, status);
-  hyb_backward_token_kernel<T, NCH><<<warp_blocks(gu.T), 256, 0, s>>>(
-      h, static_cast<const T*>(dy), static_cast<const T*>(Wg_t), static_cast<const T*>(Wu_t),
-      static_cast<const T*>(Wd), d, lam, w.e0, w.pay, dx, dx_dtype);
+  // per-token pass: dh, du, dz, dx and one record per entry
+  cudaError_t e = launch_hybrid_gather_backward(dy, gu, Wg_t, Wu_t, Wd, d, lam, w.e0, w.pay, dx,
+                                                dx_dtype, engine_ws, status, s);
+  if (e != cudaSuccess) return e;
+  // weight gradients: records transposed to unit-major, token order kept
   hyb_count_kernel<T><<<nb, 256, hist_bytes, s>>>(h, w.cntb);
   hyb_colscan_kernel<<<(gu.F + 255) / 256, 256, 0, s>>>(nb, gu.F, w.cntb, w.unit_total);
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.unit_total, 0, w.unit_off, nullptr, 0,
@@ -674,27 +518,17 @@ cudaError_t launch_twell_to_hybrid(const tw_twell& g, const tw_hybrid& out, int3
                             : to_hybrid_t<float>(g, out, status, stream);
 }
 
+size_t hybrid_forward_ws_bytes(int T, int d) { return fused_ws_bytes(T, d); }
+
 cudaError_t launch_hybrid_forward(const void* x, const tw_hybrid& gu, const void* Wu_t,
-                                  const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                  const void* Wd, int d, void* y, tw_dtype y_dtype, void* ws,
                                   int32_t* status, cudaStream_t stream) {
-  (void)status;
   if (gu.T == 0) return cudaSuccess;
-  if (gu.dtype == TW_BF16) {
-    if (d <= 256) return forward_t<uint16_t, 1>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-    if (d <= 512) return forward_t<uint16_t, 2>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-    if (d <= 1024) return forward_t<uint16_t, 4>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-    return forward_t<uint16_t, 8>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-  }
-  if (d <= 128) return forward_t<float, 1>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-  if (d <= 256) return forward_t<float, 2>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-  if (d <= 512) return forward_t<float, 4>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-  if (d <= 1024) return forward_t<float, 8>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
-  return forward_t<float, 16>(x, gu, Wu_t, Wd, d, y, y_dtype, stream);
+  return launch_hybrid_gather_forward(x, gu, Wu_t, Wd, d, y, y_dtype, ws, status, stream);
 }
 
 size_t hybrid_backward_ws_bytes(int T, int d, int F, int C_h, int backup_cap) {
-  (void)d;
-  return carve(nullptr, T, F, C_h, backup_cap).bytes;
+  return carve(nullptr, T, F, C_h, backup_cap).bytes + fused_ws_bytes(T, d);
 }
 
 cudaError_t launch_hybrid_backward(const void* x, const void* dy, const tw_hybrid& gu,
@@ -709,21 +543,11 @@ cudaError_t launch_hybrid_backward(const void* x, const void* dy, const tw_hybri
     cudaMemsetAsync(dWd, 0, sizeof(float) * (size_t)gu.F * d, stream);
     return cudaGetLastError();
   }
-#define TW_BWD(TY, N)                                                                          \
-  return backward_t<TY, N>(x, dy, gu, Wg_t, Wu_t, Wd, d, lam, dx, dx_dtype, dWg_t, dWu_t, dWd, \
-                           ws, status, stream)
-  if (gu.dtype == TW_BF16) {
-    if (d <= 256) TW_BWD(uint16_t, 1);
-    if (d <= 512) TW_BWD(uint16_t, 2);
-    if (d <= 1024) TW_BWD(uint16_t, 4);
-    TW_BWD(uint16_t, 8);
-  }
-  if (d <= 128) TW_BWD(float, 1);
-  if (d <= 256) TW_BWD(float, 2);
-  if (d <= 512) TW_BWD(float, 4);
-  if (d <= 1024) TW_BWD(float, 8);
-  TW_BWD(float, 16);
-#undef TW_BWD
+  return gu.dtype == TW_BF16
+             ? backward_t<uint16_t>(x, dy, gu, Wg_t, Wu_t, Wd, d, lam, dx, dx_dtype, dWg_t, dWu_t,
+                                    dWd, ws, status, stream)
+             : backward_t<float>(x, dy, gu, Wg_t, Wu_t, Wd, d, lam, dx, dx_dtype, dWg_t, dWu_t,
+                                 dWd, ws, status, stream);
 }
 
 }  // namespace tw

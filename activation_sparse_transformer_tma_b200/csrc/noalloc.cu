@@ -71,7 +71,7 @@ extern "C" tw_status twell_fused_updown_noalloc(const void* x, const tw_twell* g
   if (!g->cnt || !g->spill_ref || !g->spill_n) return TW_ERR_INVALID_ARG;
   if (g->C > 0 && (!g->val || !g->idx)) return TW_ERR_INVALID_ARG;
   if (g->spill_cap > 0 && (!g->spill_tk || !g->spill_val)) return TW_ERR_INVALID_ARG;
-  if (d % 8 != 0 || d > 2048) return TW_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || d > (g->dtype == TW_BF16 ? 2048 : 1024)) return TW_ERR_UNSUPPORTED;
   if (!al16(x) || !al16(Wu_t) || !al16(Wd) || !al16(y) || (g->val && !al16(g->val)) ||
       (g->idx && !al16(g->idx)) || (g->spill_val && !al16(g->spill_val)))
     return TW_ERR_ALIGNMENT;

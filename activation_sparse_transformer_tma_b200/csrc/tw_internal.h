@@ -38,11 +38,29 @@ cudaError_t launch_dense_gateup_tc(const void* x, const void* Wg_t, const void* 
                                    int d, int F, void* h, int32_t* status, cudaStream_t stream);
 cudaError_t launch_dense_down_tc(const void* h, const void* Wd_dense, int T, int d, int F,
                                  void* y, int32_t* status, cudaStream_t stream);
+// One active (t, j) entry of the hybrid backward, recorded for the
+// weight-gradient pass: h = g u, du, dz.
+struct Payload {
+  int32_t t;
+  float h, du, dz;
+};
+
+// Gather engine, hybrid modes (fused_updown.cu); ws holds fused_ws_bytes(T, d).
+cudaError_t launch_hybrid_gather_forward(const void* x, const tw_hybrid& gu, const void* Wu_t,
+                                         const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                         void* ws, int32_t* status, cudaStream_t stream);
+cudaError_t launch_hybrid_gather_backward(const void* dy, const tw_hybrid& gu, const void* Wg_t,
+                                          const void* Wu_t, const void* Wd, int d, float lam,
+                                          const int32_t* e0, Payload* pay, void* dx,
+                                          tw_dtype dx_dtype, void* ws, int32_t* status,
+                                          cudaStream_t stream);
+
 // Hybrid (training) kernels.
 cudaError_t launch_twell_to_hybrid(const tw_twell& g, const tw_hybrid& out, int32_t* status,
                                    cudaStream_t stream);
+size_t hybrid_forward_ws_bytes(int T, int d);
 cudaError_t launch_hybrid_forward(const void* x, const tw_hybrid& gu, const void* Wu_t,
-                                  const void* Wd, int d, void* y, tw_dtype y_dtype,
+                                  const void* Wd, int d, void* y, tw_dtype y_dtype, void* ws,
                                   int32_t* status, cudaStream_t stream);
 size_t hybrid_backward_ws_bytes(int T, int d, int F, int C_h, int backup_cap);
 cudaError_t launch_hybrid_backward(const void* x, const void* dy, const tw_hybrid& gu,

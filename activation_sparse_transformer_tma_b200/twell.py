@@ -23,7 +23,8 @@ STATUS = ["TW_OK", "TW_ERR_INVALID_ARG", "TW_ERR_UNSUPPORTED", "TW_ERR_ALIGNMENT
           "TW_ERR_CUDA", "TW_ERR_SPILL_CAPACITY", "TW_ERR_BACKUP_CAPACITY",
           "TW_ERR_TIMEOUT", "TW_ERR_WORKSPACE"]
 EXPORTS = ["twell_gate_gemm", "twell_fused_updown_workspace_size", "twell_fused_updown",
-           "twell_fused_updown_noalloc", "twell_to_hybrid", "hybrid_ffn_forward",
+           "twell_fused_updown_noalloc", "twell_to_hybrid", "hybrid_ffn_forward_workspace_size",
+           "hybrid_ffn_forward",
            "hybrid_ffn_backward_workspace_size", "hybrid_ffn_backward", "dense_ffn_forward",
            "tw_status_string", "twell_version"]
 
@@ -74,7 +75,10 @@ def lib():
         L.twell_fused_updown_noalloc.argtypes = [vp, PT, vp, vp, i32, vp, ctypes.c_int, vp, vp]
         L.twell_fused_updown_noalloc.restype = st
         L.twell_to_hybrid.argtypes = [PT, PH, vp, vp]
-        L.hybrid_ffn_forward.argtypes = [vp, PH, vp, vp, i32, vp, ctypes.c_int, vp, vp]
+        L.hybrid_ffn_forward_workspace_size.argtypes = [i32, i32]
+        L.hybrid_ffn_forward_workspace_size.restype = ctypes.c_size_t
+        L.hybrid_ffn_forward.argtypes = [vp, PH, vp, vp, i32, vp, ctypes.c_int, vp,
+                                         ctypes.c_size_t, vp, vp]
         L.hybrid_ffn_backward_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         L.hybrid_ffn_backward_workspace_size.restype = ctypes.c_size_t
         L.hybrid_ffn_backward.argtypes = [vp, vp, PH, vp, vp, vp, i32, ctypes.c_float, vp,
@@ -212,11 +216,20 @@ def twell_to_hybrid(g: Twell, out: Hybrid, dev_status=None, stream=None):
         ctypes.byref(sg), ctypes.byref(sh), _ptr(dev_status), _stream(stream)))
 
 
-def hybrid_ffn_forward(x, gu: Hybrid, Wu_t, Wd, y, dev_status=None, stream=None):
+def hybrid_ffn_forward_workspace_size(T, d):
+    return int(lib().hybrid_ffn_forward_workspace_size(T, d))
+
+
+def hybrid_ffn_forward(x, gu: Hybrid, Wu_t, Wd, y, ws=None, dev_status=None, stream=None):
+    """ws: caller-owned workspace (hybrid_ffn_forward_workspace_size bytes);
+    when None, one is allocated with torch for this call."""
+    if ws is None:
+        ws = torch.empty(hybrid_ffn_forward_workspace_size(x.shape[0], x.shape[1]),
+                         dtype=torch.uint8, device=x.device)
     s = gu.struct()
     _check("hybrid_ffn_forward", lib().hybrid_ffn_forward(
-        _ptr(x), ctypes.byref(s), _ptr(Wu_t), _ptr(Wd), x.shape[1], _ptr(y), _dt(y),
-        _ptr(dev_status), _stream(stream)))
+        _ptr(x), ctypes.byref(s), _ptr(Wu_t), _ptr(Wd), x.shape[1], _ptr(y), _dt(y), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
 
 
 def hybrid_ffn_backward_workspace_size(T, d, F, C_h, backup_cap):

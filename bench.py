@@ -403,6 +403,7 @@ def training_leg(torch, tw):
     dW = [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
     ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, C_h, cap), dtype=torch.uint8,
                      device="cuda")
+    fws = torch.empty(tw.hybrid_ffn_forward_workspace_size(T, d), dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     names = ["gate_twell_gemm", "twell_to_hybrid", "hybrid_ffn_forward", "hybrid_ffn_backward"]
     times = {n: [] for n in names}
@@ -413,7 +414,7 @@ def training_leg(torch, tw):
         e[1].record()
         tw.twell_to_hybrid(g, hy, st)
         e[2].record()
-        tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], y, st)
+        tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], y, fws, st)
         e[3].record()
         tw.hybrid_ffn_backward(dev["x"], dev["dy"], hy, dev["Wg_t"], dev["Wu_t"], dev["Wd"],
                                w["lam"], dx, dW[0], dW[1], dW[2], ws, st)

@@ -32,7 +32,8 @@
  *             dev_status may be NULL.  The caller zeroes it and reads it after
  *             synchronising; tw_status_string names each code.
  * Limits      W == 128; 0 <= C <= 32; F % W == 0; d % 8 == 0; 8 <= d <= 2048
- *             for the fused and hybrid kernels; T >= 1.  F <= 65536 (hybrid
+ *             (bf16 rows) or d <= 1024 (fp32 rows) for the fused and hybrid
+ *             kernels; T >= 1.  F <= 65536 (hybrid
  *             indices are uint16).
  */
 #ifndef TWELL_H
@@ -196,15 +197,21 @@ TW_API tw_status twell_fused_updown_noalloc(const void* x, const tw_twell* g, co
 TW_API tw_status twell_to_hybrid(const tw_twell* g, const tw_hybrid* out, int32_t* dev_status,
                           cudaStream_t stream);
 
+/* Bytes of workspace hybrid_ffn_forward needs for T tokens of width d. */
+TW_API size_t hybrid_ffn_forward_workspace_size(int32_t T, int32_t d);
+
 /*
  * Training forward on the hybrid pattern (sections 2.3-2.4): u = x Wu sampled
  * at the active positions -> gu->ell_u / gu->backup_u (rounded to gu->dtype,
  * +0 off the pattern), then y = (g * u) Wd with fp32 accumulation and the
  * unrounded u.  x, Wu_t, Wd have gu->dtype.  y [T][d] in y_dtype.
+ * ws: device workspace of at least hybrid_ffn_forward_workspace_size bytes
+ * (the same work plan as twell_fused_updown; calls sharing one workspace must
+ * not overlap on the device).
  */
 TW_API tw_status hybrid_ffn_forward(const void* x, const tw_hybrid* gu, const void* Wu_t,
-                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype,
-                             int32_t* dev_status, cudaStream_t stream);
+                             const void* Wd, int32_t d, void* y, tw_dtype y_dtype, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, cudaStream_t stream);
 
 /* Bytes of workspace hybrid_ffn_backward needs for these sizes. */
 TW_API size_t hybrid_ffn_backward_workspace_size(int32_t T, int32_t d, int32_t F, int32_t C_h,

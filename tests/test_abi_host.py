@@ -97,6 +97,11 @@ def test_fused_validation(L):
     assert f(*args(512, yd=7)) == INVALID
     assert f(*args(512, n=ws - 1)) == 8        # TW_ERR_WORKSPACE
     assert f(*args(512, w=None)) == INVALID
+    # fp32 rows: one warp's ring of 1024-column fp32 slices is the shared-memory limit
+    tw32 = _tw(dtype=twell.TW_F32)
+    ws32 = L.twell_fused_updown_workspace_size(256, 2048)
+    assert f(FAKE, ctypes.byref(tw32), FAKE, FAKE, 2048, FAKE, twell.TW_F32, FAKE, ws32,
+             None, None) == UNSUPPORTED
 
 
 def _hy(T=256, F=1024, C_h=64, cap=32, dtype=twell.TW_BF16, base=FAKE):

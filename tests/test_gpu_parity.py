@@ -260,7 +260,7 @@ def run_hybrid(w, backup_cap=None):
     hy = tw.Hybrid(T, F, w["C_h"], dtype=torch.bfloat16, backup_cap=backup_cap)
     tw.twell_to_hybrid(g, hy, st)
     yh = torch.empty((T, d), dtype=torch.float32, device="cuda")
-    tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, st)
+    tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, dev_status=st)
     hy.ell_u_after_forward = hy.ell_u.clone()  # diagnostics: u before the backward runs
     ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, w["C_h"], hy.backup_cap),
                      dtype=torch.uint8, device="cuda")
