@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="ffn_2b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip comparator/training/decode legs")
+    ap.add_argument("--legs", default="dense,decode,training",
+                    help="comma-separated extra legs to run after the timed step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -326,12 +328,16 @@ def run_ours(args, rank, world, local_rank):
 
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_leg(w, y)
-    if rank == 0 and not args.no_extras:
-        line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
+    legs = set() if args.no_extras else {s.strip() for s in args.legs.split(",") if s.strip()}
+    if rank == 0 and legs:
+        if "dense" in legs:
+            line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
         del x, Wg, Wu, Wd, g, y, ws, xh, yh
         torch.cuda.empty_cache()
-        line["decode"] = decode_leg(torch, tw, hbm)
-        line["training"] = training_leg(torch, tw)
+        if "decode" in legs:
+            line["decode"] = decode_leg(torch, tw, hbm)
+        if "training" in legs:
+            line["training"] = training_leg(torch, tw)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
