@@ -31,18 +31,23 @@
 //
 // Teams.  An item is processed by a team of kTeam warps; warp w of the team
 // owns one contiguous range of the d columns (the token's row and the output
-// of that range live in its registers).  Per entry every warp forms its
-// partial dot product, the partials meet in shared memory behind a named
-// barrier and are added in warp order, and every warp updates its own
-// columns.
+// of that range live in its registers).  Entries are taken in pairs: the two
+// warps form their partial dot products, the partials meet in shared memory
+// behind one named barrier per pair and are added in warp order, and every
+// warp updates its own columns.
 //
-// Data movement.  Each warp owns a ring of shared-memory stages; lane 0
-// gathers its column range of the weight rows of upcoming entries with 1-D
-// bulk copies (cp.async.bulk, completion on one mbarrier per stage, no
-// multicast) while the warp computes on earlier stages.  Every lane owns
-// 16-byte column slices: conflict-free shared loads.  bf16 dot products use
-// the mixed-precision FMA (bf16 inputs, fp32 accumulator); the scaled-row
-// updates widen bf16 pairs exactly and use packed fp32x2 FMA.
+// Data movement.  Weight rows are gathered with plain 16-byte vector loads
+// straight into registers (each lane owns 16-byte column slices, so a warp's
+// load of a row slice is fully coalesced).  Two register sets hold the rows
+// of one entry pair; each set is reloaded with the next pair's rows as soon
+// as it has been consumed, so the loads of the next pair overlap the rest of
+// the current one.  (Bulk copies into shared memory were the first design;
+// the copy engine spends a roughly fixed time per copy, which bounded that
+// version by the number of row slices, not by bytes.)
+//
+// Arithmetic.  bf16 dot products run on the tensor pipe (mma.sync with a
+// diagonal-extraction layout, see dot2); the scaled-row updates widen bf16
+// pairs exactly and use packed fp32x2 FMA.
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -56,7 +61,6 @@ constexpr int kMinPart = 8;        // lower bound of the part size
 constexpr int kTeam = 2;           // warps per work item
 constexpr int kTeams = 8;          // teams per CTA
 constexpr int kWarps = kTeam * kTeams;
-constexpr int kRingBytes = 12288;  // shared-memory ring per warp
 constexpr int kListCap = 64;       // entry window collected at a time
 
 enum : int { kModeTwell = 0, kModeHybFwd = 1, kModeHybBwd = 2 };
@@ -170,23 +174,43 @@ TW_DEV int block_exclusive_scan(int v, int* warp_sums, int* total) {
   return excl;
 }
 
+// Largest T whose per-token counts are staged in shared memory by the planner
+// (with one padding word per run of tokens).
+constexpr int kScanSmemTokens = 40960;
+size_t plan_scan_smem(int T) {
+  if (T > kScanSmemTokens) return 0;
+  const int run = (T + kScanThreads - 1) / kScanThreads;
+  return sizeof(int32_t) * ((size_t)T + T / (run > 0 ? run : 1) + 1);
+}
+
 // One CTA: the part size, partial rows of split tokens (in token order,
 // within capacity), then one descriptor per work item.  The part size is
 // kPart, lowered to about two items per team when there are few entries in
 // all (small batches), but not below kMinPart; it is stored in hdr[2].
 // Each thread owns a contiguous run of tokens, so each of the three passes
-// needs a single block-wide scan.
+// needs a single block-wide scan.  The counts are first copied into shared
+// memory with coalesced loads (a padding word after every run keeps the
+// threads' strided reads free of bank conflicts); beyond kScanSmemTokens the
+// passes read them from global memory.
 __global__ void __launch_bounds__(kScanThreads)
     plan_scan_kernel(int T, const int32_t* __restrict__ nnz, int parts_cap, int max_items,
                      int n_teams, int32_t* slot_off, int4* item_desc, int32_t* hdr) {
   __shared__ int warp_sums[32];
   __shared__ int part_sh;
+  extern __shared__ int32_t staged[];
   const int run = (T + kScanThreads - 1) / kScanThreads;
   const int t0 = threadIdx.x * run;
   const int t1 = min(T, t0 + run);
+  const bool in_smem = T <= kScanSmemTokens;
+  if (in_smem) {
+#pragma unroll 8
+    for (int i = threadIdx.x; i < T; i += kScanThreads) staged[i + i / run] = nnz[i];
+    __syncthreads();
+  }
+  auto count = [&](int t) { return in_smem ? staged[t + t / run] : nnz[t]; };
   // pass 0: total number of entries -> part size
   int local = 0;
-  for (int t = t0; t < t1; ++t) local += nnz[t];
+  for (int t = t0; t < t1; ++t) local += count(t);
   int total;
   block_exclusive_scan(local, warp_sums, &total);
   if (threadIdx.x == 0) {
@@ -200,33 +224,38 @@ __global__ void __launch_bounds__(kScanThreads)
   // would pass the capacity (and every later one) stays unsplit
   local = 0;
   for (int t = t0; t < t1; ++t) {
-    const int n = nnz[t];
+    const int n = count(t);
     local += n > part ? (n + part - 1) / part : 0;
   }
   int tot;
-  int ex = block_exclusive_scan(local, warp_sums, &tot);
+  const int ex1 = block_exclusive_scan(local, warp_sums, &tot);
+  // pass 2: one descriptor per work item (the slot decision of pass 1 is
+  // recomputed from the same running offset)
+  local = 0;
+  int ex = ex1;
   for (int t = t0; t < t1; ++t) {
-    const int n = nnz[t];
+    const int n = count(t);
     const int parts = n > part ? (n + part - 1) / part : 0;
-    slot_off[t] = (parts > 0 && ex + parts <= parts_cap) ? ex : -1;
+    const bool split = parts > 0 && ex + parts <= parts_cap;
+    slot_off[t] = split ? ex : -1;
+    local += split ? parts : 1;
     ex += parts;
   }
-  // pass 2: one descriptor per work item
-  local = 0;
-  for (int t = t0; t < t1; ++t)
-    local += slot_off[t] >= 0 ? (nnz[t] + part - 1) / part : 1;
-  ex = block_exclusive_scan(local, warp_sums, &tot);
+  int exd = block_exclusive_scan(local, warp_sums, &tot);
+  ex = ex1;
   for (int t = t0; t < t1; ++t) {
-    const int n = nnz[t], so = slot_off[t];
-    if (so < 0) {
-      if (ex < max_items) item_desc[ex] = make_int4(t, 0, n, -1);
-      ++ex;
+    const int n = count(t);
+    const int parts = n > part ? (n + part - 1) / part : 0;
+    const bool split = parts > 0 && ex + parts <= parts_cap;
+    if (!split) {
+      if (exd < max_items) item_desc[exd] = make_int4(t, 0, n, -1);
+      ++exd;
     } else {
-      const int parts = (n + part - 1) / part;
-      for (int p = 0; p < parts && ex + p < max_items; ++p)
-        item_desc[ex + p] = make_int4(t, p * part, min(n, (p + 1) * part), so + p);
-      ex += parts;
+      for (int q = 0; q < parts && exd + q < max_items; ++q)
+        item_desc[exd + q] = make_int4(t, q * part, min(n, (q + 1) * part), ex + q);
+      exd += parts;
     }
+    ex += parts;
   }
   if (threadIdx.x == 0) hdr[1] = tot < max_items ? tot : max_items;
 }
@@ -286,16 +315,117 @@ struct Elem<float> {
   }
 };
 
-TW_DEV void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+// D (16x8 fp32) += A (16x16 bf16, row-major) . B (16x8 bf16, column-major).
+TW_DEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                           uint32_t b0, uint32_t b1) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes),
-        "r"(smem_u32(bar))
-      : "memory");
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-TW_DEV void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+
+// Sum over the warp of p0 (result in lane 0) and of p1 (result in lane 16)
+// with five shuffle steps.
+TW_DEV void warp_sum2(float p0, float p1, int lane, float& s0, float& s1) {
+  const bool hi = (lane & 16) != 0;
+  float v = hi ? p1 : p0;
+  v += __shfl_xor_sync(FULL, hi ? p0 : p1, 16);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+  s0 = __shfl_sync(FULL, v, 0);
+  s1 = __shfl_sync(FULL, v, 16);
 }
+
+// This warp's partial dot products of the token row (xr) with the rows of
+// two entries (w[0], w[1]), all held in registers as this lane's 16-byte
+// slices of the warp's column range; a missing second entry is all zeros.
+// dot2_issue leaves per-lane partial sums in D; dot2_reduce turns them into
+// the two warp sums, so independent work can be placed between the two.
+//
+// bf16: on the tensor pipe.  One m16n8k16 MMA takes, from lane (g, q) =
+// (lane / 4, lane % 4), four consecutive columns of its slice: A row g holds
+// them for the first entry, A row g + 8 for the second, B column g holds the
+// token's values at the same columns.  The diagonal D[g][g] (D[g + 8][g]) is
+// then the dot product of the first (second) row with the token over the 16
+// columns of lanes 4g..4g+3; the other products are not used.  D[g][g] sits
+// in lane 4g + g/2, register g & 1 (+2 for the second entry).  Products of
+// bf16 are exact and the MMA accumulates in fp32; two accumulators halve the
+// chain of dependent MMAs.
+template <typename Tin, int NCHW>
+TW_DEV void dot2_issue(const uint4 (&xr)[NCHW], const uint4 (&w)[2][NCHW], float (&D)[2][4]) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) D[k][i] = 0.f;
+  if constexpr (sizeof(Tin) == 2) {
+#pragma unroll
+    for (int c = 0; c < NCHW; ++c) {
+      mma_bf16_16816(D[0], w[0][c].x, w[1][c].x, w[0][c].y, w[1][c].y, xr[c].x, xr[c].y);
+      mma_bf16_16816(D[1], w[0][c].z, w[1][c].z, w[0][c].w, w[1][c].w, xr[c].z,
+                     xr[c].w);
+    }
+  } else {
+    // fp32: D[0] and D[1] hold four running sums per entry
+#pragma unroll
+    for (int c = 0; c < NCHW; ++c) {
+      Elem<Tin>::dot(xr[c], w[0][c], D[0]);
+      Elem<Tin>::dot(xr[c], w[1][c], D[1]);
+    }
+  }
+}
+
+template <typename Tin>
+TW_DEV void dot2_reduce(const float (&D)[2][4], int lane, float& v0, float& v1) {
+  float p0, p1;
+  if constexpr (sizeof(Tin) == 2) {
+    float d[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = D[0][i] + D[1][i];
+    const int g = lane >> 2;
+    const bool diag = (lane & 3) == (g >> 1);
+    p0 = diag ? ((g & 1) ? d[1] : d[0]) : 0.f;
+    p1 = diag ? ((g & 1) ? d[3] : d[2]) : 0.f;
+  } else {
+    p0 = (D[0][0] + D[0][1]) + (D[0][2] + D[0][3]);
+    p1 = (D[1][0] + D[1][1]) + (D[1][2] + D[1][3]);
+  }
+  warp_sum2(p0, p1, lane, v0, v1);
+}
+
+// Rows j0 and (when `two`) j1 of a row-major [F][d] weight, this lane's
+// slices of columns [c0, c0 + my_cols), into registers (zeros elsewhere).
+// Read-only 16-byte load that asks L2 to keep the line (weight rows are
+// gathered again by other tokens; activations and outputs stream past them).
+TW_DEV uint4 ldg_keep(const uint4* p, uint64_t policy) {
+  uint4 r;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p), "l"(policy));
+  return r;
+}
+TW_DEV uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+template <typename Tin, int NCHW>
+TW_DEV void load_rows2(uint4 (&w)[2][NCHW], const Tin* base, int j0, int j1, bool two, int d,
+                       int c0, int my_cols, int lane, uint64_t pol) {
+  constexpr int E = Elem<Tin>::E;
+  constexpr int SPAN = 32 * E;
+  const uint4* p0 = reinterpret_cast<const uint4*>(base + (size_t)j0 * d + c0);
+  const uint4* p1 = reinterpret_cast<const uint4*>(base + (size_t)j1 * d + c0);
+#pragma unroll
+  for (int c = 0; c < NCHW; ++c) {
+    const int lc = c * SPAN + lane * E;
+    const bool in = lc < my_cols;
+    w[0][c] = in ? ldg_keep(p0 + lc / E, pol) : make_uint4(0, 0, 0, 0);
+    w[1][c] = in && two ? ldg_keep(p1 + lc / E, pol) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 // Named barrier over the kTeam warps of one team (ids 1..kTeams; 0 is
 // __syncthreads).  Every warp of a team executes the same sequence of these.
 TW_DEV void team_bar(int team) {
@@ -337,9 +467,6 @@ struct GatherArgs {
   void* out;
   int32_t* status;
   FusedWs ws;
-  int stages;       // ring depth per warp
-  int slice_bytes;  // bytes of one row's column range of one warp (max over warps)
-  unsigned long long timeout_ns;
 };
 
 // Shared state of one team.
@@ -348,8 +475,7 @@ struct TeamSmem {
   int32_t j[kListCap];
   int32_t pos[kListCap];  // hybrid position of the entry (u is saved / read there)
   float u[kListCap];      // saved u of the entry (backward)
-  float red[2][kTeam];    // partial dot products, double-buffered by entry parity
-  int ok[2][kTeam];       // wait results, same buffering
+  float red[2][kTeam][2];  // partial dot products of an entry pair, double-buffered
   int4 desc[2];           // current item, double-buffered by item parity
   int n;                  // entries in the current window
   int prev;               // split-token finisher broadcast
@@ -460,56 +586,32 @@ TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, TeamS
 }
 
 // NCHW: 16-byte column slices per lane for one warp of a team.
+// Teams per CTA: fewer for the widest rows, whose register sets of row slices
+// need more than 128 registers per thread (three sets in the backward).
+template <int NCHW, int MODE>
+constexpr int teams_for() { return NCHW < 4 ? kTeams : (MODE == kModeHybBwd ? 4 : 6); }
+
 template <typename Tin, int NCHW, bool kOutBf16, int MODE>
-__global__ void __launch_bounds__(32 * kWarps, 1) gather_kernel(const GatherArgs<Tin> a) {
+__global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
+    gather_kernel(const GatherArgs<Tin> a) {
   using L = Elem<Tin>;
   constexpr int E = L::E;
   constexpr int P = L::P;
-  constexpr int SPAN = 32 * E;             // columns of one warp-wide slice
-  constexpr int COLS = NCHW * SPAN;        // columns owned by one warp
-  constexpr int NROWS = MODE == kModeHybBwd ? 3 : 2;  // weight rows per entry
-  extern __shared__ __align__(128) uint8_t smem_raw[];
+  constexpr int SPAN = 32 * E;       // columns of one warp-wide slice
+  constexpr int COLS = NCHW * SPAN;  // columns owned by one warp
+  constexpr bool kBwd = MODE == kModeHybBwd;
+  __shared__ TeamSmem team_smem[teams_for<NCHW, MODE>()];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int team = wid / kTeam;
-  const int tw = wid % kTeam;              // this warp's place in its team
+  const int tw = wid % kTeam;  // this warp's place in its team
   const int d = a.d;
-  const int c0 = tw * COLS;                // first column of this warp
+  const int c0 = tw * COLS;    // first column of this warp
   const int my_cols = d - c0 < COLS ? (d - c0 > 0 ? d - c0 : 0) : COLS;
-  const uint32_t my_bytes = (uint32_t)my_cols * sizeof(Tin);
-  const size_t stage_bytes = (size_t)NROWS * a.slice_bytes;
-
-  // shared memory: [kTeams] TeamSmem, then per warp: barriers + ring
-  TeamSmem& ts = reinterpret_cast<TeamSmem*>(smem_raw)[team];
-  const size_t team_bytes = (sizeof(TeamSmem) * kTeams + 127) & ~size_t(127);
-  const size_t per_warp = 128 + (size_t)a.stages * stage_bytes;
-  uint8_t* mine = smem_raw + team_bytes + (size_t)wid * per_warp;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(mine);
-  uint8_t* ring = mine + 128;
-  if (lane == 0) {
-    for (int i = 0; i < a.stages; ++i) mbar_init(&bar[i], 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-
-  int never = 0;
-  // Ring position of this warp, advanced incrementally (no division):
-  // cst/cph next stage to wait on and its phase parity, pst next stage to
-  // fill, inflight stages filled but not yet waited on.
-  uint32_t cst = 0, cph = 0, pst = 0, inflight = 0;
-  bool failed = false;
+  TeamSmem& ts = team_smem[team];
   const int n_items = a.ws.hdr[1];
   const bool leader = tw == 0;
-
-  auto issue = [&](int j) {
-    uint8_t* dst = ring + (size_t)pst * stage_bytes;
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&bar[pst], NROWS * my_bytes);
-    bulk_g2s(dst, a.rdot + (size_t)j * d + c0, my_bytes, &bar[pst]);
-    bulk_g2s(dst + a.slice_bytes, a.rax1 + (size_t)j * d + c0, my_bytes, &bar[pst]);
-    if (MODE == kModeHybBwd)
-      bulk_g2s(dst + 2 * a.slice_bytes, a.rax2 + (size_t)j * d + c0, my_bytes, &bar[pst]);
-  };
+  const uint64_t pol = policy_evict_last();
 
   int ticket = 0;
   if (leader && lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);
@@ -534,12 +636,12 @@ __global__ void __launch_bounds__(32 * kWarps, 1) gather_kernel(const GatherArgs
 #pragma unroll
     for (int c = 0; c < NCHW; ++c) {
       const int col = c0 + c * SPAN + lane * E;
-      xr[c] = col < d ? __ldg(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
+      xr[c] = col < d ? __ldcs(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
     }
 
-    for (int w0 = lo; w0 < hi && !failed; w0 += kListCap) {
+    for (int w0 = lo; w0 < hi; w0 += kListCap) {
       if (leader) {
         const int w1 = min(hi, w0 + kListCap);
         const int n = MODE == kModeTwell ? collect_twell(a, t, w0, w1, ts, lane)
@@ -548,104 +650,100 @@ __global__ void __launch_bounds__(32 * kWarps, 1) gather_kernel(const GatherArgs
       }
       team_bar(team);
       const int n = ts.n;
-      const int pre = n < a.stages ? n : a.stages;
-      for (int e = 0; e < pre; ++e) {
-        if (lane == 0 && my_bytes) issue(ts.j[e]);
-        pst = pst + 1 == (uint32_t)a.stages ? 0u : pst + 1;
-        ++inflight;
-      }
-      for (int e = 0; e < n; ++e) {
-        const uint32_t st = cst;
-        bool ok = true;
-        if (my_bytes) ok = mbar_wait(&bar[st], cph, &never, a.timeout_ns);
-        ok = __all_sync(FULL, ok);
-        const uint8_t* stage = ring + (size_t)st * stage_bytes;
-        const uint4* rd = reinterpret_cast<const uint4*>(stage);
-        const uint4* r1 = reinterpret_cast<const uint4*>(stage + a.slice_bytes);
-        const uint4* r2 = reinterpret_cast<const uint4*>(stage + 2 * a.slice_bytes);
-        float pa[4] = {0.f, 0.f, 0.f, 0.f};
-        float pb[4] = {0.f, 0.f, 0.f, 0.f};
-        if (ok) {
-#pragma unroll
-          for (int c = 0; c < NCHW; ++c) {
-            const int lc = c * SPAN + lane * E;  // column within this warp's range
-            if (lc < my_cols) {
-              if (c & 1) L::dot(xr[c], rd[lc / E], pb);
-              else L::dot(xr[c], rd[lc / E], pa);
-            }
-          }
-        }
-        const float part = warp_sum(((pa[0] + pb[0]) + (pa[1] + pb[1])) +
-                                    ((pa[2] + pb[2]) + (pa[3] + pb[3])));
-        const int rb = e & 1;  // exchange buffer of this entry
+      const int npairs = (n + 1) / 2;
+      auto jof = [&](int e) { return e < n ? ts.j[e] : 0; };
+      // Register sets of row slices of one entry pair: A rows of the
+      // dot-product weight, B (and C, backward) rows of the update weights.
+      uint4 A[2][NCHW], B[2][NCHW], C[2][NCHW];
+      // The team's dot products of a pair: partial sums meet in shared
+      // memory behind one barrier; the scalars of the pair follow.
+      auto exchange = [&](int pp, float v0, float v1, float& s1a, float& s2a, float& s1b,
+                          float& s2b) {
+        const int rb = pp & 1;
         if (lane == 0) {
-          ts.red[rb][tw] = part;
-          ts.ok[rb][tw] = ok ? 1 : 0;
+          ts.red[rb][tw][0] = v0;
+          ts.red[rb][tw][1] = v1;
         }
-        team_bar(team);  // unconditional: every warp of the team reaches it
-        float dotv = 0.f;
-        bool all_ok = true;
+        team_bar(team);
+        float dv[2] = {0.f, 0.f};
 #pragma unroll
         for (int q = 0; q < kTeam; ++q) {
-          dotv += ts.red[rb][q];
-          all_ok = all_ok && ts.ok[rb][q] != 0;
+          dv[0] += ts.red[rb][q][0];
+          dv[1] += ts.red[rb][q][1];
         }
-        if (!all_ok) {  // the same decision in every warp of the team
-          failed = true;
-          break;
-        }
-        --inflight;
-        if (++cst == (uint32_t)a.stages) {
-          cst = 0;
-          cph ^= 1u;
-        }
-        const float gv = ts.g[e];
-        float s1, s2 = 0.f;
-        if (MODE == kModeHybBwd) {
-          const float uv = ts.u[e];
-          s1 = dotv * gv;                    // du
-          s2 = fmaf(dotv, uv, a.lam);        // dz
-          if (leader && lane == 0) {
-            Payload p;
-            p.t = t;
-            p.h = gv * uv;
-            p.du = s1;
-            p.dz = s2;
-            a.pay[a.e0[t] + w0 + e] = p;
+        float s1[2] = {0.f, 0.f}, s2[2] = {0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int ee = 2 * pp + k;
+          if (ee >= n) break;
+          const float gv = ts.g[ee];
+          if (kBwd) {
+            const float uv = ts.u[ee];
+            s1[k] = dv[k] * gv;              // du
+            s2[k] = fmaf(dv[k], uv, a.lam);  // dz
+            if (leader && lane == 0) {
+              Payload pl;
+              pl.t = t;
+              pl.h = gv * uv;
+              pl.du = s1[k];
+              pl.dz = s2[k];
+              a.pay[a.e0[t] + w0 + ee] = pl;
+            }
+          } else {
+            s1[k] = gv * dv[k];  // h
+            if (MODE == kModeHybFwd && leader && lane == 0)
+              L::store((to_backup ? a.backup_u : a.ell_u) + ts.pos[ee], dv[k]);
           }
-        } else {
-          s1 = gv * dotv;                    // h
-          if (MODE == kModeHybFwd && leader && lane == 0)
-            L::store((to_backup ? a.backup_u : a.ell_u) + ts.pos[e], dotv);
         }
-        const float2 h1 = make_float2(s1, s1);
-        const float2 h2 = make_float2(s2, s2);
+        s1a = s1[0];
+        s1b = s1[1];
+        s2a = s2[0];
+        s2b = s2[1];
+      };
+      // rows of a missing second entry are zeros, so both rows always update
+      auto update = [&](const uint4 (&R)[2][NCHW], float sa, float sb) {
+        const float2 ha = make_float2(sa, sa), hb = make_float2(sb, sb);
 #pragma unroll
         for (int c = 0; c < NCHW; ++c) {
-          const int lc = c * SPAN + lane * E;
-          if (lc < my_cols) {
-            float2 w[P];
-            L::pairs(r1[lc / E], w);
+          float2 w[P];
+          L::pairs(R[0][c], w);
 #pragma unroll
-            for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(h1, w[q], acc[c][q]);
-            if (MODE == kModeHybBwd) {
-              L::pairs(r2[lc / E], w);
+          for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(ha, w[q], acc[c][q]);
+          L::pairs(R[1][c], w);
 #pragma unroll
-              for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(h2, w[q], acc[c][q]);
-            }
-          }
+          for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(hb, w[q], acc[c][q]);
         }
-        __syncwarp();  // every lane is done with this stage
-        const int nxt = e + a.stages;
-        if (nxt < n) {  // refill the stage just freed (the ring was full)
-          if (lane == 0 && my_bytes) issue(ts.j[nxt]);
-          pst = pst + 1 == (uint32_t)a.stages ? 0u : pst + 1;
-          ++inflight;
+      };
+      auto load = [&](uint4 (&R)[2][NCHW], const Tin* base, int pp) {
+        load_rows2<Tin, NCHW>(R, base, jof(2 * pp), jof(2 * pp + 1), 2 * pp + 1 < n, d, c0,
+                              my_cols, lane, pol);
+      };
+      // Each register set is reloaded with the next pair's rows as soon as it
+      // has been consumed, so those loads overlap the rest of the pair.
+      if (npairs > 0) {
+        load(A, a.rdot, 0);
+        load(B, a.rax1, 0);
+      }
+      for (int pp = 0; pp < npairs; ++pp) {
+        const bool next = pp + 1 < npairs;
+        float D[2][4];
+        dot2_issue<Tin, NCHW>(xr, A, D);
+        if (kBwd)  // A now takes the rows of the second update weight
+          load(C, a.rax2, pp);
+        else if (next)
+          load(A, a.rdot, pp + 1);
+        float v0, v1, s1a, s2a, s1b, s2b;
+        dot2_reduce<Tin>(D, lane, v0, v1);
+        exchange(pp, v0, v1, s1a, s2a, s1b, s2b);
+        update(B, s1a, s1b);
+        if (next) load(B, a.rax1, pp + 1);
+        if (kBwd) {
+          if (next) load(A, a.rdot, pp + 1);
+          update(C, s2a, s2b);
         }
       }
       team_bar(team);  // the list may be overwritten by the next window
     }
-    if (failed) break;
 
     // ------------------------------------------------------------ output --
     const bool split = prow >= 0;
@@ -657,9 +755,14 @@ __global__ void __launch_bounds__(32 * kWarps, 1) gather_kernel(const GatherArgs
       if (split || !kOutBf16) {
         float* dst = split ? out_row + col : static_cast<float*>(a.out) + (size_t)t * d + col;
 #pragma unroll
-        for (int q = 0; q < P / 2; ++q)
-          reinterpret_cast<float4*>(dst)[q] = make_float4(acc[c][2 * q].x, acc[c][2 * q].y,
-                                                          acc[c][2 * q + 1].x, acc[c][2 * q + 1].y);
+        for (int q = 0; q < P / 2; ++q) {
+          const float4 v = make_float4(acc[c][2 * q].x, acc[c][2 * q].y, acc[c][2 * q + 1].x,
+                                       acc[c][2 * q + 1].y);
+          if (split)
+            reinterpret_cast<float4*>(dst)[q] = v;
+          else
+            __stcs(reinterpret_cast<float4*>(dst) + q, v);
+        }
       } else {
         uint16_t* yt = static_cast<uint16_t*>(a.out) + (size_t)t * d + col;
 #pragma unroll
@@ -695,39 +798,17 @@ __global__ void __launch_bounds__(32 * kWarps, 1) gather_kernel(const GatherArgs
       }
     }
   }
-
-  if (failed) {
-    if (lane == 0) set_status(a.status, kStatusTimeout);
-    // let the copies still in flight land before the CTA may exit
-    for (uint32_t q = 0; q < inflight; ++q) {
-      if (my_bytes) mbar_wait(&bar[cst], cph, &never, a.timeout_ns);
-      if (++cst == (uint32_t)a.stages) {
-        cst = 0;
-        cph ^= 1u;
-      }
-    }
-  }
 }
 
 template <typename Tin, int NCHW, int MODE>
 cudaError_t launch_nchw(GatherArgs<Tin> a, bool out_bf16, cudaStream_t stream) {
-  constexpr int SPAN = 32 * Elem<Tin>::E;
-  constexpr int NROWS = MODE == kModeHybBwd ? 3 : 2;
-  a.slice_bytes = NCHW * SPAN * (int)sizeof(Tin);
-  a.stages = kRingBytes / (NROWS * a.slice_bytes);
-  if (a.stages > 8) a.stages = 8;
-  if (a.stages < 2) a.stages = 2;
-  const size_t team_bytes = (sizeof(TeamSmem) * kTeams + 127) & ~size_t(127);
-  const size_t per_warp = 128 + (size_t)a.stages * NROWS * a.slice_bytes;
-  const size_t smem = team_bytes + per_warp * kWarps;
   auto kern = out_bf16 ? gather_kernel<Tin, NCHW, true, MODE> : gather_kernel<Tin, NCHW, false, MODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  constexpr int threads = 32 * kTeam * teams_for<NCHW, MODE>();
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * kWarps, smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  kern<<<num_sms() * per_sm, 32 * kWarps, smem, stream>>>(a);
+  kern<<<num_sms() * per_sm, threads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -740,7 +821,6 @@ cudaError_t launch_mode(const GatherArgs<Tin>& a, bool out_bf16, cudaStream_t st
   if (per <= 1) return launch_nchw<Tin, 1, MODE>(a, out_bf16, stream);
   if (per <= 2) return launch_nchw<Tin, 2, MODE>(a, out_bf16, stream);
   if (per <= 4) return launch_nchw<Tin, 4, MODE>(a, out_bf16, stream);
-  if constexpr (sizeof(Tin) == 4) return launch_nchw<Tin, 8, MODE>(a, out_bf16, stream);
   return cudaErrorInvalidValue;  // d beyond the validated maximum
 }
 
@@ -752,7 +832,13 @@ cudaError_t run_engine(GatherArgs<Tin> a, bool out_bf16, void* base, CountFn cou
   cudaError_t e = cudaMemsetAsync(base, 0, a.ws.zero_bytes, stream);
   if (e != cudaSuccess) return e;
   count();
-  plan_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.T, a.ws.nnz, a.ws.parts_cap,
+  const size_t scan_smem = plan_scan_smem(a.T);
+  if (scan_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(plan_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)plan_scan_smem(kScanSmemTokens));
+    if (e != cudaSuccess) return e;
+  }
+  plan_scan_kernel<<<1, kScanThreads, scan_smem, stream>>>(a.T, a.ws.nnz, a.ws.parts_cap,
                                                    a.ws.max_items, num_sms() * kTeams,
                                                    a.ws.slot_off, a.ws.item_desc, a.ws.hdr);
   return launch_mode<Tin, MODE>(a, out_bf16, stream);
@@ -779,7 +865,6 @@ cudaError_t twell_fused_t(const void* x, const tw_twell& g, const void* Wu_t, co
   a.out = y;
   a.status = status;
   a.ws = w;
-  a.timeout_ns = kWaitTimeoutNs;
   const int T = g.T, K = g.F / W;
   return run_engine<Tin, kModeTwell>(
       a, y_dtype == TW_BF16, base,
@@ -823,7 +908,6 @@ cudaError_t hybrid_t(const void* xin, const tw_hybrid& h, const void* rdot, cons
   a.out = out;
   a.status = status;
   a.ws = w;
-  a.timeout_ns = kWaitTimeoutNs;
   const int T = h.T;
   return run_engine<Tin, MODE>(
       a, out_dtype == TW_BF16, base,

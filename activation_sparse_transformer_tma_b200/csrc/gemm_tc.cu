@@ -18,10 +18,7 @@
 // accumulator).  Every wait is bounded: on timeout the CTA raises an abort
 // flag, flags TW_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees its
 // TMEM and returns.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
+#include "tmap.h"
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -395,31 +392,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ----------------------------------------------------------------- host ----
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // Row-major bf16 matrix [rows][cols]; boxes of 64 columns x box_rows rows.
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tmap_bf16(m, base, rows, cols, BK, box_rows);
 }
 
 template <class Epi>

@@ -87,12 +87,15 @@ def test_bf16_gate_and_fused_small(T, d, F, C, kind, ma):
     check_y(f64(y), w64, rows, TOL[synth.BF16])
 
 
-def test_bf16_output_y():
-    w = synth.make_workload(T=300, d=320, F=640, W=128, C=8, dtype=synth.BF16, kind="dead20",
+@pytest.mark.parametrize("d", [320, 256])  # CUDA-core gather engine / tensor-core path
+def test_bf16_output_y(d):
+    w = synth.make_workload(T=300, d=d, F=640, W=128, C=8, dtype=synth.BF16, kind="dead20",
                             mean_active=29.0, seed=620)
     _, g, gd, y, st = run_forward(w, y_dtype=torch.bfloat16)
     _, _, _, y32, _ = run_forward(w)
-    # the bf16 output is the fp32 result rounded once
+    _, _, _, y32b, _ = run_forward(w)
+    # both paths are deterministic, and the bf16 output is the fp32 result rounded once
+    assert torch.equal(y32, y32b)
     assert torch.equal(y, y32.to(torch.bfloat16))
     check_y(f64(y), widened(w), np.arange(300, dtype=np.int32), TOL[synth.BF16],
             elem_rel=2.0 ** -8)
