@@ -62,7 +62,8 @@ tw_status check_hybrid(const tw_hybrid* h) {
   if (h->T < 0 || h->F <= 0 || h->C_h < 0 || h->C_h > h->F || h->backup_cap < 0 ||
       !dtype_ok(h->dtype))
     return TW_ERR_INVALID_ARG;
-  if (h->F > 51200) return TW_ERR_UNSUPPORTED;  // unit histograms live in shared memory
+  // unit histograms live in shared memory; dense rows are read 16 bytes at a time
+  if (h->F > 51200 || h->F % 8 != 0) return TW_ERR_UNSUPPORTED;
   if ((size_t)h->T * (size_t)h->C_h + (size_t)h->backup_cap * (size_t)h->F > 0x7FFFFFFFull)
     return TW_ERR_UNSUPPORTED;  // entry numbers are int32
   if (!h->row_nnz || !h->row_slot || !h->n_backup) return TW_ERR_INVALID_ARG;

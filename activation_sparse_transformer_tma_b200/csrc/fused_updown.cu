@@ -566,20 +566,53 @@ TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, TeamS
       }
     }
   } else {
+    // dense row: 16-byte loads (V values per lane), ranks from a warp scan
+    constexpr int V = 16 / (int)sizeof(Tin);
+    const Tin* row = a.backup_g + (size_t)slot * a.F;
     int base = 0;
-    for (int c0 = 0; c0 < a.F && base < hi; c0 += 32) {
-      const int c = c0 + lane;
-      const size_t pos = (size_t)slot * a.F + c;
-      const float v = c < a.F ? Elem<Tin>::scalar(a.backup_g[pos]) : 0.f;
-      const unsigned m = __ballot_sync(FULL, v != 0.f);
-      const int r = base + __popc(m & lanemask_lt());
-      if (v != 0.f && r >= lo && r < hi) {
-        s.g[r - lo] = v;
-        s.j[r - lo] = c;
-        s.pos[r - lo] = (int)pos;
-        if (MODE == kModeHybBwd) s.u[r - lo] = Elem<Tin>::scalar(a.backup_u[pos]);
+    for (int c0 = 0; c0 < a.F && base < hi; c0 += 32 * V) {
+      const int cl = c0 + lane * V;
+      const uint4 raw =
+          cl < a.F ? *reinterpret_cast<const uint4*>(row + cl) : make_uint4(0, 0, 0, 0);
+      float v[V];
+      if constexpr (sizeof(Tin) == 2) {
+        float2 pr[4];
+        Elem<uint16_t>::pairs(raw, pr);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[2 * i] = pr[i].x;
+          v[2 * i + 1] = pr[i].y;
+        }
+      } else {
+        v[0] = __uint_as_float(raw.x);
+        v[1] = __uint_as_float(raw.y);
+        v[2] = __uint_as_float(raw.z);
+        v[3] = __uint_as_float(raw.w);
       }
-      base += __popc(m);
+      unsigned mask = 0;
+#pragma unroll
+      for (int i = 0; i < V; ++i) mask |= (v[i] != 0.f ? 1u : 0u) << i;
+      const int nz = __popc(mask);
+      int incl = nz;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += u;
+      }
+      unsigned m = mask;
+      while (m) {
+        const int i = __ffs(m) - 1;
+        m &= m - 1;
+        const int r = base + incl - nz + __popc(mask & ((1u << i) - 1u));
+        if (r >= lo && r < hi) {
+          const size_t pos = (size_t)slot * a.F + cl + i;
+          s.g[r - lo] = v[i];
+          s.j[r - lo] = cl + i;
+          s.pos[r - lo] = (int)pos;
+          if (MODE == kModeHybBwd) s.u[r - lo] = Elem<Tin>::scalar(a.backup_u[pos]);
+        }
+      }
+      base += __shfl_sync(FULL, incl, 31);
     }
   }
   return hi - lo;

@@ -25,6 +25,24 @@ TW_DEV float ld_scalar<uint16_t>(const uint16_t* p, size_t i) { return bf16_to_f
 template <>
 TW_DEV float ld_scalar<float>(const float* p, size_t i) { return p[i]; }
 
+// The V = 16 / sizeof(T) values of row[cl .. cl + V) widened exactly to
+// fp32 (zeros past n).  row + cl must be 16-byte aligned (n % V == 0).
+template <typename T>
+TW_DEV void load_vec(const T* row, int cl, int n, float (&v)[16 / sizeof(T)]) {
+  const uint4 r = cl < n ? *reinterpret_cast<const uint4*>(row + cl) : make_uint4(0, 0, 0, 0);
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(w[i]);
+  }
+}
+
 template <typename T>
 TW_DEV void st_scalar(T* p, size_t i, float v);
 template <>
@@ -92,16 +110,35 @@ TW_DEV void for_each_chunk(const HView<T>& h, int t, int lane, Fn&& fn) {
       fn(v, j, g, pos, true, s);
     }
   } else if (slot < h.backup_cap) {
+    // dense row: 16-byte loads (V values per lane), ranks from a warp scan of
+    // the per-lane non-zero counts; fn is called for the non-zeros only
+    constexpr int V = 16 / (int)sizeof(T);
+    const T* row = h.backup_g + (size_t)slot * h.F;
     int base = 0;
-    for (int c0 = 0; c0 < h.F; c0 += 32) {
-      const int j = c0 + lane;
-      const size_t pos = (size_t)slot * h.F + (j < h.F ? j : 0);
-      const float g = j < h.F ? ld_scalar<T>(h.backup_g, pos) : 0.f;
-      const bool v = g != 0.f;
-      const unsigned m = __ballot_sync(FULL, v);
-      if (m == 0u) continue;
-      fn(v, j, g, pos, false, base + __popc(m & lanemask_lt()));
-      base += __popc(m);
+#pragma unroll 2
+    for (int c0 = 0; c0 < h.F; c0 += 32 * V) {
+      const int cl = c0 + lane * V;
+      float v[V];
+      load_vec<T>(row, cl, h.F, v);
+      unsigned mask = 0;
+#pragma unroll
+      for (int i = 0; i < V; ++i) mask |= (v[i] != 0.f ? 1u : 0u) << i;
+      const int nz = __popc(mask);
+      int incl = nz;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += u;
+      }
+      const int total = __shfl_sync(FULL, incl, 31);
+      unsigned m = mask;
+      while (m) {
+        const int i = __ffs(m) - 1;
+        m &= m - 1;
+        fn(true, cl + i, v[i], (size_t)slot * h.F + cl + i, false,
+           base + incl - nz + __popc(mask & ((1u << i) - 1u)));
+      }
+      base += total;
     }
   }
 }
@@ -273,22 +310,30 @@ __global__ void __launch_bounds__(256)
   if (slot >= nb) return;
   const int t = backup_rows[slot];
   T* row = backup_g + (size_t)slot * F;
-  for (int j = lane; j < F; j += 32) row[j] = T(0);
+  uint4* row4 = reinterpret_cast<uint4*>(row);
+  for (int i = lane; i < F * (int)sizeof(T) / 16; i += 32) row4[i] = make_uint4(0, 0, 0, 0);
   __syncwarp();
+  // lane k handles tile k (its slots); spilled tiles are copied by the warp
   const int K = F / W;
-  for (int k = 0; k < K; ++k) {
+  for (int kb = 0; kb < K; kb += 32) {
+    const int k = kb + lane;
     const size_t kt = (size_t)k * Tn + t;
-    const int n = cnt[kt];
-    if (n == 0) continue;
-    if (n <= C) {
-      if (lane < n) row[k * W + idx[kt * C + lane]] = val[kt * C + lane];
-    } else {
-      const int ref = spill_ref[kt];
-      if (ref >= 0 && ref < spill_cap) {
-        for (int c = lane; c < W; c += 32) row[k * W + c] = spill_val[(size_t)ref * W + c];
-      } else if (lane < C) {
-        row[k * W + idx[kt * C + lane]] = val[kt * C + lane];
-      }
+    const int n = k < K ? cnt[kt] : 0;
+    int ref = -1;
+    if (n > C) {
+      ref = spill_ref[kt];
+      if (ref >= spill_cap) ref = -1;
+    }
+    if (n > 0 && ref < 0) {
+      const int m = n < C ? n : C;
+      for (int s2 = 0; s2 < m; ++s2) row[k * W + idx[kt * C + s2]] = val[kt * C + s2];
+    }
+    unsigned sp = __ballot_sync(FULL, ref >= 0);
+    while (sp) {
+      const int src = __ffs(sp) - 1;
+      sp &= sp - 1;
+      const int rb = __shfl_sync(FULL, ref, src);
+      for (int c = lane; c < W; c += 32) row[(kb + src) * W + c] = spill_val[(size_t)rb * W + c];
     }
   }
 }
@@ -299,60 +344,114 @@ __global__ void __launch_bounds__(256)
 // (fused_updown.cu), which splits heavy rows and streams the weight rows
 // through shared memory.  The weight gradients below use its records.
 
-constexpr int TB = 32;  // tokens per block of the transposition
+// The records of the backward are in token-major order (entry e0[t] + rank).
+// The weight gradients sum them per unit in ascending token order, so they
+// are transposed to a unit-major list with a stable counting sort:
+//   1. hyb_count_kernel   entries per (block of TB tokens, unit), written
+//                         unit-major: cnt[j][b];
+//   2. hyb_colscan_kernel one warp per unit: exclusive prefix over blocks
+//                         (in place) and the unit's total;
+//   3. scan_kernel        exclusive prefix of the totals -> unit_off;
+//   4. hyb_fill_kernel    each block walks its tokens again and writes every
+//                         entry's record index at its place.
+// A block is TB_WARPS warps, each owning TB_TOK consecutive tokens with a
+// private uint8 histogram of the F units in shared memory; within a block the
+// warps' histograms become exclusive offsets, so the warps place their
+// entries in parallel and the token order inside each unit is kept.
+constexpr int TB_WARPS = 4;
+constexpr int TB_TOK = 16;               // tokens per warp
+constexpr int TB = TB_WARPS * TB_TOK;    // tokens per block
+static_assert((TB_WARPS - 1) * TB_TOK < 256, "per-warp offsets must fit in uint8");
 
-// Per (token block, unit) entry counts: cntb[b][j].
+// Shared memory of the count and fill kernels: TB_WARPS x F uint8.
+inline size_t tb_hist_bytes(int F) { return (size_t)TB_WARPS * F; }
+
+// Per-warp histogram of the units of the warp's tokens (zeroed first).
 template <typename T>
-__global__ void __launch_bounds__(256)
-    hyb_count_kernel(const HView<T> h, int32_t* cntb) {
-  extern __shared__ int32_t hist[];
-  const int b = blockIdx.x;
-  for (int j = threadIdx.x; j < h.F; j += blockDim.x) hist[j] = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  for (int tt = wid; tt < TB; tt += blockDim.x / 32) {
-    const int t = b * TB + tt;
+TW_DEV void warp_unit_hist(const HView<T>& h, uint8_t* hist, int b, int warp, int lane) {
+  for (int j = lane; j < h.F; j += 32) hist[j] = 0;
+  __syncwarp();
+  for (int k = 0; k < TB_TOK; ++k) {
+    const int t = b * TB + warp * TB_TOK + k;
     if (t >= h.T) break;
+    // the units of one row are distinct, so these increments never collide
     for_each_chunk<T>(h, t, lane, [&](bool v, int j, float, size_t, bool, int) {
-      if (v) atomicAdd(&hist[j], 1);
+      if (v) hist[j] = (uint8_t)(hist[j] + 1);
     });
+    __syncwarp();
   }
-  __syncthreads();
-  for (int j = threadIdx.x; j < h.F; j += blockDim.x) cntb[(size_t)b * h.F + j] = hist[j];
 }
 
-// Column-wise exclusive prefix over token blocks; totals per unit.
-__global__ void hyb_colscan_kernel(int nblocks, int F, int32_t* cntb, int32_t* unit_total) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= F) return;
-  int run = 0;
-  for (int b = 0; b < nblocks; ++b) {
-    const int c = cntb[(size_t)b * F + j];
-    cntb[(size_t)b * F + j] = run;
-    run += c;
-  }
-  unit_total[j] = run;
-}
-
-// Fill the unit-major list with token-major entry indices, tokens ascending.
 template <typename T>
-__global__ void __launch_bounds__(256)
-    hyb_fill_kernel(const HView<T> h, const int32_t* cntb, const int32_t* unit_off,
-                    const int32_t* e0, int32_t* list) {
-  extern __shared__ int32_t next[];
+__global__ void __launch_bounds__(32 * TB_WARPS)
+    hyb_count_kernel(const HView<T> h, int nb, int32_t* cnt) {
+  extern __shared__ uint8_t hist[];  // [TB_WARPS][F]
   const int b = blockIdx.x;
-  for (int j = threadIdx.x; j < h.F; j += blockDim.x)
-    next[j] = unit_off[j] + cntb[(size_t)b * h.F + j];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  warp_unit_hist<T>(h, hist + (size_t)warp * h.F, b, warp, lane);
   __syncthreads();
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
-  for (int tt = 0; tt < TB; ++tt) {
-    const int t = b * TB + tt;
+  for (int j = threadIdx.x; j < h.F; j += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < TB_WARPS; ++w) c += hist[(size_t)w * h.F + j];
+    cnt[(size_t)j * nb + b] = c;
+  }
+}
+
+// One warp per unit: exclusive prefix of the unit's block counts, in place.
+__global__ void hyb_colscan_kernel(int nb, int F, int32_t* cnt, int32_t* unit_total) {
+  const int j = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= F) return;
+  int32_t* row = cnt + (size_t)j * nb;
+  int carry = 0;
+  for (int b0 = 0; b0 < nb; b0 += 32) {
+    const int b = b0 + lane;
+    const int v = b < nb ? row[b] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (b < nb) row[b] = carry + incl - v;
+    carry += __shfl_sync(FULL, incl, 31);
+  }
+  if (lane == 0) unit_total[j] = carry;
+}
+
+// Fill the unit-major list with token-major record indices, tokens ascending
+// within each unit.
+template <typename T>
+__global__ void __launch_bounds__(32 * TB_WARPS)
+    hyb_fill_kernel(const HView<T> h, int nb, const int32_t* cnt, const int32_t* unit_off,
+                    const int32_t* e0, int32_t* list) {
+  extern __shared__ uint8_t hist[];  // [TB_WARPS][F] -> per-warp offsets inside the block
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* mine = hist + (size_t)warp * h.F;
+  warp_unit_hist<T>(h, mine, b, warp, lane);
+  __syncthreads();
+  for (int j = threadIdx.x; j < h.F; j += blockDim.x) {
+    int r = 0;
+#pragma unroll
+    for (int w = 0; w < TB_WARPS; ++w) {
+      const int c = hist[(size_t)w * h.F + j];
+      hist[(size_t)w * h.F + j] = (uint8_t)r;
+      r += c;
+    }
+  }
+  __syncthreads();
+  for (int k = 0; k < TB_TOK; ++k) {
+    const int t = b * TB + warp * TB_TOK + k;
     if (t >= h.T) break;
     const int ebase = e0[t];
     for_each_chunk<T>(h, t, lane, [&](bool v, int j, float, size_t, bool, int rank) {
-      // the units of one row are distinct, so these increments never collide
-      if (v) list[next[j]++] = ebase + rank;
+      if (v) {
+        const int o = mine[j];
+        mine[j] = (uint8_t)(o + 1);
+        list[unit_off[j] + cnt[(size_t)j * nb + b] + o] = ebase + rank;
+      }
     });
     __syncwarp();
   }
@@ -373,6 +472,7 @@ __global__ void __launch_bounds__(256)
     float ad[E], au[E], ag[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) ad[e] = au[e] = ag[e] = 0.f;
+#pragma unroll 4
     for (int q = e_begin; q < e_end; ++q) {
       const Payload p = pay[list[q]];
       float xf[E], df[E];
@@ -399,7 +499,7 @@ __global__ void __launch_bounds__(256)
 struct BwdWs {  // the gather engine's own workspace follows these arrays
   int32_t* e0;        // [T+1]
   Payload* pay;       // [Emax]
-  int32_t* cntb;      // [NB][F]
+  int32_t* cnt;       // [F][NB], unit-major
   int32_t* unit_total;// [F]
   int32_t* unit_off;  // [F+1]
   int32_t* list;      // [Emax]
@@ -420,7 +520,7 @@ BwdWs carve(void* base, int T, int F, int C_h, int backup_cap) {
   };
   const size_t o_e0 = take(sizeof(int32_t) * ((size_t)T + 1));
   const size_t o_pay = take(sizeof(Payload) * (emax > 0 ? emax : 1));
-  const size_t o_cntb = take(sizeof(int32_t) * nb * F);
+  const size_t o_cnt = take(sizeof(int32_t) * nb * F);
   const size_t o_tot = take(sizeof(int32_t) * (size_t)F);
   const size_t o_off = take(sizeof(int32_t) * ((size_t)F + 1));
   const size_t o_list = take(sizeof(int32_t) * (emax > 0 ? emax : 1));
@@ -429,7 +529,7 @@ BwdWs carve(void* base, int T, int F, int C_h, int backup_cap) {
     char* p = static_cast<char*>(base);
     w.e0 = reinterpret_cast<int32_t*>(p + o_e0);
     w.pay = reinterpret_cast<Payload*>(p + o_pay);
-    w.cntb = reinterpret_cast<int32_t*>(p + o_cntb);
+    w.cnt = reinterpret_cast<int32_t*>(p + o_cnt);
     w.unit_total = reinterpret_cast<int32_t*>(p + o_tot);
     w.unit_off = reinterpret_cast<int32_t*>(p + o_off);
     w.list = reinterpret_cast<int32_t*>(p + o_list);
@@ -482,7 +582,7 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
   const BwdWs w = carve(ws, gu.T, gu.F, gu.C_h, gu.backup_cap);
   void* engine_ws = static_cast<char*>(ws) + w.bytes;
   const int nb = (gu.T + TB - 1) / TB;
-  const size_t hist_bytes = sizeof(int32_t) * (size_t)gu.F;
+  const size_t hist_bytes = tb_hist_bytes(gu.F);
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(hyb_count_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -499,11 +599,13 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
                                                 dx_dtype, engine_ws, status, s);
   if (e != cudaSuccess) return e;
   // weight gradients: records transposed to unit-major, token order kept
-  hyb_count_kernel<T><<<nb, 256, hist_bytes, s>>>(h, w.cntb);
-  hyb_colscan_kernel<<<(gu.F + 255) / 256, 256, 0, s>>>(nb, gu.F, w.cntb, w.unit_total);
+  hyb_count_kernel<T><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt);
+  hyb_colscan_kernel<<<(unsigned)(((size_t)gu.F * 32 + 255) / 256), 256, 0, s>>>(nb, gu.F, w.cnt,
+                                                                                w.unit_total);
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.unit_total, 0, w.unit_off, nullptr, 0,
                                          nullptr, status);
-  hyb_fill_kernel<T><<<nb, 256, hist_bytes, s>>>(h, w.cntb, w.unit_off, w.e0, w.list);
+  hyb_fill_kernel<T><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt, w.unit_off, w.e0,
+                                                          w.list);
   hyb_wgrad_kernel<T><<<gu.F, 256, 0, s>>>(gu.F, d, static_cast<const T*>(x),
                                            static_cast<const T*>(dy), w.unit_off, w.list, w.pay,
                                            dWg_t, dWu_t, dWd);

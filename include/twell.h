@@ -34,7 +34,8 @@
  * Limits      W == 128; 0 <= C <= 32; F % W == 0; d % 8 == 0; 8 <= d <= 2048
  *             (bf16 rows) or d <= 1024 (fp32 rows) for the fused and hybrid
  *             kernels; T >= 1.  F <= 65536 (hybrid
- *             indices are uint16).
+ *             indices are uint16); for hybrid arguments F % 8 == 0 and
+ *             F <= 51200.
  */
 #ifndef TWELL_H
 #define TWELL_H

@@ -121,6 +121,11 @@ def test_hybrid_validation(L):
     args2 = list(args)
     args2[0] = FAKE + 2
     assert L.hybrid_ffn_backward(*args2, ws, None, None) == ALIGN
+    # dense backup rows are read 16 bytes at a time: F must be a multiple of 8
+    odd = _hy(F=1020)
+    fws = L.hybrid_ffn_forward_workspace_size(256, 512)
+    assert L.hybrid_ffn_forward(FAKE, ctypes.byref(odd), FAKE, FAKE, 512, FAKE, twell.TW_F32, FAKE,
+                                fws, None, None) == UNSUPPORTED
 
 
 def test_workspace_size_grows_with_capacity(L):
