@@ -329,15 +329,17 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_leg(w, y)
     legs = set() if args.no_extras else {s.strip() for s in args.legs.split(",") if s.strip()}
-    if rank == 0 and legs:
-        if "dense" in legs:
+    if legs:
+        if rank == 0 and "dense" in legs:
             line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
         del x, Wg, Wu, Wd, g, y, ws, xh, yh
         torch.cuda.empty_cache()
-        if "decode" in legs:
+        if rank == 0 and "decode" in legs:
             line["decode"] = decode_leg(torch, tw, hbm)
-        if "training" in legs:
-            line["training"] = training_leg(torch, tw)
+        if "training" in legs:  # every rank: data-parallel, one gradient all-reduce per step
+            tr = training_leg(torch, tw, dist, world)
+            if rank == 0:
+                line["training"] = tr
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -394,9 +396,13 @@ def decode_leg(torch, tw, hbm):
     return out
 
 
-def training_leg(torch, tw):
-    """One training step of the hybrid path at the train_2b shape: gate GEMM ->
-    TwELL -> hybrid, hybrid forward, hybrid backward (with the L1 term)."""
+def training_leg(torch, tw, dist=None, world=1):
+    """One training step of the hybrid path at the train_2b shape per GPU: gate
+    GEMM -> TwELL -> hybrid, hybrid forward, hybrid backward (with the L1
+    term); on N GPUs each rank takes its own train_2b batch (weak scaling)
+    and the weight gradients are summed with one all-reduce (NCCL)."""
+    from activation_sparse_transformer_tma_b200 import dp
+
     w = synth.make_workload("train_2b")
     T, d, F, C, C_h = w["T"], w["d"], w["F"], w["C"], w["C_h"]
     dev = {k: torch.from_numpy(w[k].view(np.int16)).cuda().view(torch.bfloat16)
@@ -406,15 +412,17 @@ def training_leg(torch, tw):
     hy = tw.Hybrid(T, F, C_h, dtype=torch.bfloat16, backup_cap=cap)
     y = torch.empty((T, d), dtype=torch.float32, device="cuda")
     dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
-    dW = [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+    grads = dp.GradBuffer(F, d, "cuda")
     ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, C_h, cap), dtype=torch.uint8,
                      device="cuda")
     fws = torch.empty(tw.hybrid_ffn_forward_workspace_size(T, d), dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     names = ["gate_twell_gemm", "twell_to_hybrid", "hybrid_ffn_forward", "hybrid_ffn_backward"]
+    if world > 1:
+        names.append("grad_allreduce")
     times = {n: [] for n in names}
     for it in range(8):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         e[0].record()
         tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, None, st)
         e[1].record()
@@ -423,17 +431,27 @@ def training_leg(torch, tw):
         tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], y, fws, st)
         e[3].record()
         tw.hybrid_ffn_backward(dev["x"], dev["dy"], hy, dev["Wg_t"], dev["Wu_t"], dev["Wd"],
-                               w["lam"], dx, dW[0], dW[1], dW[2], ws, st)
+                               w["lam"], dx, grads.dWg_t, grads.dWu_t, grads.dWd, ws, st)
         e[4].record()
+        if world > 1:
+            grads.allreduce()
+            e[5].record()
         torch.cuda.synchronize()
         if it >= 3:
             for i, n in enumerate(names):
                 times[n].append(e[i].elapsed_time(e[i + 1]))
     ms = {n: float(np.median(v)) for n, v in times.items()}
     step = sum(ms.values())
-    return {"workload": "train_2b", "T": T, "d": d, "F": F, "C": C, "C_h": C_h,
-            "ms": ms, "ms_per_step": step, "tokens_per_s": T / (step * 1e-3),
-            "n_backup": int(hy.n_backup.item()), "backup_cap": cap, "device_status": int(st.item())}
+    if world > 1:  # the slowest rank sets the step time
+        tt = torch.tensor([step], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        step = float(tt.item())
+    out = {"workload": "train_2b", "T": T, "d": d, "F": F, "C": C, "C_h": C_h,
+           "ms": ms, "ms_per_step": step, "tokens_per_s": world * T / (step * 1e-3),
+           "n_backup": int(hy.n_backup.item()), "backup_cap": cap, "device_status": int(st.item())}
+    if world > 1:
+        out["parallelism"] = f"dp{world}: one fp32 all-reduce of dWg, dWu, dWd ({3 * F * d * 4} B)"
+    return out
 
 
 def dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_sparse, args):
