@@ -26,16 +26,30 @@ namespace tw {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 64;  // 64 bf16 = 128 B = one swizzle atom row
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
-constexpr int TMEM_COLS = 2 * BN;
 constexpr int EPI_SLOTS = 32;  // largest TwELL capacity C this epilogue packs
 
+// Tile widths: BN = 256 with a 4-stage ring, or BN = 128 with a 6-stage ring
+// when there are too few 256-wide tiles to occupy every SM (small T).
+template <int BN>
+struct Shape {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
+};
+
+// Per-thread staging of the TwELL epilogue.
+struct EpiStage {
+  alignas(16) uint16_t slot_val[128 * EPI_SLOTS];  // read back with 16-byte loads
+  alignas(16) uint8_t slot_idx[128 * EPI_SLOTS];   // read back with 8-byte loads
+};
+static_assert(offsetof(EpiStage, slot_val) % 16 == 0 && offsetof(EpiStage, slot_idx) % 16 == 0,
+              "epilogue staging must be 16-byte aligned");
+
+template <int STAGES>
 struct SmemTail {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -45,13 +59,16 @@ struct SmemTail {
   uint32_t tmem_base;
   int abort;
   int never;
-  alignas(16) uint16_t slot_val[128 * EPI_SLOTS];  // read back with 16-byte loads
-  alignas(16) uint8_t slot_idx[128 * EPI_SLOTS];   // read back with 8-byte loads
+  EpiStage epi;
 };
-static_assert(offsetof(SmemTail, slot_val) % 16 == 0 && offsetof(SmemTail, slot_idx) % 16 == 0,
-              "epilogue staging must be 16-byte aligned");
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+template <int BN>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)Shape<BN>::STAGES * Shape<BN>::STAGE_BYTES +
+         sizeof(SmemTail<Shape<BN>::STAGES>);
+}
+static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024,
+              "shared memory budget");
 
 // ReLU on fp32 bits: negative numbers and -0 (sign bit set) become +0.
 TW_DEV uint32_t relu_bits(uint32_t b) { return (int32_t)b > 0 ? b : 0u; }
@@ -70,15 +87,17 @@ struct EpiTwell {
   uint16_t* dump;
   int32_t* status;
 
-  // taddr: TMEM address of this warp's lane block at column 0 of the tile.
-  TW_DEV void run(uint32_t taddr, int row, int nb, int ethread, SmemTail* sm) const {
+  // taddr: TMEM address of this warp's lane block at column 0 of the tile;
+  // the tile holds KT TwELL tiles of 128 columns.
+  template <int KT>
+  TW_DEV void run(uint32_t taddr, int row, int nb, int ethread, EpiStage* st) const {
     const bool row_ok = row < T;
     const int K = F / 128;
-    uint16_t* sv = sm->slot_val + ethread * EPI_SLOTS;
-    uint8_t* si = sm->slot_idx + ethread * EPI_SLOTS;
+    uint16_t* sv = st->slot_val + ethread * EPI_SLOTS;
+    uint8_t* si = st->slot_idx + ethread * EPI_SLOTS;
 #pragma unroll 1
-    for (int kt = 0; kt < 2; ++kt) {
-      const int k = nb * 2 + kt;
+    for (int kt = 0; kt < KT; ++kt) {
+      const int k = nb * KT + kt;
       if (k >= K) break;  // uniform across the CTA
       for (int s = 0; s < C; ++s) {
         sv[s] = 0;
@@ -181,7 +200,9 @@ struct EpiGateUp {
   static constexpr bool kDualB = true;
   int T, F;
   uint16_t* h;
-  TW_DEV void run(uint32_t taddr, int row, int nb, int, SmemTail*) const {
+  template <int KT>
+  TW_DEV void run(uint32_t taddr, int row, int nb, int, EpiStage*) const {
+    static_assert(KT == 2, "gate and up halves of a 256-wide tile");
     const bool row_ok = row < T;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
@@ -210,11 +231,12 @@ struct EpiStore {
   static constexpr bool kDualB = false;
   int T, N;
   uint16_t* y;
-  TW_DEV void run(uint32_t taddr, int row, int nb, int, SmemTail*) const {
+  template <int KT>
+  TW_DEV void run(uint32_t taddr, int row, int nb, int, EpiStage*) const {
     const bool row_ok = row < T;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      const int col0 = nb * BN + c * 32;
+    for (int c = 0; c < KT * 4; ++c) {
+      const int col0 = nb * KT * 128 + c * 32;
       if (col0 >= N) break;  // uniform
       uint32_t r[32];
       tmem_ld_32x32b_x32(taddr + c * 32, r);
@@ -233,16 +255,20 @@ struct EpiStore {
 };
 
 // --------------------------------------------------------------- kernel ----
-template <class Epi>
+template <class Epi, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, int Kdim, int n_tiles_n,
                    int num_tiles, const Epi epi, int32_t* status,
                    unsigned long long timeout_ns) {
+  constexpr int STAGES = Shape<BN>::STAGES;
+  constexpr int STAGE_BYTES = Shape<BN>::STAGE_BYTES;
+  constexpr int B_BYTES = Shape<BN>::B_BYTES;
+  constexpr int TMEM_COLS = Shape<BN>::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SmemTail* sm = reinterpret_cast<SmemTail*>(smem + (size_t)STAGES * STAGE_BYTES);
+  auto* sm = reinterpret_cast<SmemTail<STAGES>*>(smem + (size_t)STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int kblocks = (Kdim + BK - 1) / BK;
@@ -377,7 +403,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int row = m_blk * BM + q * 32 + lane;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-      epi.run(taddr, row, n_blk, ethread, sm);
+      epi.template run<BN / 128>(taddr, row, n_blk, ethread, &sm->epi);
       tc_fence_before();
       mbar_arrive(&sm->tmem_empty[acc]);
     }
@@ -397,22 +423,22 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   return make_tmap_bf16(m, base, rows, cols, BK, box_rows);
 }
 
-template <class Epi>
+template <class Epi, int BN>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, int Kdim,
                    int n_tiles_m, int n_tiles_n, const Epi& epi, int32_t* status,
                    cudaStream_t stream) {
   static bool attr_set = false;  // per template instance; idempotent
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<Epi>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<Epi, BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+                                         (int)smem_bytes<BN>());
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int num_tiles = n_tiles_m * n_tiles_n;
   if (num_tiles == 0) return cudaSuccess;
   const int grid = num_tiles < num_sms() ? num_tiles : num_sms();
-  gemm_tc_kernel<Epi><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(
+  gemm_tc_kernel<Epi, BN><<<grid, NUM_THREADS, smem_bytes<BN>(), stream>>>(
       a, b0, b1, Kdim, n_tiles_n, num_tiles, epi, status, kWaitTimeoutNs);
   return cudaGetLastError();
 }
@@ -422,8 +448,12 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
 cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, int F,
                                  const tw_twell& out, void* dump, int32_t* status,
                                  cudaStream_t stream) {
+  // 128-wide tiles when 256-wide ones would leave SMs idle (small T)
+  const int m_tiles = (T + BM - 1) / BM;
+  const bool narrow = (long long)m_tiles * ((F + 255) / 256) < num_sms();
   CUtensorMap ma, mb;
-  if (!make_map(&ma, x, T, d, BM) || !make_map(&mb, Wg_t, F, d, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&ma, x, T, d, BM) || !make_map(&mb, Wg_t, F, d, narrow ? 128 : 256))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(out.spill_n, 0, sizeof(int32_t), stream);
   if (e != cudaSuccess) return e;
   EpiTwell epi;
@@ -440,32 +470,34 @@ cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, 
   epi.spill_n = out.spill_n;
   epi.dump = static_cast<uint16_t*>(dump);
   epi.status = status;
-  return launch(ma, mb, mb, d, (T + BM - 1) / BM, (F + BN - 1) / BN, epi, status, stream);
+  return narrow ? launch<EpiTwell, 128>(ma, mb, mb, d, m_tiles, F / 128, epi, status, stream)
+                : launch<EpiTwell, 256>(ma, mb, mb, d, m_tiles, (F + 255) / 256, epi, status, stream);
 }
 
 cudaError_t launch_dense_gateup_tc(const void* x, const void* Wg_t, const void* Wu_t, int T,
                                    int d, int F, void* h, int32_t* status, cudaStream_t stream) {
   CUtensorMap ma, mg, mu;
-  if (!make_map(&ma, x, T, d, BM) || !make_map(&mg, Wg_t, F, d, BN / 2) ||
-      !make_map(&mu, Wu_t, F, d, BN / 2))
+  if (!make_map(&ma, x, T, d, BM) || !make_map(&mg, Wg_t, F, d, 128) ||
+      !make_map(&mu, Wu_t, F, d, 128))
     return cudaErrorInvalidValue;
   EpiGateUp epi;
   epi.T = T;
   epi.F = F;
   epi.h = static_cast<uint16_t*>(h);
-  return launch(ma, mg, mu, d, (T + BM - 1) / BM, F / (BN / 2), epi, status, stream);
+  return launch<EpiGateUp, 256>(ma, mg, mu, d, (T + BM - 1) / BM, F / 128, epi, status, stream);
 }
 
 cudaError_t launch_dense_down_tc(const void* h, const void* Wd_dense, int T, int d, int F,
                                  void* y, int32_t* status, cudaStream_t stream) {
   CUtensorMap ma, mb;
-  if (!make_map(&ma, h, T, F, BM) || !make_map(&mb, Wd_dense, d, F, BN))
+  if (!make_map(&ma, h, T, F, BM) || !make_map(&mb, Wd_dense, d, F, 256))
     return cudaErrorInvalidValue;
   EpiStore epi;
   epi.T = T;
   epi.N = d;
   epi.y = static_cast<uint16_t*>(y);
-  return launch(ma, mb, mb, F, (T + BM - 1) / BM, (d + BN - 1) / BN, epi, status, stream);
+  return launch<EpiStore, 256>(ma, mb, mb, F, (T + BM - 1) / BM, (d + 255) / 256, epi, status,
+                               stream);
 }
 
 }  // namespace tw
