@@ -377,7 +377,7 @@ def decode_leg(torch, tw, hbm):
         ws = tw.fused_workspace(T, d)
         tg, tf = [], []
         for it in range(25):
-            torch.sum(flush, out=sink)
+            torch.sum(flush, dim=0, out=sink)
             e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             e[0].record()
             tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g)
