@@ -259,7 +259,7 @@ template <class Epi, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, int Kdim, int n_tiles_n,
-                   int num_tiles, const Epi epi, int32_t* status,
+                   int num_tiles, uint32_t a_bytes, const Epi epi, int32_t* status,
                    unsigned long long timeout_ns) {
   constexpr int STAGES = Shape<BN>::STAGES;
   constexpr int STAGE_BYTES = Shape<BN>::STAGE_BYTES;
@@ -319,7 +319,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           uint8_t* a = smem + (size_t)s * STAGE_BYTES;
           uint8_t* b = a + A_BYTES;
-          mbar_arrive_expect_tx(&sm->full[s], STAGE_BYTES);
+          // the x box may be narrower than the 128-row tile (one small m-tile);
+          // rows past it are stale and only reach output rows that are not stored
+          mbar_arrive_expect_tx(&sm->full[s], a_bytes + B_BYTES);
           tma_load_2d(a, &tmA, &sm->full[s], kb * BK, m_blk * BM);
           if (Epi::kDualB) {
             tma_load_2d(b, &tmB0, &sm->full[s], kb * BK, n_blk * (BN / 2));
@@ -426,7 +428,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 template <class Epi, int BN>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, int Kdim,
                    int n_tiles_m, int n_tiles_n, const Epi& epi, int32_t* status,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, uint32_t a_bytes = A_BYTES) {
   static bool attr_set = false;  // per template instance; idempotent
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<Epi, BN>,
@@ -439,7 +441,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   if (num_tiles == 0) return cudaSuccess;
   const int grid = num_tiles < num_sms() ? num_tiles : num_sms();
   gemm_tc_kernel<Epi, BN><<<grid, NUM_THREADS, smem_bytes<BN>(), stream>>>(
-      a, b0, b1, Kdim, n_tiles_n, num_tiles, epi, status, kWaitTimeoutNs);
+      a, b0, b1, Kdim, n_tiles_n, num_tiles, a_bytes, epi, status, kWaitTimeoutNs);
   return cudaGetLastError();
 }
 
@@ -451,8 +453,10 @@ cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, 
   // 128-wide tiles when 256-wide ones would leave SMs idle (small T)
   const int m_tiles = (T + BM - 1) / BM;
   const bool narrow = (long long)m_tiles * ((F + 255) / 256) < num_sms();
+  // with a single m-tile, load only the x rows that exist (rounded up to 16)
+  const uint32_t a_rows = T < BM ? (uint32_t)((T + 15) / 16 * 16) : (uint32_t)BM;
   CUtensorMap ma, mb;
-  if (!make_map(&ma, x, T, d, BM) || !make_map(&mb, Wg_t, F, d, narrow ? 128 : 256))
+  if (!make_map(&ma, x, T, d, a_rows) || !make_map(&mb, Wg_t, F, d, narrow ? 128 : 256))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(out.spill_n, 0, sizeof(int32_t), stream);
   if (e != cudaSuccess) return e;
@@ -470,8 +474,11 @@ cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, 
   epi.spill_n = out.spill_n;
   epi.dump = static_cast<uint16_t*>(dump);
   epi.status = status;
-  return narrow ? launch<EpiTwell, 128>(ma, mb, mb, d, m_tiles, F / 128, epi, status, stream)
-                : launch<EpiTwell, 256>(ma, mb, mb, d, m_tiles, (F + 255) / 256, epi, status, stream);
+  const uint32_t a_bytes = a_rows * BK * 2;
+  return narrow ? launch<EpiTwell, 128>(ma, mb, mb, d, m_tiles, F / 128, epi, status, stream,
+                                        a_bytes)
+                : launch<EpiTwell, 256>(ma, mb, mb, d, m_tiles, (F + 255) / 256, epi, status,
+                                        stream, a_bytes);
 }
 
 cudaError_t launch_dense_gateup_tc(const void* x, const void* Wg_t, const void* Wu_t, int T,

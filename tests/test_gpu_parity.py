@@ -70,6 +70,9 @@ SMALL = [
     (129, 64, 256, 0, "dead20", 29.0),       # C = 0: every non-empty tile spills
     (257, 2048, 1280, 32, "zipf", 40.0),     # full-width rows, largest C
     (128, 512, 2048, 16, "uniform4", 29.0),
+    (40, 512, 640, 2, "dead20", 60.0),       # small batch: x box narrower than the tile, spills
+    (64, 1024, 1024, 8, "zipf", 29.0),
+    (65, 256, 1024, 8, "zipf", 29.0),
 ]
 
 
@@ -154,8 +157,10 @@ def test_decode_sizes(T):
     dev, g, gd, y, st = run_forward(w)
     assert int(st.item()) == 0
     w64 = widened(w)
+    rows = np.arange(T, dtype=np.int32)
+    check_gate_values(f64(gd), w64["x"], w64["Wg_t"], rows)
     assert_twell_matches_oracle(g, f64(gd))
-    check_y(f64(y), w64, np.arange(T, dtype=np.int32), TOL[synth.BF16])
+    check_y(f64(y), w64, rows, TOL[synth.BF16])
 
 
 def test_fused_without_dump_matches_dump_run():
