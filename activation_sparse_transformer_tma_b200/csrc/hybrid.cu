@@ -97,10 +97,17 @@ struct HView {
 // entry's position among the row's non-zeros.  Rows whose backup slot was
 // dropped for lack of capacity have no entries.
 template <typename T, class Fn>
+TW_DEV void for_each_chunk(const HView<T>& h, int t, int slot, int nnz, int lane, Fn&& fn);
+
+template <typename T, class Fn>
 TW_DEV void for_each_chunk(const HView<T>& h, int t, int lane, Fn&& fn) {
-  const int slot = h.row_slot[t];
+  for_each_chunk<T>(h, t, h.row_slot[t], h.row_nnz[t], lane, fn);
+}
+
+// The same with the row's slot and count already loaded.
+template <typename T, class Fn>
+TW_DEV void for_each_chunk(const HView<T>& h, int t, int slot, int nnz, int lane, Fn&& fn) {
   if (slot < 0) {
-    const int nnz = h.row_nnz[t];
     for (int s0 = 0; s0 < nnz; s0 += 32) {
       const int s = s0 + lane;
       const bool v = s < nnz;
@@ -347,9 +354,8 @@ __global__ void __launch_bounds__(256)
 // The records of the backward are in token-major order (entry e0[t] + rank).
 // The weight gradients sum them per unit in ascending token order, so they
 // are transposed to a unit-major list with a stable counting sort:
-//   1. hyb_count_kernel   entries per (block of TB tokens, unit), written
-//                         unit-major: cnt[j][b];
-//   2. hyb_colscan_kernel one warp per unit: exclusive prefix over blocks
+//   1. hyb_count_kernel   entries per (block of TB tokens, unit): cnt[b][j];
+//   2. hyb_colscan_kernel one thread per unit: exclusive prefix over blocks
 //                         (in place) and the unit's total;
 //   3. scan_kernel        exclusive prefix of the totals -> unit_off;
 //   4. hyb_fill_kernel    each block walks its tokens again and writes every
@@ -359,7 +365,7 @@ __global__ void __launch_bounds__(256)
 // warps' histograms become exclusive offsets, so the warps place their
 // entries in parallel and the token order inside each unit is kept.
 constexpr int TB_WARPS = 4;
-constexpr int TB_TOK = 16;               // tokens per warp
+constexpr int TB_TOK = 8;                // tokens per warp
 constexpr int TB = TB_WARPS * TB_TOK;    // tokens per block
 static_assert((TB_WARPS - 1) * TB_TOK < 256, "per-warp offsets must fit in uint8");
 
@@ -367,15 +373,30 @@ static_assert((TB_WARPS - 1) * TB_TOK < 256, "per-warp offsets must fit in uint8
 inline size_t tb_hist_bytes(int F) { return (size_t)TB_WARPS * F; }
 
 // Per-warp histogram of the units of the warp's tokens (zeroed first).
+// Slot and count of the warp's TB_TOK tokens, loaded in one round (lane k
+// holds token k's), so the walk over the tokens does not wait for them.
+template <typename T>
+TW_DEV void warp_token_meta(const HView<T>& h, int t0, int lane, int& slot, int& nnz) {
+  const int t = t0 + lane;
+  const bool ok = lane < TB_TOK && t < h.T;
+  slot = ok ? h.row_slot[t] : -1;
+  nnz = ok ? h.row_nnz[t] : 0;
+}
+
 template <typename T>
 TW_DEV void warp_unit_hist(const HView<T>& h, uint8_t* hist, int b, int warp, int lane) {
-  for (int j = lane; j < h.F; j += 32) hist[j] = 0;
+  const int t0 = b * TB + warp * TB_TOK;
+  int mslot, mnnz;
+  warp_token_meta<T>(h, t0, lane, mslot, mnnz);
+  uint32_t* h4 = reinterpret_cast<uint32_t*>(hist);
+  for (int j = lane; j < h.F / 4; j += 32) h4[j] = 0u;
   __syncwarp();
   for (int k = 0; k < TB_TOK; ++k) {
-    const int t = b * TB + warp * TB_TOK + k;
+    const int t = t0 + k;
     if (t >= h.T) break;
+    const int slot = __shfl_sync(FULL, mslot, k), nnz = __shfl_sync(FULL, mnnz, k);
     // the units of one row are distinct, so these increments never collide
-    for_each_chunk<T>(h, t, lane, [&](bool v, int j, float, size_t, bool, int) {
+    for_each_chunk<T>(h, t, slot, nnz, lane, [&](bool v, int j, float, size_t, bool, int) {
       if (v) hist[j] = (uint8_t)(hist[j] + 1);
     });
     __syncwarp();
@@ -394,30 +415,28 @@ __global__ void __launch_bounds__(32 * TB_WARPS)
     int c = 0;
 #pragma unroll
     for (int w = 0; w < TB_WARPS; ++w) c += hist[(size_t)w * h.F + j];
-    cnt[(size_t)j * nb + b] = c;
+    cnt[(size_t)b * h.F + j] = c;  // block-major: coalesced
   }
 }
 
-// One warp per unit: exclusive prefix of the unit's block counts, in place.
+// One thread per unit: exclusive prefix over the blocks of the unit's counts
+// (block-major, so a warp reads 32 consecutive units per block), in place;
+// eight blocks are loaded ahead of the running sum.
 __global__ void hyb_colscan_kernel(int nb, int F, int32_t* cnt, int32_t* unit_total) {
-  const int j = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= F) return;
-  int32_t* row = cnt + (size_t)j * nb;
-  int carry = 0;
-  for (int b0 = 0; b0 < nb; b0 += 32) {
-    const int b = b0 + lane;
-    const int v = b < nb ? row[b] : 0;
-    int incl = v;
+  int run = 0;
+  for (int b0 = 0; b0 < nb; b0 += 8) {
+    int v[8];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(FULL, incl, o);
-      if (lane >= o) incl += u;
+    for (int i = 0; i < 8; ++i) v[i] = b0 + i < nb ? cnt[(size_t)(b0 + i) * F + j] : 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (b0 + i < nb) cnt[(size_t)(b0 + i) * F + j] = run;
+      run += v[i];
     }
-    if (b < nb) row[b] = carry + incl - v;
-    carry += __shfl_sync(FULL, incl, 31);
   }
-  if (lane == 0) unit_total[j] = carry;
+  unit_total[j] = run;
 }
 
 // Fill the unit-major list with token-major record indices, tokens ascending
@@ -442,15 +461,20 @@ __global__ void __launch_bounds__(32 * TB_WARPS)
     }
   }
   __syncthreads();
+  const int t0 = b * TB + warp * TB_TOK;
+  int mslot, mnnz;
+  warp_token_meta<T>(h, t0, lane, mslot, mnnz);
+  const int mbase = lane < TB_TOK && t0 + lane < h.T ? e0[t0 + lane] : 0;
   for (int k = 0; k < TB_TOK; ++k) {
-    const int t = b * TB + warp * TB_TOK + k;
+    const int t = t0 + k;
     if (t >= h.T) break;
-    const int ebase = e0[t];
-    for_each_chunk<T>(h, t, lane, [&](bool v, int j, float, size_t, bool, int rank) {
+    const int ebase = __shfl_sync(FULL, mbase, k);
+    const int slot = __shfl_sync(FULL, mslot, k), nnz = __shfl_sync(FULL, mnnz, k);
+    for_each_chunk<T>(h, t, slot, nnz, lane, [&](bool v, int j, float, size_t, bool, int rank) {
       if (v) {
         const int o = mine[j];
         mine[j] = (uint8_t)(o + 1);
-        list[unit_off[j] + cnt[(size_t)j * nb + b] + o] = ebase + rank;
+        list[unit_off[j] + cnt[(size_t)b * h.F + j] + o] = ebase + rank;
       }
     });
     __syncwarp();
@@ -499,7 +523,7 @@ __global__ void __launch_bounds__(256)
 struct BwdWs {  // the gather engine's own workspace follows these arrays
   int32_t* e0;        // [T+1]
   Payload* pay;       // [Emax]
-  int32_t* cnt;       // [F][NB], unit-major
+  int32_t* cnt;       // [NB][F], block-major
   int32_t* unit_total;// [F]
   int32_t* unit_off;  // [F+1]
   int32_t* list;      // [Emax]
@@ -600,8 +624,7 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
   if (e != cudaSuccess) return e;
   // weight gradients: records transposed to unit-major, token order kept
   hyb_count_kernel<T><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt);
-  hyb_colscan_kernel<<<(unsigned)(((size_t)gu.F * 32 + 255) / 256), 256, 0, s>>>(nb, gu.F, w.cnt,
-                                                                                w.unit_total);
+  hyb_colscan_kernel<<<(gu.F + 255) / 256, 256, 0, s>>>(nb, gu.F, w.cnt, w.unit_total);
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.unit_total, 0, w.unit_off, nullptr, 0,
                                          nullptr, status);
   hyb_fill_kernel<T><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt, w.unit_off, w.e0,
