@@ -265,7 +265,7 @@ def test_dense_comparator_2b_shape_sampled():
 def run_hybrid(w, backup_cap=None):
     T, d, F = w["T"], w["d"], w["F"]
     dev, g, gd, y, st = run_forward(w)
-    hy = tw.Hybrid(T, F, w["C_h"], dtype=torch.bfloat16, backup_cap=backup_cap)
+    hy = tw.Hybrid(T, F, w["C_h"], dtype=TDT[w["dtype"]], backup_cap=backup_cap)
     tw.twell_to_hybrid(g, hy, st)
     yh = torch.empty((T, d), dtype=torch.float32, device="cuda")
     tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, dev_status=st)
@@ -323,9 +323,10 @@ def check_hybrid_all(w, res):
             f"u mismatch at {where}: gpu {ug[i]} oracle {ur[i]}, {int((viol > 0).sum())} "
             f"violations; rows (t, nnz, slot) {info}; u right after the forward "
             f"{u_fwd[i]}; y row errors {yerr} (rms {rms(y_ref)})")
-    assert np.max(np.abs(f64(yh) - y_ref)) <= TOL[synth.BF16] * rms(y_ref)
+    tol = TOL[w["dtype"]]
+    assert np.max(np.abs(f64(yh) - y_ref)) <= tol * rms(y_ref)
     # the hybrid forward y equals the inference y up to rounding
-    assert np.max(np.abs(f64(yh) - f64(y))) <= TOL[synth.BF16] * rms(y_ref)
+    assert np.max(np.abs(f64(yh) - f64(y))) <= tol * rms(y_ref)
     # backward, conditioned on the GPU's saved g and u
     got_u = dict(got)
     grads = oracle.hybrid_backward(w64["x"], w64["dy"], got, f64(hy.ell_u),
@@ -333,7 +334,7 @@ def check_hybrid_all(w, res):
                                    w["lam"])
     for name, a, b in zip(("dx", "dWg_t", "dWu_t", "dWd"), (dx, dW[0], dW[1], dW[2]), grads):
         err = np.max(np.abs(f64(a) - b))
-        assert err <= TOL[synth.BF16] * rms(b), (name, err, rms(b))
+        assert err <= tol * rms(b), (name, err, rms(b))
     return got_u
 
 
@@ -353,6 +354,42 @@ def test_hybrid_extreme_caps(C_h):
         assert got["n_backup"] == int((got["row_nnz"] > 0).sum())
     else:
         assert got["n_backup"] == 0
+
+
+def test_hybrid_fp32_small():
+    # fp32 activations: fp32 gate on the CUDA cores, fp32 gather engine (FMA dot products)
+    w = synth.make_workload(T=150, d=128, F=512, W=128, C=4, C_h=8, dtype=synth.F32,
+                            kind="pareto", lam=2e-5, seed=12, mean_active=10.0)
+    got = check_hybrid_all(w, run_hybrid(w, backup_cap=150))
+    assert 0 < got["n_backup"] < 150
+
+
+def test_hybrid_bf16_outputs_are_the_fp32_results_rounded():
+    w = synth.make_workload(T=300, d=256, F=640, W=128, C=8, C_h=16, dtype=synth.BF16,
+                            kind="pareto", lam=2e-5, seed=13, mean_active=14.0)
+    T, d, F = w["T"], w["d"], w["F"]
+    dev, g, gd, y, st = run_forward(w)
+    hy = tw.Hybrid(T, F, w["C_h"], dtype=torch.bfloat16, backup_cap=T)
+    tw.twell_to_hybrid(g, hy, st)
+    ws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, w["C_h"], T),
+                     dtype=torch.uint8, device="cuda")
+    outs = {}
+    for dt in (torch.float32, torch.bfloat16):
+        yh = torch.empty((T, d), dtype=dt, device="cuda")
+        tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, dev_status=st)
+        dx = torch.empty((T, d), dtype=dt, device="cuda")
+        dW = [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+        tw.hybrid_ffn_backward(dev["x"], dev["dy"], hy, dev["Wg_t"], dev["Wu_t"], dev["Wd"],
+                               w["lam"], dx, dW[0], dW[1], dW[2], ws, st)
+        torch.cuda.synchronize()
+        outs[dt] = (yh, dx, dW)
+    assert int(st.item()) == 0, tw.status_bits(st)
+    y32, dx32, dW32 = outs[torch.float32]
+    y16, dx16, dW16 = outs[torch.bfloat16]
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    assert torch.equal(dx16, dx32.to(torch.bfloat16))
+    for a, b in zip(dW16, dW32):  # the weight gradients do not depend on the dx dtype
+        assert torch.equal(a, b)
 
 
 def test_hybrid_backup_capacity_overflow_is_flagged():
