@@ -48,8 +48,9 @@ tw_status check_twell(const tw_twell* g) {
     return TW_ERR_INVALID_ARG;
   if (g->W != kTileW || g->F % kTileW != 0 || g->C > kMaxC) return TW_ERR_UNSUPPORTED;
   if (g->F > 65536) return TW_ERR_UNSUPPORTED;
-  if (!g->cnt || !g->spill_ref || !g->spill_n) return TW_ERR_INVALID_ARG;
-  if (g->C > 0 && (!g->val || !g->idx)) return TW_ERR_INVALID_ARG;
+  // arrays sized by T may be NULL for an empty batch
+  if (!g->spill_n || (g->T > 0 && (!g->cnt || !g->spill_ref))) return TW_ERR_INVALID_ARG;
+  if (g->T > 0 && g->C > 0 && (!g->val || !g->idx)) return TW_ERR_INVALID_ARG;
   if (g->spill_cap > 0 && (!g->spill_tk || !g->spill_val)) return TW_ERR_INVALID_ARG;
   if ((g->val && !aligned16(g->val)) || (g->idx && !aligned16(g->idx)) ||
       (g->spill_val && !aligned16(g->spill_val)))
@@ -66,8 +67,9 @@ tw_status check_hybrid(const tw_hybrid* h) {
   if (h->F > 51200 || h->F % 8 != 0) return TW_ERR_UNSUPPORTED;
   if ((size_t)h->T * (size_t)h->C_h + (size_t)h->backup_cap * (size_t)h->F > 0x7FFFFFFFull)
     return TW_ERR_UNSUPPORTED;  // entry numbers are int32
-  if (!h->row_nnz || !h->row_slot || !h->n_backup) return TW_ERR_INVALID_ARG;
-  if (h->C_h > 0 && (!h->ell_g || !h->ell_idx)) return TW_ERR_INVALID_ARG;
+  // arrays sized by T may be NULL for an empty batch
+  if (!h->n_backup || (h->T > 0 && (!h->row_nnz || !h->row_slot))) return TW_ERR_INVALID_ARG;
+  if (h->T > 0 && h->C_h > 0 && (!h->ell_g || !h->ell_idx)) return TW_ERR_INVALID_ARG;
   if (h->backup_cap > 0 && (!h->backup_rows || !h->backup_g)) return TW_ERR_INVALID_ARG;
   return TW_OK;
 }
@@ -98,7 +100,7 @@ tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int32_t d,
                           int32_t* dev_status, cudaStream_t stream) {
   tw_status st = check_twell(out);
   if (st != TW_OK) return st;
-  if (!x || !Wg_t) return TW_ERR_INVALID_ARG;
+  if ((T > 0 && !x) || !Wg_t) return TW_ERR_INVALID_ARG;
   if (T < 0 || d <= 0 || F <= 0 || out->T != T || out->F != F || out->dtype != dtype)
     return TW_ERR_INVALID_ARG;
   if (d % 8 != 0) return TW_ERR_UNSUPPORTED;
@@ -126,13 +128,14 @@ tw_status twell_fused_updown(const void* x, const tw_twell* g, const void* Wu_t,
                              int32_t* dev_status, cudaStream_t stream) {
   tw_status st = check_twell(g);
   if (st != TW_OK) return st;
-  if (!x || !Wu_t || !Wd || !y || !ws || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
+  const bool any = g->T > 0;  // with no tokens x, y and ws are not touched
+  if ((any && (!x || !y || !ws)) || !Wu_t || !Wd || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
   if (d <= 0) return TW_ERR_INVALID_ARG;
   if (!row_d_ok(d, g->dtype)) return TW_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y) || !aligned16(ws))
     return TW_ERR_ALIGNMENT;
+  if (!any) return TW_OK;
   if (ws_bytes < tw::fused_ws_bytes(g->T, d)) return TW_ERR_WORKSPACE;
-  if (g->T == 0) return TW_OK;
   return from_cuda(
       tw::launch_fused_updown(x, *g, Wu_t, Wd, d, y, y_dtype, ws, dev_status, stream));
 }
@@ -158,14 +161,15 @@ tw_status hybrid_ffn_forward(const void* x, const tw_hybrid* gu, const void* Wu_
                              size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
   tw_status st = check_hybrid(gu);
   if (st != TW_OK) return st;
-  if (!x || !Wu_t || !Wd || !y || !ws || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
-  if ((gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
+  const bool any = gu->T > 0;  // with no tokens x, y, ws and ell_u are not touched
+  if ((any && (!x || !y || !ws)) || !Wu_t || !Wd || !dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
+  if ((any && gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
     return TW_ERR_INVALID_ARG;
   if (d <= 0) return TW_ERR_INVALID_ARG;
   if (!row_d_ok(d, gu->dtype)) return TW_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(Wu_t) || !aligned16(Wd) || !aligned16(y) || !aligned16(ws))
     return TW_ERR_ALIGNMENT;
-  if (ws_bytes < tw::hybrid_forward_ws_bytes(gu->T, d)) return TW_ERR_WORKSPACE;
+  if (any && ws_bytes < tw::hybrid_forward_ws_bytes(gu->T, d)) return TW_ERR_WORKSPACE;
   return from_cuda(
       tw::launch_hybrid_forward(x, *gu, Wu_t, Wd, d, y, y_dtype, ws, dev_status, stream));
 }
@@ -183,17 +187,18 @@ tw_status hybrid_ffn_backward(const void* x, const void* dy, const tw_hybrid* gu
                               int32_t* dev_status, cudaStream_t stream) {
   tw_status st = check_hybrid(gu);
   if (st != TW_OK) return st;
-  if (!x || !dy || !Wg_t || !Wu_t || !Wd || !dx || !dWg_t || !dWu_t || !dWd || !ws ||
+  const bool any = gu->T > 0;  // with no tokens only the weight gradients are written
+  if ((any && (!x || !dy || !dx || !ws)) || !Wg_t || !Wu_t || !Wd || !dWg_t || !dWu_t || !dWd ||
       !dtype_ok(dx_dtype))
     return TW_ERR_INVALID_ARG;
-  if ((gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
+  if ((any && gu->C_h > 0 && !gu->ell_u) || (gu->backup_cap > 0 && !gu->backup_u))
     return TW_ERR_INVALID_ARG;
   if (d <= 0) return TW_ERR_INVALID_ARG;
   if (!row_d_ok(d, gu->dtype)) return TW_ERR_UNSUPPORTED;
   const void* ptrs[] = {x, dy, Wg_t, Wu_t, Wd, dx, dWg_t, dWu_t, dWd, ws};
   for (const void* p : ptrs)
     if (!aligned16(p)) return TW_ERR_ALIGNMENT;
-  if (ws_bytes < tw::hybrid_backward_ws_bytes(gu->T, d, gu->F, gu->C_h, gu->backup_cap))
+  if (any && ws_bytes < tw::hybrid_backward_ws_bytes(gu->T, d, gu->F, gu->C_h, gu->backup_cap))
     return TW_ERR_WORKSPACE;
   return from_cuda(tw::launch_hybrid_backward(x, dy, *gu, Wg_t, Wu_t, Wd, d, l1_lambda, dx,
                                               dx_dtype, dWg_t, dWu_t, dWd, ws, ws_bytes,

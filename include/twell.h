@@ -33,7 +33,10 @@
  *             synchronising; tw_status_string names each code.
  * Limits      W == 128; 0 <= C <= 32; F % W == 0; d % 8 == 0; 8 <= d <= 2048
  *             (bf16 rows) or d <= 1024 (fp32 rows) for the fused and hybrid
- *             kernels; T >= 1.  F <= 65536 (hybrid
+ *             kernels; T >= 0.  With T == 0 the arrays sized by T (x, y, dy,
+ *             dx, the TwELL and hybrid per-token arrays, the workspaces) may
+ *             be NULL: the calls only reset spill_n / n_backup and write zero
+ *             weight gradients.  F <= 65536 (hybrid
  *             indices are uint16); for hybrid arguments F % 8 == 0 and
  *             F <= 51200.
  */

@@ -104,6 +104,19 @@ def test_fused_validation(L):
              None, None) == UNSUPPORTED
 
 
+def test_empty_batch_needs_no_token_buffers(L):
+    # T == 0: the arrays sized by T may be NULL; the fused call returns before any launch
+    tw0 = twell.TwTwellC(0, 1024, 128, 8, twell.TW_BF16, None, None, None, None, 0, None, None,
+                         FAKE)
+    assert L.twell_fused_updown(None, ctypes.byref(tw0), FAKE, FAKE, 512, None, twell.TW_F32,
+                                None, 0, None, None) == 0
+    # with tokens the same NULL buffers are rejected
+    tw1 = twell.TwTwellC(1, 1024, 128, 8, twell.TW_BF16, None, None, None, None, 0, None, None,
+                         FAKE)
+    assert L.twell_fused_updown(None, ctypes.byref(tw1), FAKE, FAKE, 512, None, twell.TW_F32,
+                                None, 0, None, None) == INVALID
+
+
 def _hy(T=256, F=1024, C_h=64, cap=32, dtype=twell.TW_BF16, base=FAKE):
     return twell.TwHybridC(T, F, C_h, dtype, base, base, base, base, base, cap, base, base, base, base)
 

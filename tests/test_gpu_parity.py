@@ -392,6 +392,32 @@ def test_hybrid_bf16_outputs_are_the_fp32_results_rounded():
         assert torch.equal(a, b)
 
 
+def test_empty_batch_through_every_entry_point():
+    d, F, C, C_h = 256, 512, 8, 16
+    rng = np.random.default_rng(14)
+    bf = lambda a: torch.from_numpy(synth.to_storage(a, synth.BF16).view(np.int16)).cuda().view(
+        torch.bfloat16)
+    x = torch.empty((0, d), dtype=torch.bfloat16, device="cuda")
+    Wg, Wu, Wd = (bf(rng.standard_normal((F, d)) / 16) for _ in range(3))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = tw.Twell(0, F, C, dtype=torch.bfloat16)
+    tw.twell_gate_gemm(x, Wg, g, None, st)
+    y = torch.empty((0, d), dtype=torch.float32, device="cuda")
+    tw.twell_fused_updown(x, g, Wu, Wd, y, tw.fused_workspace(0, d), st)
+    hy = tw.Hybrid(0, F, C_h, dtype=torch.bfloat16, backup_cap=4)
+    tw.twell_to_hybrid(g, hy, st)
+    tw.hybrid_ffn_forward(x, hy, Wu, Wd, y, dev_status=st)
+    ws = torch.empty(max(1, tw.hybrid_ffn_backward_workspace_size(0, d, F, C_h, 4)),
+                     dtype=torch.uint8, device="cuda")
+    dW = [torch.full((F, d), 7.0, dtype=torch.float32, device="cuda") for _ in range(3)]
+    tw.hybrid_ffn_backward(x, x, hy, Wg, Wu, Wd, 2e-5, y, dW[0], dW[1], dW[2], ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert int(g.spill_n.item()) == 0 and int(hy.n_backup.item()) == 0
+    for a in dW:  # no tokens: the weight gradients are zero, not left unwritten
+        assert float(a.abs().max().item()) == 0.0
+
+
 def test_hybrid_backup_capacity_overflow_is_flagged():
     w = synth.make_workload(T=256, d=128, F=512, W=128, C=8, C_h=2, dtype=synth.BF16,
                             kind="pareto", lam=2e-5, seed=11, mean_active=10.0)
