@@ -46,7 +46,7 @@
 // version by the number of row slices, not by bytes.)
 //
 // Arithmetic.  bf16 dot products run on the tensor pipe (mma.sync with a
-// diagonal-extraction layout, see dot2); the scaled-row updates widen bf16
+// diagonal-extraction layout, see dot2_issue); the scaled-row updates widen bf16
 // pairs exactly and use packed fp32x2 FMA.
 #include "tw_common.cuh"
 #include "tw_internal.h"

@@ -4,11 +4,11 @@
 //   * TwELL -> hybrid: each token row becomes a compact ELL row (global unit
 //     indices, ascending) when it has at most C_h non-zeros, otherwise a dense
 //     backup row; backup slots follow ascending token order;
-//   * hybrid forward (dense x times dense Wu sampled on the hybrid pattern,
-//     then the sparse pattern times dense Wd);
-//   * hybrid backward with the L1 term: per-token pass for dh, du, dz and dx,
-//     then weight gradients per unit from a deterministic, token-ordered
-//     transposition of the pattern (counting sort by unit; no float atomics).
+//   * hybrid forward and the per-token pass of the backward (dh, du, dz, dx
+//     with the L1 term) run on the gather engine of fused_updown.cu;
+//   * the weight gradients are summed per unit from the backward's per-entry
+//     records after a deterministic, token-ordered transposition (stable
+//     counting sort by unit; no float atomics).
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
