@@ -17,11 +17,14 @@
 // Work decomposition.  Per-token activity is very uneven (a few tokens carry
 // tens of times the median number of active units), so a token with more
 // than `part` active units is split into parts:
-//   1. plan_count_*        entries per token;
+//   1. plan_count_*        entries per token, and per-block partials;
 //   2. plan_scan_kernel    (one CTA) the part size (adapted to the total work),
 //                          partial-buffer rows for split tokens (bounded by
 //                          the workspace), one descriptor {t, first entry,
-//                          end entry, partial row} per work item;
+//                          end entry, partial row} per work item; when the
+//                          part size is the largest and every split fits,
+//                          only the block partials are scanned and
+//                          plan_write_kernel writes the same plan in parallel;
 //   3. gather_kernel       persistent teams take work items from a ticket
 //                          counter (the next ticket is fetched while the
 //                          current item runs).
@@ -62,16 +65,19 @@ constexpr int kTeam = 2;           // warps per work item
 constexpr int kTeams = 8;          // teams per CTA
 constexpr int kWarps = kTeam * kTeams;
 constexpr int kListCap = 64;       // entry window collected at a time
+constexpr int kCountBlock = 256;   // tokens per block of the count kernels
 
 enum : int { kModeTwell = 0, kModeHybFwd = 1, kModeHybBwd = 2 };
 
 // --------------------------------------------------------------- workspace --
 struct FusedWs {
-  int32_t* hdr;        // [0] item ticket, [1] number of items, [2] part size
+  int32_t* hdr;        // [0] item ticket, [1] number of items, [2] part size, [3] fast plan
   int32_t* done;       // [T] parts finished (split tokens)
   int32_t* nnz;        // [T]
   int32_t* slot_off;   // [T] first partial row of a split token, -1 if whole
   int4* item_desc;     // [max_items] {t, lo, hi, partial row or -1}
+  int4* bpart;         // [nb] per block of kCountBlock tokens: entries, split parts and items
+                       // with the largest part size; the planner's fast path scans them
   float* partial;      // [parts_cap][d]
   int parts_cap, max_items;
   size_t bytes;
@@ -94,6 +100,7 @@ FusedWs layout(void* base, int T, int d, int cap) {
   const size_t o_nnz = take(sizeof(int32_t) * (size_t)T);
   const size_t o_slot = take(sizeof(int32_t) * (size_t)T);
   const size_t o_desc = take(sizeof(int4) * (size_t)w.max_items);
+  const size_t o_bpart = take(sizeof(int4) * ((size_t)T / kCountBlock + 1));
   const size_t o_part = take(sizeof(float) * (size_t)(cap > 0 ? cap : 1) * d);
   w.bytes = off;
   if (base) {
@@ -103,6 +110,7 @@ FusedWs layout(void* base, int T, int d, int cap) {
     w.nnz = reinterpret_cast<int32_t*>(p + o_nnz);
     w.slot_off = reinterpret_cast<int32_t*>(p + o_slot);
     w.item_desc = reinterpret_cast<int4*>(p + o_desc);
+    w.bpart = reinterpret_cast<int4*>(p + o_bpart);
     w.partial = reinterpret_cast<float*>(p + o_part);
   }
   return w;
@@ -126,23 +134,56 @@ bool carve_within(void* base, int T, int d, size_t limit, FusedWs* out) {
 }
 
 // -------------------------------------------------------------------- plan --
-__global__ void plan_count_twell_kernel(int T, int K, const uint8_t* __restrict__ cnt,
-                                        int32_t* nnz) {
+// Per-block partials for the planner's fast path: entries, split parts and
+// work items of the block's tokens with the part size kPart (thread 0 writes).
+TW_DEV void count_block_partials(int n, bool valid, int4* bpart) {
+  __shared__ int red[3][kCountBlock / 32];
+  const int parts = n > kPart ? (n + kPart - 1) / kPart : 0;
+  int v[3] = {n, parts, valid ? (parts > 0 ? parts : 1) : 0};
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[i] += __shfl_xor_sync(FULL, v[i], o);
+    if (lane == 0) red[i][wid] = v[i];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int4 r = make_int4(0, 0, 0, 0);
+    for (int w2 = 0; w2 < kCountBlock / 32; ++w2) {
+      r.x += red[0][w2];
+      r.y += red[1][w2];
+      r.z += red[2][w2];
+    }
+    bpart[blockIdx.x] = r;
+  }
+}
+
+__global__ void __launch_bounds__(kCountBlock)
+    plan_count_twell_kernel(int T, int K, const uint8_t* __restrict__ cnt, int32_t* nnz,
+                            int4* bpart) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
   int s = 0;
-  for (int k = 0; k < K; ++k) s += cnt[(size_t)k * T + t];
-  nnz[t] = s;
+  if (t < T) {
+    for (int k = 0; k < K; ++k) s += cnt[(size_t)k * T + t];
+    nnz[t] = s;
+  }
+  count_block_partials(s, t < T, bpart);
 }
 
 // Hybrid rows: the row's non-zero count, or 0 for a backup row that was not
 // stored (capacity exceeded, flagged by the conversion).
-__global__ void plan_count_hybrid_kernel(int T, const int32_t* __restrict__ row_nnz,
-                                         const int32_t* __restrict__ row_slot, int cap,
-                                         int32_t* nnz) {
+__global__ void __launch_bounds__(kCountBlock)
+    plan_count_hybrid_kernel(int T, const int32_t* __restrict__ row_nnz,
+                             const int32_t* __restrict__ row_slot, int cap, int32_t* nnz,
+                             int4* bpart) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  nnz[t] = row_slot[t] >= cap ? 0 : row_nnz[t];
+  int s = 0;
+  if (t < T) {
+    s = row_slot[t] >= cap ? 0 : row_nnz[t];
+    nnz[t] = s;
+  }
+  count_block_partials(s, t < T, bpart);
 }
 
 constexpr int kScanThreads = 1024;
@@ -194,10 +235,50 @@ size_t plan_scan_smem(int T) {
 // passes read them from global memory.
 __global__ void __launch_bounds__(kScanThreads)
     plan_scan_kernel(int T, const int32_t* __restrict__ nnz, int parts_cap, int max_items,
-                     int n_teams, int32_t* slot_off, int4* item_desc, int32_t* hdr) {
+                     int n_teams, int32_t* slot_off, int4* item_desc, int32_t* hdr, int4* bpart,
+                     int nb) {
   __shared__ int warp_sums[32];
   __shared__ int part_sh;
   extern __shared__ int32_t staged[];
+  // Fast path, from the count kernels' per-block partials: when there is
+  // enough work for the largest part size and every split token fits the
+  // partial rows, the plan below would use part = kPart and split every token
+  // with more entries.  Then only the block partials are scanned here (into
+  // per-block offsets of split parts and items) and plan_write_kernel writes
+  // the same plan with one thread per token.
+  {
+    int e = 0, sp = 0, it = 0;
+    for (int b = threadIdx.x; b < nb; b += kScanThreads) {
+      const int4 v = bpart[b];
+      e += v.x;
+      sp += v.y;
+      it += v.z;
+    }
+    int te, tsp, tit;
+    block_exclusive_scan(e, warp_sums, &te);
+    block_exclusive_scan(sp, warp_sums, &tsp);
+    block_exclusive_scan(it, warp_sums, &tit);
+    if (te / (2 * n_teams) >= kPart && tsp <= parts_cap) {
+      int carry_s = 0, carry_i = 0;
+      for (int b0 = 0; b0 < nb; b0 += kScanThreads) {
+        const int b = b0 + threadIdx.x;
+        const int4 v = b < nb ? bpart[b] : make_int4(0, 0, 0, 0);
+        int ts2, ti2;
+        const int xs = block_exclusive_scan(v.y, warp_sums, &ts2);
+        const int xi = block_exclusive_scan(v.z, warp_sums, &ti2);
+        if (b < nb) bpart[b] = make_int4(carry_s + xs, carry_i + xi, 0, 0);
+        carry_s += ts2;
+        carry_i += ti2;
+      }
+      if (threadIdx.x == 0) {
+        hdr[1] = tit < max_items ? tit : max_items;
+        hdr[2] = kPart;
+        hdr[3] = 1;
+      }
+      return;
+    }
+    if (threadIdx.x == 0) hdr[3] = 0;
+  }
   const int run = (T + kScanThreads - 1) / kScanThreads;
   const int t0 = threadIdx.x * run;
   const int t1 = min(T, t0 + run);
@@ -258,6 +339,35 @@ __global__ void __launch_bounds__(kScanThreads)
     ex += parts;
   }
   if (threadIdx.x == 0) hdr[1] = tot < max_items ? tot : max_items;
+}
+
+// The fast-path plan, one thread per token: split parts and items of the
+// token from its count, block-local offsets from a block scan plus the
+// block's offsets from the planner.  The same plan as the single-CTA path
+// with part = kPart.  Does nothing unless the planner took the fast path.
+__global__ void __launch_bounds__(kCountBlock)
+    plan_write_kernel(int T, const int32_t* __restrict__ nnz, int max_items, int32_t* slot_off,
+                      int4* item_desc, const int32_t* hdr, const int4* bpart) {
+  __shared__ int warp_sums[32];
+  if (hdr[3] == 0) return;  // uniform
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n = t < T ? nnz[t] : 0;
+  const int parts = n > kPart ? (n + kPart - 1) / kPart : 0;
+  const int items = t < T ? (parts > 0 ? parts : 1) : 0;
+  int tot;
+  const int xs = block_exclusive_scan(parts, warp_sums, &tot);
+  const int xi = block_exclusive_scan(items, warp_sums, &tot);
+  if (t >= T) return;
+  const int4 off = bpart[blockIdx.x];
+  const int so = parts > 0 ? off.x + xs : -1;
+  slot_off[t] = so;
+  const int base = off.y + xi;
+  if (parts == 0) {
+    if (base < max_items) item_desc[base] = make_int4(t, 0, n, -1);
+  } else {
+    for (int q = 0; q < parts && base + q < max_items; ++q)
+      item_desc[base + q] = make_int4(t, q * kPart, min(n, (q + 1) * kPart), so + q);
+  }
 }
 
 // ------------------------------------------------------------- arithmetic --
@@ -871,9 +981,13 @@ cudaError_t run_engine(GatherArgs<Tin> a, bool out_bf16, void* base, CountFn cou
                              (int)plan_scan_smem(kScanSmemTokens));
     if (e != cudaSuccess) return e;
   }
+  const int nb = (a.T + kCountBlock - 1) / kCountBlock;
   plan_scan_kernel<<<1, kScanThreads, scan_smem, stream>>>(a.T, a.ws.nnz, a.ws.parts_cap,
                                                    a.ws.max_items, num_sms() * kTeams,
-                                                   a.ws.slot_off, a.ws.item_desc, a.ws.hdr);
+                                                   a.ws.slot_off, a.ws.item_desc, a.ws.hdr,
+                                                   a.ws.bpart, nb);
+  plan_write_kernel<<<nb, kCountBlock, 0, stream>>>(a.T, a.ws.nnz, a.ws.max_items, a.ws.slot_off,
+                                                    a.ws.item_desc, a.ws.hdr, a.ws.bpart);
   return launch_mode<Tin, MODE>(a, out_bf16, stream);
 }
 
@@ -901,7 +1015,10 @@ cudaError_t twell_fused_t(const void* x, const tw_twell& g, const void* Wu_t, co
   const int T = g.T, K = g.F / W;
   return run_engine<Tin, kModeTwell>(
       a, y_dtype == TW_BF16, base,
-      [&] { plan_count_twell_kernel<<<(T + 255) / 256, 256, 0, stream>>>(T, K, g.cnt, w.nnz); },
+      [&] {
+        plan_count_twell_kernel<<<(T + kCountBlock - 1) / kCountBlock, kCountBlock, 0, stream>>>(
+            T, K, g.cnt, w.nnz, w.bpart);
+      },
       stream);
 }
 
@@ -945,8 +1062,9 @@ cudaError_t hybrid_t(const void* xin, const tw_hybrid& h, const void* rdot, cons
   return run_engine<Tin, MODE>(
       a, out_dtype == TW_BF16, base,
       [&] {
-        plan_count_hybrid_kernel<<<(T + 255) / 256, 256, 0, stream>>>(T, h.row_nnz, h.row_slot,
-                                                                       h.backup_cap, w.nnz);
+        plan_count_hybrid_kernel<<<(T + kCountBlock - 1) / kCountBlock, kCountBlock, 0,
+                                   stream>>>(T, h.row_nnz, h.row_slot, h.backup_cap, w.nnz,
+                                             w.bpart);
       },
       stream);
 }
