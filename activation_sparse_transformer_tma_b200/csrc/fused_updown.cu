@@ -955,6 +955,115 @@ cudaError_t launch_nchw(GatherArgs<Tin> a, bool out_bf16, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Small batches (T <= kDecodeMaxT, decoding): one CTA per token, no work
+// plan.  The work per token is small and its rows come from HBM, so the
+// aim is to have as many row loads in flight as possible:
+//   warp 0 collects a window of the token's entries into shared memory;
+//   each warp takes every kDecWarps-th entry, two at a time, and forms
+//     h = g * (x_t . Wu_t[j]) with a warp reduction;
+//   each thread then accumulates its own columns of y over all entries of
+//     the window, eight rows of Wd in flight.
+// Entries are summed in their (tile-major) order, so y is deterministic.
+constexpr int kDecWarps = 8;
+constexpr int kDecodeMaxT = 16;
+
+template <typename Tin, bool kOutBf16>
+__global__ void __launch_bounds__(32 * kDecWarps) decode_kernel(const GatherArgs<Tin> a) {
+  using L = Elem<Tin>;
+  constexpr int E = L::E;
+  constexpr int P = L::P;
+  constexpr int SPAN = 32 * E;   // columns of one warp-wide slice
+  constexpr int NCH = 8;         // slices per lane: d <= 8 * SPAN (the validated maximum)
+  __shared__ TeamSmem lst;
+  __shared__ float hsh[kListCap];
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = a.d;
+  const Tin* xt = a.xin + (size_t)t * d;
+  uint4 xr[NCH];  // the whole token row in every warp, for the dot products
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const int cc = c * SPAN + lane * E;
+    xr[c] = cc < d ? __ldg(reinterpret_cast<const uint4*>(xt + cc)) : make_uint4(0, 0, 0, 0);
+  }
+  const int col = threadIdx.x * E;  // this thread's output columns
+  float2 acc[P];
+#pragma unroll
+  for (int q = 0; q < P; ++q) acc[q] = make_float2(0.f, 0.f);
+
+  for (int w0 = 0;; w0 += kListCap) {
+    if (warp == 0) {
+      const int n = collect_twell(a, t, w0, w0 + kListCap, lst, lane);
+      if (lane == 0) lst.n = n;
+    }
+    __syncthreads();
+    const int n = lst.n;
+    // h of each entry: two entries per warp at a time
+    for (int e = warp; e < n; e += 2 * kDecWarps) {
+      const int e2 = e + kDecWarps;
+      const bool two = e2 < n;
+      const uint4* r0 = reinterpret_cast<const uint4*>(a.rdot + (size_t)lst.j[e] * d);
+      const uint4* r1 = reinterpret_cast<const uint4*>(a.rdot + (size_t)(two ? lst.j[e2] : 0) * d);
+      uint4 w0v[NCH], w1v[NCH];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        const int cc = c * SPAN + lane * E;
+        w0v[c] = cc < d ? __ldg(r0 + cc / E) : make_uint4(0, 0, 0, 0);
+        w1v[c] = cc < d && two ? __ldg(r1 + cc / E) : make_uint4(0, 0, 0, 0);
+      }
+      float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        L::dot(xr[c], w0v[c], p0);
+        L::dot(xr[c], w1v[c], p1);
+      }
+      const float u0 = warp_sum((p0[0] + p0[1]) + (p0[2] + p0[3]));
+      const float u1 = warp_sum((p1[0] + p1[1]) + (p1[2] + p1[3]));
+      if (lane == 0) {
+        hsh[e] = lst.g[e] * u0;
+        if (two) hsh[e2] = lst.g[e2] * u1;
+      }
+    }
+    __syncthreads();
+    // y columns of this thread over the window's entries
+    if (col < d) {
+      for (int e0 = 0; e0 < n; e0 += 8) {
+        uint4 w[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          w[u] = e0 + u < n ? __ldg(reinterpret_cast<const uint4*>(a.rax1 + (size_t)lst.j[e0 + u] * d + col))
+                            : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (e0 + u >= n) break;
+          const float h = hsh[e0 + u];
+          const float2 hh = make_float2(h, h);
+          float2 wv[P];
+          L::pairs(w[u], wv);
+#pragma unroll
+          for (int q = 0; q < P; ++q) acc[q] = __ffma2_rn(hh, wv[q], acc[q]);
+        }
+      }
+    }
+    __syncthreads();  // the window's list and h are reused
+    if (n < kListCap) break;
+  }
+  if (col < d) {
+    if (kOutBf16) {
+      uint16_t* yt = static_cast<uint16_t*>(a.out) + (size_t)t * d + col;
+#pragma unroll
+      for (int q = 0; q < P; ++q)
+        reinterpret_cast<uint32_t*>(yt)[q] = pack_bf16x2(acc[q].x, acc[q].y);
+    } else {
+      float* yt = static_cast<float*>(a.out) + (size_t)t * d + col;
+#pragma unroll
+      for (int q = 0; q < P / 2; ++q)
+        reinterpret_cast<float4*>(yt)[q] = make_float4(acc[2 * q].x, acc[2 * q].y,
+                                                       acc[2 * q + 1].x, acc[2 * q + 1].y);
+    }
+  }
+}
+
 template <typename Tin, int MODE>
 cudaError_t launch_mode(const GatherArgs<Tin>& a, bool out_bf16, cudaStream_t stream) {
   // chunks of one 16-byte slice per lane, split over the kTeam warps
@@ -1013,6 +1122,14 @@ cudaError_t twell_fused_t(const void* x, const tw_twell& g, const void* Wu_t, co
   a.status = status;
   a.ws = w;
   const int T = g.T, K = g.F / W;
+  // A handful of tokens: one CTA per token, no plan.  Above that the planned
+  // path wins, because it splits the heavy tokens of the batch over teams
+  // (at T = 64 of the 2B workload: 115 us planned, 282 us one CTA per token).
+  if (T <= kDecodeMaxT) {
+    auto kern = y_dtype == TW_BF16 ? decode_kernel<Tin, true> : decode_kernel<Tin, false>;
+    kern<<<T, 32 * kDecWarps, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
   return run_engine<Tin, kModeTwell>(
       a, y_dtype == TW_BF16, base,
       [&] {

@@ -90,9 +90,11 @@ def test_bf16_gate_and_fused_small(T, d, F, C, kind, ma):
     check_y(f64(y), w64, rows, TOL[synth.BF16])
 
 
-@pytest.mark.parametrize("d", [320, 256])  # CUDA-core gather engine / tensor-core path
-def test_bf16_output_y(d):
-    w = synth.make_workload(T=300, d=d, F=640, W=128, C=8, dtype=synth.BF16, kind="dead20",
+# planned gather engine with both slice widths, and the one-CTA-per-token
+# small-batch kernel (T <= 16)
+@pytest.mark.parametrize("d,T", [(320, 300), (256, 300), (256, 12)])
+def test_bf16_output_y(d, T):
+    w = synth.make_workload(T=T, d=d, F=640, W=128, C=8, dtype=synth.BF16, kind="dead20",
                             mean_active=29.0, seed=620)
     _, g, gd, y, st = run_forward(w, y_dtype=torch.bfloat16)
     _, _, _, y32, _ = run_forward(w)
@@ -100,13 +102,13 @@ def test_bf16_output_y(d):
     # both paths are deterministic, and the bf16 output is the fp32 result rounded once
     assert torch.equal(y32, y32b)
     assert torch.equal(y, y32.to(torch.bfloat16))
-    check_y(f64(y), widened(w), np.arange(300, dtype=np.int32), TOL[synth.BF16],
+    check_y(f64(y), widened(w), np.arange(T, dtype=np.int32), TOL[synth.BF16],
             elem_rel=2.0 ** -8)
 
 
-@pytest.mark.parametrize("C", [16, 2])
-def test_fp32_tiny_config(C):
-    w = synth.make_workload("tiny_fp32")
+@pytest.mark.parametrize("C,T", [(16, None), (2, None), (2, 10)])  # T=10: small-batch kernel
+def test_fp32_tiny_config(C, T):
+    w = synth.make_workload("tiny_fp32") if T is None else synth.make_workload("tiny_fp32", T=T)
     dev, g, gd, y, st = run_forward(w, C=C)
     assert int(st.item()) == 0
     w64 = widened(w)
