@@ -109,6 +109,9 @@ tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int32_t d,
   if (T == 0) return from_cuda(cudaMemsetAsync(out->spill_n, 0, sizeof(int32_t), stream));
   if (dtype == TW_BF16) {
     if (d < 64) return TW_ERR_UNSUPPORTED;
+    if (T <= tw::kFewMaxT)
+      return from_cuda(tw::launch_gate_twell_few(x, Wg_t, T, d, F, *out, g_dense_dump,
+                                                 dev_status, stream));
     return from_cuda(tw::launch_gate_twell_tc(x, Wg_t, T, d, F, *out, g_dense_dump, dev_status,
                                               stream));
   }

@@ -28,9 +28,11 @@
 //   3. gather_kernel       persistent teams take work items from a ticket
 //                          counter (the next ticket is fetched while the
 //                          current item runs).
-// A split token's parts write fp32 partial rows to the workspace; the part
-// that finishes last (atomic counter per token) sums them in part order, so
-// the output is deterministic.
+// A split token's parts are added up a binary tree over the part index
+// through fp32 partial rows in the workspace (one arrival counter per tree
+// node); the tree's shape is fixed by the number of parts, so the output is
+// deterministic, and its depth, not the number of parts, sets the time the
+// last part spends on the sum.
 //
 // Teams.  An item is processed by a team of kTeam warps; warp w of the team
 // owns one contiguous range of the d columns (the token's row and the output
@@ -72,7 +74,7 @@ enum : int { kModeTwell = 0, kModeHybFwd = 1, kModeHybBwd = 2 };
 // --------------------------------------------------------------- workspace --
 struct FusedWs {
   int32_t* hdr;        // [0] item ticket, [1] number of items, [2] part size, [3] fast plan
-  int32_t* done;       // [T] parts finished (split tokens)
+  int32_t* done;       // [parts_cap] arrivals per internal node of a split token's sum tree
   int32_t* nnz;        // [T]
   int32_t* slot_off;   // [T] first partial row of a split token, -1 if whole
   int4* item_desc;     // [max_items] {t, lo, hi, partial row or -1}
@@ -95,7 +97,7 @@ FusedWs layout(void* base, int T, int d, int cap) {
   size_t off = 0;
   auto take = [&](size_t b) { size_t o = off; off = al256(off + b); return o; };
   const size_t o_hdr = take(4 * sizeof(int32_t));
-  const size_t o_done = take(sizeof(int32_t) * (size_t)T);
+  const size_t o_done = take(sizeof(int32_t) * (size_t)(cap > 0 ? cap : 1));
   w.zero_bytes = off;
   const size_t o_nnz = take(sizeof(int32_t) * (size_t)T);
   const size_t o_slot = take(sizeof(int32_t) * (size_t)T);
@@ -588,7 +590,7 @@ struct TeamSmem {
   float red[2][kTeam][2];  // partial dot products of an entry pair, double-buffered
   int4 desc[2];           // current item, double-buffered by item parity
   int n;                  // entries in the current window
-  int prev;               // split-token finisher broadcast
+  int prev;               // arrival count at a sum-tree node, broadcast to the team
 };
 
 // TwELL: the entries of token t with ordinal in [lo, hi) (tile-major order,
@@ -889,54 +891,88 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
     }
 
     // ------------------------------------------------------------ output --
-    const bool split = prow >= 0;
-    float* out_row = split ? a.ws.partial + (size_t)prow * d : nullptr;
-#pragma unroll
-    for (int c = 0; c < NCHW; ++c) {
-      const int col = c0 + c * SPAN + lane * E;
-      if (col >= d) continue;
-      if (split || !kOutBf16) {
-        float* dst = split ? out_row + col : static_cast<float*>(a.out) + (size_t)t * d + col;
-#pragma unroll
-        for (int q = 0; q < P / 2; ++q) {
-          const float4 v = make_float4(acc[c][2 * q].x, acc[c][2 * q].y, acc[c][2 * q + 1].x,
-                                       acc[c][2 * q + 1].y);
-          if (split)
-            reinterpret_cast<float4*>(dst)[q] = v;
-          else
-            __stcs(reinterpret_cast<float4*>(dst) + q, v);
-        }
-      } else {
-        uint16_t* yt = static_cast<uint16_t*>(a.out) + (size_t)t * d + col;
-#pragma unroll
-        for (int q = 0; q < P; ++q)
-          reinterpret_cast<uint32_t*>(yt)[q] = pack_bf16x2(acc[c][q].x, acc[c][q].y);
-      }
-    }
-    if (split) {
-      // the last part to finish sums the partial rows in part order
-      __threadfence();
-      team_bar(team);  // both halves of this part's row are written
+    // A split token's parts are summed up a binary tree over the part index:
+    // node [L, L + 2s) adds its children [L, L + s) and [L + s, L + 2s), and
+    // a node's sum is published in the partial row of its first part L.  Of
+    // two children, the one that finishes second (arrival counter per
+    // internal node, keyed by its right child's first part) loads the
+    // other's row into its registers and goes up; the first one stops.
+    // Floating-point addition is commutative, so every node's sum, and y, is
+    // the same whichever part finishes first.  The team that completes the
+    // root writes the output row.
+    bool complete = true;
+    if (prow >= 0) {
       const int part = a.ws.hdr[2];
       const int parts = (a.ws.nnz[t] + part - 1) / part;
-      if (leader && lane == 0) ts.prev = atomicAdd(&a.ws.done[t], 1);
-      team_bar(team);
-      if (ts.prev == parts - 1) {
+      const int leaf = lo / part;
+      const int row0 = prow - leaf;  // the token's first partial row
+      int node = leaf;
+      for (int span = 1; span < parts; span *= 2) {
+        const int left = node & ~(2 * span - 1);
+        const int right = left + span;
+        if (right >= parts) {  // no right sibling: the node is its own parent
+          node = left;
+          continue;
+        }
+        float* mine = a.ws.partial + (size_t)(row0 + node) * d;
+#pragma unroll
+        for (int c = 0; c < NCHW; ++c) {
+          const int col = c0 + c * SPAN + lane * E;
+          if (col >= d) continue;
+#pragma unroll
+          for (int q = 0; q < P / 2; ++q)
+            reinterpret_cast<float4*>(mine + col)[q] =
+                make_float4(acc[c][2 * q].x, acc[c][2 * q].y, acc[c][2 * q + 1].x,
+                            acc[c][2 * q + 1].y);
+        }
         __threadfence();
-        const float* part0 = a.ws.partial + (size_t)(prow - lo / part) * d;
-        for (int col = c0 + lane * 4; col < c0 + my_cols; col += 128) {
-          float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int q = 0; q < parts; ++q) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(part0 + (size_t)q * d + col));
-            sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        team_bar(team);  // both halves of the row are written
+        if (leader && lane == 0) ts.prev = atomicAdd(&a.ws.done[row0 + right], 1);
+        team_bar(team);
+        if (ts.prev == 0) {  // the sibling is still running; it goes on
+          complete = false;
+          break;
+        }
+        __threadfence();
+        const float* other = a.ws.partial + (size_t)(row0 + (node == left ? right : left)) * d;
+        float4 sib[NCHW][P / 2];
+#pragma unroll
+        for (int c = 0; c < NCHW; ++c) {
+          const int col = c0 + c * SPAN + lane * E;
+#pragma unroll
+          for (int q = 0; q < P / 2; ++q)
+            sib[c][q] = col < d ? __ldcg(reinterpret_cast<const float4*>(other + col) + q)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int c = 0; c < NCHW; ++c)
+#pragma unroll
+          for (int q = 0; q < P / 2; ++q) {
+            acc[c][2 * q].x += sib[c][q].x;
+            acc[c][2 * q].y += sib[c][q].y;
+            acc[c][2 * q + 1].x += sib[c][q].z;
+            acc[c][2 * q + 1].y += sib[c][q].w;
           }
-          if (kOutBf16) {
-            uint16_t* yt = static_cast<uint16_t*>(a.out) + (size_t)t * d + col;
-            reinterpret_cast<uint2*>(yt)[0] = make_uint2(pack_bf16x2(sum.x, sum.y),
-                                                         pack_bf16x2(sum.z, sum.w));
-          } else {
-            *reinterpret_cast<float4*>(static_cast<float*>(a.out) + (size_t)t * d + col) = sum;
-          }
+        node = left;
+      }
+    }
+    if (complete) {
+#pragma unroll
+      for (int c = 0; c < NCHW; ++c) {
+        const int col = c0 + c * SPAN + lane * E;
+        if (col >= d) continue;
+        if (!kOutBf16) {
+          float* dst = static_cast<float*>(a.out) + (size_t)t * d + col;
+#pragma unroll
+          for (int q = 0; q < P / 2; ++q)
+            __stcs(reinterpret_cast<float4*>(dst) + q,
+                   make_float4(acc[c][2 * q].x, acc[c][2 * q].y, acc[c][2 * q + 1].x,
+                               acc[c][2 * q + 1].y));
+        } else {
+          uint16_t* yt = static_cast<uint16_t*>(a.out) + (size_t)t * d + col;
+#pragma unroll
+          for (int q = 0; q < P; ++q)
+            reinterpret_cast<uint32_t*>(yt)[q] = pack_bf16x2(acc[c][q].x, acc[c][q].y);
         }
       }
     }

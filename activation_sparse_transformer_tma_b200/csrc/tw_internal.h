@@ -18,6 +18,12 @@ constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, int F,
                                  const tw_twell& out, void* dump, int32_t* status,
                                  cudaStream_t stream);
+// The same GEMM and packing for small batches (1 <= T <= kFewMaxT): units on
+// the MMA's M side, the reduction over d split across a thread-block cluster.
+constexpr int kFewMaxT = 64;
+cudaError_t launch_gate_twell_few(const void* x, const void* Wg_t, int T, int d, int F,
+                                  const tw_twell& out, void* dump, int32_t* status,
+                                  cudaStream_t stream);
 // fp32 CUDA-core gate with the same TwELL packing.
 cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int d, int F,
                                   const tw_twell& out, float* dump, int32_t* status,

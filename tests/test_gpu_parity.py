@@ -153,6 +153,52 @@ def test_ffn_2b_full_size():
     check_y(f64(y), w64, rows, TOL[synth.BF16])
 
 
+# Small batches (T <= 64) take the cluster split-K gate; the cases cover
+# cluster sizes 8, 8 with uneven k-block shares (d = 520), 2 (partials of
+# 48 tokens), 1 (more tiles than SMs), C = 0 and the largest C.  The last
+# case splits every token into tens of parts of the fused kernel.
+FEW = [
+    # T, d, F, C, kind, mean_active
+    (1, 1024, 1024, 8, "zipf", 29.0),
+    (5, 520, 2048, 2, "dead20", 60.0),
+    (33, 2048, 4096, 8, "zipf", 29.0),
+    (17, 256, 19200, 8, "zipf", 29.0),
+    (64, 128, 640, 0, "dead20", 29.0),
+    (16, 2048, 1280, 32, "zipf", 40.0),
+    (20, 512, 8192, 8, "zipf", 400.0),  # dozens of parts per token: deep sum trees
+]
+
+
+@pytest.mark.parametrize("T,d,F,C,kind,ma", FEW)
+def test_small_batch_gate(T, d, F, C, kind, ma):
+    w = synth.make_workload(T=T, d=d, F=F, W=128, C=C, dtype=synth.BF16, kind=kind,
+                            mean_active=ma, seed=T * 7 + d)
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    w64 = widened(w)
+    g64 = f64(gd)
+    rows = np.arange(T, dtype=np.int32)
+    check_gate_values(g64, w64["x"], w64["Wg_t"], rows)
+    assert_twell_matches_oracle(g, g64)
+    check_y(f64(y), w64, rows, TOL[synth.BF16])
+    # the same launch without the dense dump writes the same TwELL
+    _, g2, _, _, _ = run_forward(w, dump=False)
+    assert torch.equal(g.cnt, g2.cnt) and torch.equal(g.spill_n, g2.spill_n)
+    if C > 0:
+        assert torch.equal(g.val, g2.val) and torch.equal(g.idx, g2.idx)
+
+
+def test_small_batch_spill_capacity_overflow_is_flagged():
+    w = synth.make_workload(T=40, d=256, F=512, W=128, C=2, dtype=synth.BF16, kind="dead20",
+                            mean_active=60.0, seed=41)
+    _, g, gd, y, st = run_forward(w, spill_cap=4)
+    assert int(g.spill_n.item()) > 4
+    assert "TW_ERR_SPILL_CAPACITY" in tw.status_bits(st)
+    ref = oracle.twell_encode(f64(gd), 128, 2)
+    assert np.array_equal(raw(g.cnt), ref["cnt"])
+    assert int(g.spill_n.item()) == ref["n_spill"]
+
+
 @pytest.mark.parametrize("T", [1, 8, 64])
 def test_decode_sizes(T):
     w = synth.make_workload("decode_2b", T=T)
