@@ -140,7 +140,9 @@ typedef struct {
  * z = x Wg accumulated in fp32 and g rounded to out->dtype, packed straight
  * into *out by the matmul's epilogue.  x [T][d] and Wg_t [F][d] have `dtype`,
  * which must equal out->dtype.  bf16 runs on the tcgen05 tensor cores fed by
- * TMA; fp32 runs at full fp32 precision on the CUDA cores.  out->T, out->F
+ * TMA (for T <= 64 with the d reduction split over a thread-block cluster,
+ * summed in a fixed order); fp32 runs at full fp32 precision on the CUDA
+ * cores.  out->T, out->F
  * must equal T, F.  g_dense_dump, if not NULL, receives the dense rounded g
  * [T][F] (dtype) -- a test aid; pass NULL for speed.
  */
