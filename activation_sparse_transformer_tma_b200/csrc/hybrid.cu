@@ -91,61 +91,73 @@ struct HView {
   V* backup_u;
 };
 
-// Enumerates the active entries of token t in ascending unit order, 32 at a
-// time.  fn(valid, j, g, pos, is_ell, rank) receives one lane-distributed
-// chunk; pos indexes ell_* (ELL row) or backup_* (backup row); rank is the
-// entry's position among the row's non-zeros.  Rows whose backup slot was
-// dropped for lack of capacity have no entries.
-template <typename T, class Fn>
-TW_DEV void for_each_chunk(const HView<T>& h, int t, int slot, int nnz, int lane, Fn&& fn);
-
-template <typename T, class Fn>
-TW_DEV void for_each_chunk(const HView<T>& h, int t, int lane, Fn&& fn) {
-  for_each_chunk<T>(h, t, h.row_slot[t], h.row_nnz[t], lane, fn);
+// Bit i set when value i of the 16-byte chunk r is non-zero (as a float
+// compare would say: -0 is zero, NaN is not).
+template <typename T>
+TW_DEV unsigned nonzero_mask(const uint4& r) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+  unsigned m = 0;
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m |= ((w[i] & 0x7FFFu) != 0u ? 1u : 0u) << (2 * i);
+      m |= ((w[i] & 0x7FFF0000u) != 0u ? 1u : 0u) << (2 * i + 1);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m |= ((w[i] & 0x7FFFFFFFu) != 0u ? 1u : 0u) << i;
+  }
+  return m;
 }
 
-// The same with the row's slot and count already loaded.
-template <typename T, class Fn>
-TW_DEV void for_each_chunk(const HView<T>& h, int t, int slot, int nnz, int lane, Fn&& fn) {
+constexpr int kDenseGroup = 8;  // 16-byte chunks per lane loaded together
+
+// Enumerates the active entries of token t in ascending unit order.
+//  * ELL row: ell_fn(valid, j, rank) once per lane for 32 entries at a time.
+//  * backup row: dense_fn(cl, mask, rank0) for this lane's V = 16 / sizeof(T)
+//    columns [cl, cl + V) that hold a non-zero: bit i of mask marks column
+//    cl + i, whose rank among the row's non-zeros is
+//    rank0 + popc(mask & ((1 << i) - 1)).  The row is read kDenseGroup
+//    chunks per lane at a time (one load latency per group, not per chunk);
+//    ranks come from a warp scan of the per-lane counts.
+// Rows whose backup slot was dropped for lack of capacity have no entries.
+template <typename T, class EllFn, class DenseFn>
+TW_DEV void for_each_chunk(const HView<T>& h, int t, int slot, int nnz, int lane, EllFn&& ell_fn,
+                           DenseFn&& dense_fn) {
   if (slot < 0) {
     for (int s0 = 0; s0 < nnz; s0 += 32) {
       const int s = s0 + lane;
       const bool v = s < nnz;
       const size_t pos = (size_t)t * h.C_h + (v ? s : 0);
       const int j = v ? (int)h.ell_idx[pos] : 0;
-      const float g = v ? ld_scalar<T>(h.ell_g, pos) : 0.f;
-      fn(v, j, g, pos, true, s);
+      ell_fn(v, j, s);
     }
   } else if (slot < h.backup_cap) {
-    // dense row: 16-byte loads (V values per lane), ranks from a warp scan of
-    // the per-lane non-zero counts; fn is called for the non-zeros only
     constexpr int V = 16 / (int)sizeof(T);
     const T* row = h.backup_g + (size_t)slot * h.F;
     int base = 0;
-#pragma unroll 2
-    for (int c0 = 0; c0 < h.F; c0 += 32 * V) {
-      const int cl = c0 + lane * V;
-      float v[V];
-      load_vec<T>(row, cl, h.F, v);
-      unsigned mask = 0;
+    for (int c0 = 0; c0 < h.F; c0 += 32 * V * kDenseGroup) {
+      uint4 r[kDenseGroup];
 #pragma unroll
-      for (int i = 0; i < V; ++i) mask |= (v[i] != 0.f ? 1u : 0u) << i;
-      const int nz = __popc(mask);
-      int incl = nz;
+      for (int q = 0; q < kDenseGroup; ++q) {
+        const int cl = c0 + (q * 32 + lane) * V;
+        r[q] = cl < h.F ? *reinterpret_cast<const uint4*>(row + cl) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(FULL, incl, o);
-        if (lane >= o) incl += u;
+      for (int q = 0; q < kDenseGroup; ++q) {
+        const int cl = c0 + (q * 32 + lane) * V;
+        const unsigned mask = nonzero_mask<T>(r[q]);
+        const int nz = __popc(mask);
+        int incl = nz;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(FULL, incl, o);
+          if (lane >= o) incl += u;
+        }
+        const int total = __shfl_sync(FULL, incl, 31);
+        if (mask != 0u) dense_fn(cl, mask, base + incl - nz);
+        base += total;
       }
-      const int total = __shfl_sync(FULL, incl, 31);
-      unsigned m = mask;
-      while (m) {
-        const int i = __ffs(m) - 1;
-        m &= m - 1;
-        fn(true, cl + i, v[i], (size_t)slot * h.F + cl + i, false,
-           base + incl - nz + __popc(mask & ((1u << i) - 1u)));
-      }
-      base += total;
     }
   }
 }
@@ -190,7 +202,32 @@ __global__ void __launch_bounds__(256)
       if (lane >= o) incl += v;
     }
     const int excl = incl - n;
-    unsigned act = __ballot_sync(FULL, n > 0);
+    // tiles within capacity: each lane copies its own tile's slots, eight
+    // loads in flight before the stores
+    if (n > 0 && n <= C) {
+      const size_t kt = (size_t)k * Tn + t;
+      const size_t q0 = rbase + pos + excl;
+      for (int s0 = 0; s0 < n; s0 += 8) {
+        T v[8];
+        uint8_t ix[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (s0 + i < n) {
+            v[i] = val[kt * C + s0 + i];
+            ix[i] = idx[kt * C + s0 + i];
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (s0 + i < n) {
+            ell_g[q0 + s0 + i] = v[i];
+            ell_idx[q0 + s0 + i] = (uint16_t)(k * W + ix[i]);
+          }
+        }
+      }
+    }
+    // overflowing tiles: the warp reads each one's spilled segment
+    unsigned act = __ballot_sync(FULL, n > C);
     while (act) {
       const int b = __ffs(act) - 1;
       act &= act - 1;
@@ -198,12 +235,7 @@ __global__ void __launch_bounds__(256)
       const int p0 = pos + __shfl_sync(FULL, excl, b);
       const int kk = kb + b;
       const size_t kt = (size_t)kk * Tn + t;
-      if (nk <= C) {
-        if (lane < nk) {
-          ell_g[rbase + p0 + lane] = val[kt * C + lane];
-          ell_idx[rbase + p0 + lane] = (uint16_t)(kk * W + idx[kt * C + lane]);
-        }
-      } else {
+      {
         const int ref = spill_ref[kt];
         if (ref < 0 || ref >= spill_cap) {
           // Dropped spill entry: only the C slots are known.
@@ -331,9 +363,22 @@ __global__ void __launch_bounds__(256)
       ref = spill_ref[kt];
       if (ref >= spill_cap) ref = -1;
     }
-    if (n > 0 && ref < 0) {
+    if (n > 0 && ref < 0) {  // the slots, eight loads in flight before the stores
       const int m = n < C ? n : C;
-      for (int s2 = 0; s2 < m; ++s2) row[k * W + idx[kt * C + s2]] = val[kt * C + s2];
+      for (int s0 = 0; s0 < m; s0 += 8) {
+        T v[8];
+        uint8_t ix[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (s0 + i < m) {
+            v[i] = val[kt * C + s0 + i];
+            ix[i] = idx[kt * C + s0 + i];
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (s0 + i < m) row[k * W + ix[i]] = v[i];
+      }
     }
     unsigned sp = __ballot_sync(FULL, ref >= 0);
     while (sp) {
@@ -396,9 +441,16 @@ TW_DEV void warp_unit_hist(const HView<T>& h, uint8_t* hist, int b, int warp, in
     if (t >= h.T) break;
     const int slot = __shfl_sync(FULL, mslot, k), nnz = __shfl_sync(FULL, mnnz, k);
     // the units of one row are distinct, so these increments never collide
-    for_each_chunk<T>(h, t, slot, nnz, lane, [&](bool v, int j, float, size_t, bool, int) {
-      if (v) hist[j] = (uint8_t)(hist[j] + 1);
-    });
+    for_each_chunk<T>(
+        h, t, slot, nnz, lane,
+        [&](bool v, int j, int) {
+          if (v) hist[j] = (uint8_t)(hist[j] + 1);
+        },
+        [&](int cl, unsigned mask, int) {
+#pragma unroll
+          for (int i = 0; i < 16 / (int)sizeof(T); ++i)
+            if ((mask >> i) & 1u) hist[cl + i] = (uint8_t)(hist[cl + i] + 1);
+        });
     __syncwarp();
   }
 }
@@ -470,13 +522,34 @@ __global__ void __launch_bounds__(32 * TB_WARPS)
     if (t >= h.T) break;
     const int ebase = __shfl_sync(FULL, mbase, k);
     const int slot = __shfl_sync(FULL, mslot, k), nnz = __shfl_sync(FULL, mnnz, k);
-    for_each_chunk<T>(h, t, slot, nnz, lane, [&](bool v, int j, float, size_t, bool, int rank) {
-      if (v) {
-        const int o = mine[j];
-        mine[j] = (uint8_t)(o + 1);
-        list[unit_off[j] + cnt[(size_t)b * h.F + j] + o] = ebase + rank;
-      }
-    });
+    for_each_chunk<T>(
+        h, t, slot, nnz, lane,
+        [&](bool v, int j, int rank) {
+          if (v) {
+            const int o = mine[j];
+            mine[j] = (uint8_t)(o + 1);
+            list[unit_off[j] + cnt[(size_t)b * h.F + j] + o] = ebase + rank;
+          }
+        },
+        [&](int cl, unsigned mask, int rank0) {
+          // the places of this lane's entries first (independent loads), then
+          // the per-warp offsets and the stores
+          constexpr int V = 16 / (int)sizeof(T);
+          int place[V];
+#pragma unroll
+          for (int i = 0; i < V; ++i)
+            place[i] = (mask >> i) & 1u ? unit_off[cl + i] + cnt[(size_t)b * h.F + cl + i] : 0;
+          int rank = rank0;
+#pragma unroll
+          for (int i = 0; i < V; ++i) {
+            if ((mask >> i) & 1u) {
+              const int o = mine[cl + i];
+              mine[cl + i] = (uint8_t)(o + 1);
+              list[place[i] + o] = ebase + rank;
+              ++rank;
+            }
+          }
+        });
     __syncwarp();
   }
 }
