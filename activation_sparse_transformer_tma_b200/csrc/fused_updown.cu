@@ -1160,7 +1160,7 @@ cudaError_t twell_fused_t(const void* x, const tw_twell& g, const void* Wu_t, co
   const int T = g.T, K = g.F / W;
   // A handful of tokens: one CTA per token, no plan.  Above that the planned
   // path wins, because it splits the heavy tokens of the batch over teams
-  // (at T = 64 of the 2B workload: 115 us planned, 282 us one CTA per token).
+  // (at T = 64 of the 2B workload: 50 us planned, 282 us one CTA per token).
   if (T <= kDecodeMaxT) {
     auto kern = y_dtype == TW_BF16 ? decode_kernel<Tin, true> : decode_kernel<Tin, false>;
     kern<<<T, 32 * kDecWarps, 0, stream>>>(a);

@@ -380,12 +380,27 @@ __global__ void __launch_bounds__(256)
           if (s0 + i < m) row[k * W + ix[i]] = v[i];
       }
     }
+    // spilled tiles: the warp copies four segments at a time, all loads first
     unsigned sp = __ballot_sync(FULL, ref >= 0);
     while (sp) {
-      const int src = __ffs(sp) - 1;
-      sp &= sp - 1;
-      const int rb = __shfl_sync(FULL, ref, src);
-      for (int c = lane; c < W; c += 32) row[(kb + src) * W + c] = spill_val[(size_t)rb * W + c];
+      int src[4], rb[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        src[q] = sp ? __ffs(sp) - 1 : -1;
+        if (sp) sp &= sp - 1;
+        rb[q] = __shfl_sync(FULL, ref, src[q] < 0 ? 0 : src[q]);
+      }
+      T v[4][W / 32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 0; c < W / 32; ++c)
+          if (src[q] >= 0) v[q][c] = spill_val[(size_t)rb[q] * W + c * 32 + lane];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 0; c < W / 32; ++c)
+          if (src[q] >= 0) row[(kb + src[q]) * W + c * 32 + lane] = v[q][c];
     }
   }
 }
@@ -415,7 +430,7 @@ constexpr int TB = TB_WARPS * TB_TOK;    // tokens per block
 static_assert((TB_WARPS - 1) * TB_TOK < 256, "per-warp offsets must fit in uint8");
 
 // Shared memory of the count and fill kernels: TB_WARPS x F uint8.
-inline size_t tb_hist_bytes(int F) { return (size_t)TB_WARPS * F; }
+__host__ __device__ inline size_t tb_hist_bytes(int F) { return (size_t)TB_WARPS * F; }
 
 // Per-warp histogram of the units of the warp's tokens (zeroed first).
 // Slot and count of the warp's TB_TOK tokens, loaded in one round (lane k
@@ -493,16 +508,28 @@ __global__ void hyb_colscan_kernel(int nb, int F, int32_t* cnt, int32_t* unit_to
 
 // Fill the unit-major list with token-major record indices, tokens ascending
 // within each unit.
-template <typename T>
+// With kSmemBase the block's first list position of every unit,
+// unit_off[j] + cnt[b][j], is staged in shared memory behind the histograms,
+// so placing an entry needs no global load.
+template <typename T, bool kSmemBase>
 __global__ void __launch_bounds__(32 * TB_WARPS)
     hyb_fill_kernel(const HView<T> h, int nb, const int32_t* cnt, const int32_t* unit_off,
                     const int32_t* e0, int32_t* list) {
   extern __shared__ uint8_t hist[];  // [TB_WARPS][F] -> per-warp offsets inside the block
+  int32_t* bases = reinterpret_cast<int32_t*>(hist + tb_hist_bytes(h.F));  // [F] if kSmemBase
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* mine = hist + (size_t)warp * h.F;
+  if (kSmemBase) {
+#pragma unroll 8
+    for (int j = threadIdx.x; j < h.F; j += blockDim.x)
+      bases[j] = unit_off[j] + cnt[(size_t)b * h.F + j];
+  }
   warp_unit_hist<T>(h, mine, b, warp, lane);
   __syncthreads();
+  auto base_of = [&](int j) {
+    return kSmemBase ? bases[j] : unit_off[j] + cnt[(size_t)b * h.F + j];
+  };
   for (int j = threadIdx.x; j < h.F; j += blockDim.x) {
     int r = 0;
 #pragma unroll
@@ -528,7 +555,7 @@ __global__ void __launch_bounds__(32 * TB_WARPS)
           if (v) {
             const int o = mine[j];
             mine[j] = (uint8_t)(o + 1);
-            list[unit_off[j] + cnt[(size_t)b * h.F + j] + o] = ebase + rank;
+            list[base_of(j) + o] = ebase + rank;
           }
         },
         [&](int cl, unsigned mask, int rank0) {
@@ -538,7 +565,7 @@ __global__ void __launch_bounds__(32 * TB_WARPS)
           int place[V];
 #pragma unroll
           for (int i = 0; i < V; ++i)
-            place[i] = (mask >> i) & 1u ? unit_off[cl + i] + cnt[(size_t)b * h.F + cl + i] : 0;
+            place[i] = (mask >> i) & 1u ? base_of(cl + i) : 0;
           int rank = rank0;
 #pragma unroll
           for (int i = 0; i < V; ++i) {
@@ -684,7 +711,9 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
   if (!attr_set) {
     cudaFuncSetAttribute(hyb_count_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          200 * 1024);
-    cudaFuncSetAttribute(hyb_fill_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(hyb_fill_kernel<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         200 * 1024);
+    cudaFuncSetAttribute(hyb_fill_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          200 * 1024);
     attr_set = true;
   }
@@ -700,8 +729,13 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
   hyb_colscan_kernel<<<(gu.F + 255) / 256, 256, 0, s>>>(nb, gu.F, w.cnt, w.unit_total);
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.unit_total, 0, w.unit_off, nullptr, 0,
                                          nullptr, status);
-  hyb_fill_kernel<T><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt, w.unit_off, w.e0,
-                                                          w.list);
+  const size_t base_bytes = sizeof(int32_t) * (size_t)gu.F;
+  if (hist_bytes + base_bytes <= 200 * 1024)
+    hyb_fill_kernel<T, true><<<nb, 32 * TB_WARPS, hist_bytes + base_bytes, s>>>(
+        h, nb, w.cnt, w.unit_off, w.e0, w.list);
+  else
+    hyb_fill_kernel<T, false><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt, w.unit_off,
+                                                                   w.e0, w.list);
   hyb_wgrad_kernel<T><<<gu.F, 256, 0, s>>>(gu.F, d, static_cast<const T*>(x),
                                            static_cast<const T*>(dy), w.unit_off, w.list, w.pay,
                                            dWg_t, dWu_t, dWd);
