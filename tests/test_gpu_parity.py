@@ -393,6 +393,16 @@ def test_hybrid_small_ragged():
     assert 0 < got["n_backup"] < 700
 
 
+def test_hybrid_wide_rows():
+    # 4 * F bytes of per-warp histograms plus 4 * F bytes of list positions
+    # exceed the transposition's shared-memory budget at F = 26624, so the
+    # fill reads the positions from global memory instead
+    w = synth.make_workload(T=96, d=128, F=26624, W=128, C=8, C_h=16, dtype=synth.BF16,
+                            kind="pareto", lam=2e-5, seed=12, mean_active=12.0)
+    got = check_hybrid_all(w, run_hybrid(w))
+    assert got["n_backup"] > 0
+
+
 @pytest.mark.parametrize("C_h", [0, 1024])
 def test_hybrid_extreme_caps(C_h):
     w = synth.make_workload(T=130, d=128, F=1024, W=128, C=8, C_h=C_h, dtype=synth.BF16,
