@@ -3,6 +3,9 @@
 // allocates device memory and never synchronises the caller's stream.
 #include <atomic>
 #include <cstdint>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "tw_internal.h"
 
@@ -21,25 +24,41 @@ int num_sms() {
   return v;
 }
 
+cudaError_t set_smem_limit(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;  // (kernel, device) -> bytes set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({func, dev});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[{func, dev}] = bytes;
+  return e;
+}
+
 }  // namespace tw
 
 namespace {
 
 constexpr int kTileW = 128;
-constexpr int kMaxC = 32;
+constexpr int kMaxC = kTileW;  // any capacity up to the tile width
 constexpr int kMaxRowD = 2048;
 
+}  // namespace
+
+namespace tw {
+
 // Row width d: a multiple of 8, at most 2048 for bf16 rows and 1024 for fp32
-// rows (one warp's column range of up to three weight rows, double-buffered,
-// for sixteen warps must fit the shared memory of one SM).
+// rows (the gather engine keeps one token's row slices and its fp32 output
+// slices in the registers of one team of warps).
 bool row_d_ok(int d, tw_dtype t) {
   return d % 8 == 0 && d <= (t == TW_BF16 ? kMaxRowD : kMaxRowD / 2);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool dtype_ok(tw_dtype t) { return t == TW_F32 || t == TW_BF16; }
-
-tw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TW_OK : TW_ERR_CUDA; }
 
 // Shared checks of a TwELL descriptor.
 tw_status check_twell(const tw_twell* g) {
@@ -57,6 +76,17 @@ tw_status check_twell(const tw_twell* g) {
     return TW_ERR_ALIGNMENT;
   return TW_OK;
 }
+
+}  // namespace tw
+
+namespace {
+
+using tw::aligned16;
+using tw::check_twell;
+using tw::dtype_ok;
+using tw::row_d_ok;
+
+tw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TW_OK : TW_ERR_CUDA; }
 
 tw_status check_hybrid(const tw_hybrid* h) {
   if (!h) return TW_ERR_INVALID_ARG;

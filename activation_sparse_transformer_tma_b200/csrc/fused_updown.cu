@@ -1122,8 +1122,8 @@ cudaError_t run_engine(GatherArgs<Tin> a, bool out_bf16, void* base, CountFn cou
   count();
   const size_t scan_smem = plan_scan_smem(a.T);
   if (scan_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(plan_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)plan_scan_smem(kScanSmemTokens));
+    e = set_smem_limit(reinterpret_cast<const void*>(plan_scan_kernel),
+                       (int)plan_scan_smem(kScanSmemTokens));
     if (e != cudaSuccess) return e;
   }
   const int nb = (a.T + kCountBlock - 1) / kCountBlock;

@@ -102,14 +102,10 @@ __global__ void __launch_bounds__(ROWS)
 cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int d, int F,
                                   const tw_twell& out, float* dump, int32_t* status,
                                   cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gate_twell_f32_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  cudaError_t e = cudaMemsetAsync(out.spill_n, 0, sizeof(int32_t), stream);
+  cudaError_t e =
+      set_smem_limit(reinterpret_cast<const void*>(gate_twell_f32_kernel), (int)SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(out.spill_n, 0, sizeof(int32_t), stream);
   if (e != cudaSuccess) return e;
   dim3 grid((T + ROWS - 1) / ROWS, F / TILE);
   gate_twell_f32_kernel<<<grid, ROWS, SMEM, stream>>>(

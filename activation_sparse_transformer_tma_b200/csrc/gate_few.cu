@@ -344,9 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               before += __popc(bal[a][j]);
             }
-            if (lane >= n[a] && lane < C) {  // padding past the count (C <= 32)
-              out.val[off * C + lane] = 0;
-              out.idx[off * C + lane] = 0;
+            for (int sl = lane; sl < C; sl += 32) {  // padding past the count
+              if (sl >= n[a]) {
+                out.val[off * C + sl] = 0;
+                out.idx[off * C + sl] = 0;
+              }
             }
             if (lane == 0) out.cnt[off] = (uint8_t)n[a];
             if (out.dump != nullptr) {
@@ -417,18 +419,13 @@ cudaError_t launch_gate_twell_few(const void* x, const void* Wg_t, int T, int d,
   sh.stages = stages;
   const size_t smem = fixed + (size_t)stages * sh.stage_bytes;
 
-  static bool attr_set = false;  // idempotent
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gate_few_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemMax);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e =
+      set_smem_limit(reinterpret_cast<const void*>(gate_few_kernel), (int)kSmemMax);
+  if (e != cudaSuccess) return e;
   CUtensorMap mw, mx;
   if (!make_tmap_bf16(&mw, Wg_t, F, d, kBK, kUnits) || !make_tmap_bf16(&mx, x, T, d, kBK, sh.N))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(out.spill_n, 0, sizeof(int32_t), stream);
+  e = cudaMemsetAsync(out.spill_n, 0, sizeof(int32_t), stream);
   if (e != cudaSuccess) return e;
 
   FewOut o;

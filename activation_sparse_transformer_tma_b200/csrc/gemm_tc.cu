@@ -29,7 +29,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 B = one swizzle atom row
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;
-constexpr int EPI_SLOTS = 32;  // largest TwELL capacity C this epilogue packs
+constexpr int EPI_SLOTS = 32;  // TwELL slots per row staged in shared memory
 
 // Tile widths: BN = 256 with a 4-stage ring, or BN = 128 with a 6-stage ring
 // when there are too few 256-wide tiles to occupy every SM (small T).
@@ -88,18 +88,42 @@ struct EpiTwell {
   int32_t* status;
 
   // taddr: TMEM address of this warp's lane block at column 0 of the tile;
-  // the tile holds KT TwELL tiles of 128 columns.
+  // the tile holds KT TwELL tiles of 128 columns.  Capacities up to
+  // EPI_SLOTS are staged per thread in shared memory and stored with vector
+  // stores; larger ones (up to the tile width) stage their first EPI_SLOTS
+  // slots the same way and write the rest straight to global memory.
   template <int KT>
   TW_DEV void run(uint32_t taddr, int row, int nb, int ethread, EpiStage* st) const {
+    if (C <= EPI_SLOTS) run_c<KT, false>(taddr, row, nb, ethread, st);
+    else run_c<KT, true>(taddr, row, nb, ethread, st);
+  }
+
+  // Slot n (< C) of the packed row: staged, or (kWide, n >= EPI_SLOTS) direct.
+  template <bool kWide>
+  TW_DEV void put(uint16_t* sv, uint8_t* si, size_t kt_off, bool row_ok, int n, uint16_t v,
+                  uint8_t j) const {
+    if (!kWide || n < EPI_SLOTS) {
+      sv[n] = v;
+      si[n] = j;
+    } else if (row_ok) {
+      val[kt_off * C + n] = v;
+      idx[kt_off * C + n] = j;
+    }
+  }
+
+  template <int KT, bool kWide>
+  TW_DEV void run_c(uint32_t taddr, int row, int nb, int ethread, EpiStage* st) const {
     const bool row_ok = row < T;
     const int K = F / 128;
+    const int CS = kWide ? EPI_SLOTS : C;  // slots staged in shared memory
     uint16_t* sv = st->slot_val + ethread * EPI_SLOTS;
     uint8_t* si = st->slot_idx + ethread * EPI_SLOTS;
 #pragma unroll 1
     for (int kt = 0; kt < KT; ++kt) {
       const int k = nb * KT + kt;
       if (k >= K) break;  // uniform across the CTA
-      for (int s = 0; s < C; ++s) {
+      const size_t kt_off = (size_t)k * T + row;
+      for (int s = 0; s < CS; ++s) {
         sv[s] = 0;
         si[s] = 0;
       }
@@ -117,17 +141,15 @@ struct EpiTwell {
           packed[i] = p;
           if (p != 0u) {
             if ((p & 0xFFFFu) != 0u) {
-              if (n < C) {
-                sv[n] = (uint16_t)(p & 0xFFFFu);
-                si[n] = (uint8_t)(c * 32 + 2 * i);
-              }
+              if (n < C)
+                put<kWide>(sv, si, kt_off, row_ok, n, (uint16_t)(p & 0xFFFFu),
+                           (uint8_t)(c * 32 + 2 * i));
               ++n;
             }
             if ((p >> 16) != 0u) {
-              if (n < C) {
-                sv[n] = (uint16_t)(p >> 16);
-                si[n] = (uint8_t)(c * 32 + 2 * i + 1);
-              }
+              if (n < C)
+                put<kWide>(sv, si, kt_off, row_ok, n, (uint16_t)(p >> 16),
+                           (uint8_t)(c * 32 + 2 * i + 1));
               ++n;
             }
           }
@@ -140,21 +162,26 @@ struct EpiTwell {
         }
       }
       if (row_ok) {
-        const size_t kt_off = (size_t)k * T + row;
         cnt[kt_off] = (uint8_t)n;
         if ((C & 7) == 0) {
           uint4* dv = reinterpret_cast<uint4*>(val + kt_off * C);
           uint2* di = reinterpret_cast<uint2*>(idx + kt_off * C);
           const uint4* svv = reinterpret_cast<const uint4*>(sv);
           const uint2* sii = reinterpret_cast<const uint2*>(si);
-          for (int s = 0; s < C / 8; ++s) {
+          for (int s = 0; s < CS / 8; ++s) {
             dv[s] = svv[s];
             di[s] = sii[s];
           }
         } else {
-          for (int s = 0; s < C; ++s) {
+          for (int s = 0; s < CS; ++s) {
             val[kt_off * C + s] = sv[s];
             idx[kt_off * C + s] = si[s];
+          }
+        }
+        if (kWide) {  // padding past the count beyond the staged slots
+          for (int s = n > EPI_SLOTS ? n : EPI_SLOTS; s < C; ++s) {
+            val[kt_off * C + s] = 0;
+            idx[kt_off * C + s] = 0;
           }
         }
       }
@@ -429,14 +456,9 @@ template <class Epi, int BN>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, int Kdim,
                    int n_tiles_m, int n_tiles_n, const Epi& epi, int32_t* status,
                    cudaStream_t stream, uint32_t a_bytes = A_BYTES) {
-  static bool attr_set = false;  // per template instance; idempotent
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<Epi, BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<BN>());
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(gemm_tc_kernel<Epi, BN>),
+                                 (int)smem_bytes<BN>());
+  if (e != cudaSuccess) return e;
   const int num_tiles = n_tiles_m * n_tiles_n;
   if (num_tiles == 0) return cudaSuccess;
   const int grid = num_tiles < num_sms() ? num_tiles : num_sms();

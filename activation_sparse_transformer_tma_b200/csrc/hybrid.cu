@@ -240,9 +240,9 @@ __global__ void __launch_bounds__(256)
         if (ref < 0 || ref >= spill_cap) {
           // Dropped spill entry: only the C slots are known.
           if (lane == 0) set_status(status, kStatusSpill);
-          if (lane < C) {
-            ell_g[rbase + p0 + lane] = val[kt * C + lane];
-            ell_idx[rbase + p0 + lane] = (uint16_t)(kk * W + idx[kt * C + lane]);
+          for (int s = lane; s < C; s += 32) {
+            ell_g[rbase + p0 + s] = val[kt * C + s];
+            ell_idx[rbase + p0 + s] = (uint16_t)(kk * W + idx[kt * C + s]);
           }
           for (int s = C + lane; s < nk; s += 32) {  // keep the row's slots defined
             ell_g[rbase + p0 + s] = T(0);
@@ -707,15 +707,11 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
   void* engine_ws = static_cast<char*>(ws) + w.bytes;
   const int nb = (gu.T + TB - 1) / TB;
   const size_t hist_bytes = tb_hist_bytes(gu.F);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(hyb_count_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         200 * 1024);
-    cudaFuncSetAttribute(hyb_fill_kernel<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         200 * 1024);
-    cudaFuncSetAttribute(hyb_fill_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         200 * 1024);
-    attr_set = true;
+  for (const void* f : {reinterpret_cast<const void*>(hyb_count_kernel<T>),
+                        reinterpret_cast<const void*>(hyb_fill_kernel<T, false>),
+                        reinterpret_cast<const void*>(hyb_fill_kernel<T, true>)}) {
+    const cudaError_t ea = set_smem_limit(f, 200 * 1024);
+    if (ea != cudaSuccess) return ea;
   }
   // entry offsets of every token (token-major order)
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(2, gu.T, gu.row_nnz, 0, w.e0, gu.row_slot,

@@ -13,7 +13,14 @@
 // The array is part of the library's device image: every GPU on which the
 // library's kernels are loaded holds kScratchBytes of it until the process
 // exits.  Its device address is looked up once per device (first call on that
-// device, with that device current) and cached.
+// device, with that device current) and cached for the life of the process;
+// after cudaDeviceReset the cached address is stale, so the entry point must
+// not be used across a device reset.
+//
+// Capacity: the plan of T tokens takes about 24 bytes per token (counts,
+// split offsets and one work item each) plus the partial rows of split
+// tokens.  T <= 696,848 fits for every supported d; the partial-row capacity
+// is whatever the rest of the array holds.
 #include <atomic>
 #include <cstdint>
 #include <mutex>
@@ -55,29 +62,25 @@ void* scratch_on_current_device(cudaError_t* err) {
   return p;
 }
 
-bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 extern "C" tw_status twell_fused_updown_noalloc(const void* x, const tw_twell* g,
                                                 const void* Wu_t, const void* Wd, int32_t d,
                                                 void* y, tw_dtype y_dtype, int32_t* dev_status,
                                                 cudaStream_t stream) {
-  if (!g || !x || !Wu_t || !Wd || !y) return TW_ERR_INVALID_ARG;
-  if (g->T < 0 || g->F <= 0 || g->C < 0 || g->spill_cap < 0 || d <= 0) return TW_ERR_INVALID_ARG;
-  if ((g->dtype != TW_F32 && g->dtype != TW_BF16) || (y_dtype != TW_F32 && y_dtype != TW_BF16))
-    return TW_ERR_INVALID_ARG;
-  if (g->W != 128 || g->F % 128 != 0 || g->C > 32 || g->F > 65536) return TW_ERR_UNSUPPORTED;
-  if (!g->cnt || !g->spill_ref || !g->spill_n) return TW_ERR_INVALID_ARG;
-  if (g->C > 0 && (!g->val || !g->idx)) return TW_ERR_INVALID_ARG;
-  if (g->spill_cap > 0 && (!g->spill_tk || !g->spill_val)) return TW_ERR_INVALID_ARG;
-  if (d % 8 != 0 || d > (g->dtype == TW_BF16 ? 2048 : 1024)) return TW_ERR_UNSUPPORTED;
-  if (!al16(x) || !al16(Wu_t) || !al16(Wd) || !al16(y) || (g->val && !al16(g->val)) ||
-      (g->idx && !al16(g->idx)) || (g->spill_val && !al16(g->spill_val)))
+  // the same checks as twell_fused_updown: with T == 0 the token-sized
+  // buffers may be NULL and nothing is launched
+  tw_status st = tw::check_twell(g);
+  if (st != TW_OK) return st;
+  const bool any = g->T > 0;
+  if ((any && (!x || !y)) || !Wu_t || !Wd || !tw::dtype_ok(y_dtype)) return TW_ERR_INVALID_ARG;
+  if (d <= 0) return TW_ERR_INVALID_ARG;
+  if (!tw::row_d_ok(d, g->dtype)) return TW_ERR_UNSUPPORTED;
+  if (!tw::aligned16(x) || !tw::aligned16(Wu_t) || !tw::aligned16(Wd) || !tw::aligned16(y))
     return TW_ERR_ALIGNMENT;
+  if (!any) return TW_OK;
   // the work plan of T tokens must fit the fixed scratch area
   if (!tw::fused_plan_fits(g->T, d, kScratchBytes)) return TW_ERR_UNSUPPORTED;
-  if (g->T == 0) return TW_OK;
   cudaError_t err = cudaSuccess;
   void* scratch = scratch_on_current_device(&err);
   if (!scratch) return TW_ERR_CUDA;

@@ -11,6 +11,18 @@ namespace tw {
 // Device properties cached per device.
 int num_sms();
 
+// Raise `func`'s dynamic shared-memory limit to `bytes` on the current device.
+// The attribute belongs to the device, so it is set once per (kernel, device)
+// and remembered under a lock; a process that drives several GPUs gets it set
+// on each of them.
+cudaError_t set_smem_limit(const void* func, int bytes);
+
+// Host-side argument checks shared by the entry points (abi.cu).
+bool row_d_ok(int d, tw_dtype t);
+bool aligned16(const void* p);
+bool dtype_ok(tw_dtype t);
+tw_status check_twell(const tw_twell* g);
+
 // Default upper bound on any single pipeline wait inside a kernel (ns).
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 

@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--workload", default="ffn_2b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip comparator/training/decode legs")
-    ap.add_argument("--legs", default="dense,decode,training",
+    ap.add_argument("--legs", default="dense,energy,decode,training",
                     help="comma-separated extra legs to run after the timed step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -320,12 +320,14 @@ def run_ours(args, rank, world, local_rank):
     flops_fused = 2.0 * 2 * d * nnz          # one dot and one axpy of length d per entry
     tflops_fused = flops_fused / (ms_fused * 1e-3) / 1e12
     Kt = F // 128
-    unique_bytes = 2 * T * d + 4 * T * d + Kt * T * (3 * C + 1)  # x, fp32 y, TwELL
+    live = live_units(torch, g)
+    # x, fp32 y, TwELL, and one Wu and one Wd row of every unit active in the batch
+    unique_bytes = 2 * T * d + 4 * T * d + Kt * T * (3 * C + 1) + live * 2 * d * 2
     roof_gate = {"kernel": "twell_gate_gemm (tcgen05 + TwELL epilogue)", "bound": "tensor",
-                 "achieved": tflops_gate, "peak": tf_sust, "unit": "TFLOP/s",
-                 "frac": tflops_gate / tf_sust,
-                 "peak_source": f"{src} bf16 sustained (kernel timed inside a long loop)",
-                 "frac_of_burst_peak": tflops_gate / tf_burst,
+                 "achieved": tflops_gate, "peak": tf_burst, "unit": "TFLOP/s",
+                 "frac": tflops_gate / tf_burst,
+                 "peak_source": f"{src} bf16 burst (the timed region is well under a second)",
+                 "frac_of_sustained_peak": tflops_gate / tf_sust,
                  "traffic": profiled_traffic("gate_twell_gemm_ffn_2b.md",
                                              src_sha("gemm_tc.cu", "tw_common.cuh")),
                  "algorithmic": f"2*T*d*F = {flops_gate:.4g} FLOP per launch"}
@@ -337,6 +339,7 @@ def run_ours(args, rank, world, local_rank):
                                               src_sha("fused_updown.cu", "tw_common.cuh")),
                   "algorithmic": f"4*d*nnz = {flops_fused:.4g} FLOP per launch (nnz = {nnz})",
                   "gathered_GBps": nnz * 4 * d / (ms_fused * 1e-3) / 1e9,
+                  "unique_hbm_bytes": unique_bytes, "live_units": live,
                   "unique_hbm_GBps": unique_bytes / (ms_fused * 1e-3) / 1e9,
                   "unique_hbm_frac": unique_bytes / (ms_fused * 1e-3) / 1e9 / hbm}
     dominant = roof_fused if ms_fused >= ms_gate else roof_gate
@@ -359,6 +362,9 @@ def run_ours(args, rank, world, local_rank):
     if legs:
         if rank == 0 and "dense" in legs:
             line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
+        if rank == 0 and "energy" in legs:
+            line["energy"] = energy_leg(torch, tw, x, Wg, Wu, Wd, g, y, ws, status, T, d, F,
+                                        local_rank)
         del x, Wg, Wu, Wd, g, y, ws, xh, yh
         torch.cuda.empty_cache()
         if rank == 0 and "decode" in legs:
@@ -377,6 +383,90 @@ def run_ours(args, rank, world, local_rank):
 # kernels of one inference step: gate GEMM; plan count, plan scan, plan write,
 # fused kernel (the two workspace clears are memsets, not kernels)
 KERNELS_PER_STEP = 5
+
+
+def live_units(torch, g):
+    """Number of units active anywhere in the batch, read from the TwELL
+    (slots below each tile's count, and the non-zeros of spilled segments)."""
+    K = g.F // g.W
+    used = torch.zeros(g.F, dtype=torch.bool, device="cuda")
+    base = (torch.arange(K, device="cuda") * g.W).view(K, 1, 1)
+    if g.C:
+        slot = torch.arange(g.C, device="cuda").view(1, 1, g.C)
+        valid = slot < g.cnt.long().unsqueeze(2)
+        used[(g.idx.long() + base)[valid]] = True
+    n = min(int(g.spill_n.item()), g.spill_cap)
+    if n:
+        tk = g.spill_tk[:n].long()
+        nz = g.spill_val[:n] != 0
+        cols = torch.arange(g.W, device="cuda").view(1, g.W)
+        used[(tk[:, 1:2] * g.W + cols)[nz]] = True
+    return int(used.sum().item())
+
+
+def nvml_handle(torch, local_rank):
+    """NVML handle of this process's GPU (matched by UUID), or None."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        u = str(torch.cuda.get_device_properties(local_rank).uuid)
+        for cand in (u, "GPU-" + u):
+            try:
+                return pynvml.nvmlDeviceGetHandleByUUID(cand)
+            except Exception:
+                pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = int(vis.split(",")[local_rank]) if vis else local_rank
+        return pynvml.nvmlDeviceGetHandleByIndex(idx)
+    except Exception:
+        return None
+
+
+def energy_leg(torch, tw, x, Wg, Wu, Wd, g, y, ws, status, T, d, F, local_rank):
+    """Energy per token of the sparse step and of the in-library dense FFN of
+    the same shape.  NVML's cumulative energy counter (read-only, mJ) is read
+    around a loop of about two seconds of each; the ratio is dense / sparse."""
+    h = nvml_handle(torch, local_rank)
+    if h is None:
+        return {"unavailable": "NVML energy counter not readable"}
+    import pynvml
+    Wd_dense = Wd.t().contiguous()
+    hbuf = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    yd = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+
+    def sparse():
+        tw.twell_gate_gemm(x, Wg, g, None, status)
+        tw.twell_fused_updown(x, g, Wu, Wd, y, ws, status)
+
+    def dense():
+        tw.dense_ffn_forward(x, Wg, Wu, Wd_dense, hbuf, yd)
+
+    def measure(fn, seconds=2.0):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(20):
+            fn()
+        torch.cuda.synchronize()
+        n = max(50, int(seconds / ((time.perf_counter() - t0) / 20)))
+        e0 = pynvml.nvmlDeviceGetTotalEnergyConsumption(h)
+        t0 = time.perf_counter()
+        for _ in range(n):
+            fn()
+        torch.cuda.synchronize()
+        el = time.perf_counter() - t0
+        joules = (pynvml.nvmlDeviceGetTotalEnergyConsumption(h) - e0) / 1e3
+        return {"steps": n, "seconds": el, "joules": joules, "avg_watts": joules / el,
+                "j_per_token": joules / (n * T)}
+
+    sp = measure(sparse)
+    dn = measure(dense)
+    del hbuf, yd, Wd_dense
+    return {"sparse": sp, "dense": dn,
+            "dense_over_sparse_j_per_token": dn["j_per_token"] / sp["j_per_token"],
+            "method": "NVML total-energy counter around each loop (whole-GPU energy, "
+                      "idle power included); wall clock for the loop length"}
 
 
 def sm_max_mhz():

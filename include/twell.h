@@ -31,7 +31,7 @@
  *             into the caller's `dev_status` word as bit (1 << tw_status);
  *             dev_status may be NULL.  The caller zeroes it and reads it after
  *             synchronising; tw_status_string names each code.
- * Limits      W == 128; 0 <= C <= 32; F % W == 0; d % 8 == 0; 8 <= d <= 2048
+ * Limits      W == 128; 0 <= C <= W; F % W == 0; d % 8 == 0; 8 <= d <= 2048
  *             (bf16 rows) or d <= 1024 (fp32 rows) for the fused and hybrid
  *             kernels; T >= 0.  With T == 0 the arrays sized by T (x, y, dy,
  *             dx, the TwELL and hybrid per-token arrays, the workspaces) may
@@ -180,13 +180,18 @@ TW_API tw_status twell_fused_updown(const void* x, const tw_twell* g, const void
  *   - No cudaMalloc or cudaFree is called; the caller passes inputs and
  *     outputs exactly as for twell_fused_updown.
  *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
- *   - The plan of T tokens must fit 16 MiB: T up to 800,000 always fits (the
- *     exact bound is a little higher and depends on d); a T whose plan does
- *     not fit returns TW_ERR_UNSUPPORTED.  When fewer heavy tokens can be split than
+ *     that device current) and caches it for the life of the process; make
+ *     that first call before any stream capture, and do not use the entry
+ *     point across cudaDeviceReset (the cached address would be stale).
+ *   - The plan of T tokens must fit 16 MiB, about 24 bytes per token: T up to
+ *     696,848 fits for every supported d; a T whose plan does not fit returns
+ *     TW_ERR_UNSUPPORTED before any device work.  The rest of the array holds
+ *     partial rows of split tokens; when fewer heavy tokens can be split than
  *     the workspace version would split, the rest run unsplit: y is the same
  *     up to fp32 summation order.
+ *   - Arguments are checked as for twell_fused_updown; with T == 0 the
+ *     token-sized buffers (x, y and the TwELL per-token arrays) may be NULL
+ *     and the call returns TW_OK without device work.
  *   - Every call shares the one array, and the call clears the part that must
  *     start at zero.  Calls whose work overlaps on the GPU (different streams
  *     or host threads without ordering) race on it and give wrong results.

@@ -71,7 +71,7 @@ def test_gate_validation(L):
     assert _gate(L, _tw(), x=None) == INVALID
     assert _gate(L, _tw(), x=FAKE + 8) == ALIGN
     assert _gate(L, _tw(W=64)) == UNSUPPORTED            # tile width must be 128
-    assert _gate(L, _tw(C=33)) == UNSUPPORTED            # capacity above the epilogue's 32
+    assert _gate(L, _tw(C=129)) == UNSUPPORTED           # capacity above the tile width
     assert _gate(L, _tw(F=1000), F=1000) == UNSUPPORTED  # F not a multiple of W
     assert _gate(L, _tw(T=255)) == INVALID               # out->T != T
     assert _gate(L, _tw(), d=500) == UNSUPPORTED         # d % 8 != 0

@@ -125,6 +125,52 @@ def test_fp32_tiny_config(C, T):
     check_y(f64(y), w64, rows, TOL[synth.F32], g_round="f32")
 
 
+# Capacities above 32 up to the tile width.  Half the units of a tile are
+# active on average (mean_active = 300 of 512 live units), so at C = 64 many
+# tiles spill and the slots past 32 are written straight from the epilogue;
+# at C = W = 128 the TwELL holds every tile whole and nothing spills.  T = 300
+# runs the tile GEMM, T <= 64 the small-batch gate, and fp32 its own kernel.
+WIDE_C = [
+    # T, C, dtype
+    (300, 64, synth.BF16),
+    (300, 128, synth.BF16),
+    (300, 40, synth.BF16),     # not a multiple of 8: scalar stores of the staged slots
+    (40, 64, synth.BF16),
+    (40, 128, synth.BF16),
+    (1, 128, synth.BF16),
+    (130, 64, synth.F32),
+    (130, 128, synth.F32),
+]
+
+
+@pytest.mark.parametrize("T,C,dt", WIDE_C)
+def test_capacity_up_to_tile_width(T, C, dt):
+    d = 256 if dt == synth.F32 else 320
+    w = synth.make_workload(T=T, d=d, F=640, W=128, C=C, dtype=dt, kind="dead20",
+                            mean_active=300.0, seed=T + C)
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    w64 = widened(w)
+    g64 = f64(gd)
+    ref = assert_twell_matches_oracle(g, g64)
+    cnt = raw(g.cnt)
+    assert cnt.max() > 32  # the rows past the staged slots are exercised
+    if C == 128:
+        assert int(g.spill_n.item()) == 0 and ref["n_spill"] == 0
+    else:
+        assert int(g.spill_n.item()) > 0
+    rows = np.arange(T, dtype=np.int32)
+    check_y(f64(y), w64, rows, TOL[dt], g_round="bf16" if dt == synth.BF16 else "f32")
+
+
+def test_hybrid_from_wide_capacity_twell():
+    """TwELL -> hybrid with C = 64: tiles with more than 32 slots feed ELL rows."""
+    w = synth.make_workload(T=300, d=256, F=640, W=128, C=64, C_h=155, dtype=synth.BF16,
+                            kind="dead20", lam=2e-5, seed=77, mean_active=150.0, with_dy=True)
+    got = check_hybrid_all(w, run_hybrid(w))
+    assert 0 < got["n_backup"] < 300
+
+
 def test_ffn_0p5b_full_size():
     w = synth.make_workload("ffn_0p5b")
     dev, g, gd, y, st = run_forward(w)
