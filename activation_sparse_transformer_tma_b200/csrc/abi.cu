@@ -38,13 +38,22 @@ cudaError_t set_smem_limit(const void* func, int bytes) {
   return e;
 }
 
+namespace {
+std::atomic<unsigned long long> g_withheld_gate_wait{0};
+}  // namespace
+
+unsigned long long take_withheld_gate_wait() { return g_withheld_gate_wait.exchange(0); }
+
 }  // namespace tw
 
 namespace {
 
-constexpr int kTileW = 128;
-constexpr int kMaxC = kTileW;  // any capacity up to the tile width
+constexpr int kTileW = 128;    // the tile width of the dense comparators' F tiles
 constexpr int kMaxRowD = 2048;
+
+// TwELL tile widths: 64, 128 (the default) or 256 (tile-local indices are
+// uint8).  Any capacity C up to the tile width.
+bool tile_width_ok(int W) { return W == 64 || W == 128 || W == 256; }
 
 }  // namespace
 
@@ -65,7 +74,7 @@ tw_status check_twell(const tw_twell* g) {
   if (!g) return TW_ERR_INVALID_ARG;
   if (g->T < 0 || g->F <= 0 || g->C < 0 || g->spill_cap < 0 || !dtype_ok(g->dtype))
     return TW_ERR_INVALID_ARG;
-  if (g->W != kTileW || g->F % kTileW != 0 || g->C > kMaxC) return TW_ERR_UNSUPPORTED;
+  if (!tile_width_ok(g->W) || g->F % g->W != 0 || g->C > g->W) return TW_ERR_UNSUPPORTED;
   if (g->F > 65536) return TW_ERR_UNSUPPORTED;
   // arrays sized by T may be NULL for an empty batch
   if (!g->spill_n || (g->T > 0 && (!g->cnt || !g->spill_ref))) return TW_ERR_INVALID_ARG;
@@ -125,6 +134,10 @@ const char* tw_status_string(tw_status s) {
 
 int32_t twell_version(void) { return 100; }
 
+void tw_test_withhold_next_gate_loads(uint64_t wait_limit_ns) {
+  tw::g_withheld_gate_wait.store(wait_limit_ns > 0 ? wait_limit_ns : 1);
+}
+
 tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int32_t d, int32_t F,
                           tw_dtype dtype, const tw_twell* out, void* g_dense_dump,
                           int32_t* dev_status, cudaStream_t stream) {
@@ -139,7 +152,7 @@ tw_status twell_gate_gemm(const void* x, const void* Wg_t, int32_t T, int32_t d,
   if (T == 0) return from_cuda(cudaMemsetAsync(out->spill_n, 0, sizeof(int32_t), stream));
   if (dtype == TW_BF16) {
     if (d < 64) return TW_ERR_UNSUPPORTED;
-    if (T <= tw::kFewMaxT)
+    if (T <= tw::kFewMaxT && out->W == 128)
       return from_cuda(tw::launch_gate_twell_few(x, Wg_t, T, d, F, *out, g_dense_dump,
                                                  dev_status, stream));
     return from_cuda(tw::launch_gate_twell_tc(x, Wg_t, T, d, F, *out, g_dense_dump, dev_status,
@@ -251,6 +264,102 @@ tw_status dense_ffn_forward(const void* x, const void* Wg_t, const void* Wu_t,
   cudaError_t e = tw::launch_dense_gateup_tc(x, Wg_t, Wu_t, T, d, F, h_ws, dev_status, stream);
   if (e != cudaSuccess) return TW_ERR_CUDA;
   return from_cuda(tw::launch_dense_down_tc(h_ws, Wd_dense, T, d, F, y, dev_status, stream));
+}
+
+size_t twell_ffn_small_batch_workspace_size(int32_t T, int32_t d, int32_t F) {
+  if (T < 0 || d <= 0 || F <= 0) return 0;
+  return tw::decode_ws_bytes(T, d, F);
+}
+
+tw_status twell_ffn_small_batch(const void* x, const void* Wg_t, const void* Wu_t, const void* Wd,
+                                int32_t T, int32_t d, int32_t F, const tw_twell* g,
+                                void* g_dense_dump, void* y, tw_dtype y_dtype, void* ws,
+                                size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
+  tw_status st = check_twell(g);
+  if (st != TW_OK) return st;
+  if (g->T != T || g->F != F || T < 0 || d <= 0) return TW_ERR_INVALID_ARG;
+  if ((T > 0 && (!x || !y || !ws)) || !Wg_t || !Wu_t || !Wd || !dtype_ok(y_dtype))
+    return TW_ERR_INVALID_ARG;
+  if (g->dtype != TW_BF16 || g->W != 128 || T > tw::kDecodeStepMaxT || d % 8 != 0 || d < 64 ||
+      d > kMaxRowD)
+    return TW_ERR_UNSUPPORTED;
+  const void* ptrs[] = {x, Wg_t, Wu_t, Wd, y, ws, g_dense_dump};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return TW_ERR_ALIGNMENT;
+  if (T == 0) return from_cuda(cudaMemsetAsync(g->spill_n, 0, sizeof(int32_t), stream));
+  if (ws_bytes < tw::decode_ws_bytes(T, d, F)) return TW_ERR_WORKSPACE;
+  return from_cuda(tw::launch_decode_step(x, Wg_t, Wu_t, Wd, T, d, F, *g, g_dense_dump, y,
+                                          y_dtype, ws, dev_status, stream));
+}
+
+// Workspace of the dense training comparator: g, u, h (saved by the forward
+// for the backward) then du, dz (backward scratch), each [T][F] bf16.
+static size_t dense_train_part(int32_t T, int32_t F) {
+  return ((size_t)T * (size_t)F * 2 + 255) & ~size_t(255);
+}
+
+size_t dense_ffn_train_workspace_size(int32_t T, int32_t F) {
+  if (T < 0 || F <= 0) return 0;
+  return 5 * dense_train_part(T, F);
+}
+
+size_t dense_ffn_train_saved_bytes(int32_t T, int32_t F) {
+  if (T < 0 || F <= 0) return 0;
+  return 3 * dense_train_part(T, F);
+}
+
+static tw_status check_dense_train(int32_t T, int32_t d, int32_t F, const void* ws,
+                                   size_t ws_bytes) {
+  if (T < 0 || d <= 0 || F <= 0) return TW_ERR_INVALID_ARG;
+  if (d % 32 != 0 || d < 64 || F % kTileW != 0) return TW_ERR_UNSUPPORTED;
+  if (T > 0 && !ws) return TW_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return TW_ERR_ALIGNMENT;
+  if (T > 0 && ws_bytes < 5 * dense_train_part(T, F)) return TW_ERR_WORKSPACE;
+  return TW_OK;
+}
+
+tw_status dense_ffn_train_forward(const void* x, const void* Wg_t, const void* Wu_t,
+                                  const void* Wd, int32_t T, int32_t d, int32_t F, void* ws,
+                                  size_t ws_bytes, float* y, int32_t* dev_status,
+                                  cudaStream_t stream) {
+  tw_status st = check_dense_train(T, d, F, ws, ws_bytes);
+  if (st != TW_OK) return st;
+  if ((T > 0 && (!x || !y)) || !Wg_t || !Wu_t || !Wd) return TW_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, Wg_t, Wu_t, Wd, y};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return TW_ERR_ALIGNMENT;
+  if (T == 0) return TW_OK;
+  uint16_t* base = static_cast<uint16_t*>(ws);
+  const size_t part = dense_train_part(T, F) / 2;
+  return from_cuda(tw::launch_dense_train_forward(x, Wg_t, Wu_t, Wd, T, d, F, base,
+                                                  base + part, base + 2 * part, y, dev_status,
+                                                  stream));
+}
+
+tw_status dense_ffn_train_backward(const void* x, const void* dy, const void* Wg_t,
+                                   const void* Wu_t, const void* Wd, int32_t T, int32_t d,
+                                   int32_t F, float l1_lambda, void* ws, size_t ws_bytes,
+                                   float* dx, float* dWg_t, float* dWu_t, float* dWd,
+                                   int32_t* dev_status, cudaStream_t stream) {
+  tw_status st = check_dense_train(T, d, F, ws, ws_bytes);
+  if (st != TW_OK) return st;
+  if ((T > 0 && (!x || !dy || !dx)) || !Wg_t || !Wu_t || !Wd || !dWg_t || !dWu_t || !dWd)
+    return TW_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, dy, Wg_t, Wu_t, Wd, dx, dWg_t, dWu_t, dWd};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return TW_ERR_ALIGNMENT;
+  if (T == 0) {  // no tokens: zero weight gradients
+    const size_t b = sizeof(float) * (size_t)F * d;
+    cudaError_t e = cudaMemsetAsync(dWg_t, 0, b, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dWu_t, 0, b, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dWd, 0, b, stream);
+    return from_cuda(e);
+  }
+  uint16_t* base = static_cast<uint16_t*>(ws);
+  const size_t part = dense_train_part(T, F) / 2;
+  return from_cuda(tw::launch_dense_train_backward(
+      x, dy, Wg_t, Wu_t, Wd, T, d, F, l1_lambda, base, base + part, base + 2 * part,
+      base + 3 * part, base + 4 * part, dx, dWg_t, dWu_t, dWd, dev_status, stream));
 }
 
 }  // extern "C"

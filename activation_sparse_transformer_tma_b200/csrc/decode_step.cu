@@ -1,0 +1,472 @@
+// decode_step.cu -- the whole gated FFN of a small batch (1 <= T <= 16
+// tokens, decoding) in ONE persistent, cooperative launch: the gate
+// projection with its TwELL packing ("Sparser, Faster, Lighter Transformer
+// Language Models", technical summary, section 2.1) and the fused up + down
+// projection over the active units (section 2.2).
+//
+// With a handful of tokens the step is bound by streaming Wg from HBM
+// (d x F bf16, 33.5 MB at d = 2048, F = 8192) plus a few dozen gathered
+// weight rows per token; the separate launches of the gate and the fused
+// kernels (and their set-up) cost more than the data movement itself.  Here
+// one grid, one CTA per SM, runs four phases separated by grid barriers:
+//
+//   A  gate: work items of 16 units x 256 columns of d, spread over every
+//      warp of the grid; a warp streams its 16 Wg rows (16-byte loads, eight
+//      32-column steps in flight) and multiplies them with the tokens' x
+//      (staged in shared memory) on the tensor pipe: mma.sync m16n8k16 with
+//      the units on M and the tokens on N.  The reduction over d is split
+//      into slices: each item writes fp32 partial sums zpart[slice][t][u].
+//   B  packing: one warp per (tile k, token t) adds the slices in a fixed
+//      order, applies ReLU, rounds g to bf16 and packs the tile's TwELL slots
+//      exactly as the gate GEMM's epilogue does (ascending units, count,
+//      padding, lossless spill of the whole segment past C).  It also writes
+//      every non-zero of the tile (unit and g) to a per-token list at stride
+//      W per tile.
+//   C  dot products: the warps of each token split its tiles (and a hot
+//      tile's entries); for an entry (j, g) a warp forms u = x_t . Wu_t[j]
+//      (fp32) and stores h = g u, with j, at the entry's ordinal in the
+//      token's compact list (ordinal = prefix of the tile counts).
+//   D  updates: one CTA per (token, 256-column slice of d); its warps take
+//      the token's entries round-robin, accumulate h Wd[j] over their
+//      columns in fp32, and the CTA adds the warps' partial rows in warp
+//      order.  y is therefore deterministic.
+//
+// Grid barriers: an arrival counter in the workspace that every CTA bumps and
+// then polls (bounded by a timeout that flags TW_ERR_TIMEOUT); after the last
+// phase a departure counter lets the last CTA reset both to zero, so the
+// workspace is ready for the next call.  The cooperative launch guarantees
+// that every CTA of the grid is resident, so a barrier cannot wait on a CTA
+// that never starts.
+#include "tw_common.cuh"
+#include "tw_internal.h"
+
+namespace tw {
+namespace {
+
+constexpr unsigned FULL = 0xFFFFFFFFu;
+constexpr int kWarpsD = 8;
+constexpr int kThreadsD = 32 * kWarpsD;
+constexpr int kW = 128;          // TwELL tile width of this path
+constexpr int kSlice = 256;      // columns of d per gate work item
+constexpr int kSteps = kSlice / 32;
+constexpr int kMaxTokD = 16;
+
+struct DecodeArgs {
+  const uint16_t* x;
+  const uint16_t* Wg;
+  const uint16_t* Wu;
+  const uint16_t* Wd;
+  int T, d, F, C, S;  // S: slices of d
+  // TwELL output
+  uint16_t* val;
+  uint8_t* idx;
+  uint8_t* cnt;
+  int32_t* spill_ref;
+  int spill_cap;
+  int32_t* spill_tk;
+  uint16_t* spill_val;
+  int32_t* spill_n;
+  uint16_t* dump;
+  // y
+  void* y;
+  int y_bf16;
+  // workspace
+  int32_t* bar;    // [0] arrivals, [1] departures
+  float* zpart;    // [S][T][F]
+  int32_t* jtile;  // [T][F]: units of tile k at [k * W, k * W + cnt)
+  float* gtile;    // [T][F]: their g
+  int32_t* jc;     // [T][F]: compact entry list (units)
+  float* hc;       // [T][F]: compact entry list (h)
+  int32_t* nent;   // [T]
+  int32_t* status;
+  unsigned long long timeout_ns;
+};
+
+TW_DEV void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                     uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+TW_DEV int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier number `b` (1-based) of this launch.  Bounded: a CTA that
+// has waited longer than timeout_ns flags TW_ERR_TIMEOUT and goes on.
+TW_DEV void grid_barrier(const DecodeArgs& a, int b) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(&a.bar[0], 1);
+    const int target = b * (int)gridDim.x;
+    uint64_t t0 = 0;
+    for (uint32_t i = 0; ld_acquire(&a.bar[0]) < target; ++i) {
+      __nanosleep(64);
+      if ((i & 63u) == 63u) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) {
+          t0 = now;
+        } else if (now - t0 > a.timeout_ns) {
+          set_status(a.status, kStatusTimeout);
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int T = a.T, d = a.d, F = a.F, K = F / kW;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [16][d] bf16, rows >= T zero
+  float* red = reinterpret_cast<float*>(smem + (size_t)kMaxTokD * d * 2);  // [8][256]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = gridDim.x * kWarpsD;
+  const int gw = blockIdx.x * kWarpsD + warp;
+
+  // stage x (16-byte chunks), zero rows past T
+  for (int i = threadIdx.x; i < kMaxTokD * d / 8; i += kThreadsD) {
+    const int t = i / (d / 8);
+    reinterpret_cast<uint4*>(xs)[i] =
+        t < T ? reinterpret_cast<const uint4*>(a.x)[i] : make_uint4(0, 0, 0, 0);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.spill_n = 0;  // before any spill (phase B)
+  __syncthreads();
+
+  // ------------------------------------------------ A: gate partial sums --
+  {
+    const int g = lane >> 2, q = lane & 3;
+    const int n_items = (F / 16) * a.S;
+    const bool two_n = T > 8;
+    for (int item = gw; item < n_items; item += nwarps) {
+      const int grp = item / a.S, s = item % a.S;
+      const int u0 = grp * 16, c0 = s * kSlice;
+      const uint16_t* r_lo = a.Wg + (size_t)(u0 + g) * d;
+      const uint16_t* r_hi = a.Wg + (size_t)(u0 + g + 8) * d;
+      uint4 alo[kSteps], ahi[kSteps];
+#pragma unroll
+      for (int i = 0; i < kSteps; ++i) {
+        const int col = c0 + i * 32 + 8 * q;
+        const bool in = col < d;
+        alo[i] = in ? __ldcs(reinterpret_cast<const uint4*>(r_lo + col)) : make_uint4(0, 0, 0, 0);
+        ahi[i] = in ? __ldcs(reinterpret_cast<const uint4*>(r_hi + col)) : make_uint4(0, 0, 0, 0);
+      }
+      float D0[4] = {0.f, 0.f, 0.f, 0.f}, D1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < kSteps; ++i) {
+        const int col = c0 + i * 32 + 8 * q;
+        // The 8 columns a lane loaded take the k-indices of its A fragment
+        // (the same permutation of k for every unit row and token column),
+        // so the products pair Wg[u][col] with x[t][col].
+        const uint4 xb = col < d ? *reinterpret_cast<const uint4*>(xs + (size_t)g * d + col)
+                                 : make_uint4(0, 0, 0, 0);
+        mma16816(D0, alo[i].x, ahi[i].x, alo[i].y, ahi[i].y, xb.x, xb.y);
+        mma16816(D0, alo[i].z, ahi[i].z, alo[i].w, ahi[i].w, xb.z, xb.w);
+        if (two_n) {
+          const uint4 xc = col < d
+                               ? *reinterpret_cast<const uint4*>(xs + (size_t)(g + 8) * d + col)
+                               : make_uint4(0, 0, 0, 0);
+          mma16816(D1, alo[i].x, ahi[i].x, alo[i].y, ahi[i].y, xc.x, xc.y);
+          mma16816(D1, alo[i].z, ahi[i].z, alo[i].w, ahi[i].w, xc.z, xc.w);
+        }
+      }
+      // D[m][n]: lane (g, q) holds (g, 2q), (g, 2q+1), (g+8, 2q), (g+8, 2q+1)
+      float* zp = a.zpart + (size_t)s * T * F;
+      const int t0 = 2 * q;
+      if (t0 < T) {
+        zp[(size_t)t0 * F + u0 + g] = D0[0];
+        zp[(size_t)t0 * F + u0 + g + 8] = D0[2];
+      }
+      if (t0 + 1 < T) {
+        zp[(size_t)(t0 + 1) * F + u0 + g] = D0[1];
+        zp[(size_t)(t0 + 1) * F + u0 + g + 8] = D0[3];
+      }
+      if (two_n) {
+        if (t0 + 8 < T) {
+          zp[(size_t)(t0 + 8) * F + u0 + g] = D1[0];
+          zp[(size_t)(t0 + 8) * F + u0 + g + 8] = D1[2];
+        }
+        if (t0 + 9 < T) {
+          zp[(size_t)(t0 + 9) * F + u0 + g] = D1[1];
+          zp[(size_t)(t0 + 9) * F + u0 + g + 8] = D1[3];
+        }
+      }
+    }
+  }
+  grid_barrier(a, 1);
+
+  // ------------------------------------------------------ B: TwELL pack --
+  {
+    const unsigned lt = (1u << lane) - 1u;
+    for (int item = gw; item < K * T; item += nwarps) {
+      const int k = item / T, t = item % T;
+      uint16_t gv[4];
+      unsigned bal[4];
+      int n = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int u = k * kW + lane + 32 * i;
+        float z = 0.f;
+        for (int s = 0; s < a.S; ++s) z += a.zpart[((size_t)s * T + t) * F + u];
+        const float zr = (int32_t)__float_as_uint(z) > 0 ? z : 0.0f;  // ReLU, -0 -> +0
+        gv[i] = f32_to_bf16(zr);
+        bal[i] = __ballot_sync(FULL, gv[i] != 0);
+        n += __popc(bal[i]);
+        if (a.dump) a.dump[(size_t)t * F + u] = gv[i];
+      }
+      const size_t off = (size_t)k * T + t;
+      const int C = a.C;
+      int before = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int pos = before + __popc(bal[i] & lt);
+        if (gv[i] != 0) {
+          if (pos < C) {
+            a.val[off * C + pos] = gv[i];
+            a.idx[off * C + pos] = (uint8_t)(lane + 32 * i);
+          }
+          a.jtile[(size_t)t * F + k * kW + pos] = k * kW + lane + 32 * i;
+          a.gtile[(size_t)t * F + k * kW + pos] = bf16_to_f32(gv[i]);
+        }
+        before += __popc(bal[i]);
+      }
+      for (int sl = lane; sl < C; sl += 32) {
+        if (sl >= n) {
+          a.val[off * C + sl] = 0;
+          a.idx[off * C + sl] = 0;
+        }
+      }
+      if (lane == 0) a.cnt[off] = (uint8_t)n;
+      if (n > C) {  // uniform across the warp
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(a.spill_n, 1);
+        slot = __shfl_sync(FULL, slot, 0);
+        if (slot < a.spill_cap) {
+          if (lane == 0) {
+            a.spill_ref[off] = slot;
+            a.spill_tk[2 * (size_t)slot] = t;
+            a.spill_tk[2 * (size_t)slot + 1] = k;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a.spill_val[(size_t)slot * kW + lane + 32 * i] = gv[i];
+        } else if (lane == 0) {
+          a.spill_ref[off] = -1;
+          set_status(a.status, kStatusSpill);
+        }
+      }
+    }
+  }
+  grid_barrier(a, 2);
+
+  // ------------------------------------------- C: h = g (x_t . Wu_t[j]) --
+  {
+    const int R = nwarps / T;  // warps per token
+    const int t = gw % T, r = gw / T;
+    if (r < R) {
+      const int m = R >= K ? R / K : 1;  // warps per tile
+      const bool spread = R >= K;
+      const int k_first = spread ? r % K : r;
+      const int sub = spread ? r / K : 0;
+      const bool active = !spread || r < m * K;
+      for (int k = k_first; active && k < K; k += spread ? K : R) {
+        const int n = a.cnt[(size_t)k * T + t];
+        if (n == 0) continue;
+        // ordinal of the tile's first entry: the counts of the tiles below k
+        int pre = 0;
+        for (int kb = 0; kb < k; kb += 32) {
+          const int kk = kb + lane;
+          pre += kk < k ? (int)a.cnt[(size_t)kk * T + t] : 0;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(FULL, pre, o);
+        for (int s = sub; s < n; s += m) {
+          const int j = a.jtile[(size_t)t * F + k * kW + s];
+          const float gval = a.gtile[(size_t)t * F + k * kW + s];
+          const uint16_t* wr = a.Wu + (size_t)j * d;
+          float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+          for (int c = lane * 8; c < d; c += 256) {
+            const uint4 w = __ldg(reinterpret_cast<const uint4*>(wr + c));
+            const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)t * d + c);
+            p[0] = fmaf(bf16_lo(xv.x), bf16_lo(w.x), p[0]);
+            p[1] = fmaf(bf16_hi(xv.x), bf16_hi(w.x), p[1]);
+            p[2] = fmaf(bf16_lo(xv.y), bf16_lo(w.y), p[2]);
+            p[3] = fmaf(bf16_hi(xv.y), bf16_hi(w.y), p[3]);
+            p[0] = fmaf(bf16_lo(xv.z), bf16_lo(w.z), p[0]);
+            p[1] = fmaf(bf16_hi(xv.z), bf16_hi(w.z), p[1]);
+            p[2] = fmaf(bf16_lo(xv.w), bf16_lo(w.w), p[2]);
+            p[3] = fmaf(bf16_hi(xv.w), bf16_hi(w.w), p[3]);
+          }
+          const float u = warp_sum((p[0] + p[1]) + (p[2] + p[3]));
+          if (lane == 0) {
+            a.jc[(size_t)t * F + pre + s] = j;
+            a.hc[(size_t)t * F + pre + s] = gval * u;
+          }
+        }
+      }
+      // the token's entry count, once per token
+      if (r == 0) {
+        int tot = 0;
+        for (int kb = 0; kb < K; kb += 32) {
+          const int kk = kb + lane;
+          tot += kk < K ? (int)a.cnt[(size_t)kk * T + t] : 0;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(FULL, tot, o);
+        if (lane == 0) a.nent[t] = tot;
+      }
+    }
+  }
+  grid_barrier(a, 3);
+
+  // ------------------------------------------------ D: y_t = sum h Wd[j] --
+  {
+    const int nsl = (d + kSlice - 1) / kSlice;
+    for (int task = blockIdx.x; task < T * nsl; task += gridDim.x) {
+      const int t = task / nsl, sl = task % nsl;
+      const int col = sl * kSlice + lane * 8;
+      const bool in = col < d;
+      const int n = a.nent[t];
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int e0 = warp; e0 < n; e0 += 4 * kWarpsD) {
+        int jj[4];
+        float hh[4];
+        uint4 wv[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int e = e0 + b * kWarpsD;
+          jj[b] = e < n ? a.jc[(size_t)t * F + e] : 0;
+          hh[b] = e < n ? a.hc[(size_t)t * F + e] : 0.f;
+        }
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          wv[b] = in && e0 + b * kWarpsD < n
+                      ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
+                      : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          acc[0] = fmaf(hh[b], bf16_lo(wv[b].x), acc[0]);
+          acc[1] = fmaf(hh[b], bf16_hi(wv[b].x), acc[1]);
+          acc[2] = fmaf(hh[b], bf16_lo(wv[b].y), acc[2]);
+          acc[3] = fmaf(hh[b], bf16_hi(wv[b].y), acc[3]);
+          acc[4] = fmaf(hh[b], bf16_lo(wv[b].z), acc[4]);
+          acc[5] = fmaf(hh[b], bf16_hi(wv[b].z), acc[5]);
+          acc[6] = fmaf(hh[b], bf16_lo(wv[b].w), acc[6]);
+          acc[7] = fmaf(hh[b], bf16_hi(wv[b].w), acc[7]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) red[warp * kSlice + lane * 8 + i] = acc[i];
+      __syncthreads();
+      if (warp == 0 && in) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = red[lane * 8 + i];
+        for (int w = 1; w < kWarpsD; ++w)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] += red[w * kSlice + lane * 8 + i];
+        if (a.y_bf16) {
+          uint16_t* yt = static_cast<uint16_t*>(a.y) + (size_t)t * d + col;
+          *reinterpret_cast<uint4*>(yt) =
+              make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+        } else {
+          float4* yt = reinterpret_cast<float4*>(static_cast<float*>(a.y) + (size_t)t * d + col);
+          yt[0] = make_float4(v[0], v[1], v[2], v[3]);
+          yt[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+      }
+      __syncthreads();  // red is reused by the next task
+    }
+  }
+
+  // leave the barrier counters at zero for the next call: the last CTA to
+  // depart (all CTAs have passed every barrier) resets them
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int prev = atomicAdd(&a.bar[1], 1);
+    if (prev == (int)gridDim.x - 1) {
+      atomicExch(&a.bar[0], 0);
+      atomicExch(&a.bar[1], 0);
+    }
+  }
+}
+
+size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace layout for (T, d, F); pointers set when base is not null.
+size_t decode_layout(void* base, int T, int d, int F, DecodeArgs* a) {
+  const int S = (d + kSlice - 1) / kSlice;
+  size_t off = 0;
+  auto take = [&](size_t b) { const size_t o = off; off = al256(off + b); return o; };
+  const size_t o_bar = take(2 * sizeof(int32_t));
+  const size_t o_z = take(sizeof(float) * (size_t)S * T * F);
+  const size_t o_jt = take(sizeof(int32_t) * (size_t)T * F);
+  const size_t o_gt = take(sizeof(float) * (size_t)T * F);
+  const size_t o_jc = take(sizeof(int32_t) * (size_t)T * F);
+  const size_t o_hc = take(sizeof(float) * (size_t)T * F);
+  const size_t o_n = take(sizeof(int32_t) * (size_t)T);
+  if (base && a) {
+    char* p = static_cast<char*>(base);
+    a->S = S;
+    a->bar = reinterpret_cast<int32_t*>(p + o_bar);
+    a->zpart = reinterpret_cast<float*>(p + o_z);
+    a->jtile = reinterpret_cast<int32_t*>(p + o_jt);
+    a->gtile = reinterpret_cast<float*>(p + o_gt);
+    a->jc = reinterpret_cast<int32_t*>(p + o_jc);
+    a->hc = reinterpret_cast<float*>(p + o_hc);
+    a->nent = reinterpret_cast<int32_t*>(p + o_n);
+  }
+  return off;
+}
+
+}  // namespace
+
+size_t decode_ws_bytes(int T, int d, int F) { return decode_layout(nullptr, T, d, F, nullptr); }
+
+cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t, const void* Wd,
+                               int T, int d, int F, const tw_twell& out, void* dump, void* y,
+                               tw_dtype y_dtype, void* ws, int32_t* status, cudaStream_t stream) {
+  DecodeArgs a{};
+  decode_layout(ws, T, d, F, &a);
+  a.x = static_cast<const uint16_t*>(x);
+  a.Wg = static_cast<const uint16_t*>(Wg_t);
+  a.Wu = static_cast<const uint16_t*>(Wu_t);
+  a.Wd = static_cast<const uint16_t*>(Wd);
+  a.T = T;
+  a.d = d;
+  a.F = F;
+  a.C = out.C;
+  a.val = static_cast<uint16_t*>(out.val);
+  a.idx = out.idx;
+  a.cnt = out.cnt;
+  a.spill_ref = out.spill_ref;
+  a.spill_cap = out.spill_cap;
+  a.spill_tk = out.spill_tk;
+  a.spill_val = static_cast<uint16_t*>(out.spill_val);
+  a.spill_n = out.spill_n;
+  a.dump = static_cast<uint16_t*>(dump);
+  a.y = y;
+  a.y_bf16 = y_dtype == TW_BF16;
+  a.status = status;
+  a.timeout_ns = kWaitTimeoutNs;
+  const size_t smem = (size_t)kMaxTokD * d * 2 + sizeof(float) * kWarpsD * kSlice;
+  cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(decode_step_kernel), (int)smem);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&a};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(decode_step_kernel),
+                                     dim3(num_sms()), dim3(kThreadsD), args, smem, stream);
+}
+
+}  // namespace tw

@@ -2,8 +2,9 @@
 // the CUDA cores ("Sparser, Faster, Lighter Transformer Language Models",
 // technical summary, section 2.1).  TF32 tensor cores would not reach fp32
 // accuracy, so the fp32 path uses FMA with a fixed accumulation order
-// (i = 0 .. d-1).  One CTA computes one 128-token x 128-unit tile of z in
-// shared memory, then each thread packs its own token row.
+// (i = 0 .. d-1).  One CTA computes one 128-token x W-unit tile of z in
+// shared memory (W the TwELL tile width), then each thread packs its own
+// token row.
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -11,19 +12,24 @@ namespace tw {
 namespace {
 
 constexpr int ROWS = 128;   // tokens per CTA
-constexpr int TILE = 128;   // TwELL tile width W
 constexpr int KC = 64;      // reduction chunk staged in shared memory
 constexpr int UC = 32;      // units per register chunk
 constexpr int XS_LD = KC + 1;
-constexpr int SEG_LD = TILE + 1;
-constexpr size_t SMEM = sizeof(float) * ((size_t)ROWS * XS_LD + (size_t)UC * XS_LD +
-                                         (size_t)ROWS * SEG_LD);
 
+// TILE: the TwELL tile width W (64, 128 or 256).
+template <int TILE>
+constexpr size_t smem_f32() {
+  return sizeof(float) *
+         ((size_t)ROWS * XS_LD + (size_t)UC * XS_LD + (size_t)ROWS * (TILE + 1));
+}
+
+template <int TILE>
 __global__ void __launch_bounds__(ROWS)
     gate_twell_f32_kernel(const float* __restrict__ x, const float* __restrict__ Wg_t, int T,
                           int d, int F, int C, float* val, uint8_t* idx, uint8_t* cnt,
                           int32_t* spill_ref, int spill_cap, int32_t* spill_tk, float* spill_val,
                           int32_t* spill_n, float* dump, int32_t* status) {
+  constexpr int SEG_LD = TILE + 1;
   extern __shared__ float sh[];
   float* xs = sh;                      // [ROWS][XS_LD]
   float* wsm = xs + ROWS * XS_LD;      // [UC][XS_LD]
@@ -79,7 +85,9 @@ __global__ void __launch_bounds__(ROWS)
     val[kt * C + s] = 0.f;
     idx[kt * C + s] = 0;
   }
-  cnt[kt] = (uint8_t)n;
+  // a full 256-wide tile has no uint8 count: stored as 255 and flagged
+  if (n > 255) set_status(status, 1 << TW_ERR_UNSUPPORTED);
+  cnt[kt] = (uint8_t)(n < 255 ? n : 255);
   if (n > C) {
     const int slot = atomicAdd(spill_n, 1);
     if (slot < spill_cap) {
@@ -99,19 +107,31 @@ __global__ void __launch_bounds__(ROWS)
 
 }  // namespace
 
-cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int d, int F,
-                                  const tw_twell& out, float* dump, int32_t* status,
-                                  cudaStream_t stream) {
-  cudaError_t e =
-      set_smem_limit(reinterpret_cast<const void*>(gate_twell_f32_kernel), (int)SMEM);
+namespace {
+
+template <int TILE>
+cudaError_t launch_f32_w(const float* x, const float* Wg_t, int T, int d, int F,
+                         const tw_twell& out, float* dump, int32_t* status, cudaStream_t stream) {
+  cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(gate_twell_f32_kernel<TILE>),
+                                 (int)smem_f32<TILE>());
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(out.spill_n, 0, sizeof(int32_t), stream);
   if (e != cudaSuccess) return e;
   dim3 grid((T + ROWS - 1) / ROWS, F / TILE);
-  gate_twell_f32_kernel<<<grid, ROWS, SMEM, stream>>>(
+  gate_twell_f32_kernel<TILE><<<grid, ROWS, smem_f32<TILE>(), stream>>>(
       x, Wg_t, T, d, F, out.C, static_cast<float*>(out.val), out.idx, out.cnt, out.spill_ref,
       out.spill_cap, out.spill_tk, static_cast<float*>(out.spill_val), out.spill_n, dump, status);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int d, int F,
+                                  const tw_twell& out, float* dump, int32_t* status,
+                                  cudaStream_t stream) {
+  if (out.W == 64) return launch_f32_w<64>(x, Wg_t, T, d, F, out, dump, status, stream);
+  if (out.W == 256) return launch_f32_w<256>(x, Wg_t, T, d, F, out, dump, status, stream);
+  return launch_f32_w<128>(x, Wg_t, T, d, F, out, dump, status, stream);
 }
 
 }  // namespace tw

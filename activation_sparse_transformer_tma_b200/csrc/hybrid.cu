@@ -16,7 +16,6 @@ namespace tw {
 namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
-constexpr int W = 128;
 
 template <typename T>
 TW_DEV float ld_scalar(const T* p, size_t i);
@@ -166,7 +165,7 @@ TW_DEV void for_each_chunk(const HView<T>& h, int t, int slot, int nnz, int lane
 // Warp per token: row_nnz, and the ELL row when nnz <= C_h.
 template <typename T>
 __global__ void __launch_bounds__(256)
-    hyb_rows_kernel(int Tn, int F, int C, const uint8_t* cnt, const T* val, const uint8_t* idx,
+    hyb_rows_kernel(int Tn, int F, int W, int C, const uint8_t* cnt, const T* val, const uint8_t* idx,
                     const int32_t* spill_ref, int spill_cap, const T* spill_val, int C_h,
                     T* ell_g, uint16_t* ell_idx, int32_t* row_nnz, int32_t* status) {
   const int lane = threadIdx.x & 31;
@@ -337,7 +336,7 @@ __global__ void __launch_bounds__(SCAN_THREADS)
 }
 
 // Warp per backup slot: dense g row from TwELL (zero fill, then scatter).
-template <typename T>
+template <typename T, int W>
 __global__ void __launch_bounds__(256)
     hyb_backup_kernel(int Tn, int F, int C, const uint8_t* cnt, const T* val, const uint8_t* idx,
                       const int32_t* spill_ref, int spill_cap, const T* spill_val,
@@ -684,16 +683,19 @@ template <typename T>
 cudaError_t to_hybrid_t(const tw_twell& g, const tw_hybrid& o, int32_t* status, cudaStream_t s) {
   if (g.T == 0) return cudaSuccess;
   hyb_rows_kernel<T><<<warp_blocks(g.T), 256, 0, s>>>(
-      g.T, g.F, g.C, g.cnt, static_cast<const T*>(g.val), g.idx, g.spill_ref, g.spill_cap,
+      g.T, g.F, g.W, g.C, g.cnt, static_cast<const T*>(g.val), g.idx, g.spill_ref, g.spill_cap,
       static_cast<const T*>(g.spill_val), o.C_h, static_cast<T*>(o.ell_g), o.ell_idx, o.row_nnz,
       status);
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(0, g.T, o.row_nnz, o.C_h, o.row_slot, o.backup_rows,
                                          o.backup_cap, o.n_backup, status);
-  if (o.backup_cap > 0)
-    hyb_backup_kernel<T><<<warp_blocks(o.backup_cap), 256, 0, s>>>(
+  if (o.backup_cap > 0) {
+    auto kern = g.W == 64 ? hyb_backup_kernel<T, 64>
+                          : (g.W == 256 ? hyb_backup_kernel<T, 256> : hyb_backup_kernel<T, 128>);
+    kern<<<warp_blocks(o.backup_cap), 256, 0, s>>>(
         g.T, g.F, g.C, g.cnt, static_cast<const T*>(g.val), g.idx, g.spill_ref, g.spill_cap,
         static_cast<const T*>(g.spill_val), o.backup_rows, o.n_backup, o.backup_cap,
         static_cast<T*>(o.backup_g));
+  }
   return cudaGetLastError();
 }
 

@@ -196,13 +196,29 @@ TW_DEV uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return desc;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile written by TMA
+// in boxes of 64 rows (K) x 64 bf16 (MN, 128 B) with 128-byte swizzling: one
+// swizzle atom is 8 K-rows x 64 MN-elements (1024 B), K-row groups of 8 are
+// 1024 B apart (stride offset) and the next 64 MN-elements start one box,
+// lbo_bytes, later (leading offset).  The tile base must be 1024-B aligned.
+TW_DEV uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+  uint64_t desc = 0;
+  desc |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  desc |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  desc |= (uint64_t)(1024u >> 4) << 32;
+  desc |= (uint64_t)1 << 46;
+  desc |= (uint64_t)2 << 61;
+  return desc;
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D.
 // Bits: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B
-// format (1 = bf16), [15] A major, [16] B major (0 = K), [17,23) N>>3,
+// format (1 = bf16), [15] A major, [16] B major (0 = K, 1 = MN), [17,23) N>>3,
 // [24,29) M>>4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false,
+                                                     bool b_mn = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace tw

@@ -26,6 +26,11 @@ tw_status check_twell(const tw_twell* g);
 // Default upper bound on any single pipeline wait inside a kernel (ns).
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 
+// Test aid of the bounded waits: the wait limit armed by
+// tw_test_withhold_next_gate_loads (0 if none), consumed by the next tile-GEMM
+// gate launch.
+unsigned long long take_withheld_gate_wait();
+
 // tcgen05 bf16 gate GEMM with TwELL epilogue.  Shapes validated by caller.
 cudaError_t launch_gate_twell_tc(const void* x, const void* Wg_t, int T, int d, int F,
                                  const tw_twell& out, void* dump, int32_t* status,
@@ -40,6 +45,13 @@ cudaError_t launch_gate_twell_few(const void* x, const void* Wg_t, int T, int d,
 cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int d, int F,
                                   const tw_twell& out, float* dump, int32_t* status,
                                   cudaStream_t stream);
+// The whole FFN of 1 <= T <= kDecodeStepMaxT tokens (bf16, W = 128) in one
+// cooperative launch: gate + TwELL packing, then the fused up + down.
+constexpr int kDecodeStepMaxT = 16;
+size_t decode_ws_bytes(int T, int d, int F);
+cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t, const void* Wd,
+                               int T, int d, int F, const tw_twell& out, void* dump, void* y,
+                               tw_dtype y_dtype, void* ws, int32_t* status, cudaStream_t stream);
 // Fused up+down over TwELL (plan + persistent gather kernel).
 size_t fused_ws_bytes(int T, int d);
 cudaError_t launch_fused_updown(const void* x, const tw_twell& g, const void* Wu_t,
@@ -56,6 +68,18 @@ cudaError_t launch_dense_gateup_tc(const void* x, const void* Wg_t, const void* 
                                    int d, int F, void* h, int32_t* status, cudaStream_t stream);
 cudaError_t launch_dense_down_tc(const void* h, const void* Wd_dense, int T, int d, int F,
                                  void* y, int32_t* status, cudaStream_t stream);
+// Dense training comparator (bf16, tcgen05): forward saves g, u, h [T][F]
+// bf16 and writes y fp32; backward uses du, dz [T][F] bf16 scratch.
+cudaError_t launch_dense_train_forward(const void* x, const void* Wg_t, const void* Wu_t,
+                                       const void* Wd, int T, int d, int F, uint16_t* g,
+                                       uint16_t* u, uint16_t* h, float* y, int32_t* status,
+                                       cudaStream_t stream);
+cudaError_t launch_dense_train_backward(const void* x, const void* dy, const void* Wg_t,
+                                        const void* Wu_t, const void* Wd, int T, int d, int F,
+                                        float lam, const uint16_t* g, const uint16_t* u,
+                                        const uint16_t* h, uint16_t* du, uint16_t* dz, float* dx,
+                                        float* dWg_t, float* dWu_t, float* dWd, int32_t* status,
+                                        cudaStream_t stream);
 // One active (t, j) entry of the hybrid backward, recorded for the
 // weight-gradient pass: h = g u, du, dz.
 struct Payload {

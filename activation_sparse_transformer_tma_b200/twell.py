@@ -23,10 +23,13 @@ STATUS = ["TW_OK", "TW_ERR_INVALID_ARG", "TW_ERR_UNSUPPORTED", "TW_ERR_ALIGNMENT
           "TW_ERR_CUDA", "TW_ERR_SPILL_CAPACITY", "TW_ERR_BACKUP_CAPACITY",
           "TW_ERR_TIMEOUT", "TW_ERR_WORKSPACE"]
 EXPORTS = ["twell_gate_gemm", "twell_fused_updown_workspace_size", "twell_fused_updown",
-           "twell_fused_updown_noalloc", "twell_to_hybrid", "hybrid_ffn_forward_workspace_size",
+           "twell_fused_updown_noalloc", "twell_ffn_small_batch_workspace_size",
+           "twell_ffn_small_batch", "twell_to_hybrid", "hybrid_ffn_forward_workspace_size",
            "hybrid_ffn_forward",
            "hybrid_ffn_backward_workspace_size", "hybrid_ffn_backward", "dense_ffn_forward",
-           "tw_status_string", "twell_version"]
+           "dense_ffn_train_workspace_size", "dense_ffn_train_saved_bytes",
+           "dense_ffn_train_forward", "dense_ffn_train_backward",
+           "tw_test_withhold_next_gate_loads", "tw_status_string", "twell_version"]
 
 
 class TwellError(RuntimeError):
@@ -74,6 +77,10 @@ def lib():
                                          ctypes.c_size_t, vp, vp]
         L.twell_fused_updown_noalloc.argtypes = [vp, PT, vp, vp, i32, vp, ctypes.c_int, vp, vp]
         L.twell_fused_updown_noalloc.restype = st
+        L.twell_ffn_small_batch_workspace_size.argtypes = [i32, i32, i32]
+        L.twell_ffn_small_batch_workspace_size.restype = ctypes.c_size_t
+        L.twell_ffn_small_batch.argtypes = [vp, vp, vp, vp, i32, i32, i32, PT, vp, vp,
+                                            ctypes.c_int, vp, ctypes.c_size_t, vp, vp]
         L.twell_to_hybrid.argtypes = [PT, PH, vp, vp]
         L.hybrid_ffn_forward_workspace_size.argtypes = [i32, i32]
         L.hybrid_ffn_forward_workspace_size.restype = ctypes.c_size_t
@@ -84,11 +91,23 @@ def lib():
         L.hybrid_ffn_backward.argtypes = [vp, vp, PH, vp, vp, vp, i32, ctypes.c_float, vp,
                                           ctypes.c_int, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
         L.dense_ffn_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
+        L.dense_ffn_train_workspace_size.argtypes = [i32, i32]
+        L.dense_ffn_train_workspace_size.restype = ctypes.c_size_t
+        L.dense_ffn_train_saved_bytes.argtypes = [i32, i32]
+        L.dense_ffn_train_saved_bytes.restype = ctypes.c_size_t
+        L.dense_ffn_train_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, ctypes.c_size_t,
+                                              vp, vp, vp]
+        L.dense_ffn_train_backward.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, ctypes.c_float,
+                                               vp, ctypes.c_size_t, vp, vp, vp, vp, vp, vp]
+        L.tw_test_withhold_next_gate_loads.argtypes = [ctypes.c_uint64]
+        L.tw_test_withhold_next_gate_loads.restype = None
         L.tw_status_string.argtypes = [st]
         L.tw_status_string.restype = ctypes.c_char_p
         L.twell_version.restype = i32
-        for name in ("twell_gate_gemm", "twell_fused_updown", "twell_to_hybrid",
-                     "hybrid_ffn_forward", "hybrid_ffn_backward", "dense_ffn_forward"):
+        for name in ("twell_gate_gemm", "twell_fused_updown", "twell_ffn_small_batch",
+                     "twell_to_hybrid",
+                     "hybrid_ffn_forward", "hybrid_ffn_backward", "dense_ffn_forward",
+                     "dense_ffn_train_forward", "dense_ffn_train_backward"):
             getattr(L, name).restype = st
         _lib = L
     return _lib
@@ -210,6 +229,28 @@ def twell_fused_updown_noalloc(x, g: Twell, Wu_t, Wd, y, dev_status=None, stream
         _ptr(dev_status), _stream(stream)))
 
 
+def twell_ffn_small_batch_workspace_size(T, d, F):
+    return int(lib().twell_ffn_small_batch_workspace_size(T, d, F))
+
+
+def small_batch_workspace(T, d, F, device="cuda"):
+    """A zero-filled workspace for twell_ffn_small_batch (its barrier counters
+    must start at zero; each call leaves them at zero)."""
+    return torch.zeros(twell_ffn_small_batch_workspace_size(T, d, F), dtype=torch.uint8,
+                       device=device)
+
+
+def twell_ffn_small_batch(x, Wg_t, Wu_t, Wd, g: Twell, y, ws, g_dense_dump=None, dev_status=None,
+                          stream=None):
+    T, d = x.shape
+    F = Wg_t.shape[0]
+    s = g.struct()
+    _check("twell_ffn_small_batch", lib().twell_ffn_small_batch(
+        _ptr(x), _ptr(Wg_t), _ptr(Wu_t), _ptr(Wd), T, d, F, ctypes.byref(s), _ptr(g_dense_dump),
+        _ptr(y), _dt(y), _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status),
+        _stream(stream)))
+
+
 def twell_to_hybrid(g: Twell, out: Hybrid, dev_status=None, stream=None):
     sg, sh = g.struct(), out.struct()
     _check("twell_to_hybrid", lib().twell_to_hybrid(
@@ -251,6 +292,43 @@ def dense_ffn_forward(x, Wg_t, Wu_t, Wd_dense, h_ws, y, dev_status=None, stream=
     _check("dense_ffn_forward", lib().dense_ffn_forward(
         _ptr(x), _ptr(Wg_t), _ptr(Wu_t), _ptr(Wd_dense), T, d, F, _ptr(h_ws), _ptr(y),
         _ptr(dev_status), _stream(stream)))
+
+
+def dense_ffn_train_workspace_size(T, F):
+    return int(lib().dense_ffn_train_workspace_size(T, F))
+
+
+def dense_ffn_train_saved_bytes(T, F):
+    return int(lib().dense_ffn_train_saved_bytes(T, F))
+
+
+def dense_train_workspace(T, F, device="cuda"):
+    """A caller-owned workspace tensor for the dense training comparator."""
+    return torch.empty(dense_ffn_train_workspace_size(T, F), dtype=torch.uint8, device=device)
+
+
+def dense_ffn_train_forward(x, Wg_t, Wu_t, Wd, ws, y, dev_status=None, stream=None):
+    T, d = x.shape
+    F = Wg_t.shape[0]
+    _check("dense_ffn_train_forward", lib().dense_ffn_train_forward(
+        _ptr(x), _ptr(Wg_t), _ptr(Wu_t), _ptr(Wd), T, d, F, _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(y), _ptr(dev_status), _stream(stream)))
+
+
+def dense_ffn_train_backward(x, dy, Wg_t, Wu_t, Wd, l1_lambda, ws, dx, dWg_t, dWu_t, dWd,
+                             dev_status=None, stream=None):
+    T, d = x.shape
+    F = Wg_t.shape[0]
+    _check("dense_ffn_train_backward", lib().dense_ffn_train_backward(
+        _ptr(x), _ptr(dy), _ptr(Wg_t), _ptr(Wu_t), _ptr(Wd), T, d, F, float(l1_lambda),
+        _ptr(ws), ws.numel() * ws.element_size(), _ptr(dx), _ptr(dWg_t), _ptr(dWu_t), _ptr(dWd),
+        _ptr(dev_status), _stream(stream)))
+
+
+def dense_train_saved(ws, T, F):
+    """Views of the g, u, h [T][F] bf16 tensors the training forward saved in ws."""
+    part = (T * F * 2 + 255) // 256 * 256
+    return [ws[i * part:i * part + T * F * 2].view(torch.bfloat16).view(T, F) for i in range(3)]
 
 
 def status_bits(dev_status) -> list:

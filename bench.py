@@ -478,14 +478,17 @@ def sm_max_mhz():
 
 
 def decode_leg(torch, tw, hbm):
-    """Small batches (T = 1, 8, 64) of the 2B shape with a cold L2: a 512 MB
+    """Small batches (T = 1, 8, 16, 64) of the 2B shape with a cold L2: a 512 MB
     buffer is READ between iterations, which leaves L2 full of clean lines of
     that buffer (a write flush would leave ~126 MB of dirty lines whose
-    write-back the next kernel would pay for).  The gate streams Wg from HBM."""
+    write-back the next kernel would pay for).  Two paths: the gate and fused
+    calls (twell_gate_gemm + twell_fused_updown), and for T <= 16 the whole
+    FFN in one cooperative launch (twell_ffn_small_batch).  The step streams
+    Wg (33.5 MB) and gathers one Wu and one Wd row per active entry."""
     flush = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device="cuda")
     sink = torch.empty((), dtype=torch.float32, device="cuda")
     out = {}
-    for T in (1, 8, 64):
+    for T in (1, 8, 16, 64):
         w = synth.make_workload("decode_2b", T=T)
         d, F, C = w["d"], w["F"], w["C"]
         dev = {k: torch.from_numpy(w[k].view(np.int16)).cuda().view(torch.bfloat16)
@@ -493,7 +496,8 @@ def decode_leg(torch, tw, hbm):
         g = tw.Twell(T, F, C, dtype=torch.bfloat16, spill_cap=4096)
         y = torch.empty((T, d), dtype=torch.float32, device="cuda")
         ws = tw.fused_workspace(T, d)
-        tg, tf = [], []
+        sws = tw.small_batch_workspace(T, d, F) if T <= 16 else None
+        tg, tf, ts = [], [], []
         for it in range(25):
             torch.sum(flush, dim=0, out=sink)
             e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
@@ -502,17 +506,37 @@ def decode_leg(torch, tw, hbm):
             e[1].record()
             tw.twell_fused_updown(dev["x"], g, dev["Wu_t"], dev["Wd"], y, ws)
             e[2].record()
+            if sws is not None:
+                torch.sum(flush, dim=0, out=sink)
+                e1 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e1[0].record()
+                tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, y, sws)
+                e1[1].record()
             torch.cuda.synchronize()
             if it >= 5:
                 tg.append(e[0].elapsed_time(e[1]))
                 tf.append(e[1].elapsed_time(e[2]))
+                if sws is not None:
+                    ts.append(e1[0].elapsed_time(e1[1]))
         nnz = int(g.cnt.to(torch.int64).sum().item())
         mg, mf = float(np.median(tg)), float(np.median(tf))
-        gate_gbs = F * d * 2 / (mg * 1e-3) / 1e9
+        wg_bytes = F * d * 2
+        gate_gbs = wg_bytes / (mg * 1e-3) / 1e9
         rows = nnz * 2 * d * 2  # Wu and Wd rows gathered (an upper bound on unique bytes)
-        out[f"T{T}"] = {"l2": "cold (512 MB read between iterations)", "gate_us": mg * 1e3, "fused_us": mf * 1e3, "tokens_per_s": T / ((mg + mf) * 1e-3),
-                        "gate_hbm_GBps": gate_gbs, "gate_hbm_frac": gate_gbs / hbm,
-                        "fused_gathered_GBps": rows / (mf * 1e-3) / 1e9, "nnz": nnz}
+        r = {"l2": "cold (512 MB read between iterations)", "nnz": nnz,
+             "two_calls": {"gate_us": mg * 1e3, "fused_us": mf * 1e3,
+                           "tokens_per_s": T / ((mg + mf) * 1e-3),
+                           "gate_hbm_GBps": gate_gbs, "gate_hbm_frac": gate_gbs / hbm,
+                           "fused_gathered_GBps": rows / (mf * 1e-3) / 1e9,
+                           "library_launches": 2 if T <= 16 else 5}}
+        if ts:
+            ms = float(np.median(ts))
+            step_gbs = (wg_bytes + rows) / (ms * 1e-3) / 1e9
+            r["single_launch"] = {"step_us": ms * 1e3, "tokens_per_s": T / (ms * 1e-3),
+                                  "bytes": wg_bytes + rows, "hbm_GBps": step_gbs,
+                                  "hbm_frac": step_gbs / hbm, "library_launches": 1,
+                                  "speedup_vs_two_calls": (mg + mf) / ms}
+        out[f"T{T}"] = r
     del flush
     return out
 
@@ -563,13 +587,69 @@ def training_leg(torch, tw, dist=None, world=1):
                 times[n].append(e[i].elapsed_time(e[i + 1]))
     ms = {n: float(np.median(v)) for n, v in times.items()}
     step = sum(ms.values())
+    n_backup = int(hy.n_backup.item())
+    st_sparse = int(st.item())
+    # bytes of the hybrid step: activations kept from the forward for the
+    # backward (the hybrid g and u with indices and row metadata), and the
+    # calls' transient workspaces; exact from the tensors and size queries
+    esz = 2
+    ell = T * C_h * (esz + esz + 2) + 2 * 4 * T
+    saved_alloc = ell + cap * (4 + 2 * F * esz) + 4
+    saved_fit = ell + n_backup * (4 + 2 * F * esz) + 4
+    twell_bytes = sum(t.numel() * t.element_size() for t in (g.val, g.idx, g.cnt, g.spill_ref,
+                                                              g.spill_tk, g.spill_val, g.spill_n))
+    sparse_ws = fws.numel() + ws.numel()
+    del g, hy, fws, ws
+    torch.cuda.empty_cache()
+
+    # the in-library dense bf16 training FFN of the same shape: forward
+    # (saves g, u, h) and backward (dx, dWg, dWu, dWd), tcgen05 GEMMs
+    dws = tw.dense_train_workspace(T, F)
+    dst = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dn = {"dense_forward": [], "dense_backward": []}
+    for it in range(8):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        tw.dense_ffn_train_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], dws, y, dst)
+        e[1].record()
+        tw.dense_ffn_train_backward(dev["x"], dev["dy"], dev["Wg_t"], dev["Wu_t"], dev["Wd"],
+                                    w["lam"], dws, dx, grads.dWg_t, grads.dWu_t, grads.dWd, dst)
+        e[2].record()
+        torch.cuda.synchronize()
+        if it >= 3:
+            dn["dense_forward"].append(e[0].elapsed_time(e[1]))
+            dn["dense_backward"].append(e[1].elapsed_time(e[2]))
+    dms = {n: float(np.median(v)) for n, v in dn.items()}
+    dense_step = sum(dms.values())
+    dense_saved = tw.dense_ffn_train_saved_bytes(T, F)
+    dense_ws = tw.dense_ffn_train_workspace_size(T, F)
+    del dws
     if world > 1:  # the slowest rank sets the step time
         tt = torch.tensor([step], device="cuda")
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         step = float(tt.item())
     out = {"workload": "train_2b", "T": T, "d": d, "F": F, "C": C, "C_h": C_h,
            "ms": ms, "ms_per_step": step, "tokens_per_s": world * T / (step * 1e-3),
-           "n_backup": int(hy.n_backup.item()), "backup_cap": cap, "device_status": int(st.item())}
+           "n_backup": n_backup, "backup_cap": cap, "device_status": st_sparse,
+           "dense": {"ms": dms, "ms_per_step": dense_step,
+                     "tokens_per_s": T / (dense_step * 1e-3),
+                     "flops_per_step": 9 * 2.0 * T * d * F,
+                     "tflops": 9 * 2.0 * T * d * F / (dense_step * 1e-3) / 1e12,
+                     "device_status": int(dst.item())},
+           "sparse_speedup_vs_dense": dense_step / step,
+           "memory_bytes": {
+               "what": "FFN-layer activation bytes per GPU, excluding x, dy, the weights and "
+                       "their gradients (the same for both paths)",
+               "sparse_saved_fwd_to_bwd": saved_alloc,
+               "sparse_saved_fwd_to_bwd_exact_fit": saved_fit,
+               "sparse_twell_transient": twell_bytes,
+               "sparse_workspaces": sparse_ws,
+               "sparse_peak": saved_alloc + max(twell_bytes, sparse_ws),
+               "dense_saved_fwd_to_bwd": dense_saved,
+               "dense_workspace": dense_ws,
+               "dense_peak": dense_ws,
+               "peak_ratio_sparse_over_dense": (saved_alloc + max(twell_bytes, sparse_ws))
+                                               / dense_ws}}
     if world > 1:
         out["parallelism"] = f"dp{world}: one fp32 all-reduce of dWg, dWu, dWd ({3 * F * d * 4} B)"
     return out

@@ -31,7 +31,7 @@
  *             into the caller's `dev_status` word as bit (1 << tw_status);
  *             dev_status may be NULL.  The caller zeroes it and reads it after
  *             synchronising; tw_status_string names each code.
- * Limits      W == 128; 0 <= C <= W; F % W == 0; d % 8 == 0; 8 <= d <= 2048
+ * Limits      W in {64, 128, 256}; 0 <= C <= W; F % W == 0; d % 8 == 0; 8 <= d <= 2048
  *             (bf16 rows) or d <= 1024 (fp32 rows) for the fused and hybrid
  *             kernels; T >= 0.  With T == 0 the arrays sized by T (x, y, dy,
  *             dx, the TwELL and hybrid per-token arrays, the workspaces) may
@@ -89,6 +89,9 @@ typedef enum { TW_F32 = 0, TW_BF16 = 1 } tw_dtype;
  * Array shapes: val [K][T][C] (dtype), idx [K][T][C] uint8, cnt [K][T] uint8,
  * spill_ref [K][T] int32, spill_tk [spill_cap][2] int32, spill_val
  * [spill_cap][W] (dtype), spill_n one int32.  With C == 0 val/idx may be NULL.
+ * A uint8 count holds 0..255: a 256-wide tile whose 256 units are all active
+ * is stored with cnt = 255 and flags TW_ERR_UNSUPPORTED in dev_status (its
+ * spilled segment, when C < 256, still holds every value).
  */
 typedef struct {
   int32_t T, F, W, C;
@@ -201,6 +204,31 @@ TW_API tw_status twell_fused_updown_noalloc(const void* x, const tw_twell* g, co
                                             int32_t* dev_status, cudaStream_t stream);
 
 /*
+ * The whole FFN of a small batch -- decoding, 1 <= T <= 16 tokens -- in ONE
+ * launch (sections 2.1 and 2.2): g = ReLU(x Wg) packed into *g as
+ * twell_gate_gemm packs it, then y = sum over the active units of
+ * g (x . Wu_t[j]) Wd[j], as twell_fused_updown computes it (fp32 accumulation,
+ * deterministic).  bf16 only, g->W == 128, 64 <= d <= 2048, d % 8 == 0.
+ * A small batch is bound by streaming Wg from HBM; separate gate and fused
+ * launches spend more on launches and set-up than on that stream, so this
+ * call runs one persistent cooperative grid (one CTA per SM) whose phases
+ * are separated by grid-wide barriers.  g_dense_dump as in twell_gate_gemm.
+ * ws: at least twell_ffn_small_batch_workspace_size(T, d, F) bytes.  Its
+ * first 256 bytes are barrier counters that must be zero when a call starts:
+ * allocate the workspace zero-filled once; every call leaves them at zero
+ * (after a call that flagged TW_ERR_TIMEOUT, zero them again).  Calls that
+ * share one workspace must not overlap on the device.  The launch fails with
+ * TW_ERR_CUDA if the device cannot hold one CTA per SM for a cooperative
+ * launch.
+ */
+TW_API size_t twell_ffn_small_batch_workspace_size(int32_t T, int32_t d, int32_t F);
+TW_API tw_status twell_ffn_small_batch(const void* x, const void* Wg_t, const void* Wu_t,
+                                       const void* Wd, int32_t T, int32_t d, int32_t F,
+                                       const tw_twell* g, void* g_dense_dump, void* y,
+                                       tw_dtype y_dtype, void* ws, size_t ws_bytes,
+                                       int32_t* dev_status, cudaStream_t stream);
+
+/*
  * TwELL -> hybrid conversion (section 2.3).  out->T, out->F equal g->T,
  * g->F and out->dtype equals g->dtype.  Fills ell_g, ell_idx, row_nnz,
  * row_slot, backup_rows, backup_g, n_backup.
@@ -254,6 +282,48 @@ TW_API tw_status hybrid_ffn_backward(const void* x, const void* dy, const tw_hyb
 TW_API tw_status dense_ffn_forward(const void* x, const void* Wg_t, const void* Wu_t,
                             const void* Wd_dense, int32_t T, int32_t d, int32_t F, void* h_ws,
                             void* y, int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Dense training comparator (the non-sparse baseline of the training results
+ * of section 4), bf16 only, on the same tcgen05 pipeline and with the same
+ * weight layouts as the sparse path (Wg_t, Wu_t, Wd all [F][d]).  One training
+ * step of the gated FFN for the loss L = sum(y * dy) + l1_lambda * sum(g):
+ *   forward   z = x Wg, u = x Wu, g = ReLU(z), h = g u, y = h Wd (y fp32);
+ *   backward  dh = dy Wd^T, du = dh g, dz = (dh u + l1_lambda) where g > 0,
+ *             dx = du Wu^T + dz Wg^T (fp32), and the fp32 weight gradients
+ *             dWd = h^T dy, dWu_t = du^T x, dWg_t = dz^T x ([F][d]).
+ * g, u, h are stored bf16 (g rounded first, as the sparse path stores it);
+ * du and dz are rounded to bf16 as the operands of the dx and weight-gradient
+ * matmuls.  d % 32 == 0, d >= 64, F % 128 == 0, any T >= 0.
+ * ws: at least dense_ffn_train_workspace_size(T, F) bytes: g, u, h [T][F]
+ * bf16 (the activations the forward saves for the backward,
+ * dense_ffn_train_saved_bytes(T, F) bytes) followed by du, dz [T][F] bf16
+ * (backward scratch).  The backward reads what the forward saved in the same
+ * workspace; calls sharing it must not overlap on the device.
+ */
+TW_API size_t dense_ffn_train_workspace_size(int32_t T, int32_t F);
+TW_API size_t dense_ffn_train_saved_bytes(int32_t T, int32_t F);
+TW_API tw_status dense_ffn_train_forward(const void* x, const void* Wg_t, const void* Wu_t,
+                                         const void* Wd, int32_t T, int32_t d, int32_t F,
+                                         void* ws, size_t ws_bytes, float* y,
+                                         int32_t* dev_status, cudaStream_t stream);
+TW_API tw_status dense_ffn_train_backward(const void* x, const void* dy, const void* Wg_t,
+                                          const void* Wu_t, const void* Wd, int32_t T, int32_t d,
+                                          int32_t F, float l1_lambda, void* ws, size_t ws_bytes,
+                                          float* dx, float* dWg_t, float* dWu_t, float* dWd,
+                                          int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Test aid for the bounded pipeline waits; not needed in normal use.  The
+ * next twell_gate_gemm call that runs the tile GEMM (T > 64, or any T when
+ * W != 128) withholds its TMA loads and bounds its waits by wait_limit_ns:
+ * the MMA issuer's first wait can then never complete, so every CTA must give
+ * up after about wait_limit_ns, flag TW_ERR_TIMEOUT in dev_status, stop its
+ * roles, free its tensor memory and return (nothing is in flight, since
+ * nothing was issued).  The TwELL output of that call is not written.  The
+ * setting is consumed by that one call; later calls run normally.
+ */
+TW_API void tw_test_withhold_next_gate_loads(uint64_t wait_limit_ns);
 
 /* Human-readable name of a status code. */
 TW_API const char* tw_status_string(tw_status s);

@@ -70,7 +70,9 @@ def _gate(L, tw, x=FAKE, w=FAKE, T=256, d=512, F=1024, dtype=twell.TW_BF16):
 def test_gate_validation(L):
     assert _gate(L, _tw(), x=None) == INVALID
     assert _gate(L, _tw(), x=FAKE + 8) == ALIGN
-    assert _gate(L, _tw(W=64)) == UNSUPPORTED            # tile width must be 128
+    assert _gate(L, _tw(W=32)) == UNSUPPORTED            # tile widths: 64, 128, 256
+    assert _gate(L, _tw(W=192)) == UNSUPPORTED
+    assert _gate(L, _tw(W=64, C=65)) == UNSUPPORTED      # capacity above the tile width
     assert _gate(L, _tw(C=129)) == UNSUPPORTED           # capacity above the tile width
     assert _gate(L, _tw(F=1000), F=1000) == UNSUPPORTED  # F not a multiple of W
     assert _gate(L, _tw(T=255)) == INVALID               # out->T != T
@@ -153,3 +155,40 @@ def test_dense_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, 256, 100, 1024, FAKE, FAKE, None, None) == UNSUPPORTED
     assert f(FAKE, FAKE, FAKE, FAKE, 256, 512, 1000, FAKE, FAKE, None, None) == UNSUPPORTED
     assert f(None, FAKE, FAKE, FAKE, 256, 512, 1024, FAKE, FAKE, None, None) == INVALID
+
+
+def test_small_batch_validation(L):
+    f = L.twell_ffn_small_batch
+    ws = L.twell_ffn_small_batch_workspace_size(8, 512, 1024)
+    assert ws > 0
+
+    def call(T=8, d=512, F=1024, W=128, dtype=twell.TW_BF16, n=ws, y=FAKE):
+        tw = _tw(T=T, F=F, W=W, dtype=dtype)
+        return f(FAKE, FAKE, FAKE, FAKE, T, d, F, ctypes.byref(tw), None, y, twell.TW_F32, FAKE,
+                 n, None, None)
+
+    assert call(T=17) == UNSUPPORTED                 # up to 16 tokens in one launch
+    assert call(W=64) == UNSUPPORTED                 # tile width 128 only
+    assert call(dtype=twell.TW_F32) == UNSUPPORTED   # bf16 only
+    assert call(d=4096) == UNSUPPORTED               # x of 16 tokens staged in shared memory
+    assert call(d=500) == UNSUPPORTED
+    assert call(n=ws - 1) == 8                       # TW_ERR_WORKSPACE
+    assert call(y=None) == INVALID
+    assert call(y=FAKE + 4) == ALIGN
+
+
+def test_dense_training_validation(L):
+    ws = L.dense_ffn_train_workspace_size(256, 1024)
+    assert ws == 5 * 256 * 1024 * 2
+    assert L.dense_ffn_train_saved_bytes(256, 1024) == 3 * 256 * 1024 * 2
+    fwd = L.dense_ffn_train_forward
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 256, 500, 1024, FAKE, ws, FAKE, None, None) == UNSUPPORTED
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 256, 512, 1000, FAKE, ws, FAKE, None, None) == UNSUPPORTED
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 256, 512, 1024, FAKE, ws - 1, FAKE, None, None) == 8
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 256, 512, 1024, None, ws, FAKE, None, None) == INVALID
+    bwd = L.dense_ffn_train_backward
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 256, 512, 1024, 2e-5, FAKE, ws, FAKE, FAKE, FAKE]
+    assert bwd(*args, None, None, None) == INVALID    # dWd missing
+    args2 = list(args)
+    args2[1] = FAKE + 8
+    assert bwd(*args2, FAKE, None, None) == ALIGN

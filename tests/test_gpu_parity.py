@@ -32,9 +32,10 @@ def run_forward(w, C=None, spill_cap=None, dump=True, y_dtype=torch.float32):
     T, d, F = w["T"], w["d"], w["F"]
     C = w["C"] if C is None else C
     dt = TDT[w["dtype"]]
+    W = w.get("W", 128)
     if spill_cap is None:
-        spill_cap = (F // 128) * T  # room for every (t, k) to spill
-    g = tw.Twell(T, F, C, dtype=dt, spill_cap=spill_cap)
+        spill_cap = (F // W) * T  # room for every (t, k) to spill
+    g = tw.Twell(T, F, C, dtype=dt, spill_cap=spill_cap, W=W)
     gd = torch.empty((T, F), dtype=dt, device="cuda") if dump else None
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, gd, st)
@@ -163,11 +164,50 @@ def test_capacity_up_to_tile_width(T, C, dt):
     check_y(f64(y), w64, rows, TOL[dt], g_round="bf16" if dt == synth.BF16 else "f32")
 
 
+# Tile widths other than 128: the tile GEMM packs BN / W TwELL tiles per
+# accumulator tile (W = 256 always on the 256-wide accumulator), also for
+# small batches; the fp32 gate sizes its tile by W; the fused kernel and the
+# hybrid conversion read W from the TwELL descriptor.
+TILE_W = [
+    # W, T, C, dtype
+    (64, 300, 8, synth.BF16),
+    (256, 300, 8, synth.BF16),
+    (256, 300, 64, synth.BF16),
+    (64, 40, 4, synth.BF16),
+    (256, 33, 16, synth.BF16),
+    (64, 130, 8, synth.F32),
+    (256, 130, 8, synth.F32),
+]
+
+
+@pytest.mark.parametrize("W,T,C,dt", TILE_W)
+def test_tile_widths(W, T, C, dt):
+    d = 256 if dt == synth.F32 else 320
+    w = synth.make_workload(T=T, d=d, F=1024, W=W, C=C, dtype=dt, kind="dead20",
+                            mean_active=60.0, seed=W + T + C)
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    w64 = widened(w)
+    g64 = f64(gd)
+    assert_twell_matches_oracle(g, g64)
+    assert int(g.spill_n.item()) > 0 or C >= 64
+    check_y(f64(y), w64, np.arange(T, dtype=np.int32), TOL[dt],
+            g_round="bf16" if dt == synth.BF16 else "f32")
+
+
+@pytest.mark.parametrize("W", [64, 256])
+def test_hybrid_from_other_tile_widths(W):
+    w = synth.make_workload(T=300, d=256, F=1024, W=W, C=8, C_h=64, dtype=synth.BF16,
+                            kind="pareto", lam=2e-5, seed=W, mean_active=30.0, with_dy=True)
+    got = check_hybrid_all(w, run_hybrid(w, backup_cap=300))
+    assert 0 < got["n_backup"] < 300
+
+
 def test_hybrid_from_wide_capacity_twell():
     """TwELL -> hybrid with C = 64: tiles with more than 32 slots feed ELL rows."""
     w = synth.make_workload(T=300, d=256, F=640, W=128, C=64, C_h=155, dtype=synth.BF16,
                             kind="dead20", lam=2e-5, seed=77, mean_active=150.0, with_dy=True)
-    got = check_hybrid_all(w, run_hybrid(w))
+    got = check_hybrid_all(w, run_hybrid(w, backup_cap=300))
     assert 0 < got["n_backup"] < 300
 
 
@@ -255,6 +295,102 @@ def test_decode_sizes(T):
     check_gate_values(f64(gd), w64["x"], w64["Wg_t"], rows)
     assert_twell_matches_oracle(g, f64(gd))
     check_y(f64(y), w64, rows, TOL[synth.BF16])
+
+
+# One cooperative launch for the whole small-batch FFN: gate partial sums on
+# mma.sync over every SM, TwELL packing, dot products, updates.  T crosses the
+# 8-token MMA column tile; d and F are ragged against the 256-column slices.
+SMALL_STEP = [
+    # T, d, F, C, kind, mean_active
+    (1, 2048, 8192, 8, "zipf", 29.0),
+    (5, 320, 640, 2, "dead20", 60.0),
+    (8, 512, 1024, 8, "zipf", 29.0),
+    (9, 256, 1280, 0, "dead20", 29.0),
+    (16, 2048, 4096, 8, "zipf", 29.0),
+    (16, 1024, 1024, 64, "dead20", 300.0),
+    (3, 64, 256, 128, "dead20", 100.0),
+]
+
+
+@pytest.mark.parametrize("T,d,F,C,kind,ma", SMALL_STEP)
+def test_small_batch_single_launch(T, d, F, C, kind, ma):
+    w = synth.make_workload(T=T, d=d, F=F, W=128, C=C, dtype=synth.BF16, kind=kind,
+                            mean_active=ma, seed=T * 13 + d)
+    dev = inputs(w)
+    g = tw.Twell(T, F, C, dtype=torch.bfloat16, spill_cap=(F // 128) * T)
+    gd = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    ws = tw.small_batch_workspace(T, d, F)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ys = []
+    for _ in range(3):  # the barrier counters reset themselves between calls
+        y = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+        tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, y, ws, gd, st)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, tw.status_bits(st)
+    assert int(ws[:8].view(torch.int32).abs().sum().item()) == 0
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    w64 = widened(w)
+    g64 = f64(gd)
+    rows = np.arange(T, dtype=np.int32)
+    check_gate_values(g64, w64["x"], w64["Wg_t"], rows)
+    assert_twell_matches_oracle(g, g64)
+    check_y(f64(ys[0]), w64, rows, TOL[synth.BF16])
+    # bf16 y: the fp32 result rounded once
+    yb = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, yb, ws, None, st)
+    torch.cuda.synchronize()
+    assert torch.equal(yb, ys[0].to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("T", [1, 8, 16])
+def test_small_batch_single_launch_decode_2b(T):
+    """The decoding workload (the 2B weights, the first T tokens) in the launch
+    configuration the benchmark times."""
+    w = synth.make_workload("decode_2b", T=T)
+    dev = inputs(w)
+    d, F, C = w["d"], w["F"], w["C"]
+    g = tw.Twell(T, F, C, dtype=torch.bfloat16, spill_cap=4096)
+    gd = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, y,
+                             tw.small_batch_workspace(T, d, F), gd, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, tw.status_bits(st)
+    w64 = widened(w)
+    g64 = f64(gd)
+    assert_twell_matches_oracle(g, g64)
+    check_y(f64(y), w64, np.arange(T, dtype=np.int32), TOL[synth.BF16])
+
+
+def test_bounded_wait_runs_out_and_the_next_call_is_correct():
+    """The tile GEMM's waits are bounded.  With its loads withheld (a test aid),
+    the MMA issuer waits on a barrier that no copy will complete; after the
+    20 ms limit every CTA flags TW_ERR_TIMEOUT, frees its tensor memory and
+    returns.  A normal call right after it, on the same stream, packs the
+    TwELL bit-exactly."""
+    import time
+    w = synth.make_workload(T=300, d=256, F=640, W=128, C=8, dtype=synth.BF16, kind="dead20",
+                            mean_active=29.0, seed=5)
+    dev = inputs(w)
+    g = tw.Twell(300, 640, 8, dtype=torch.bfloat16, spill_cap=5 * 300)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    tw.lib().tw_test_withhold_next_gate_loads(20_000_000)
+    t0 = time.perf_counter()
+    tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, None, st)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 2.0
+    assert "TW_ERR_TIMEOUT" in tw.status_bits(st)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gd = torch.empty((300, 640), dtype=torch.bfloat16, device="cuda")
+    tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, gd, st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0, tw.status_bits(st2)
+    g64 = f64(gd)
+    check_gate_values(g64, widened(w)["x"], widened(w)["Wg_t"], np.arange(300, dtype=np.int32))
+    assert_twell_matches_oracle(g, g64)
 
 
 def test_fused_without_dump_matches_dump_run():
@@ -353,6 +489,116 @@ def test_dense_comparator_2b_shape_sampled():
     hr = dense["g"] * dense["u"]
     bound = 2.0 ** -8 * (np.abs(hr) @ np.abs(w64["Wd"])) + 2.0 ** -8 * np.abs(dense["y"])
     assert np.all(np.abs(f64(y)[rows] - dense["y"]) <= bound + 1e-2 * rms(dense["y"]))
+
+
+# ----------------------------------------------------- dense training FFN ---
+def run_dense_training(w):
+    dev = inputs(w)
+    T, d, F = w["T"], w["d"], w["F"]
+    ws = tw.dense_train_workspace(T, F)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    dW = [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+    tw.dense_ffn_train_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], ws, y, st)
+    tw.dense_ffn_train_backward(dev["x"], dev["dy"], dev["Wg_t"], dev["Wu_t"], dev["Wd"],
+                                w["lam"], ws, dx, dW[0], dW[1], dW[2], st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, tw.status_bits(st)
+    g, u, h = tw.dense_train_saved(ws, T, F)
+    return f64(g), f64(u), f64(h), f64(y), f64(dx), [f64(a) for a in dW]
+
+
+def dense_grad_bounds(w64, g64, u64, lam, rows=None, units=None):
+    """Elementwise error bounds of the dense training comparator's gradients
+    from its own arithmetic: du and dz enter the dx and weight-gradient
+    matmuls rounded to bf16 (at most 2^-9 relative each), h enters dWd as
+    bf16(g u) with u unrounded, while the conditioned oracle uses g times the
+    stored u (two bf16 roundings apart); the fp32 accumulation adds far less.
+    Each bound is twice the first-order sum of those roundings, sum |a| |b|
+    over the matmul, so (dx, dWg_t, dWu_t, dWd) on the rows / units given."""
+    x, dy, Wg, Wu, Wd = (w64[k] for k in ("x", "dy", "Wg_t", "Wu_t", "Wd"))
+    if rows is not None:
+        x, dy, g64, u64 = x[rows], dy[rows], g64[rows], u64[rows]
+    dh = dy @ (Wd if units is None else Wd[units]).T
+    if units is not None:
+        g64, u64 = g64[:, units], u64[:, units]
+    du = np.abs(dh * g64)
+    dz = np.abs(np.where(g64 > 0, dh * u64 + lam, 0.0))
+    hh = np.abs(g64 * u64)
+    if units is None:
+        bdx = 2.0 ** -8 * (du @ np.abs(Wu) + dz @ np.abs(Wg))
+    else:
+        bdx = None
+    ax, ady = np.abs(x), np.abs(dy)
+    return bdx, 2.0 ** -8 * (dz.T @ ax), 2.0 ** -8 * (du.T @ ax), 2.0 ** -7 * (hh.T @ ady)
+
+
+def dense_grads_oracle(w64, g64, u64, lam, rows=None, units=None):
+    """The oracle's backward conditioned on the GPU's saved g and u: every
+    token row with a non-zero g is a dense backup row of a hybrid split with
+    C_h = 0, u is kept on the pattern; optionally restricted to token rows
+    (exact for dx of those rows) or to units (exact for their weight rows)."""
+    x, dy, Wg, Wu, Wd = (w64[k] for k in ("x", "dy", "Wg_t", "Wu_t", "Wd"))
+    if rows is not None:
+        x, dy, g64, u64 = x[rows], dy[rows], g64[rows], u64[rows]
+    if units is not None:
+        Wg, Wu, Wd, g64, u64 = Wg[units], Wu[units], Wd[units], g64[:, units], u64[:, units]
+    hy = oracle.hybrid_split(g64, 0)
+    bu = (u64 * (g64 != 0))[hy["backup_rows"]]
+    return oracle.hybrid_backward(x, dy, hy, np.zeros((len(x), 0)), bu, Wg, Wu, Wd, lam)
+
+
+@pytest.mark.parametrize("T,d,F", [(300, 256, 640), (260, 320, 1024), (128, 64, 128)])
+def test_dense_training_comparator(T, d, F):
+    """Ragged T (partial 128-row tiles and 64-row k-blocks of the weight
+    gradients), F not a multiple of 256, d not a multiple of 256."""
+    w = synth.make_workload(T=T, d=d, F=F, W=128, C=8, C_h=64, dtype=synth.BF16, kind="pareto",
+                            lam=2e-5, seed=T + F, mean_active=40.0, with_dy=True)
+    g, u, h, y, dx, dW = run_dense_training(w)
+    w64 = widened(w)
+    rows = np.arange(T, dtype=np.int32)
+    check_gate_values(g, w64["x"], w64["Wg_t"], rows)
+    # u = x Wu rounded once to bf16; h = g u (fp32 u) rounded once to bf16, so
+    # against g times the stored u it is off by at most two bf16 roundings
+    u_ref = w64["x"] @ w64["Wu_t"].T
+    assert np.all(np.abs(u - u_ref) <= 2.0 ** -8 * np.abs(u_ref) + 1e-4 * rms(u_ref))
+    assert np.all(np.abs(h - g * u) <= 2.0 ** -7 * np.abs(g * u))
+    # y against the fp64 FFN: each term of y rounds h once to bf16 (2^-9 relative)
+    out = oracle.dense_ffn(w64["x"], w64["Wg_t"], w64["Wu_t"], w64["Wd"], g_round="bf16")
+    bound = 2.0 ** -8 * (np.abs(out["g"] * out["u"]) @ np.abs(w64["Wd"]))
+    assert np.all(np.abs(y - out["y"]) <= bound + 1e-2 * rms(out["y"]))
+    # gradients: oracle conditioned on the GPU's saved g and u, elementwise
+    # within the bf16-operand bound plus 1e-2 rms
+    ref = dense_grads_oracle(w64, g, u, w["lam"])
+    bnd = dense_grad_bounds(w64, g, u, w["lam"])
+    for name, a, b, e in zip(("dx", "dWg_t", "dWu_t", "dWd"), [dx] + dW, ref, bnd):
+        viol = np.abs(a - b) - (e + 1e-2 * rms(b))
+        assert np.all(viol <= 0), (name, float(np.max(np.abs(a - b))), rms(b), float(viol.max()))
+
+
+def test_dense_training_comparator_train_2b_sampled():
+    """The training workload's full shape (T=8192, d=2048, F=8192): dx on a
+    seeded sample of token rows, the weight gradients on a seeded sample of
+    units, each exact for the rows / units it covers."""
+    w = synth.make_workload("train_2b")
+    g, u, h, y, dx, dW = run_dense_training(w)
+    w64 = widened(w)
+    T, F = w["T"], w["F"]
+    rows = synth.subsample_rows(T, 48, seed=11)
+    units = synth.subsample_rows(F, 48, seed=12)
+    check_gate_values(g, w64["x"], w64["Wg_t"], rows)
+    ref_r = dense_grads_oracle(w64, g, u, w["lam"], rows=rows)
+    bdx = dense_grad_bounds(w64, g, u, w["lam"], rows=rows)[0]
+    assert np.all(np.abs(dx[rows] - ref_r[0]) <= bdx + 1e-2 * rms(ref_r[0]))
+    ref_u = dense_grads_oracle(w64, g, u, w["lam"], units=units)
+    bnd_u = dense_grad_bounds(w64, g, u, w["lam"], units=units)[1:]
+    for name, a, b, e in zip(("dWg_t", "dWu_t", "dWd"), dW, ref_u[1:], bnd_u):
+        err = np.abs(a[units] - b)
+        assert np.all(err <= e + 1e-2 * rms(b)), (name, float(err.max()), rms(b))
+    out = oracle.dense_ffn(w64["x"][rows], w64["Wg_t"], w64["Wu_t"], w64["Wd"], g_round="bf16")
+    bound = 2.0 ** -8 * (np.abs(out["g"] * out["u"]) @ np.abs(w64["Wd"]))
+    assert np.all(np.abs(y[rows] - out["y"]) <= bound + 1e-2 * rms(out["y"]))
 
 
 # ----------------------------------------------------------------- hybrid ---
