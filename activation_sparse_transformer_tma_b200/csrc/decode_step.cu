@@ -8,7 +8,8 @@
 // (d x F bf16, 33.5 MB at d = 2048, F = 8192) plus a few dozen gathered
 // weight rows per token; the separate launches of the gate and the fused
 // kernels (and their set-up) cost more than the data movement itself.  Here
-// one grid, one CTA per SM, runs four phases separated by grid barriers:
+// one grid, one CTA of 16 warps per SM, runs three phases separated by grid
+// barriers:
 //
 //   A  gate: work items of 16 units x 256 columns of d, spread over every
 //      warp of the grid; a warp streams its 16 Wg rows (16-byte loads, eight
@@ -16,27 +17,19 @@
 //      (staged in shared memory) on the tensor pipe: mma.sync m16n8k16 with
 //      the units on M and the tokens on N.  The reduction over d is split
 //      into slices: each item writes fp32 partial sums zpart[slice][t][u].
-//   B  packing: one warp per (tile k, token t) adds the slices in a fixed
-//      order, applies ReLU, rounds g to bf16 and packs the tile's TwELL slots
+//   B  packing and dot products: each (tile k, token t) gets one or more
+//      warps.  Every one of them adds the slices in a fixed order, applies
+//      ReLU and rounds g to bf16; the first packs the tile's TwELL slots
 //      exactly as the gate GEMM's epilogue does (ascending units, count,
-//      padding, lossless spill of the whole segment past C).  It also writes
-//      every non-zero of the tile (unit and g) to a per-token list at stride
-//      W per tile.
-//   C  dot products: the warps of each token split its tiles (and a hot
-//      tile's entries); for an entry (j, g) a warp forms u = x_t . Wu_t[j]
-//      (fp32) and stores h = g u, with j, at the entry's ordinal in the
-//      token's compact list (ordinal = prefix of the tile counts).
-//   D  updates: one CTA per (token, 256-column slice of d); its warps take
-//      the token's entries round-robin, accumulate h Wd[j] over their
+//      padding, lossless spill of the whole segment past C).  The warps then
+//      split the tile's non-zeros: for an entry (j, g) a warp forms
+//      u = x_t . Wu_t[j] (fp32) and stores h = g u and j at the entry's place
+//      in the tile (stride W per tile, ascending within it).
+//   C  updates: one CTA per (token, 256-column slice of d); warp w takes the
+//      tiles k = w (mod 16) in ascending order, accumulates h Wd[j] over its
 //      columns in fp32, and the CTA adds the warps' partial rows in warp
 //      order.  y is therefore deterministic.
 //
-// Grid barriers: an arrival counter in the workspace that every CTA bumps and
-// then polls (bounded by a timeout that flags TW_ERR_TIMEOUT); after the last
-// phase a departure counter lets the last CTA reset both to zero, so the
-// workspace is ready for the next call.  The cooperative launch guarantees
-// that every CTA of the grid is resident, so a barrier cannot wait on a CTA
-// that never starts.
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -44,7 +37,7 @@ namespace tw {
 namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
-constexpr int kWarpsD = 8;
+constexpr int kWarpsD = 16;
 constexpr int kThreadsD = 32 * kWarpsD;
 constexpr int kW = 128;          // TwELL tile width of this path
 constexpr int kSlice = 256;      // columns of d per gate work item
@@ -73,11 +66,8 @@ struct DecodeArgs {
   // workspace
   int32_t* bar;    // [0] arrivals, [1] departures
   float* zpart;    // [S][T][F]
-  int32_t* jtile;  // [T][F]: units of tile k at [k * W, k * W + cnt)
-  float* gtile;    // [T][F]: their g
-  int32_t* jc;     // [T][F]: compact entry list (units)
-  float* hc;       // [T][F]: compact entry list (h)
-  int32_t* nent;   // [T]
+  int32_t* jtile;  // [T][F]: units of the non-zeros of tile k at [k * W, k * W + cnt)
+  float* htile;    // [T][F]: their h = g u
   int32_t* status;
   unsigned long long timeout_ns;
 };
@@ -102,12 +92,13 @@ TW_DEV int ld_acquire(const int32_t* p) {
 TW_DEV void grid_barrier(const DecodeArgs& a, int b) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(&a.bar[0], 1);
+    // release: the CTA's writes (ordered before this thread by the CTA
+    // barrier) become visible before the arrival does
+    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(&a.bar[0]) : "memory");
     const int target = b * (int)gridDim.x;
     uint64_t t0 = 0;
     for (uint32_t i = 0; ld_acquire(&a.bar[0]) < target; ++i) {
-      __nanosleep(64);
+      __nanosleep(32);
       if ((i & 63u) == 63u) {
         const uint64_t now = globaltimer_ns();
         if (t0 == 0) {
@@ -118,7 +109,6 @@ TW_DEV void grid_barrier(const DecodeArgs& a, int b) {
         }
       }
     }
-    __threadfence();
   }
   __syncthreads();
 }
@@ -127,13 +117,15 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   extern __shared__ __align__(16) uint8_t smem[];
   const int T = a.T, d = a.d, F = a.F, K = F / kW;
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [16][d] bf16, rows >= T zero
-  float* red = reinterpret_cast<float*>(smem + (size_t)kMaxTokD * d * 2);  // [8][256]
+  float* red = reinterpret_cast<float*>(smem + (size_t)kMaxTokD * d * 2);  // [16][256]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = gridDim.x * kWarpsD;
   const int gw = blockIdx.x * kWarpsD + warp;
 
-  // stage x (16-byte chunks), zero rows past T
-  for (int i = threadIdx.x; i < kMaxTokD * d / 8; i += kThreadsD) {
+  // stage x (16-byte chunks): the token rows the MMAs read (8 or 16), zeros
+  // past T
+  const int xrows = T <= 8 ? 8 : kMaxTokD;
+  for (int i = threadIdx.x; i < xrows * d / 8; i += kThreadsD) {
     const int t = i / (d / 8);
     reinterpret_cast<uint4*>(xs)[i] =
         t < T ? reinterpret_cast<const uint4*>(a.x)[i] : make_uint4(0, 0, 0, 0);
@@ -203,10 +195,14 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   }
   grid_barrier(a, 1);
 
-  // ------------------------------------------------------ B: TwELL pack --
+  // -------------------------------------- B: TwELL pack, h = g (x_t . Wu_t[j]) --
   {
     const unsigned lt = (1u << lane) - 1u;
-    for (int item = gw; item < K * T; item += nwarps) {
+    const int n_it = K * T;
+    const int m = nwarps >= n_it ? nwarps / n_it : 1;  // warps per (tile, token)
+    const int sub = nwarps >= n_it ? gw / n_it : 0;
+    for (int item = nwarps >= n_it ? gw % n_it : gw; sub < m && item < n_it;
+         item += nwarps >= n_it ? n_it : nwarps) {
       const int k = item / T, t = item % T;
       uint16_t gv[4];
       unsigned bal[4];
@@ -215,81 +211,63 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       for (int i = 0; i < 4; ++i) {
         const int u = k * kW + lane + 32 * i;
         float z = 0.f;
-        for (int s = 0; s < a.S; ++s) z += a.zpart[((size_t)s * T + t) * F + u];
+        for (int s2 = 0; s2 < a.S; ++s2) z += a.zpart[((size_t)s2 * T + t) * F + u];
         const float zr = (int32_t)__float_as_uint(z) > 0 ? z : 0.0f;  // ReLU, -0 -> +0
         gv[i] = f32_to_bf16(zr);
         bal[i] = __ballot_sync(FULL, gv[i] != 0);
         n += __popc(bal[i]);
-        if (a.dump) a.dump[(size_t)t * F + u] = gv[i];
       }
       const size_t off = (size_t)k * T + t;
       const int C = a.C;
-      int before = 0;
+      if (sub == 0) {  // the tile's TwELL slots, count, padding and spill
+        int before = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int pos = before + __popc(bal[i] & lt);
-        if (gv[i] != 0) {
-          if (pos < C) {
+        for (int i = 0; i < 4; ++i) {
+          const int pos = before + __popc(bal[i] & lt);
+          if (gv[i] != 0 && pos < C) {
             a.val[off * C + pos] = gv[i];
             a.idx[off * C + pos] = (uint8_t)(lane + 32 * i);
           }
-          a.jtile[(size_t)t * F + k * kW + pos] = k * kW + lane + 32 * i;
-          a.gtile[(size_t)t * F + k * kW + pos] = bf16_to_f32(gv[i]);
+          before += __popc(bal[i]);
+          if (a.dump) a.dump[(size_t)t * F + k * kW + lane + 32 * i] = gv[i];
         }
-        before += __popc(bal[i]);
-      }
-      for (int sl = lane; sl < C; sl += 32) {
-        if (sl >= n) {
-          a.val[off * C + sl] = 0;
-          a.idx[off * C + sl] = 0;
-        }
-      }
-      if (lane == 0) a.cnt[off] = (uint8_t)n;
-      if (n > C) {  // uniform across the warp
-        int slot = 0;
-        if (lane == 0) slot = atomicAdd(a.spill_n, 1);
-        slot = __shfl_sync(FULL, slot, 0);
-        if (slot < a.spill_cap) {
-          if (lane == 0) {
-            a.spill_ref[off] = slot;
-            a.spill_tk[2 * (size_t)slot] = t;
-            a.spill_tk[2 * (size_t)slot + 1] = k;
+        for (int sl = lane; sl < C; sl += 32) {
+          if (sl >= n) {
+            a.val[off * C + sl] = 0;
+            a.idx[off * C + sl] = 0;
           }
+        }
+        if (lane == 0) a.cnt[off] = (uint8_t)n;
+        if (n > C) {  // uniform across the warp
+          int slot = 0;
+          if (lane == 0) slot = atomicAdd(a.spill_n, 1);
+          slot = __shfl_sync(FULL, slot, 0);
+          if (slot < a.spill_cap) {
+            if (lane == 0) {
+              a.spill_ref[off] = slot;
+              a.spill_tk[2 * (size_t)slot] = t;
+              a.spill_tk[2 * (size_t)slot + 1] = k;
+            }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) a.spill_val[(size_t)slot * kW + lane + 32 * i] = gv[i];
-        } else if (lane == 0) {
-          a.spill_ref[off] = -1;
-          set_status(a.status, kStatusSpill);
+            for (int i = 0; i < 4; ++i) a.spill_val[(size_t)slot * kW + lane + 32 * i] = gv[i];
+          } else if (lane == 0) {
+            a.spill_ref[off] = -1;
+            set_status(a.status, kStatusSpill);
+          }
         }
       }
-    }
-  }
-  grid_barrier(a, 2);
-
-  // ------------------------------------------- C: h = g (x_t . Wu_t[j]) --
-  {
-    const int R = nwarps / T;  // warps per token
-    const int t = gw % T, r = gw / T;
-    if (r < R) {
-      const int m = R >= K ? R / K : 1;  // warps per tile
-      const bool spread = R >= K;
-      const int k_first = spread ? r % K : r;
-      const int sub = spread ? r / K : 0;
-      const bool active = !spread || r < m * K;
-      for (int k = k_first; active && k < K; k += spread ? K : R) {
-        const int n = a.cnt[(size_t)k * T + t];
-        if (n == 0) continue;
-        // ordinal of the tile's first entry: the counts of the tiles below k
-        int pre = 0;
-        for (int kb = 0; kb < k; kb += 32) {
-          const int kk = kb + lane;
-          pre += kk < k ? (int)a.cnt[(size_t)kk * T + t] : 0;
-        }
+      // the tile's non-zeros, ascending; entry p goes to the warp with p % m == sub
+      int before = 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(FULL, pre, o);
-        for (int s = sub; s < n; s += m) {
-          const int j = a.jtile[(size_t)t * F + k * kW + s];
-          const float gval = a.gtile[(size_t)t * F + k * kW + s];
+      for (int i = 0; i < 4; ++i) {
+        unsigned b = bal[i];
+        while (b) {  // uniform across the warp
+          const int l = __ffs(b) - 1;
+          b &= b - 1;
+          const int pos = before + __popc(bal[i] & ((1u << l) - 1u));
+          if (pos % m != sub) continue;
+          const int j = k * kW + l + 32 * i;
+          const float gval = bf16_to_f32(__shfl_sync(FULL, gv[i], l));
           const uint16_t* wr = a.Wu + (size_t)j * d;
           float p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
@@ -307,62 +285,64 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
           }
           const float u = warp_sum((p[0] + p[1]) + (p[2] + p[3]));
           if (lane == 0) {
-            a.jc[(size_t)t * F + pre + s] = j;
-            a.hc[(size_t)t * F + pre + s] = gval * u;
+            a.jtile[(size_t)t * F + k * kW + pos] = j;
+            a.htile[(size_t)t * F + k * kW + pos] = gval * u;
           }
         }
-      }
-      // the token's entry count, once per token
-      if (r == 0) {
-        int tot = 0;
-        for (int kb = 0; kb < K; kb += 32) {
-          const int kk = kb + lane;
-          tot += kk < K ? (int)a.cnt[(size_t)kk * T + t] : 0;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(FULL, tot, o);
-        if (lane == 0) a.nent[t] = tot;
+        before += __popc(bal[i]);
       }
     }
   }
-  grid_barrier(a, 3);
+  grid_barrier(a, 2);
 
-  // ------------------------------------------------ D: y_t = sum h Wd[j] --
+  // --------------------------------------------------- C: y_t = sum h Wd[j] --
   {
     const int nsl = (d + kSlice - 1) / kSlice;
     for (int task = blockIdx.x; task < T * nsl; task += gridDim.x) {
       const int t = task / nsl, sl = task % nsl;
       const int col = sl * kSlice + lane * 8;
       const bool in = col < d;
-      const int n = a.nent[t];
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int e0 = warp; e0 < n; e0 += 4 * kWarpsD) {
+      for (int k = warp; k < K; k += kWarpsD) {
+        // the count and the tile's first entries are loaded together (the
+        // entries past the count are not used)
+        const size_t e0 = (size_t)t * F + k * kW;
+        const int n = a.cnt[(size_t)k * T + t];
         int jj[4];
         float hh[4];
-        uint4 wv[4];
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-          const int e = e0 + b * kWarpsD;
-          jj[b] = e < n ? a.jc[(size_t)t * F + e] : 0;
-          hh[b] = e < n ? a.hc[(size_t)t * F + e] : 0.f;
+          jj[b] = a.jtile[e0 + b];
+          hh[b] = a.htile[e0 + b];
         }
+        for (int s0 = 0; s0 < n; s0 += 4) {
+          uint4 wv[4];
+          if (s0 > 0) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
-          wv[b] = in && e0 + b * kWarpsD < n
-                      ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
-                      : make_uint4(0, 0, 0, 0);
+            for (int b = 0; b < 4; ++b) {
+              jj[b] = s0 + b < n ? a.jtile[e0 + s0 + b] : 0;
+              hh[b] = s0 + b < n ? a.htile[e0 + s0 + b] : 0.f;
+            }
+          }
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          acc[0] = fmaf(hh[b], bf16_lo(wv[b].x), acc[0]);
-          acc[1] = fmaf(hh[b], bf16_hi(wv[b].x), acc[1]);
-          acc[2] = fmaf(hh[b], bf16_lo(wv[b].y), acc[2]);
-          acc[3] = fmaf(hh[b], bf16_hi(wv[b].y), acc[3]);
-          acc[4] = fmaf(hh[b], bf16_lo(wv[b].z), acc[4]);
-          acc[5] = fmaf(hh[b], bf16_hi(wv[b].z), acc[5]);
-          acc[6] = fmaf(hh[b], bf16_lo(wv[b].w), acc[6]);
-          acc[7] = fmaf(hh[b], bf16_hi(wv[b].w), acc[7]);
+          for (int b = 0; b < 4; ++b)
+            wv[b] = in && s0 + b < n
+                        ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
+                        : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const float hb = s0 + b < n ? hh[b] : 0.f;  // stale values past the count
+            acc[0] = fmaf(hb, bf16_lo(wv[b].x), acc[0]);
+            acc[1] = fmaf(hb, bf16_hi(wv[b].x), acc[1]);
+            acc[2] = fmaf(hb, bf16_lo(wv[b].y), acc[2]);
+            acc[3] = fmaf(hb, bf16_hi(wv[b].y), acc[3]);
+            acc[4] = fmaf(hb, bf16_lo(wv[b].z), acc[4]);
+            acc[5] = fmaf(hb, bf16_hi(wv[b].z), acc[5]);
+            acc[6] = fmaf(hb, bf16_lo(wv[b].w), acc[6]);
+            acc[7] = fmaf(hb, bf16_hi(wv[b].w), acc[7]);
+          }
         }
       }
 #pragma unroll
@@ -413,20 +393,14 @@ size_t decode_layout(void* base, int T, int d, int F, DecodeArgs* a) {
   const size_t o_bar = take(2 * sizeof(int32_t));
   const size_t o_z = take(sizeof(float) * (size_t)S * T * F);
   const size_t o_jt = take(sizeof(int32_t) * (size_t)T * F);
-  const size_t o_gt = take(sizeof(float) * (size_t)T * F);
-  const size_t o_jc = take(sizeof(int32_t) * (size_t)T * F);
-  const size_t o_hc = take(sizeof(float) * (size_t)T * F);
-  const size_t o_n = take(sizeof(int32_t) * (size_t)T);
+  const size_t o_ht = take(sizeof(float) * (size_t)T * F);
   if (base && a) {
     char* p = static_cast<char*>(base);
     a->S = S;
     a->bar = reinterpret_cast<int32_t*>(p + o_bar);
     a->zpart = reinterpret_cast<float*>(p + o_z);
     a->jtile = reinterpret_cast<int32_t*>(p + o_jt);
-    a->gtile = reinterpret_cast<float*>(p + o_gt);
-    a->jc = reinterpret_cast<int32_t*>(p + o_jc);
-    a->hc = reinterpret_cast<float*>(p + o_hc);
-    a->nent = reinterpret_cast<int32_t*>(p + o_n);
+    a->htile = reinterpret_cast<float*>(p + o_ht);
   }
   return off;
 }

@@ -1101,343 +1101,6 @@ __global__ void __launch_bounds__(32 * kDecWarps) decode_kernel(const GatherArgs
   }
 }
 
-// ---------------------------------------------------- streamed inference --
-// The inference pass (MODE kModeTwell) with the weight rows streamed by the
-// copy engine.  One warp per work item owns all d columns (the token's row
-// and its fp32 output row live in its registers), so an item needs no team
-// barrier or cross-warp exchange.  Each warp keeps a ring of kSlots shared-
-// memory slots; a slot receives one entry's two rows, Wu_t[j] and Wd[j], each
-// by a single cp.async.bulk of d elements that signals the slot's mbarrier.
-// The ring runs over the warp's whole stream of entries, across windows and
-// work items: the entry lists of the current and the next window are
-// collected ahead (the next item's token row is loaded ahead too), and as soon
-// as a pair of entries has been consumed their slots take the next entries'
-// rows.  A whole-row copy moves up to 4 KB per instruction, so the copy
-// engine's per-copy cost stays small against the bytes it moves, and the
-// rows in flight are bounded by shared memory, not registers.
-constexpr int kSWarps = 6;  // warps per CTA, one work item each
-constexpr int kSlots = 4;   // ring slots per warp: entries whose rows are in flight
-
-struct StreamCtl {
-  uint64_t full[kSWarps][kSlots];
-  float g[kSWarps][2][kListCap];
-  int32_t j[kSWarps][2][kListCap];
-  int never;
-};
-
-// Global -> shared bulk copy of `bytes` (16-byte multiple, both addresses
-// 16-byte aligned), completion signalled on `bar`; L2 keeps the source lines
-// (evict-last), since hot rows are gathered again by other tokens.
-TW_DEV void bulk_row(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-      : "memory");
-}
-// Orders this thread's earlier shared-memory accesses (generic proxy), and
-// those its warp made visible to it, before its later bulk copies (async
-// proxy) into the same memory.
-TW_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-TW_DEV uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
-
-// Entries [w0, w0 + n) of work item (t, lo, hi, prow); n <= kListCap.
-struct Win {
-  int t, lo, hi, prow, w0, n, buf;
-  bool valid, first;
-};
-
-template <typename Tin, int NCHW, bool kOutBf16>
-__global__ void __launch_bounds__(32 * kSWarps, 1)
-    stream_kernel(const GatherArgs<Tin> a, uint32_t row_bytes, uint32_t slot_bytes,
-                  unsigned long long timeout_ns) {
-  using L = Elem<Tin>;
-  constexpr int E = L::E;
-  constexpr int P = L::P;
-  constexpr int SPAN = 32 * E;  // columns of one warp-wide 16-byte slice
-  extern __shared__ __align__(128) uint8_t dyn[];
-  __shared__ StreamCtl ctl;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) {
-    for (int w = 0; w < kSWarps; ++w)
-      for (int q = 0; q < kSlots; ++q) mbar_init(&ctl.full[w][q], 1);
-    ctl.never = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  const int d = a.d;
-  const int n_items = a.ws.hdr[1];
-  uint8_t* ring = dyn + (size_t)warp * kSlots * slot_bytes;
-  uint64_t* full = ctl.full[warp];
-  const uint64_t pol = policy_evict_last();
-
-  // first window of the next work item (from the ticket counter)
-  auto fetch = [&](Win& w, int buf) {
-    int item = 0;
-    if (lane == 0) item = atomicAdd(&a.ws.hdr[0], 1);
-    item = __shfl_sync(FULL, item, 0);
-    w.valid = item < n_items;
-    w.buf = buf;
-    w.first = true;
-    w.n = 0;
-    if (!w.valid) return;
-    const int4 dd = a.ws.item_desc[item];
-    w.t = dd.x;
-    w.lo = dd.y;
-    w.hi = dd.z;
-    w.prow = dd.w;
-    w.w0 = dd.y;
-  };
-  auto collect = [&](Win& w) {
-    const int w1 = w.hi < w.w0 + kListCap ? w.hi : w.w0 + kListCap;
-    w.n = collect_twell(a, w.t, w.w0, w1, ctl.g[warp][w.buf], ctl.j[warp][w.buf], lane);
-    __syncwarp();
-  };
-  // the window after c, collected into the other list buffer
-  auto advance = [&](const Win& c, Win& nx) {
-    if (c.w0 + kListCap < c.hi) {
-      nx = c;
-      nx.w0 = c.w0 + kListCap;
-      nx.first = false;
-      nx.buf = c.buf ^ 1;
-    } else {
-      fetch(nx, c.buf ^ 1);
-    }
-    if (nx.valid) collect(nx);
-  };
-  auto load_x = [&](int t, uint4 (&xr)[NCHW]) {
-    const Tin* xt = a.xin + (size_t)t * d;
-#pragma unroll
-    for (int c = 0; c < NCHW; ++c) {
-      const int col = c * SPAN + lane * E;
-      xr[c] = col < d ? __ldcs(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
-    }
-  };
-
-  uint32_t q_issue = 0, q_cons = 0;  // entries issued to / consumed from the ring
-  auto issue = [&](const Win& w, int e) {
-    const uint32_t slot = q_issue % kSlots;
-    if (lane == 0) {
-      const int jj = ctl.j[warp][w.buf][e];
-      uint8_t* dst = ring + (size_t)slot * slot_bytes;
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&full[slot], 2 * row_bytes);
-      bulk_row(dst, a.rdot + (size_t)jj * d, row_bytes, &full[slot], pol);
-      bulk_row(dst + row_bytes, a.rax1 + (size_t)jj * d, row_bytes, &full[slot], pol);
-    }
-    ++q_issue;
-  };
-
-  Win cur, nxt;
-  fetch(cur, 0);
-  if (cur.valid) collect(cur);
-  nxt.valid = false;
-  if (cur.valid) advance(cur, nxt);
-  int ic = 0, inx = 0;  // entries of cur / nxt already issued
-  auto fill = [&]() {
-    while (q_issue - q_cons < (uint32_t)kSlots) {
-      if (ic < cur.n) issue(cur, ic++);
-      else if (nxt.valid && inx < nxt.n) issue(nxt, inx++);
-      else break;
-    }
-  };
-  uint4 xr[NCHW], xn[NCHW];
-  if (cur.valid) load_x(cur.t, xr);
-  if (nxt.valid && nxt.first) load_x(nxt.t, xn);
-  float2 acc[NCHW][P];
-#pragma unroll
-  for (int c = 0; c < NCHW; ++c)
-#pragma unroll
-    for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
-
-  bool ok = true;
-  while (cur.valid) {
-    fill();
-    const float* lg = ctl.g[warp][cur.buf];
-    for (int e = 0; e < cur.n; e += 2) {
-      const bool two = e + 1 < cur.n;
-      const uint32_t s0 = q_cons % kSlots, s1 = (q_cons + 1) % kSlots;
-      bool got = mbar_wait(&full[s0], (q_cons / kSlots) & 1u, &ctl.never, timeout_ns);
-      if (two) got = got && mbar_wait(&full[s1], ((q_cons + 1) / kSlots) & 1u, &ctl.never,
-                                      timeout_ns);
-      ok = __all_sync(FULL, got);
-      if (!ok) break;
-      const uint8_t* r0 = ring + (size_t)s0 * slot_bytes;
-      const uint8_t* r1 = ring + (size_t)s1 * slot_bytes;
-      // u of both entries: partial dot products per lane, then one warp reduction
-      float D[2][4];
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) D[k][i] = 0.f;
-#pragma unroll
-      for (int c = 0; c < NCHW; ++c) {
-        const int col = c * SPAN + lane * E;
-        const uint32_t off = (uint32_t)col * sizeof(Tin);
-        const uint4 w0 = col < d ? lds128(r0 + off) : make_uint4(0, 0, 0, 0);
-        const uint4 w1 = col < d && two ? lds128(r1 + off) : make_uint4(0, 0, 0, 0);
-        if constexpr (sizeof(Tin) == 2) {
-          mma_bf16_16816(D[0], w0.x, w1.x, w0.y, w1.y, xr[c].x, xr[c].y);
-          mma_bf16_16816(D[1], w0.z, w1.z, w0.w, w1.w, xr[c].z, xr[c].w);
-        } else {
-          L::dot(xr[c], w0, D[0]);
-          L::dot(xr[c], w1, D[1]);
-        }
-      }
-      float u0, u1;
-      dot2_reduce<Tin>(D, lane, u0, u1);
-      const float h0 = lg[e] * u0;
-      const float h1 = two ? lg[e + 1] * u1 : 0.f;
-      const float2 ha = make_float2(h0, h0), hb = make_float2(h1, h1);
-      // y_t += h Wd[j] over this lane's columns
-#pragma unroll
-      for (int c = 0; c < NCHW; ++c) {
-        const int col = c * SPAN + lane * E;
-        const uint32_t off = row_bytes + (uint32_t)col * sizeof(Tin);
-        const uint4 v0 = col < d ? lds128(r0 + off) : make_uint4(0, 0, 0, 0);
-        const uint4 v1 = col < d && two ? lds128(r1 + off) : make_uint4(0, 0, 0, 0);
-        float2 wv[P];
-        L::pairs(v0, wv);
-#pragma unroll
-        for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(ha, wv[q], acc[c][q]);
-        L::pairs(v1, wv);
-#pragma unroll
-        for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(hb, wv[q], acc[c][q]);
-      }
-      __syncwarp();  // every lane has read the pair's slots
-      q_cons += two ? 2u : 1u;
-      fill();
-    }
-    if (!ok) break;
-
-    // window done: on the last window of its item, the item's output
-    const bool same_item = nxt.valid && !nxt.first;
-    if (!same_item) {
-      bool complete = true;
-      if (cur.prow >= 0) {
-        // split token: partial rows summed up the fixed binary tree of parts
-        const int part = a.ws.hdr[2];
-        const int parts = (a.ws.nnz[cur.t] + part - 1) / part;
-        const int leaf = cur.lo / part;
-        const int row0 = cur.prow - leaf;
-        int node = leaf;
-        for (int span = 1; span < parts; span *= 2) {
-          const int left = node & ~(2 * span - 1);
-          const int right = left + span;
-          if (right >= parts) {
-            node = left;
-            continue;
-          }
-          float* mine = a.ws.partial + (size_t)(row0 + node) * d;
-#pragma unroll
-          for (int c = 0; c < NCHW; ++c) {
-            const int col = c * SPAN + lane * E;
-            if (col >= d) continue;
-#pragma unroll
-            for (int q = 0; q < P / 2; ++q)
-              reinterpret_cast<float4*>(mine + col)[q] =
-                  make_float4(acc[c][2 * q].x, acc[c][2 * q].y, acc[c][2 * q + 1].x,
-                              acc[c][2 * q + 1].y);
-          }
-          __threadfence();
-          __syncwarp();
-          int prev = 0;
-          if (lane == 0) prev = atomicAdd(&a.ws.done[row0 + right], 1);
-          prev = __shfl_sync(FULL, prev, 0);
-          if (prev == 0) {  // the sibling is still running; it goes on
-            complete = false;
-            break;
-          }
-          __threadfence();
-          const float* other =
-              a.ws.partial + (size_t)(row0 + (node == left ? right : left)) * d;
-#pragma unroll
-          for (int c = 0; c < NCHW; ++c) {
-            const int col = c * SPAN + lane * E;
-#pragma unroll
-            for (int q = 0; q < P / 2; ++q) {
-              const float4 sb = col < d
-                                    ? __ldcg(reinterpret_cast<const float4*>(other + col) + q)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-              acc[c][2 * q].x += sb.x;
-              acc[c][2 * q].y += sb.y;
-              acc[c][2 * q + 1].x += sb.z;
-              acc[c][2 * q + 1].y += sb.w;
-            }
-          }
-          node = left;
-        }
-      }
-      if (complete) {
-#pragma unroll
-        for (int c = 0; c < NCHW; ++c) {
-          const int col = c * SPAN + lane * E;
-          if (col >= d) continue;
-          if (!kOutBf16) {
-            float* dst = static_cast<float*>(a.out) + (size_t)cur.t * d + col;
-#pragma unroll
-            for (int q = 0; q < P / 2; ++q)
-              __stcs(reinterpret_cast<float4*>(dst) + q,
-                     make_float4(acc[c][2 * q].x, acc[c][2 * q].y, acc[c][2 * q + 1].x,
-                                 acc[c][2 * q + 1].y));
-          } else {
-            uint16_t* yt = static_cast<uint16_t*>(a.out) + (size_t)cur.t * d + col;
-#pragma unroll
-            for (int q = 0; q < P; ++q)
-              reinterpret_cast<uint32_t*>(yt)[q] = pack_bf16x2(acc[c][q].x, acc[c][q].y);
-          }
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < NCHW; ++c) {
-#pragma unroll
-        for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
-        xr[c] = xn[c];
-      }
-    }
-    cur = nxt;
-    ic = inx;
-    inx = 0;
-    nxt.valid = false;
-    if (cur.valid) {
-      advance(cur, nxt);
-      if (nxt.valid && nxt.first) load_x(nxt.t, xn);
-    }
-  }
-  if (!ok) {
-    // a row copy did not land in time: flag it, let the copies already
-    // issued land (bounded) before the CTA can exit, and stop this warp
-    if (lane == 0) set_status(a.status, kStatusTimeout);
-    for (uint32_t q = q_cons; q < q_issue; ++q)
-      mbar_wait(&full[q % kSlots], (q / kSlots) & 1u, &ctl.never, timeout_ns);
-  }
-}
-
-template <typename Tin, int NCHW>
-cudaError_t launch_stream_nchw(const GatherArgs<Tin>& a, bool out_bf16, cudaStream_t stream) {
-  auto kern = out_bf16 ? stream_kernel<Tin, NCHW, true> : stream_kernel<Tin, NCHW, false>;
-  const uint32_t row_bytes = (uint32_t)a.d * sizeof(Tin);
-  const uint32_t slot_bytes = (2 * row_bytes + 127u) & ~127u;
-  const size_t smem = (size_t)kSWarps * kSlots * slot_bytes;
-  cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(kern), (int)smem);
-  if (e != cudaSuccess) return e;
-  kern<<<num_sms(), 32 * kSWarps, smem, stream>>>(a, row_bytes, slot_bytes, kWaitTimeoutNs);
-  return cudaGetLastError();
-}
-
-// d up to 8 slices of 16 bytes per lane (2048 bf16 or 1024 fp32 columns)
-template <typename Tin>
-cudaError_t launch_stream(const GatherArgs<Tin>& a, bool out_bf16, cudaStream_t stream) {
-  constexpr int SPAN = 32 * Elem<Tin>::E;
-  const int nch = (a.d + SPAN - 1) / SPAN;
-  if (nch <= 1) return launch_stream_nchw<Tin, 1>(a, out_bf16, stream);
-  if (nch <= 2) return launch_stream_nchw<Tin, 2>(a, out_bf16, stream);
-  if (nch <= 4) return launch_stream_nchw<Tin, 4>(a, out_bf16, stream);
-  if (nch <= 8) return launch_stream_nchw<Tin, 8>(a, out_bf16, stream);
-  return cudaErrorInvalidValue;  // d beyond the validated maximum
-}
-
 template <typename Tin, int MODE>
 cudaError_t launch_mode(const GatherArgs<Tin>& a, bool out_bf16, cudaStream_t stream) {
   // chunks of one 16-byte slice per lane, split over the kTeam warps
@@ -1455,8 +1118,7 @@ cudaError_t launch_mode(const GatherArgs<Tin>& a, bool out_bf16, cudaStream_t st
 template <typename Tin, int MODE, class CountFn>
 cudaError_t run_engine(GatherArgs<Tin> a, bool out_bf16, void* base, CountFn count,
                        cudaStream_t stream) {
-  // workers taking items: warps of the streamed kernel, teams of the other
-  const int n_teams = num_sms() * (MODE == kModeTwell ? kSWarps : kTeams);
+  const int n_teams = num_sms() * kTeams;  // workers taking items
   cudaError_t e = cudaMemsetAsync(base, 0, a.ws.zero_bytes, stream);
   if (e != cudaSuccess) return e;
   count();
@@ -1473,7 +1135,6 @@ cudaError_t run_engine(GatherArgs<Tin> a, bool out_bf16, void* base, CountFn cou
                                                    a.ws.bpart, nb);
   plan_write_kernel<<<nb, kCountBlock, 0, stream>>>(a.T, a.ws.nnz, a.ws.max_items, a.ws.slot_off,
                                                     a.ws.item_desc, a.ws.hdr, a.ws.bpart);
-  if (MODE == kModeTwell) return launch_stream<Tin>(a, out_bf16, stream);
   return launch_mode<Tin, MODE>(a, out_bf16, stream);
 }
 

@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--workload", default="ffn_2b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip comparator/training/decode legs")
-    ap.add_argument("--legs", default="dense,energy,decode,training",
+    ap.add_argument("--legs", default="dense,tiles,energy,decode,training",
                     help="comma-separated extra legs to run after the timed step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -362,6 +362,8 @@ def run_ours(args, rank, world, local_rank):
     if legs:
         if rank == 0 and "dense" in legs:
             line["dense_comparator"] = dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_step, args)
+        if rank == 0 and "tiles" in legs:
+            line["tile_sweep"] = tile_sweep_leg(torch, tw, x, Wg, Wu, Wd, T, d, F)
         if rank == 0 and "energy" in legs:
             line["energy"] = energy_leg(torch, tw, x, Wg, Wu, Wd, g, y, ws, status, T, d, F,
                                         local_rank)
@@ -402,6 +404,41 @@ def live_units(torch, g):
         cols = torch.arange(g.W, device="cuda").view(1, g.W)
         used[(tk[:, 1:2] * g.W + cols)[nz]] = True
     return int(used.sum().item())
+
+
+def tile_sweep_leg(torch, tw, x, Wg, Wu, Wd, T, d, F):
+    """The same 2B-shaped step with other TwELL tile widths W and capacities C:
+    spilled (token, tile) pairs per step and the step time (gate + fused)."""
+    out = []
+    for W, C in ((128, 4), (128, 8), (128, 16), (128, 32), (64, 8), (256, 16), (256, 32)):
+        g = tw.Twell(T, F, C, dtype=torch.bfloat16, spill_cap=(F // W) * T // 4, W=W)
+        y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+        ws = tw.fused_workspace(T, d)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        for _ in range(3):
+            tw.twell_gate_gemm(x, Wg, g, None, st)
+            tw.twell_fused_updown(x, g, Wu, Wd, y, ws, st)
+        torch.cuda.synchronize()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        n = 20
+        tg = tf = 0.0
+        for _ in range(n):
+            e[0].record()
+            tw.twell_gate_gemm(x, Wg, g, None, st)
+            e[1].record()
+            tw.twell_fused_updown(x, g, Wu, Wd, y, ws, st)
+            e[2].record()
+            torch.cuda.synchronize()
+            tg += e[0].elapsed_time(e[1])
+            tf += e[1].elapsed_time(e[2])
+        twell_bytes = (F // W) * T * (3 * C + 1)
+        out.append({"W": W, "C": C, "spills_per_step": int(g.spill_n.item()),
+                    "gate_ms": tg / n, "fused_ms": tf / n, "step_ms": (tg + tf) / n,
+                    "tokens_per_s": T / ((tg + tf) / n * 1e-3), "twell_bytes": twell_bytes,
+                    "device_status": int(st.item())})
+        del g, y, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def nvml_handle(torch, local_rank):
