@@ -36,17 +36,18 @@
 //
 // Teams.  An item is processed by a team of kTeam warps; warp w of the team
 // owns one contiguous range of the d columns (the token's row and the output
-// of that range live in its registers).  Entries are taken in pairs: the two
-// warps form their partial dot products, the partials meet in shared memory
-// behind one named barrier per pair and are added in warp order, and every
-// warp updates its own columns.
+// of that range live in its registers).  A window of up to kListCap entries
+// runs in two phases: each warp forms its partial dot products of all the
+// window's entries, two at a time, and leaves them in shared memory; after
+// one named barrier each warp adds the team's partials in warp order, derives
+// the entry's scalars and updates its own columns.
 //
 // Data movement.  Weight rows are gathered with plain 16-byte vector loads
 // straight into registers (each lane owns 16-byte column slices, so a warp's
-// load of a row slice is fully coalesced).  Two register sets hold the rows
-// of one entry pair; each set is reloaded with the next pair's rows as soon
-// as it has been consumed, so the loads of the next pair overlap the rest of
-// the current one.  (Bulk copies into shared memory were the first design;
+// load of a row slice is fully coalesced).  In each phase two register sets
+// hold the rows of two entry pairs; a set is reloaded with the rows of the
+// pair after next as soon as it has been consumed, so loads stay in flight
+// through the phase.  (Bulk copies into shared memory were the first design;
 // the copy engine spends a roughly fixed time per copy, which bounded that
 // version by the number of row slices, not by bytes.)
 //
@@ -586,7 +587,7 @@ struct TeamSmem {
   int32_t j[kListCap];
   int32_t pos[kListCap];  // hybrid position of the entry (u is saved / read there)
   float u[kListCap];      // saved u of the entry (backward)
-  float red[2][kTeam][2];  // partial dot products of an entry pair, double-buffered
+  float part[kTeam][kListCap];  // each warp's partial dot product per entry of the window
   int4 desc[2];           // current item, double-buffered by item parity
   int n;                  // entries in the current window
   int prev;               // arrival count at a sum-tree node, broadcast to the team
@@ -798,54 +799,6 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
       const int n = ts.n;
       const int npairs = (n + 1) / 2;
       auto jof = [&](int e) { return e < n ? ts.j[e] : 0; };
-      // Register sets of row slices of one entry pair: A rows of the
-      // dot-product weight, B (and C, backward) rows of the update weights.
-      uint4 A[2][NCHW], B[2][NCHW], C[2][NCHW];
-      // The team's dot products of a pair: partial sums meet in shared
-      // memory behind one barrier; the scalars of the pair follow.
-      auto exchange = [&](int pp, float v0, float v1, float& s1a, float& s2a, float& s1b,
-                          float& s2b) {
-        const int rb = pp & 1;
-        if (lane == 0) {
-          ts.red[rb][tw][0] = v0;
-          ts.red[rb][tw][1] = v1;
-        }
-        team_bar(team);
-        float dv[2] = {0.f, 0.f};
-#pragma unroll
-        for (int q = 0; q < kTeam; ++q) {
-          dv[0] += ts.red[rb][q][0];
-          dv[1] += ts.red[rb][q][1];
-        }
-        float s1[2] = {0.f, 0.f}, s2[2] = {0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int ee = 2 * pp + k;
-          if (ee >= n) break;
-          const float gv = ts.g[ee];
-          if (kBwd) {
-            const float uv = ts.u[ee];
-            s1[k] = dv[k] * gv;              // du
-            s2[k] = fmaf(dv[k], uv, a.lam);  // dz
-            if (leader && lane == 0) {
-              Payload pl;
-              pl.t = t;
-              pl.h = gv * uv;
-              pl.du = s1[k];
-              pl.dz = s2[k];
-              a.pay[a.e0[t] + w0 + ee] = pl;
-            }
-          } else {
-            s1[k] = gv * dv[k];  // h
-            if (MODE == kModeHybFwd && leader && lane == 0)
-              L::store((to_backup ? a.backup_u : a.ell_u) + ts.pos[ee], dv[k]);
-          }
-        }
-        s1a = s1[0];
-        s1b = s1[1];
-        s2a = s2[0];
-        s2b = s2[1];
-      };
       // rows of a missing second entry are zeros, so both rows always update
       auto update = [&](const uint4 (&R)[2][NCHW], float sa, float sb) {
         const float2 ha = make_float2(sa, sa), hb = make_float2(sb, sb);
@@ -864,31 +817,100 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
         load_rows2<Tin, NCHW>(R, base, jof(2 * pp), jof(2 * pp + 1), 2 * pp + 1 < n, d, c0,
                               my_cols, lane, pol);
       };
-      // Each register set is reloaded with the next pair's rows as soon as it
-      // has been consumed, so those loads overlap the rest of the pair.
-      if (npairs > 0) {
-        load(A, a.rdot, 0);
-        load(B, a.rax1, 0);
-      }
-      for (int pp = 0; pp < npairs; ++pp) {
-        const bool next = pp + 1 < npairs;
-        float D[2][4];
-        dot2_issue<Tin, NCHW>(xr, A, D);
-        if (kBwd)  // A now takes the rows of the second update weight
-          load(C, a.rax2, pp);
-        else if (next)
-          load(A, a.rdot, pp + 1);
-        float v0, v1, s1a, s2a, s1b, s2b;
-        dot2_reduce<Tin>(D, lane, v0, v1);
-        exchange(pp, v0, v1, s1a, s2a, s1b, s2b);
-        update(B, s1a, s1b);
-        if (next) load(B, a.rax1, pp + 1);
-        if (kBwd) {
-          if (next) load(A, a.rdot, pp + 1);
-          update(C, s2a, s2b);
+      {
+        // Two phases per window.  Phase 1: this warp's partial dot products of
+        // every entry pair, two pairs of dot rows in flight, no team barrier
+        // between pairs.  One team barrier.  Phase 2: the scalars of each
+        // entry from the team's partials (added in warp order) -- h, or in
+        // the backward du and dz with the entry's record -- and the row
+        // updates, two pairs of update rows in flight.
+        uint4 S0[2][NCHW], S1[2][NCHW];
+        if (npairs > 0) load(S0, a.rdot, 0);
+        if (npairs > 1) load(S1, a.rdot, 1);
+        auto dots = [&](uint4 (&R)[2][NCHW], int pp) {
+          float D[2][4];
+          dot2_issue<Tin, NCHW>(xr, R, D);
+          if (pp + 2 < npairs) load(R, a.rdot, pp + 2);
+          float v0, v1;
+          dot2_reduce<Tin>(D, lane, v0, v1);
+          if (lane == 0) {
+            ts.part[tw][2 * pp] = v0;
+            ts.part[tw][2 * pp + 1] = v1;
+          }
+        };
+        for (int pp = 0; pp < npairs; pp += 2) {
+          dots(S0, pp);
+          if (pp + 1 < npairs) dots(S1, pp + 1);
         }
+        if constexpr (kBwd) {
+          // S0, S1: Wu_t rows (du); T0, T1: Wg_t rows (dz)
+          uint4 T0[2][NCHW], T1[2][NCHW];
+          if (npairs > 0) {
+            load(S0, a.rax1, 0);
+            load(T0, a.rax2, 0);
+          }
+          if (npairs > 1) {
+            load(S1, a.rax1, 1);
+            load(T1, a.rax2, 1);
+          }
+          team_bar(team);
+          auto coef = [&](int e, float& du, float& dz) {
+            du = dz = 0.f;
+            if (e >= n) return;
+            float dh = 0.f;
+#pragma unroll
+            for (int q = 0; q < kTeam; ++q) dh += ts.part[q][e];
+            const float gv = ts.g[e], uv = ts.u[e];
+            du = dh * gv;
+            dz = fmaf(dh, uv, a.lam);
+            if (leader && lane == 0) {
+              Payload pl;
+              pl.t = t;
+              pl.h = gv * uv;
+              pl.du = du;
+              pl.dz = dz;
+              a.pay[a.e0[t] + w0 + e] = pl;
+            }
+          };
+          auto upd2 = [&](uint4 (&RU)[2][NCHW], uint4 (&RG)[2][NCHW], int pp) {
+            float dua, dza, dub, dzb;
+            coef(2 * pp, dua, dza);
+            coef(2 * pp + 1, dub, dzb);
+            update(RU, dua, dub);
+            if (pp + 2 < npairs) load(RU, a.rax1, pp + 2);
+            update(RG, dza, dzb);
+            if (pp + 2 < npairs) load(RG, a.rax2, pp + 2);
+          };
+          for (int pp = 0; pp < npairs; pp += 2) {
+            upd2(S0, T0, pp);
+            if (pp + 1 < npairs) upd2(S1, T1, pp + 1);
+          }
+          team_bar(team);  // the list and the partials may be overwritten by the next window
+          continue;
+        }
+        if (npairs > 0) load(S0, a.rax1, 0);
+        if (npairs > 1) load(S1, a.rax1, 1);
+        team_bar(team);
+        auto hval = [&](int e) {
+          if (e >= n) return 0.f;
+          float dv = 0.f;
+#pragma unroll
+          for (int q = 0; q < kTeam; ++q) dv += ts.part[q][e];
+          if (MODE == kModeHybFwd && leader && lane == 0)
+            L::store((to_backup ? a.backup_u : a.ell_u) + ts.pos[e], dv);
+          return ts.g[e] * dv;
+        };
+        auto upd = [&](uint4 (&R)[2][NCHW], int pp) {
+          const float ha = hval(2 * pp), hb = hval(2 * pp + 1);
+          update(R, ha, hb);
+          if (pp + 2 < npairs) load(R, a.rax1, pp + 2);
+        };
+        for (int pp = 0; pp < npairs; pp += 2) {
+          upd(S0, pp);
+          if (pp + 1 < npairs) upd(S1, pp + 1);
+        }
+        team_bar(team);  // the list and the partials may be overwritten by the next window
       }
-      team_bar(team);  // the list may be overwritten by the next window
     }
 
     // ------------------------------------------------------------ output --
