@@ -1,4 +1,4 @@
-// decode_step.cu -- the whole gated FFN of a small batch (1 <= T <= 16
+// decode_step.cu -- the whole gated FFN of a small batch (1 <= T <= 64
 // tokens, decoding) in ONE persistent, cooperative launch: the gate
 // projection with its TwELL packing ("Sparser, Faster, Lighter Transformer
 // Language Models", technical summary, section 2.1) and the fused up + down
@@ -13,18 +13,20 @@
 //
 //   A  gate: work items of 16 units x 256 columns of d, spread over every
 //      warp of the grid; a warp streams its 16 Wg rows (16-byte loads, eight
-//      32-column steps in flight) and multiplies them with the tokens' x
-//      (staged in shared memory) on the tensor pipe: mma.sync m16n8k16 with
-//      the units on M and the tokens on N.  The reduction over d is split
-//      into slices: each item writes fp32 partial sums zpart[slice][t][u].
+//      32-column steps in flight; four for more than 16 tokens) and
+//      multiplies them with the tokens' x on the tensor pipe: mma.sync
+//      m16n8k16 with the units on M and the tokens on N, one 8-token column
+//      tile per MMA.  x is staged in shared memory for up to 16 tokens and
+//      read through L1 for more.  The reduction over d is split into slices:
+//      each item writes fp32 partial sums zpart[slice][t][u].
 //   B  packing and dot products: each (tile k, token t) gets one or more
 //      warps.  Every one of them adds the slices in a fixed order, applies
 //      ReLU and rounds g to bf16; the first packs the tile's TwELL slots
 //      exactly as the gate GEMM's epilogue does (ascending units, count,
 //      padding, lossless spill of the whole segment past C).  The warps then
-//      split the tile's non-zeros: for an entry (j, g) a warp forms
-//      u = x_t . Wu_t[j] (fp32) and stores h = g u and j at the entry's place
-//      in the tile (stride W per tile, ascending within it).
+//      split the tile's non-zeros (two at a time per warp): for an entry
+//      (j, g) a warp forms u = x_t . Wu_t[j] (fp32) and stores h = g u and j
+//      at the entry's place in the tile (stride W per tile, ascending).
 //   C  updates: one CTA per (token, 256-column slice of d); warp w takes the
 //      tiles k = w (mod 16) in ascending order, accumulates h Wd[j] over its
 //      columns in fp32, and the CTA adds the warps' partial rows in warp
@@ -42,7 +44,8 @@ constexpr int kThreadsD = 32 * kWarpsD;
 constexpr int kW = 128;          // TwELL tile width of this path
 constexpr int kSlice = 256;      // columns of d per gate work item
 constexpr int kSteps = kSlice / 32;
-constexpr int kMaxTokD = 16;
+constexpr int kMaxTokD = 64;
+constexpr int kStageTok = 16;  // x is staged in shared memory up to this many tokens
 
 struct DecodeArgs {
   const uint16_t* x;
@@ -113,23 +116,33 @@ TW_DEV void grid_barrier(const DecodeArgs& a, int b) {
   __syncthreads();
 }
 
+// NT: 8-token column tiles of the gate MMAs (1, 2, 4 or 8: T <= 8 * NT).
+template <int NT>
 __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeArgs a) {
+  constexpr bool kStage = 8 * NT <= kStageTok;  // x rows in shared memory
+  constexpr int kStepsA = kStage ? kSteps : kSteps / 2;  // Wg row steps in flight
   extern __shared__ __align__(16) uint8_t smem[];
   const int T = a.T, d = a.d, F = a.F, K = F / kW;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [16][d] bf16, rows >= T zero
-  float* red = reinterpret_cast<float*>(smem + (size_t)kMaxTokD * d * 2);  // [16][256]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [8 * NT][d] bf16 if kStage, rows >= T zero
+  float* red = reinterpret_cast<float*>(smem + (kStage ? (size_t)8 * NT * d * 2 : 0));  // [16][256]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = gridDim.x * kWarpsD;
   const int gw = blockIdx.x * kWarpsD + warp;
 
-  // stage x (16-byte chunks): the token rows the MMAs read (8 or 16), zeros
-  // past T
-  const int xrows = T <= 8 ? 8 : kMaxTokD;
-  for (int i = threadIdx.x; i < xrows * d / 8; i += kThreadsD) {
-    const int t = i / (d / 8);
-    reinterpret_cast<uint4*>(xs)[i] =
-        t < T ? reinterpret_cast<const uint4*>(a.x)[i] : make_uint4(0, 0, 0, 0);
+  // stage x (16-byte chunks): the token rows the MMAs read, zeros past T
+  if (kStage) {
+    for (int i = threadIdx.x; i < 8 * NT * d / 8; i += kThreadsD) {
+      const int t = i / (d / 8);
+      reinterpret_cast<uint4*>(xs)[i] =
+          t < T ? reinterpret_cast<const uint4*>(a.x)[i] : make_uint4(0, 0, 0, 0);
+    }
   }
+  // 16 bytes of token t's x at column col (zeros past T or d)
+  auto xrow = [&](int t, int col) -> uint4 {
+    if (t >= T || col >= d) return make_uint4(0, 0, 0, 0);
+    return kStage ? *reinterpret_cast<const uint4*>(xs + (size_t)t * d + col)
+                  : __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * d + col));
+  };
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.spill_n = 0;  // before any spill (phase B)
   __syncthreads();
 
@@ -137,58 +150,52 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   {
     const int g = lane >> 2, q = lane & 3;
     const int n_items = (F / 16) * a.S;
-    const bool two_n = T > 8;
     for (int item = gw; item < n_items; item += nwarps) {
       const int grp = item / a.S, s = item % a.S;
       const int u0 = grp * 16, c0 = s * kSlice;
       const uint16_t* r_lo = a.Wg + (size_t)(u0 + g) * d;
       const uint16_t* r_hi = a.Wg + (size_t)(u0 + g + 8) * d;
-      uint4 alo[kSteps], ahi[kSteps];
+      float D[NT][4];
 #pragma unroll
-      for (int i = 0; i < kSteps; ++i) {
-        const int col = c0 + i * 32 + 8 * q;
-        const bool in = col < d;
-        alo[i] = in ? __ldcs(reinterpret_cast<const uint4*>(r_lo + col)) : make_uint4(0, 0, 0, 0);
-        ahi[i] = in ? __ldcs(reinterpret_cast<const uint4*>(r_hi + col)) : make_uint4(0, 0, 0, 0);
-      }
-      float D0[4] = {0.f, 0.f, 0.f, 0.f}, D1[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int i = 0; i < kSteps; ++i) {
-        const int col = c0 + i * 32 + 8 * q;
-        // The 8 columns a lane loaded take the k-indices of its A fragment
-        // (the same permutation of k for every unit row and token column),
-        // so the products pair Wg[u][col] with x[t][col].
-        const uint4 xb = col < d ? *reinterpret_cast<const uint4*>(xs + (size_t)g * d + col)
-                                 : make_uint4(0, 0, 0, 0);
-        mma16816(D0, alo[i].x, ahi[i].x, alo[i].y, ahi[i].y, xb.x, xb.y);
-        mma16816(D0, alo[i].z, ahi[i].z, alo[i].w, ahi[i].w, xb.z, xb.w);
-        if (two_n) {
-          const uint4 xc = col < d
-                               ? *reinterpret_cast<const uint4*>(xs + (size_t)(g + 8) * d + col)
-                               : make_uint4(0, 0, 0, 0);
-          mma16816(D1, alo[i].x, ahi[i].x, alo[i].y, ahi[i].y, xc.x, xc.y);
-          mma16816(D1, alo[i].z, ahi[i].z, alo[i].w, ahi[i].w, xc.z, xc.w);
+        for (int i = 0; i < 4; ++i) D[n][i] = 0.f;
+#pragma unroll
+      for (int i0 = 0; i0 < kSteps; i0 += kStepsA) {
+        uint4 alo[kStepsA], ahi[kStepsA];
+#pragma unroll
+        for (int i = 0; i < kStepsA; ++i) {
+          const int col = c0 + (i0 + i) * 32 + 8 * q;
+          const bool in = col < d;
+          alo[i] = in ? __ldcs(reinterpret_cast<const uint4*>(r_lo + col)) : make_uint4(0, 0, 0, 0);
+          ahi[i] = in ? __ldcs(reinterpret_cast<const uint4*>(r_hi + col)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kStepsA; ++i) {
+          const int col = c0 + (i0 + i) * 32 + 8 * q;
+          // The 8 columns a lane loaded take the k-indices of its A fragment
+          // (the same permutation of k for every unit row and token column),
+          // so the products pair Wg[u][col] with x[t][col].
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const uint4 xb = xrow(8 * n + g, col);
+            mma16816(D[n], alo[i].x, ahi[i].x, alo[i].y, ahi[i].y, xb.x, xb.y);
+            mma16816(D[n], alo[i].z, ahi[i].z, alo[i].w, ahi[i].w, xb.z, xb.w);
+          }
         }
       }
       // D[m][n]: lane (g, q) holds (g, 2q), (g, 2q+1), (g+8, 2q), (g+8, 2q+1)
       float* zp = a.zpart + (size_t)s * T * F;
-      const int t0 = 2 * q;
-      if (t0 < T) {
-        zp[(size_t)t0 * F + u0 + g] = D0[0];
-        zp[(size_t)t0 * F + u0 + g + 8] = D0[2];
-      }
-      if (t0 + 1 < T) {
-        zp[(size_t)(t0 + 1) * F + u0 + g] = D0[1];
-        zp[(size_t)(t0 + 1) * F + u0 + g + 8] = D0[3];
-      }
-      if (two_n) {
-        if (t0 + 8 < T) {
-          zp[(size_t)(t0 + 8) * F + u0 + g] = D1[0];
-          zp[(size_t)(t0 + 8) * F + u0 + g + 8] = D1[2];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int t0 = 8 * n + 2 * q;
+        if (t0 < T) {
+          zp[(size_t)t0 * F + u0 + g] = D[n][0];
+          zp[(size_t)t0 * F + u0 + g + 8] = D[n][2];
         }
-        if (t0 + 9 < T) {
-          zp[(size_t)(t0 + 9) * F + u0 + g] = D1[1];
-          zp[(size_t)(t0 + 9) * F + u0 + g + 8] = D1[3];
+        if (t0 + 1 < T) {
+          zp[(size_t)(t0 + 1) * F + u0 + g] = D[n][1];
+          zp[(size_t)(t0 + 1) * F + u0 + g + 8] = D[n][3];
         }
       }
     }
@@ -256,41 +263,66 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
           }
         }
       }
-      // the tile's non-zeros, ascending; entry p goes to the warp with p % m == sub
+      // the tile's non-zeros, ascending; entry p goes to the warp with
+      // p % m == sub, which lists (unit, g) of its entries in its slice of
+      // `red` and forms their dot products two at a time
+      float* lst = red + warp * kSlice;  // 128 (unit, g) pairs
       int before = 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        unsigned b = bal[i];
-        while (b) {  // uniform across the warp
-          const int l = __ffs(b) - 1;
-          b &= b - 1;
-          const int pos = before + __popc(bal[i] & ((1u << l) - 1u));
-          if (pos % m != sub) continue;
-          const int j = k * kW + l + 32 * i;
-          const float gval = bf16_to_f32(__shfl_sync(FULL, gv[i], l));
-          const uint16_t* wr = a.Wu + (size_t)j * d;
-          float p[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-          for (int c = lane * 8; c < d; c += 256) {
-            const uint4 w = __ldg(reinterpret_cast<const uint4*>(wr + c));
-            const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)t * d + c);
-            p[0] = fmaf(bf16_lo(xv.x), bf16_lo(w.x), p[0]);
-            p[1] = fmaf(bf16_hi(xv.x), bf16_hi(w.x), p[1]);
-            p[2] = fmaf(bf16_lo(xv.y), bf16_lo(w.y), p[2]);
-            p[3] = fmaf(bf16_hi(xv.y), bf16_hi(w.y), p[3]);
-            p[0] = fmaf(bf16_lo(xv.z), bf16_lo(w.z), p[0]);
-            p[1] = fmaf(bf16_hi(xv.z), bf16_hi(w.z), p[1]);
-            p[2] = fmaf(bf16_lo(xv.w), bf16_lo(w.w), p[2]);
-            p[3] = fmaf(bf16_hi(xv.w), bf16_hi(w.w), p[3]);
-          }
-          const float u = warp_sum((p[0] + p[1]) + (p[2] + p[3]));
-          if (lane == 0) {
-            a.jtile[(size_t)t * F + k * kW + pos] = j;
-            a.htile[(size_t)t * F + k * kW + pos] = gval * u;
-          }
+        const int pos = before + __popc(bal[i] & lt);
+        if (gv[i] != 0 && pos % m == sub) {
+          const int r = pos / m;
+          lst[2 * r] = __int_as_float(k * kW + lane + 32 * i);
+          lst[2 * r + 1] = bf16_to_f32(gv[i]);
         }
         before += __popc(bal[i]);
       }
+      __syncwarp();
+      const int nh = sub < n ? (n - sub + m - 1) / m : 0;  // entries of this warp
+      for (int r0 = 0; r0 < nh; r0 += 2) {
+        const bool two = r0 + 1 < nh;
+        const int j0 = __float_as_int(lst[2 * r0]);
+        const int j1 = two ? __float_as_int(lst[2 * r0 + 2]) : j0;
+        const uint16_t* w0 = a.Wu + (size_t)j0 * d;
+        const uint16_t* w1 = a.Wu + (size_t)j1 * d;
+        float p[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
+        for (int c = lane * 8; c < d; c += 256) {
+          const uint4 xv = xrow(t, c);
+          const uint4 wa = __ldg(reinterpret_cast<const uint4*>(w0 + c));
+          const uint4 wb = two ? __ldg(reinterpret_cast<const uint4*>(w1 + c)) : make_uint4(0, 0, 0, 0);
+          p[0][0] = fmaf(bf16_lo(xv.x), bf16_lo(wa.x), p[0][0]);
+          p[0][1] = fmaf(bf16_hi(xv.x), bf16_hi(wa.x), p[0][1]);
+          p[0][2] = fmaf(bf16_lo(xv.y), bf16_lo(wa.y), p[0][2]);
+          p[0][3] = fmaf(bf16_hi(xv.y), bf16_hi(wa.y), p[0][3]);
+          p[0][0] = fmaf(bf16_lo(xv.z), bf16_lo(wa.z), p[0][0]);
+          p[0][1] = fmaf(bf16_hi(xv.z), bf16_hi(wa.z), p[0][1]);
+          p[0][2] = fmaf(bf16_lo(xv.w), bf16_lo(wa.w), p[0][2]);
+          p[0][3] = fmaf(bf16_hi(xv.w), bf16_hi(wa.w), p[0][3]);
+          p[1][0] = fmaf(bf16_lo(xv.x), bf16_lo(wb.x), p[1][0]);
+          p[1][1] = fmaf(bf16_hi(xv.x), bf16_hi(wb.x), p[1][1]);
+          p[1][2] = fmaf(bf16_lo(xv.y), bf16_lo(wb.y), p[1][2]);
+          p[1][3] = fmaf(bf16_hi(xv.y), bf16_hi(wb.y), p[1][3]);
+          p[1][0] = fmaf(bf16_lo(xv.z), bf16_lo(wb.z), p[1][0]);
+          p[1][1] = fmaf(bf16_hi(xv.z), bf16_hi(wb.z), p[1][1]);
+          p[1][2] = fmaf(bf16_lo(xv.w), bf16_lo(wb.w), p[1][2]);
+          p[1][3] = fmaf(bf16_hi(xv.w), bf16_hi(wb.w), p[1][3]);
+        }
+        const float u0 = warp_sum((p[0][0] + p[0][1]) + (p[0][2] + p[0][3]));
+        const float u1 = warp_sum((p[1][0] + p[1][1]) + (p[1][2] + p[1][3]));
+        if (lane == 0) {
+          const int pos0 = r0 * m + sub;
+          a.jtile[(size_t)t * F + k * kW + pos0] = j0;
+          a.htile[(size_t)t * F + k * kW + pos0] = lst[2 * r0 + 1] * u0;
+          if (two) {
+            const int pos1 = (r0 + 1) * m + sub;
+            a.jtile[(size_t)t * F + k * kW + pos1] = j1;
+            a.htile[(size_t)t * F + k * kW + pos1] = lst[2 * r0 + 3] * u1;
+          }
+        }
+      }
+      __syncwarp();  // the list is rewritten by the warp's next item
     }
   }
   grid_barrier(a, 2);
@@ -310,29 +342,30 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
         // entries past the count are not used)
         const size_t e0 = (size_t)t * F + k * kW;
         const int n = a.cnt[(size_t)k * T + t];
-        int jj[4];
-        float hh[4];
+        constexpr int kB = 8;  // entries whose rows are loaded together
+        int jj[kB];
+        float hh[kB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < kB; ++b) {
           jj[b] = a.jtile[e0 + b];
           hh[b] = a.htile[e0 + b];
         }
-        for (int s0 = 0; s0 < n; s0 += 4) {
-          uint4 wv[4];
+        for (int s0 = 0; s0 < n; s0 += kB) {
+          uint4 wv[kB];
           if (s0 > 0) {
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
+            for (int b = 0; b < kB; ++b) {
               jj[b] = s0 + b < n ? a.jtile[e0 + s0 + b] : 0;
               hh[b] = s0 + b < n ? a.htile[e0 + s0 + b] : 0.f;
             }
           }
 #pragma unroll
-          for (int b = 0; b < 4; ++b)
+          for (int b = 0; b < kB; ++b)
             wv[b] = in && s0 + b < n
                         ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
                         : make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
+          for (int b = 0; b < kB; ++b) {
             const float hb = s0 + b < n ? hh[b] : 0.f;  // stale values past the count
             acc[0] = fmaf(hb, bf16_lo(wv[b].x), acc[0]);
             acc[1] = fmaf(hb, bf16_hi(wv[b].x), acc[1]);
@@ -435,12 +468,17 @@ cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t
   a.y_bf16 = y_dtype == TW_BF16;
   a.status = status;
   a.timeout_ns = kWaitTimeoutNs;
-  const size_t smem = (size_t)kMaxTokD * d * 2 + sizeof(float) * kWarpsD * kSlice;
-  cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(decode_step_kernel), (int)smem);
+  const int NT = T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : 8;
+  const size_t xs_bytes = 8 * NT <= kStageTok ? (size_t)8 * NT * d * 2 : 0;
+  const size_t smem = xs_bytes + sizeof(float) * kWarpsD * kSlice;
+  const void* kern = NT == 1 ? reinterpret_cast<const void*>(decode_step_kernel<1>)
+                     : NT == 2 ? reinterpret_cast<const void*>(decode_step_kernel<2>)
+                     : NT == 4 ? reinterpret_cast<const void*>(decode_step_kernel<4>)
+                               : reinterpret_cast<const void*>(decode_step_kernel<8>);
+  cudaError_t e = set_smem_limit(kern, (int)smem);
   if (e != cudaSuccess) return e;
   void* args[] = {&a};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(decode_step_kernel),
-                                     dim3(num_sms()), dim3(kThreadsD), args, smem, stream);
+  return cudaLaunchCooperativeKernel(kern, dim3(num_sms()), dim3(kThreadsD), args, smem, stream);
 }
 
 }  // namespace tw

@@ -47,7 +47,7 @@ cudaError_t launch_gate_twell_f32(const float* x, const float* Wg_t, int T, int 
                                   cudaStream_t stream);
 // The whole FFN of 1 <= T <= kDecodeStepMaxT tokens (bf16, W = 128) in one
 // cooperative launch: gate + TwELL packing, then the fused up + down.
-constexpr int kDecodeStepMaxT = 16;
+constexpr int kDecodeStepMaxT = 64;
 size_t decode_ws_bytes(int T, int d, int F);
 cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t, const void* Wd,
                                int T, int d, int F, const tw_twell& out, void* dump, void* y,

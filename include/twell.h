@@ -204,7 +204,7 @@ TW_API tw_status twell_fused_updown_noalloc(const void* x, const tw_twell* g, co
                                             int32_t* dev_status, cudaStream_t stream);
 
 /*
- * The whole FFN of a small batch -- decoding, 1 <= T <= 16 tokens -- in ONE
+ * The whole FFN of a small batch -- decoding, 1 <= T <= 64 tokens -- in ONE
  * launch (sections 2.1 and 2.2): g = ReLU(x Wg) packed into *g as
  * twell_gate_gemm packs it, then y = sum over the active units of
  * g (x . Wu_t[j]) Wd[j], as twell_fused_updown computes it (fp32 accumulation,

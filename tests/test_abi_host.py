@@ -167,7 +167,7 @@ def test_small_batch_validation(L):
         return f(FAKE, FAKE, FAKE, FAKE, T, d, F, ctypes.byref(tw), None, y, twell.TW_F32, FAKE,
                  n, None, None)
 
-    assert call(T=17) == UNSUPPORTED                 # up to 16 tokens in one launch
+    assert call(T=65) == UNSUPPORTED                 # up to 64 tokens in one launch
     assert call(W=64) == UNSUPPORTED                 # tile width 128 only
     assert call(dtype=twell.TW_F32) == UNSUPPORTED   # bf16 only
     assert call(d=4096) == UNSUPPORTED               # x of 16 tokens staged in shared memory

@@ -299,7 +299,8 @@ def test_decode_sizes(T):
 
 # One cooperative launch for the whole small-batch FFN: gate partial sums on
 # mma.sync over every SM, TwELL packing, dot products, updates.  T crosses the
-# 8-token MMA column tile; d and F are ragged against the 256-column slices.
+# 8-token MMA column tiles and the 16-token limit of x staged in shared
+# memory; d and F are ragged against the 256-column slices.
 SMALL_STEP = [
     # T, d, F, C, kind, mean_active
     (1, 2048, 8192, 8, "zipf", 29.0),
@@ -309,6 +310,9 @@ SMALL_STEP = [
     (16, 2048, 4096, 8, "zipf", 29.0),
     (16, 1024, 1024, 64, "dead20", 300.0),
     (3, 64, 256, 128, "dead20", 100.0),
+    (17, 320, 640, 8, "dead20", 60.0),   # x read through L1 from here on
+    (33, 2048, 2048, 8, "zipf", 29.0),
+    (64, 512, 1280, 16, "zipf", 200.0),  # heavy tokens: many entries per tile
 ]
 
 
@@ -343,7 +347,7 @@ def test_small_batch_single_launch(T, d, F, C, kind, ma):
     assert torch.equal(yb, ys[0].to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("T", [1, 8, 16])
+@pytest.mark.parametrize("T", [1, 8, 16, 64])
 def test_small_batch_single_launch_decode_2b(T):
     """The decoding workload (the 2B weights, the first T tokens) in the launch
     configuration the benchmark times."""
