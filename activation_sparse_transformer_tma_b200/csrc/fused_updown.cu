@@ -866,6 +866,7 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
             if (leader && lane == 0) {
               Payload pl;
               pl.t = t;
+              pl.j = ts.j[e];
               pl.h = gv * uv;
               pl.du = du;
               pl.dz = dz;

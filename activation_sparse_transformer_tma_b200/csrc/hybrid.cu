@@ -410,194 +410,117 @@ __global__ void __launch_bounds__(256)
 // (fused_updown.cu), which splits heavy rows and streams the weight rows
 // through shared memory.  The weight gradients below use its records.
 
-// The records of the backward are in token-major order (entry e0[t] + rank).
-// The weight gradients sum them per unit in ascending token order, so they
-// are transposed to a unit-major list with a stable counting sort:
-//   1. hyb_count_kernel   entries per (block of TB tokens, unit): cnt[b][j];
-//   2. hyb_colscan_kernel one thread per unit: exclusive prefix over blocks
-//                         (in place) and the unit's total;
-//   3. scan_kernel        exclusive prefix of the totals -> unit_off;
-//   4. hyb_fill_kernel    each block walks its tokens again and writes every
-//                         entry's record index at its place.
-// A block is TB_WARPS warps, each owning TB_TOK consecutive tokens with a
-// private uint8 histogram of the F units in shared memory; within a block the
-// warps' histograms become exclusive offsets, so the warps place their
-// entries in parallel and the token order inside each unit is kept.
-constexpr int TB_WARPS = 4;
-constexpr int TB_TOK = 8;                // tokens per warp
-constexpr int TB = TB_WARPS * TB_TOK;    // tokens per block
-static_assert((TB_WARPS - 1) * TB_TOK < 256, "per-warp offsets must fit in uint8");
+// The records of the backward are in token-major order (entry e0[t] + rank),
+// and each carries its unit.  The weight gradients sum them per unit in
+// ascending token order, i.e. ascending record index, so each unit's records
+// are gathered into a unit-major list and sorted there:
+//   1. hyb_ucount_kernel  records per unit (one atomic per record);
+//   2. scan_kernel        exclusive prefix of the counts -> unit_off;
+//   3. hyb_place_kernel   each record's index at its unit's next place (the
+//                         order inside a unit is arbitrary here);
+//   4. hyb_wgrad_kernel   one CTA per unit sorts its segment (bitonic, in
+//                         shared memory up to kSegSmem records; longer
+//                         segments as sorted runs merged by rank into a
+//                         scratch list) and sums in that order.
+// Every pass is flat over the records, so a heavy backup row costs no one
+// thread or warp more than its share.
+constexpr int kSegSmem = 2048;  // records of a unit sorted in shared memory
 
-// Shared memory of the count and fill kernels: TB_WARPS x F uint8.
-__host__ __device__ inline size_t tb_hist_bytes(int F) { return (size_t)TB_WARPS * F; }
-
-// Per-warp histogram of the units of the warp's tokens (zeroed first).
-// Slot and count of the warp's TB_TOK tokens, loaded in one round (lane k
-// holds token k's), so the walk over the tokens does not wait for them.
-template <typename T>
-TW_DEV void warp_token_meta(const HView<T>& h, int t0, int lane, int& slot, int& nnz) {
-  const int t = t0 + lane;
-  const bool ok = lane < TB_TOK && t < h.T;
-  slot = ok ? h.row_slot[t] : -1;
-  nnz = ok ? h.row_nnz[t] : 0;
+__global__ void __launch_bounds__(256)
+    hyb_ucount_kernel(const Payload* pay, const int32_t* e_total, int32_t* ucnt) {
+  const int n = *e_total;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x)
+    atomicAdd(&ucnt[pay[e].j], 1);
 }
 
-template <typename T>
-TW_DEV void warp_unit_hist(const HView<T>& h, uint8_t* hist, int b, int warp, int lane) {
-  const int t0 = b * TB + warp * TB_TOK;
-  int mslot, mnnz;
-  warp_token_meta<T>(h, t0, lane, mslot, mnnz);
-  uint32_t* h4 = reinterpret_cast<uint32_t*>(hist);
-  for (int j = lane; j < h.F / 4; j += 32) h4[j] = 0u;
-  __syncwarp();
-  for (int k = 0; k < TB_TOK; ++k) {
-    const int t = t0 + k;
-    if (t >= h.T) break;
-    const int slot = __shfl_sync(FULL, mslot, k), nnz = __shfl_sync(FULL, mnnz, k);
-    // the units of one row are distinct, so these increments never collide
-    for_each_chunk<T>(
-        h, t, slot, nnz, lane,
-        [&](bool v, int j, int) {
-          if (v) hist[j] = (uint8_t)(hist[j] + 1);
-        },
-        [&](int cl, unsigned mask, int) {
-#pragma unroll
-          for (int i = 0; i < 16 / (int)sizeof(T); ++i)
-            if ((mask >> i) & 1u) hist[cl + i] = (uint8_t)(hist[cl + i] + 1);
-        });
-    __syncwarp();
+__global__ void __launch_bounds__(256)
+    hyb_place_kernel(const Payload* pay, const int32_t* e_total, const int32_t* unit_off,
+                     int32_t* cursor, int32_t* list) {
+  const int n = *e_total;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+    const int j = pay[e].j;
+    list[unit_off[j] + atomicAdd(&cursor[j], 1)] = e;
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(32 * TB_WARPS)
-    hyb_count_kernel(const HView<T> h, int nb, int32_t* cnt) {
-  extern __shared__ uint8_t hist[];  // [TB_WARPS][F]
-  const int b = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  warp_unit_hist<T>(h, hist + (size_t)warp * h.F, b, warp, lane);
-  __syncthreads();
-  for (int j = threadIdx.x; j < h.F; j += blockDim.x) {
-    int c = 0;
-#pragma unroll
-    for (int w = 0; w < TB_WARPS; ++w) c += hist[(size_t)w * h.F + j];
-    cnt[(size_t)b * h.F + j] = c;  // block-major: coalesced
-  }
-}
-
-// One thread per unit: exclusive prefix over the blocks of the unit's counts
-// (block-major, so a warp reads 32 consecutive units per block), in place;
-// eight blocks are loaded ahead of the running sum.
-__global__ void hyb_colscan_kernel(int nb, int F, int32_t* cnt, int32_t* unit_total) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= F) return;
-  int run = 0;
-  for (int b0 = 0; b0 < nb; b0 += 8) {
-    int v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = b0 + i < nb ? cnt[(size_t)(b0 + i) * F + j] : 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (b0 + i < nb) cnt[(size_t)(b0 + i) * F + j] = run;
-      run += v[i];
+// Ascending bitonic sort of v[0, P) in shared memory (P a power of two <= the
+// array), all threads of the CTA.
+TW_DEV void block_bitonic(int32_t* v, int P) {
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        const int o = i ^ jj;
+        if (o > i) {
+          const int32_t a = v[i], b = v[o];
+          if ((a > b) == ((i & k) == 0)) {
+            v[i] = b;
+            v[o] = a;
+          }
+        }
+      }
+      __syncthreads();
     }
   }
-  unit_total[j] = run;
 }
 
-// Fill the unit-major list with token-major record indices, tokens ascending
-// within each unit.
-// With kSmemBase the block's first list position of every unit,
-// unit_off[j] + cnt[b][j], is staged in shared memory behind the histograms,
-// so placing an entry needs no global load.
-template <typename T, bool kSmemBase>
-__global__ void __launch_bounds__(32 * TB_WARPS)
-    hyb_fill_kernel(const HView<T> h, int nb, const int32_t* cnt, const int32_t* unit_off,
-                    const int32_t* e0, int32_t* list) {
-  extern __shared__ uint8_t hist[];  // [TB_WARPS][F] -> per-warp offsets inside the block
-  int32_t* bases = reinterpret_cast<int32_t*>(hist + tb_hist_bytes(h.F));  // [F] if kSmemBase
-  const int b = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* mine = hist + (size_t)warp * h.F;
-  if (kSmemBase) {
-#pragma unroll 8
-    for (int j = threadIdx.x; j < h.F; j += blockDim.x)
-      bases[j] = unit_off[j] + cnt[(size_t)b * h.F + j];
-  }
-  warp_unit_hist<T>(h, mine, b, warp, lane);
-  __syncthreads();
-  auto base_of = [&](int j) {
-    return kSmemBase ? bases[j] : unit_off[j] + cnt[(size_t)b * h.F + j];
-  };
-  for (int j = threadIdx.x; j < h.F; j += blockDim.x) {
-    int r = 0;
-#pragma unroll
-    for (int w = 0; w < TB_WARPS; ++w) {
-      const int c = hist[(size_t)w * h.F + j];
-      hist[(size_t)w * h.F + j] = (uint8_t)r;
-      r += c;
-    }
-  }
-  __syncthreads();
-  const int t0 = b * TB + warp * TB_TOK;
-  int mslot, mnnz;
-  warp_token_meta<T>(h, t0, lane, mslot, mnnz);
-  const int mbase = lane < TB_TOK && t0 + lane < h.T ? e0[t0 + lane] : 0;
-  for (int k = 0; k < TB_TOK; ++k) {
-    const int t = t0 + k;
-    if (t >= h.T) break;
-    const int ebase = __shfl_sync(FULL, mbase, k);
-    const int slot = __shfl_sync(FULL, mslot, k), nnz = __shfl_sync(FULL, mnnz, k);
-    for_each_chunk<T>(
-        h, t, slot, nnz, lane,
-        [&](bool v, int j, int rank) {
-          if (v) {
-            const int o = mine[j];
-            mine[j] = (uint8_t)(o + 1);
-            list[base_of(j) + o] = ebase + rank;
-          }
-        },
-        [&](int cl, unsigned mask, int rank0) {
-          // the places of this lane's entries first (independent loads), then
-          // the per-warp offsets and the stores
-          constexpr int V = 16 / (int)sizeof(T);
-          int place[V];
-#pragma unroll
-          for (int i = 0; i < V; ++i)
-            place[i] = (mask >> i) & 1u ? base_of(cl + i) : 0;
-          int rank = rank0;
-#pragma unroll
-          for (int i = 0; i < V; ++i) {
-            if ((mask >> i) & 1u) {
-              const int o = mine[cl + i];
-              mine[cl + i] = (uint8_t)(o + 1);
-              list[place[i] + o] = ebase + rank;
-              ++rank;
-            }
-          }
-        });
-    __syncwarp();
-  }
-}
-
-// Weight gradients of one unit per CTA, entries summed in token order.
+// Weight gradients of one unit per CTA, records summed in token order.
 template <typename T>
 __global__ void __launch_bounds__(256)
     hyb_wgrad_kernel(int F, int d, const T* x, const T* dy, const int32_t* unit_off,
-                     const int32_t* list, const Payload* pay, float* dWg_t, float* dWu_t,
-                     float* dWd) {
+                     int32_t* list, int32_t* sorted, const Payload* pay, float* dWg_t,
+                     float* dWu_t, float* dWd) {
   using S = Slice<T>;
   constexpr int E = S::E;
+  __shared__ int32_t seg[kSegSmem];
   const int j = blockIdx.x;
-  const int e_begin = unit_off[j], e_end = unit_off[j + 1];
+  const int b = unit_off[j], n = unit_off[j + 1] - b;
+  const bool small = n <= kSegSmem;
+  if (small) {
+    int P = 1;
+    while (P < n) P <<= 1;
+    for (int i = threadIdx.x; i < P; i += blockDim.x) seg[i] = i < n ? list[b + i] : INT32_MAX;
+    __syncthreads();
+    block_bitonic(seg, P);
+  } else {
+    // sorted runs of kSegSmem records, written back in place
+    for (int r0 = 0; r0 < n; r0 += kSegSmem) {
+      const int len = min(kSegSmem, n - r0);
+      for (int i = threadIdx.x; i < kSegSmem; i += blockDim.x)
+        seg[i] = i < len ? list[b + r0 + i] : INT32_MAX;
+      __syncthreads();
+      block_bitonic(seg, kSegSmem);
+      for (int i = threadIdx.x; i < len; i += blockDim.x) list[b + r0 + i] = seg[i];
+      __syncthreads();
+    }
+    // final place of a record: its rank in its own run plus, in every other
+    // run, the number of smaller records (indices are distinct)
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int32_t v = list[b + i];
+      const int own = i / kSegSmem;
+      int pos = i - own * kSegSmem;
+      for (int r = 0; r * kSegSmem < n; ++r) {
+        if (r == own) continue;
+        int lo = r * kSegSmem, hi = min(n, lo + kSegSmem);
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (list[b + mid] < v) lo = mid + 1;
+          else hi = mid;
+        }
+        pos += lo - r * kSegSmem;
+      }
+      sorted[b + pos] = v;
+    }
+    __syncthreads();
+  }
+  const int32_t* order = small ? seg : sorted + b;
   const int stride = blockDim.x * E;
   for (int col = threadIdx.x * E; col < d; col += stride) {
     float ad[E], au[E], ag[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) ad[e] = au[e] = ag[e] = 0.f;
 #pragma unroll 4
-    for (int q = e_begin; q < e_end; ++q) {
-      const Payload p = pay[list[q]];
+    for (int q = 0; q < n; ++q) {
+      const Payload p = pay[order[q]];
       float xf[E], df[E];
       S::widen(S::load(x + (size_t)p.t * d + col), xf);
       S::widen(S::load(dy + (size_t)p.t * d + col), df);
@@ -620,12 +543,13 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------ workspace ----
 struct BwdWs {  // the gather engine's own workspace follows these arrays
-  int32_t* e0;        // [T+1]
+  int32_t* e0;        // [T+1], e0[T] = number of records
   Payload* pay;       // [Emax]
-  int32_t* cnt;       // [NB][F], block-major
-  int32_t* unit_total;// [F]
+  int32_t* ucnt;      // [F] records per unit, then [F] placement cursors (zeroed together)
+  int32_t* cursor;
   int32_t* unit_off;  // [F+1]
-  int32_t* list;      // [Emax]
+  int32_t* list;      // [Emax] unit-major record indices
+  int32_t* sorted;    // [Emax] scratch for segments longer than kSegSmem
   size_t bytes;
 };
 
@@ -633,7 +557,6 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 BwdWs carve(void* base, int T, int F, int C_h, int backup_cap) {
   const size_t emax = (size_t)T * C_h + (size_t)backup_cap * F;
-  const size_t nb = ((size_t)T + TB - 1) / TB;
   BwdWs w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -643,19 +566,20 @@ BwdWs carve(void* base, int T, int F, int C_h, int backup_cap) {
   };
   const size_t o_e0 = take(sizeof(int32_t) * ((size_t)T + 1));
   const size_t o_pay = take(sizeof(Payload) * (emax > 0 ? emax : 1));
-  const size_t o_cnt = take(sizeof(int32_t) * nb * F);
-  const size_t o_tot = take(sizeof(int32_t) * (size_t)F);
+  const size_t o_cnt = take(sizeof(int32_t) * 2 * (size_t)F);
   const size_t o_off = take(sizeof(int32_t) * ((size_t)F + 1));
   const size_t o_list = take(sizeof(int32_t) * (emax > 0 ? emax : 1));
+  const size_t o_sorted = take(sizeof(int32_t) * (emax > 0 ? emax : 1));
   w.bytes = off;
   if (base) {
     char* p = static_cast<char*>(base);
     w.e0 = reinterpret_cast<int32_t*>(p + o_e0);
     w.pay = reinterpret_cast<Payload*>(p + o_pay);
-    w.cnt = reinterpret_cast<int32_t*>(p + o_cnt);
-    w.unit_total = reinterpret_cast<int32_t*>(p + o_tot);
+    w.ucnt = reinterpret_cast<int32_t*>(p + o_cnt);
+    w.cursor = w.ucnt + F;
     w.unit_off = reinterpret_cast<int32_t*>(p + o_off);
     w.list = reinterpret_cast<int32_t*>(p + o_list);
+    w.sorted = reinterpret_cast<int32_t*>(p + o_sorted);
   }
   return w;
 }
@@ -704,17 +628,8 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
                        const void* Wu_t, const void* Wd, int d, float lam, void* dx,
                        tw_dtype dx_dtype, float* dWg_t, float* dWu_t, float* dWd, void* ws,
                        int32_t* status, cudaStream_t s) {
-  const HView<T> h = view_of<T>(gu);
   const BwdWs w = carve(ws, gu.T, gu.F, gu.C_h, gu.backup_cap);
   void* engine_ws = static_cast<char*>(ws) + w.bytes;
-  const int nb = (gu.T + TB - 1) / TB;
-  const size_t hist_bytes = tb_hist_bytes(gu.F);
-  for (const void* f : {reinterpret_cast<const void*>(hyb_count_kernel<T>),
-                        reinterpret_cast<const void*>(hyb_fill_kernel<T, false>),
-                        reinterpret_cast<const void*>(hyb_fill_kernel<T, true>)}) {
-    const cudaError_t ea = set_smem_limit(f, 200 * 1024);
-    if (ea != cudaSuccess) return ea;
-  }
   // entry offsets of every token (token-major order)
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(2, gu.T, gu.row_nnz, 0, w.e0, gu.row_slot,
                                          gu.backup_cap, nullptr, status);
@@ -722,21 +637,18 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
   cudaError_t e = launch_hybrid_gather_backward(dy, gu, Wg_t, Wu_t, Wd, d, lam, w.e0, w.pay, dx,
                                                 dx_dtype, engine_ws, status, s);
   if (e != cudaSuccess) return e;
-  // weight gradients: records transposed to unit-major, token order kept
-  hyb_count_kernel<T><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt);
-  hyb_colscan_kernel<<<(gu.F + 255) / 256, 256, 0, s>>>(nb, gu.F, w.cnt, w.unit_total);
-  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.unit_total, 0, w.unit_off, nullptr, 0,
-                                         nullptr, status);
-  const size_t base_bytes = sizeof(int32_t) * (size_t)gu.F;
-  if (hist_bytes + base_bytes <= 200 * 1024)
-    hyb_fill_kernel<T, true><<<nb, 32 * TB_WARPS, hist_bytes + base_bytes, s>>>(
-        h, nb, w.cnt, w.unit_off, w.e0, w.list);
-  else
-    hyb_fill_kernel<T, false><<<nb, 32 * TB_WARPS, hist_bytes, s>>>(h, nb, w.cnt, w.unit_off,
-                                                                   w.e0, w.list);
+  // weight gradients: records grouped by unit, then each unit sorted and summed
+  e = cudaMemsetAsync(w.ucnt, 0, sizeof(int32_t) * 2 * (size_t)gu.F, s);
+  if (e != cudaSuccess) return e;
+  const int grid = num_sms() * 8;
+  const int32_t* e_total = w.e0 + gu.T;
+  hyb_ucount_kernel<<<grid, 256, 0, s>>>(w.pay, e_total, w.ucnt);
+  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.ucnt, 0, w.unit_off, nullptr, 0, nullptr,
+                                         status);
+  hyb_place_kernel<<<grid, 256, 0, s>>>(w.pay, e_total, w.unit_off, w.cursor, w.list);
   hyb_wgrad_kernel<T><<<gu.F, 256, 0, s>>>(gu.F, d, static_cast<const T*>(x),
-                                           static_cast<const T*>(dy), w.unit_off, w.list, w.pay,
-                                           dWg_t, dWu_t, dWd);
+                                           static_cast<const T*>(dy), w.unit_off, w.list,
+                                           w.sorted, w.pay, dWg_t, dWu_t, dWd);
   return cudaGetLastError();
 }
 

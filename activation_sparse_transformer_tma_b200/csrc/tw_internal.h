@@ -83,7 +83,7 @@ cudaError_t launch_dense_train_backward(const void* x, const void* dy, const voi
 // One active (t, j) entry of the hybrid backward, recorded for the
 // weight-gradient pass: h = g u, du, dz.
 struct Payload {
-  int32_t t;
+  int32_t t, j;  // token and unit
   float h, du, dz;
 };
 

@@ -203,6 +203,22 @@ def test_hybrid_from_other_tile_widths(W):
     assert 0 < got["n_backup"] < 300
 
 
+def test_hybrid_weight_gradients_of_a_unit_with_thousands_of_entries():
+    """Zipf units without the permutation: the hottest units are active for
+    half of 5000 tokens, so their records exceed the 2048 a CTA sorts in
+    shared memory and take the sorted-runs path of the weight gradients."""
+    w = synth.make_workload(T=5000, d=256, F=1024, W=128, C=8, C_h=64, dtype=synth.BF16,
+                            kind="zipf", lam=2e-5, seed=31, mean_active=29.0, permute=False,
+                            with_dy=True)
+    res = run_hybrid(w, backup_cap=5000)
+    hy = res[5]
+    got = check_hybrid_all(w, res)
+    cols = got["ell_idx"][got["ell_g"] != 0]
+    bcols = np.nonzero(got["backup_g"])[1]
+    per_unit = np.bincount(np.concatenate([cols, bcols]).astype(np.int64), minlength=1024)
+    assert per_unit.max() > 2048
+
+
 def test_hybrid_from_wide_capacity_twell():
     """TwELL -> hybrid with C = 64: tiles with more than 32 slots feed ELL rows."""
     w = synth.make_workload(T=300, d=256, F=640, W=128, C=64, C_h=155, dtype=synth.BF16,
