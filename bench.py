@@ -656,6 +656,9 @@ def training_leg(torch, tw, dist=None, world=1):
     twell_bytes = sum(t.numel() * t.element_size() for t in (g.val, g.idx, g.cnt, g.spill_ref,
                                                               g.spill_tk, g.spill_val, g.spill_n))
     sparse_ws = fws.numel() + ws.numel()
+    # the backward workspace bounds every backup row by F records; a caller
+    # that sizes its backup capacity to the rows it uses needs this much
+    sparse_ws_fit = fws.numel() + tw.hybrid_ffn_backward_workspace_size(T, d, F, C_h, n_backup)
     del g, hy, fws, ws
     torch.cuda.empty_cache()
 
@@ -702,11 +705,15 @@ def training_leg(torch, tw, dist=None, world=1):
                "sparse_twell_transient": twell_bytes,
                "sparse_workspaces": sparse_ws,
                "sparse_peak": saved_alloc + max(twell_bytes, sparse_ws),
+               "sparse_workspaces_exact_fit": sparse_ws_fit,
+               "sparse_peak_exact_fit": saved_fit + max(twell_bytes, sparse_ws_fit),
                "dense_saved_fwd_to_bwd": dense_saved,
                "dense_workspace": dense_ws,
                "dense_peak": dense_ws,
                "peak_ratio_sparse_over_dense": (saved_alloc + max(twell_bytes, sparse_ws))
-                                               / dense_ws}}
+                                               / dense_ws,
+               "peak_ratio_exact_fit": (saved_fit + max(twell_bytes, sparse_ws_fit))
+                                       / dense_ws}}
     if world > 1:
         out["parallelism"] = f"dp{world}: one fp32 all-reduce of dWg, dWu, dWd ({3 * F * d * 4} B)"
     return out
