@@ -40,7 +40,10 @@
 // runs in two phases: each warp forms its partial dot products of all the
 // window's entries, two at a time, and leaves them in shared memory; after
 // one named barrier each warp adds the team's partials in warp order, derives
-// the entry's scalars and updates its own columns.
+// the entry's scalars and updates its own columns.  Entry lists alternate
+// between two buffers and the next item's descriptor is published during the
+// current item, so a window costs two team barriers (list written, partials
+// written) and an item none of its own.
 //
 // Data movement.  Weight rows are gathered with plain 16-byte vector loads
 // straight into registers (each lane owns 16-byte column slices, so a warp's
@@ -65,7 +68,6 @@ constexpr int kPart = 64;          // entries per part of a split token (upper b
 constexpr int kMinPart = 8;        // lower bound of the part size
 constexpr int kTeam = 2;           // warps per work item
 constexpr int kTeams = 8;          // teams per CTA
-constexpr int kWarps = kTeam * kTeams;
 constexpr int kListCap = 64;       // entry window collected at a time
 constexpr int kCountBlock = 256;   // tokens per block of the count kernels
 
@@ -430,23 +432,22 @@ struct Elem<float> {
 // D (16x8 fp32) += A (16x16 bf16, row-major) . B (16x8 bf16, column-major).
 TW_DEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                            uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Sum over the warp of p0 (result in lane 0) and of p1 (result in lane 16)
-// with five shuffle steps.
-TW_DEV void warp_sum2(float p0, float p1, int lane, float& s0, float& s1) {
+// Sum over the warp of p0 and of p1 with five shuffle steps; lane 0 stores
+// the first sum to *s0 and lane 16 the second to *s1.
+TW_DEV void warp_sum2(float p0, float p1, int lane, float* s0, float* s1) {
   const bool hi = (lane & 16) != 0;
   float v = hi ? p1 : p0;
   v += __shfl_xor_sync(FULL, hi ? p0 : p1, 16);
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-  s0 = __shfl_sync(FULL, v, 0);
-  s1 = __shfl_sync(FULL, v, 16);
+  if (lane == 0) *s0 = v;
+  if (lane == 16) *s1 = v;
 }
 
 // This warp's partial dot products of the token row (xr) with the rows of
@@ -488,7 +489,7 @@ TW_DEV void dot2_issue(const uint4 (&xr)[NCHW], const uint4 (&w)[2][NCHW], float
 }
 
 template <typename Tin>
-TW_DEV void dot2_reduce(const float (&D)[2][4], int lane, float& v0, float& v1) {
+TW_DEV void dot2_reduce(const float (&D)[2][4], int lane, float* v0, float* v1) {
   float p0, p1;
   if constexpr (sizeof(Tin) == 2) {
     float d[4];
@@ -511,7 +512,7 @@ TW_DEV void dot2_reduce(const float (&D)[2][4], int lane, float& v0, float& v1) 
 // gathered again by other tokens; activations and outputs stream past them).
 TW_DEV uint4 ldg_keep(const uint4* p, uint64_t policy) {
   uint4 r;
-  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+  asm("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p), "l"(policy));
   return r;
@@ -522,19 +523,32 @@ TW_DEV uint64_t policy_evict_last() {
   return pol;
 }
 
-template <typename Tin, int NCHW>
+//
+// kFull: every lane's slices lie inside the row (d is exactly kTeam warps'
+// slices), so no load is predicated; a missing second entry then re-reads
+// the first entry's row, which its zero coefficient leaves without effect.
+template <typename Tin, int NCHW, bool kFull>
 TW_DEV void load_rows2(uint4 (&w)[2][NCHW], const Tin* base, int j0, int j1, bool two, int d,
                        int c0, int my_cols, int lane, uint64_t pol) {
   constexpr int E = Elem<Tin>::E;
   constexpr int SPAN = 32 * E;
   const uint4* p0 = reinterpret_cast<const uint4*>(base + (size_t)j0 * d + c0);
-  const uint4* p1 = reinterpret_cast<const uint4*>(base + (size_t)j1 * d + c0);
+  if constexpr (kFull) {
+    const uint4* p1 = reinterpret_cast<const uint4*>(base + (size_t)(two ? j1 : j0) * d + c0);
 #pragma unroll
-  for (int c = 0; c < NCHW; ++c) {
-    const int lc = c * SPAN + lane * E;
-    const bool in = lc < my_cols;
-    w[0][c] = in ? ldg_keep(p0 + lc / E, pol) : make_uint4(0, 0, 0, 0);
-    w[1][c] = in && two ? ldg_keep(p1 + lc / E, pol) : make_uint4(0, 0, 0, 0);
+    for (int c = 0; c < NCHW; ++c) {
+      w[0][c] = ldg_keep(p0 + c * 32 + lane, pol);
+      w[1][c] = ldg_keep(p1 + c * 32 + lane, pol);
+    }
+  } else {
+    const uint4* p1 = reinterpret_cast<const uint4*>(base + (size_t)j1 * d + c0);
+#pragma unroll
+    for (int c = 0; c < NCHW; ++c) {
+      const int lc = c * SPAN + lane * E;
+      const bool in = lc < my_cols;
+      w[0][c] = in ? ldg_keep(p0 + lc / E, pol) : make_uint4(0, 0, 0, 0);
+      w[1][c] = in && two ? ldg_keep(p1 + lc / E, pol) : make_uint4(0, 0, 0, 0);
+    }
   }
 }
 
@@ -581,31 +595,47 @@ struct GatherArgs {
   FusedWs ws;
 };
 
-// Shared state of one team.
-struct TeamSmem {
+// One window's entry list.
+struct EntryList {
   float g[kListCap];
   int32_t j[kListCap];
   int32_t pos[kListCap];  // hybrid position of the entry (u is saved / read there)
   float u[kListCap];      // saved u of the entry (backward)
-  float part[kTeam][kListCap];  // each warp's partial dot product per entry of the window
-  int4 desc[2];           // current item, double-buffered by item parity
-  int n;                  // entries in the current window
+  alignas(16) float part[kListCap][kTeam];  // each warp's partial dot product per entry
+                                           // (a pair's partials are 16 bytes)
+};
+
+// Shared state of one team.  Lists alternate by window parity and
+// descriptors by item parity, so no barrier is needed before either is
+// rewritten: a buffer is written again two windows (items) later, after both
+// warps have passed the barriers of the window (item) in between.
+struct TeamSmem {
+  EntryList list[2];
+  int4 desc[2];           // item descriptors, published one item ahead
+  int n[2];               // entries in the window, by window parity (hybrid modes)
   int prev;               // arrival count at a sum-tree node, broadcast to the team
 };
 
 // TwELL: the entries of token t with ordinal in [lo, hi) (tile-major order,
-// ascending within a tile) into the team's list; returns how many.  Each lane
-// owns one tile, so the slots of all active tiles are read in one round;
-// spilled tiles are read by the whole warp.
+// ascending within a tile) into a list; returns how many.  Each lane owns one
+// tile of a round of 32 tiles, so the slots of all active tiles of a round are
+// read at once; spilled tiles are read by the whole warp.  The rounds are
+// dealt out to `nwho` warps (this one is `who`): every warp scans every
+// round's counts, so all know each entry's ordinal and the total, and each
+// writes the entries of its own rounds.
 template <typename Tin>
 TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float* sg, int32_t* sj,
-                         int lane) {
+                         int lane, int who, int nwho) {
   const int W = a.W;
   const int K = a.F / W;
   int base = 0;  // ordinal of the first entry of tile kb
+  int n_next = lane < K ? (int)a.cnt[(size_t)lane * a.T + t] : 0;
   for (int kb = 0; kb < K && base < hi; kb += 32) {
     const int k = kb + lane;
-    const int n = k < K ? (int)a.cnt[(size_t)k * a.T + t] : 0;
+    const int n = n_next;
+    const bool mine = ((kb >> 5) % nwho) == who;
+    // the next round's count, loaded while this round is expanded
+    n_next = k + 32 < K ? (int)a.cnt[(size_t)(k + 32) * a.T + t] : 0;
     int incl = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -613,7 +643,7 @@ TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float*
       if (lane >= o) incl += u;
     }
     const int tb = base + incl - n;  // first ordinal of tile k
-    const bool over = n > 0 && tb < hi && tb + n > lo;
+    const bool over = mine && n > 0 && tb < hi && tb + n > lo;
     const size_t kt = (size_t)k * a.T + t;
     int ref = -1;
     if (over && n > a.C) {
@@ -665,7 +695,7 @@ TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float*
 // Hybrid: the entries of token t with ordinal in [lo, hi): ELL slots in order,
 // or the non-zeros of its backup row in ascending unit order.
 template <typename Tin, int MODE>
-TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, TeamSmem& s,
+TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, EntryList& s,
                           int lane) {
   const int slot = a.row_slot[t];
   if (slot < 0) {
@@ -738,7 +768,8 @@ TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, TeamS
 template <int NCHW, int MODE>
 constexpr int teams_for() { return NCHW < 4 ? kTeams : (MODE == kModeHybBwd ? 4 : 6); }
 
-template <typename Tin, int NCHW, bool kOutBf16, int MODE>
+// kFull: d is exactly the kTeam warps' slices (see load_rows2).
+template <typename Tin, int NCHW, bool kOutBf16, int MODE, bool kFull>
 __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
     gather_kernel(const GatherArgs<Tin> a) {
   using L = Elem<Tin>;
@@ -760,22 +791,27 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
   const bool leader = tw == 0;
   const uint64_t pol = policy_evict_last();
 
+  // Items come from a ticket counter.  The leader publishes the descriptor
+  // of the team's next item while the current one runs (before the team
+  // barrier in the middle of its first window), so an item starts without a
+  // barrier of its own.
   int ticket = 0;
-  if (leader && lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);
-  for (uint32_t it = 0;; ++it) {
-    // The descriptor slot alternates between items: the partner reads slot
-    // it&1 after this barrier, and the leader next writes it two items later,
-    // behind barriers the partner has passed.
+  auto publish = [&](int slot) {
     if (leader && lane == 0) {
-      const int item = ticket;
-      ts.desc[it & 1] = item < n_items ? a.ws.item_desc[item] : make_int4(-1, 0, 0, -1);
-      if (item < n_items) ticket = atomicAdd(&a.ws.hdr[0], 1);  // next, fetched early
+      ts.desc[slot] = ticket < n_items ? a.ws.item_desc[ticket] : make_int4(-1, 0, 0, -1);
+      if (ticket < n_items) ticket = atomicAdd(&a.ws.hdr[0], 1);
     }
-    team_bar(team);
+  };
+  if (leader && lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);
+  publish(0);
+  team_bar(team);
+  uint32_t win = 0;  // windows processed by the team: the list parity
+  for (uint32_t it = 0;; ++it) {
     const int4 desc = ts.desc[it & 1];
     if (desc.x < 0) break;
     const int t = desc.x, lo = desc.y, hi = desc.z, prow = desc.w;
     const bool to_backup = MODE == kModeHybFwd && a.row_slot[t] >= 0;
+    bool published = false;
 
     uint4 xr[NCHW];  // the token's row slices, kept in the input format
     float2 acc[NCHW][P];
@@ -783,22 +819,28 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
 #pragma unroll
     for (int c = 0; c < NCHW; ++c) {
       const int col = c0 + c * SPAN + lane * E;
-      xr[c] = col < d ? __ldcs(reinterpret_cast<const uint4*>(xt + col)) : make_uint4(0, 0, 0, 0);
+      xr[c] = kFull || col < d ? __ldcs(reinterpret_cast<const uint4*>(xt + col))
+                               : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
     }
 
-    for (int w0 = lo; w0 < hi; w0 += kListCap) {
-      if (leader) {
-        const int w1 = min(hi, w0 + kListCap);
-        const int n = MODE == kModeTwell ? collect_twell(a, t, w0, w1, ts.g, ts.j, lane)
-                                         : collect_hybrid<Tin, MODE>(a, t, w0, w1, ts, lane);
-        if (lane == 0) ts.n = n;
+    for (int w0 = lo; w0 < hi; w0 += kListCap, ++win) {
+      EntryList& ls = ts.list[win & 1];
+      const int w1 = min(hi, w0 + kListCap);
+      int n;
+      if constexpr (MODE == kModeTwell) {
+        n = collect_twell(a, t, w0, w1, ls.g, ls.j, lane, tw, kTeam);
+        team_bar(team);  // the list is written
+      } else {
+        if (leader) {
+          const int m = collect_hybrid<Tin, MODE>(a, t, w0, w1, ls, lane);
+          if (lane == 0) ts.n[win & 1] = m;
+        }
+        team_bar(team);  // the list is written
+        n = ts.n[win & 1];
       }
-      team_bar(team);
-      const int n = ts.n;
       const int npairs = (n + 1) / 2;
-      auto jof = [&](int e) { return e < n ? ts.j[e] : 0; };
       // rows of a missing second entry are zeros, so both rows always update
       auto update = [&](const uint4 (&R)[2][NCHW], float sa, float sb) {
         const float2 ha = make_float2(sa, sa), hb = make_float2(sb, sb);
@@ -813,9 +855,12 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
           for (int q = 0; q < P; ++q) acc[c][q] = __ffma2_rn(hb, w[q], acc[c][q]);
         }
       };
+      // rows of the entry pair pp (its first entry always exists)
       auto load = [&](uint4 (&R)[2][NCHW], const Tin* base, int pp) {
-        load_rows2<Tin, NCHW>(R, base, jof(2 * pp), jof(2 * pp + 1), 2 * pp + 1 < n, d, c0,
-                              my_cols, lane, pol);
+        const int2 jj = *reinterpret_cast<const int2*>(&ls.j[2 * pp]);
+        const bool two = 2 * pp + 1 < n;
+        load_rows2<Tin, NCHW, kFull>(R, base, jj.x, two ? jj.y : 0, two, d, c0, my_cols, lane,
+                                     pol);
       };
       {
         // Two phases per window.  Phase 1: this warp's partial dot products of
@@ -823,24 +868,28 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
         // between pairs.  One team barrier.  Phase 2: the scalars of each
         // entry from the team's partials (added in warp order) -- h, or in
         // the backward du and dz with the entry's record -- and the row
-        // updates, two pairs of update rows in flight.
+        // updates, two pairs of update rows in flight.  Outside the backward,
+        // a register set freed by the last dot pairs takes the rows of the
+        // first update pairs at once (pair q in set q & 1, as in phase 2).
         uint4 S0[2][NCHW], S1[2][NCHW];
         if (npairs > 0) load(S0, a.rdot, 0);
         if (npairs > 1) load(S1, a.rdot, 1);
         auto dots = [&](uint4 (&R)[2][NCHW], int pp) {
           float D[2][4];
           dot2_issue<Tin, NCHW>(xr, R, D);
-          if (pp + 2 < npairs) load(R, a.rdot, pp + 2);
-          float v0, v1;
-          dot2_reduce<Tin>(D, lane, v0, v1);
-          if (lane == 0) {
-            ts.part[tw][2 * pp] = v0;
-            ts.part[tw][2 * pp + 1] = v1;
-          }
+          if (pp + 2 < npairs)
+            load(R, a.rdot, pp + 2);
+          else if (!kBwd && (pp & 1) < npairs)
+            load(R, a.rax1, pp & 1);
+          dot2_reduce<Tin>(D, lane, &ls.part[2 * pp][tw], &ls.part[2 * pp + 1][tw]);
         };
         for (int pp = 0; pp < npairs; pp += 2) {
           dots(S0, pp);
           if (pp + 1 < npairs) dots(S1, pp + 1);
+        }
+        if (!published) {  // the next item's descriptor, behind the barrier below
+          publish((it + 1) & 1);
+          published = true;
         }
         if constexpr (kBwd) {
           // S0, S1: Wu_t rows (du); T0, T1: Wg_t rows (dz)
@@ -853,20 +902,20 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
             load(S1, a.rax1, 1);
             load(T1, a.rax2, 1);
           }
-          team_bar(team);
+          team_bar(team);  // the partials (and the next descriptor) are written
           auto coef = [&](int e, float& du, float& dz) {
             du = dz = 0.f;
             if (e >= n) return;
             float dh = 0.f;
 #pragma unroll
-            for (int q = 0; q < kTeam; ++q) dh += ts.part[q][e];
-            const float gv = ts.g[e], uv = ts.u[e];
+            for (int q = 0; q < kTeam; ++q) dh += ls.part[e][q];
+            const float gv = ls.g[e], uv = ls.u[e];
             du = dh * gv;
             dz = fmaf(dh, uv, a.lam);
             if (leader && lane == 0) {
               Payload pl;
               pl.t = t;
-              pl.j = ts.j[e];
+              pl.j = ls.j[e];
               pl.h = gv * uv;
               pl.du = du;
               pl.dz = dz;
@@ -886,32 +935,34 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
             upd2(S0, T0, pp);
             if (pp + 1 < npairs) upd2(S1, T1, pp + 1);
           }
-          team_bar(team);  // the list and the partials may be overwritten by the next window
           continue;
         }
-        if (npairs > 0) load(S0, a.rax1, 0);
-        if (npairs > 1) load(S1, a.rax1, 1);
-        team_bar(team);
-        auto hval = [&](int e) {
-          if (e >= n) return 0.f;
-          float dv = 0.f;
-#pragma unroll
-          for (int q = 0; q < kTeam; ++q) dv += ts.part[q][e];
-          if (MODE == kModeHybFwd && leader && lane == 0)
-            L::store((to_backup ? a.backup_u : a.ell_u) + ts.pos[e], dv);
-          return ts.g[e] * dv;
-        };
+        team_bar(team);  // the partials (and the next descriptor) are written
+        // h of the pair's entries: u from the team's partials (added in warp
+        // order), times g; 0 for a missing second entry
+        static_assert(kTeam == 2, "a pair's partials are read as one float4");
         auto upd = [&](uint4 (&R)[2][NCHW], int pp) {
-          const float ha = hval(2 * pp), hb = hval(2 * pp + 1);
-          update(R, ha, hb);
+          const float4 pt = *reinterpret_cast<const float4*>(&ls.part[2 * pp][0]);
+          const float2 gg = *reinterpret_cast<const float2*>(&ls.g[2 * pp]);
+          const bool two = 2 * pp + 1 < n;
+          const float ua = pt.x + pt.y, ub = pt.z + pt.w;
+          if (MODE == kModeHybFwd && leader && lane == 0) {
+            Tin* dst = to_backup ? a.backup_u : a.ell_u;
+            L::store(dst + ls.pos[2 * pp], ua);
+            if (two) L::store(dst + ls.pos[2 * pp + 1], ub);
+          }
+          update(R, gg.x * ua, two ? gg.y * ub : 0.f);
           if (pp + 2 < npairs) load(R, a.rax1, pp + 2);
         };
         for (int pp = 0; pp < npairs; pp += 2) {
           upd(S0, pp);
           if (pp + 1 < npairs) upd(S1, pp + 1);
         }
-        team_bar(team);  // the list and the partials may be overwritten by the next window
       }
+    }
+    if (!published) {  // an item without entries
+      publish((it + 1) & 1);
+      team_bar(team);
     }
 
     // ------------------------------------------------------------ output --
@@ -1005,7 +1056,11 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
 
 template <typename Tin, int NCHW, int MODE>
 cudaError_t launch_nchw(GatherArgs<Tin> a, bool out_bf16, cudaStream_t stream) {
-  auto kern = out_bf16 ? gather_kernel<Tin, NCHW, true, MODE> : gather_kernel<Tin, NCHW, false, MODE>;
+  const bool full = a.d == kTeam * NCHW * 32 * Elem<Tin>::E;
+  auto kern = full ? (out_bf16 ? gather_kernel<Tin, NCHW, true, MODE, true>
+                               : gather_kernel<Tin, NCHW, false, MODE, true>)
+                   : (out_bf16 ? gather_kernel<Tin, NCHW, true, MODE, false>
+                               : gather_kernel<Tin, NCHW, false, MODE, false>);
   constexpr int threads = 32 * kTeam * teams_for<NCHW, MODE>();
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
@@ -1034,7 +1089,8 @@ __global__ void __launch_bounds__(32 * kDecWarps) decode_kernel(const GatherArgs
   constexpr int P = L::P;
   constexpr int SPAN = 32 * E;   // columns of one warp-wide slice
   constexpr int NCH = 8;         // slices per lane: d <= 8 * SPAN (the validated maximum)
-  __shared__ TeamSmem lst;
+  __shared__ EntryList lst;
+  __shared__ int lst_n;
   __shared__ float hsh[kListCap];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1053,11 +1109,11 @@ __global__ void __launch_bounds__(32 * kDecWarps) decode_kernel(const GatherArgs
 
   for (int w0 = 0;; w0 += kListCap) {
     if (warp == 0) {
-      const int n = collect_twell(a, t, w0, w0 + kListCap, lst.g, lst.j, lane);
-      if (lane == 0) lst.n = n;
+      const int n = collect_twell(a, t, w0, w0 + kListCap, lst.g, lst.j, lane, 0, 1);
+      if (lane == 0) lst_n = n;
     }
     __syncthreads();
-    const int n = lst.n;
+    const int n = lst_n;
     // h of each entry: two entries per warp at a time
     for (int e = warp; e < n; e += 2 * kDecWarps) {
       const int e2 = e + kDecWarps;
