@@ -54,9 +54,9 @@
 // the copy engine spends a roughly fixed time per copy, which bounded that
 // version by the number of row slices, not by bytes.)
 //
-// Arithmetic.  bf16 dot products run on the tensor pipe (mma.sync with a
-// diagonal-extraction layout, see dot2_issue); the scaled-row updates widen bf16
-// pairs exactly and use packed fp32x2 FMA.
+// Arithmetic.  bf16 dot products use the mixed-precision FMA (bf16 operands,
+// fp32 accumulator); the scaled-row updates widen bf16 pairs exactly and use
+// packed fp32x2 FMA.
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -429,15 +429,6 @@ struct Elem<float> {
   }
 };
 
-// D (16x8 fp32) += A (16x16 bf16, row-major) . B (16x8 bf16, column-major).
-TW_DEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                           uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 // Sum over the warp of p0 and of p1 with five shuffle steps; lane 0 stores
 // the first sum to *s0 and lane 16 the second to *s1.
 TW_DEV void warp_sum2(float p0, float p1, int lane, float* s0, float* s1) {
@@ -453,56 +444,29 @@ TW_DEV void warp_sum2(float p0, float p1, int lane, float* s0, float* s1) {
 // This warp's partial dot products of the token row (xr) with the rows of
 // two entries (w[0], w[1]), all held in registers as this lane's 16-byte
 // slices of the warp's column range; a missing second entry is all zeros.
-// dot2_issue leaves per-lane partial sums in D; dot2_reduce turns them into
-// the two warp sums, so independent work can be placed between the two.
-//
-// bf16: on the tensor pipe.  One m16n8k16 MMA takes, from lane (g, q) =
-// (lane / 4, lane % 4), four consecutive columns of its slice: A row g holds
-// them for the first entry, A row g + 8 for the second, B column g holds the
-// token's values at the same columns.  The diagonal D[g][g] (D[g + 8][g]) is
-// then the dot product of the first (second) row with the token over the 16
-// columns of lanes 4g..4g+3; the other products are not used.  D[g][g] sits
-// in lane 4g + g/2, register g & 1 (+2 for the second entry).  Products of
-// bf16 are exact and the MMA accumulates in fp32; two accumulators halve the
-// chain of dependent MMAs.
+// dot2_issue leaves four running sums per entry in each lane (bf16: the
+// mixed-precision FMA, whose bf16 products are exact in fp32); dot2_reduce
+// turns them into the two warp sums, so independent work can be placed
+// between the two.  (The tensor pipe was tried for these dot products, with
+// the rows of two entries as the A fragment of an m16n8k16 MMA and the
+// diagonal of D kept: the chains of dependent MMAs made it slower.)
 template <typename Tin, int NCHW>
 TW_DEV void dot2_issue(const uint4 (&xr)[NCHW], const uint4 (&w)[2][NCHW], float (&D)[2][4]) {
 #pragma unroll
-  for (int k = 0; k < 2; ++k)
+  for (int e = 0; e < 2; ++e)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) D[k][i] = 0.f;
-  if constexpr (sizeof(Tin) == 2) {
+    for (int i = 0; i < 4; ++i) D[e][i] = 0.f;
 #pragma unroll
-    for (int c = 0; c < NCHW; ++c) {
-      mma_bf16_16816(D[0], w[0][c].x, w[1][c].x, w[0][c].y, w[1][c].y, xr[c].x, xr[c].y);
-      mma_bf16_16816(D[1], w[0][c].z, w[1][c].z, w[0][c].w, w[1][c].w, xr[c].z,
-                     xr[c].w);
-    }
-  } else {
-    // fp32: D[0] and D[1] hold four running sums per entry
-#pragma unroll
-    for (int c = 0; c < NCHW; ++c) {
-      Elem<Tin>::dot(xr[c], w[0][c], D[0]);
-      Elem<Tin>::dot(xr[c], w[1][c], D[1]);
-    }
+  for (int c = 0; c < NCHW; ++c) {
+    Elem<Tin>::dot(xr[c], w[0][c], D[0]);
+    Elem<Tin>::dot(xr[c], w[1][c], D[1]);
   }
 }
 
 template <typename Tin>
 TW_DEV void dot2_reduce(const float (&D)[2][4], int lane, float* v0, float* v1) {
-  float p0, p1;
-  if constexpr (sizeof(Tin) == 2) {
-    float d[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = D[0][i] + D[1][i];
-    const int g = lane >> 2;
-    const bool diag = (lane & 3) == (g >> 1);
-    p0 = diag ? ((g & 1) ? d[1] : d[0]) : 0.f;
-    p1 = diag ? ((g & 1) ? d[3] : d[2]) : 0.f;
-  } else {
-    p0 = (D[0][0] + D[0][1]) + (D[0][2] + D[0][3]);
-    p1 = (D[1][0] + D[1][1]) + (D[1][2] + D[1][3]);
-  }
+  const float p0 = (D[0][0] + D[0][1]) + (D[0][2] + D[0][3]);
+  const float p1 = (D[1][0] + D[1][1]) + (D[1][2] + D[1][3]);
   warp_sum2(p0, p1, lane, v0, v1);
 }
 
