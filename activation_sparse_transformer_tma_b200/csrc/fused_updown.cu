@@ -66,6 +66,10 @@ namespace {
 constexpr unsigned FULL = 0xFFFFFFFFu;
 constexpr int kPart = 64;          // entries per part of a split token (upper bound)
 constexpr int kMinPart = 8;        // lower bound of the part size
+// Items of split tokens and unsplit tokens with at least kHeavy entries are
+// handed out first: with the long items taken early, the last items of the
+// launch are short and the teams finish close together.
+constexpr int kHeavy = 32;
 constexpr int kTeam = 2;           // warps per work item
 constexpr int kTeams = 8;          // teams per CTA
 constexpr int kListCap = 64;       // entry window collected at a time
@@ -138,15 +142,17 @@ bool carve_within(void* base, int T, int d, size_t limit, FusedWs* out) {
 }
 
 // -------------------------------------------------------------------- plan --
-// Per-block partials for the planner's fast path: entries, split parts and
-// work items of the block's tokens with the part size kPart (thread 0 writes).
+// Per-block partials for the planner's fast path: entries, split parts, work
+// items and heavy items (see kHeavy) of the block's tokens with the part size
+// kPart (thread 0 writes).
 TW_DEV void count_block_partials(int n, bool valid, int4* bpart) {
-  __shared__ int red[3][kCountBlock / 32];
+  __shared__ int red[4][kCountBlock / 32];
   const int parts = n > kPart ? (n + kPart - 1) / kPart : 0;
-  int v[3] = {n, parts, valid ? (parts > 0 ? parts : 1) : 0};
+  int v[4] = {n, parts, valid ? (parts > 0 ? parts : 1) : 0,
+              valid ? (parts > 0 ? parts : (n >= kHeavy ? 1 : 0)) : 0};
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < 4; ++i) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v[i] += __shfl_xor_sync(FULL, v[i], o);
     if (lane == 0) red[i][wid] = v[i];
@@ -158,6 +164,7 @@ TW_DEV void count_block_partials(int n, bool valid, int4* bpart) {
       r.x += red[0][w2];
       r.y += red[1][w2];
       r.z += red[2][w2];
+      r.w += red[3][w2];
     }
     bpart[blockIdx.x] = r;
   }
@@ -229,7 +236,8 @@ size_t plan_scan_smem(int T) {
 }
 
 // One CTA: the part size, partial rows of split tokens (in token order,
-// within capacity), then one descriptor per work item.  The part size is
+// within capacity), then one descriptor per work item: heavy items (see
+// kHeavy) first, then the others, each group in token order.  The part size is
 // kPart, lowered to about two items per team when there are few entries in
 // all (small batches), but not below kMinPart; it is stored in hdr[2].
 // Each thread owns a contiguous run of tokens, so each of the three passes
@@ -251,28 +259,33 @@ __global__ void __launch_bounds__(kScanThreads)
   // per-block offsets of split parts and items) and plan_write_kernel writes
   // the same plan with one thread per token.
   {
-    int e = 0, sp = 0, it = 0;
+    int e = 0, sp = 0, it = 0, hv = 0;
     for (int b = threadIdx.x; b < nb; b += kScanThreads) {
       const int4 v = bpart[b];
       e += v.x;
       sp += v.y;
       it += v.z;
+      hv += v.w;
     }
-    int te, tsp, tit;
+    int te, tsp, tit, thv;
     block_exclusive_scan(e, warp_sums, &te);
     block_exclusive_scan(sp, warp_sums, &tsp);
     block_exclusive_scan(it, warp_sums, &tit);
+    block_exclusive_scan(hv, warp_sums, &thv);
     if (te / (2 * n_teams) >= kPart && tsp <= parts_cap) {
-      int carry_s = 0, carry_i = 0;
+      // per block: first split part, first heavy item, first other item
+      int carry_s = 0, carry_h = 0, carry_l = 0;
       for (int b0 = 0; b0 < nb; b0 += kScanThreads) {
         const int b = b0 + threadIdx.x;
         const int4 v = b < nb ? bpart[b] : make_int4(0, 0, 0, 0);
-        int ts2, ti2;
+        int ts2, th2, tl2;
         const int xs = block_exclusive_scan(v.y, warp_sums, &ts2);
-        const int xi = block_exclusive_scan(v.z, warp_sums, &ti2);
-        if (b < nb) bpart[b] = make_int4(carry_s + xs, carry_i + xi, 0, 0);
+        const int xh = block_exclusive_scan(v.w, warp_sums, &th2);
+        const int xl = block_exclusive_scan(v.z - v.w, warp_sums, &tl2);
+        if (b < nb) bpart[b] = make_int4(carry_s + xs, carry_h + xh, thv + carry_l + xl, 0);
         carry_s += ts2;
-        carry_i += ti2;
+        carry_h += th2;
+        carry_l += tl2;
       }
       if (threadIdx.x == 0) {
         hdr[1] = tit < max_items ? tit : max_items;
@@ -314,34 +327,43 @@ __global__ void __launch_bounds__(kScanThreads)
   }
   int tot;
   const int ex1 = block_exclusive_scan(local, warp_sums, &tot);
-  // pass 2: one descriptor per work item (the slot decision of pass 1 is
-  // recomputed from the same running offset)
-  local = 0;
+  // pass 2: one descriptor per work item, heavy items first (the slot
+  // decision of pass 1 is recomputed from the same running offset)
+  int local_h = 0, local_l = 0;
   int ex = ex1;
   for (int t = t0; t < t1; ++t) {
     const int n = count(t);
     const int parts = n > part ? (n + part - 1) / part : 0;
     const bool split = parts > 0 && ex + parts <= parts_cap;
     slot_off[t] = split ? ex : -1;
-    local += split ? parts : 1;
+    if (split)
+      local_h += parts;
+    else if (n >= kHeavy)
+      ++local_h;
+    else
+      ++local_l;
     ex += parts;
   }
-  int exd = block_exclusive_scan(local, warp_sums, &tot);
+  int tot_h, tot_l;
+  int exh = block_exclusive_scan(local_h, warp_sums, &tot_h);
+  int exl = tot_h + block_exclusive_scan(local_l, warp_sums, &tot_l);
   ex = ex1;
   for (int t = t0; t < t1; ++t) {
     const int n = count(t);
     const int parts = n > part ? (n + part - 1) / part : 0;
     const bool split = parts > 0 && ex + parts <= parts_cap;
     if (!split) {
-      if (exd < max_items) item_desc[exd] = make_int4(t, 0, n, -1);
-      ++exd;
+      int& at = n >= kHeavy ? exh : exl;
+      if (at < max_items) item_desc[at] = make_int4(t, 0, n, -1);
+      ++at;
     } else {
-      for (int q = 0; q < parts && exd + q < max_items; ++q)
-        item_desc[exd + q] = make_int4(t, q * part, min(n, (q + 1) * part), ex + q);
-      exd += parts;
+      for (int q = 0; q < parts && exh + q < max_items; ++q)
+        item_desc[exh + q] = make_int4(t, q * part, min(n, (q + 1) * part), ex + q);
+      exh += parts;
     }
     ex += parts;
   }
+  tot = tot_h + tot_l;
   if (threadIdx.x == 0) hdr[1] = tot < max_items ? tot : max_items;
 }
 
@@ -358,16 +380,19 @@ __global__ void __launch_bounds__(kCountBlock)
   const int n = t < T ? nnz[t] : 0;
   const int parts = n > kPart ? (n + kPart - 1) / kPart : 0;
   const int items = t < T ? (parts > 0 ? parts : 1) : 0;
+  const int heavy = t < T ? (parts > 0 ? parts : (n >= kHeavy ? 1 : 0)) : 0;
   int tot;
   const int xs = block_exclusive_scan(parts, warp_sums, &tot);
-  const int xi = block_exclusive_scan(items, warp_sums, &tot);
+  const int xh = block_exclusive_scan(heavy, warp_sums, &tot);
+  const int xl = block_exclusive_scan(items - heavy, warp_sums, &tot);
   if (t >= T) return;
-  const int4 off = bpart[blockIdx.x];
+  const int4 off = bpart[blockIdx.x];  // first split part, heavy item, other item
   const int so = parts > 0 ? off.x + xs : -1;
   slot_off[t] = so;
-  const int base = off.y + xi;
+  const int base = off.y + xh;
   if (parts == 0) {
-    if (base < max_items) item_desc[base] = make_int4(t, 0, n, -1);
+    const int at = heavy ? base : off.z + xl;
+    if (at < max_items) item_desc[at] = make_int4(t, 0, n, -1);
   } else {
     for (int q = 0; q < parts && base + q < max_items; ++q)
       item_desc[base + q] = make_int4(t, q * kPart, min(n, (q + 1) * kPart), so + q);
@@ -587,19 +612,50 @@ struct TeamSmem {
 // dealt out to `nwho` warps (this one is `who`): every warp scans every
 // round's counts, so all know each entry's ordinal and the total, and each
 // writes the entries of its own rounds.
+//
+// The data of a round are loaded one round ahead and in one go: the count
+// and, for a round this warp writes, the tile's slots (one 16-byte load when
+// C slots are 16 bytes) with their indices and the spill reference, whether
+// or not the tile has entries.  So a list costs one dependent trip to memory
+// (two for a token with a spilled tile) instead of one per step.
 template <typename Tin>
 TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float* sg, int32_t* sj,
                          int lane, int who, int nwho) {
+  constexpr int E = Elem<Tin>::E;  // slots in 16 bytes
   const int W = a.W;
   const int K = a.F / W;
+  const int C = a.C;
+  const bool vec = C == E;  // a tile's slots are one 16-byte load
+  struct Round {
+    int n, ref;
+    uint4 v;
+    uint2 ix;
+  };
+  auto fetch = [&](int kb) {
+    Round r{0, -1, make_uint4(0, 0, 0, 0), make_uint2(0, 0)};
+    const int k = kb + lane;
+    if (k < K) {
+      const size_t kt = (size_t)k * a.T + t;
+      r.n = a.cnt[kt];
+      if (vec && ((kb >> 5) % nwho) == who) {
+        r.v = __ldg(reinterpret_cast<const uint4*>(a.val + kt * C));
+        if constexpr (E == 8)
+          r.ix = __ldg(reinterpret_cast<const uint2*>(a.idx + kt * C));
+        else
+          r.ix.x = __ldg(reinterpret_cast<const uint32_t*>(a.idx + kt * C));
+        r.ref = a.spill_ref[kt];
+      }
+    }
+    return r;
+  };
   int base = 0;  // ordinal of the first entry of tile kb
-  int n_next = lane < K ? (int)a.cnt[(size_t)lane * a.T + t] : 0;
+  Round nxt = fetch(0);
   for (int kb = 0; kb < K && base < hi; kb += 32) {
     const int k = kb + lane;
-    const int n = n_next;
+    const Round cur = nxt;
+    if (kb + 32 < K) nxt = fetch(kb + 32);
     const bool mine = ((kb >> 5) % nwho) == who;
-    // the next round's count, loaded while this round is expanded
-    n_next = k + 32 < K ? (int)a.cnt[(size_t)(k + 32) * a.T + t] : 0;
+    const int n = cur.n;
     int incl = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -610,8 +666,8 @@ TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float*
     const bool over = mine && n > 0 && tb < hi && tb + n > lo;
     const size_t kt = (size_t)k * a.T + t;
     int ref = -1;
-    if (over && n > a.C) {
-      ref = a.spill_ref[kt];
+    if (over && n > C) {
+      ref = vec ? cur.ref : a.spill_ref[kt];
       if (ref < 0 || ref >= a.spill_cap) {
         // dropped spill entry (capacity, flagged by the producer): only the
         // C slots are known; the other entries of the tile contribute 0
@@ -620,14 +676,37 @@ TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float*
       }
     }
     if (over && ref < 0) {
-      const int m = n <= a.C ? n : a.C;
+      const int m = n <= C ? n : C;
       const int s0 = lo > tb ? lo - tb : 0;
       const int s1 = hi - tb < n ? hi - tb : n;
+      if (vec) {
+        const uint32_t vw[4] = {cur.v.x, cur.v.y, cur.v.z, cur.v.w};
+#pragma unroll
+        for (int sl = 0; sl < E; ++sl) {
+          if (sl >= s0 && sl < s1) {
+            float gv;
+            if constexpr (sizeof(Tin) == 2)
+              gv = __uint_as_float((sl & 1) ? (vw[sl >> 1] & 0xFFFF0000u) : (vw[sl >> 1] << 16));
+            else
+              gv = __uint_as_float(vw[sl]);
+            const uint32_t iw = sl < 4 ? cur.ix.x : cur.ix.y;
+            const int ix = (int)((iw >> (8 * (sl & 3))) & 0xFFu);
+            const int o = tb + sl - lo;
+            sg[o] = sl < m ? gv : 0.f;
+            sj[o] = sl < m ? k * W + ix : k * W;
+          }
+        }
+        for (int sl = s0 > E ? s0 : E; sl < s1; ++sl) {  // past the slots: a dropped spill
+          sg[tb + sl - lo] = 0.f;
+          sj[tb + sl - lo] = k * W;
+        }
+      } else {
 #pragma unroll 4
-      for (int sl = s0; sl < s1; ++sl) {
-        const int o = tb + sl - lo;
-        sg[o] = sl < m ? Elem<Tin>::scalar(a.val[kt * a.C + sl]) : 0.f;
-        sj[o] = sl < m ? k * W + a.idx[kt * a.C + sl] : k * W;
+        for (int sl = s0; sl < s1; ++sl) {
+          const int o = tb + sl - lo;
+          sg[o] = sl < m ? Elem<Tin>::scalar(a.val[kt * C + sl]) : 0.f;
+          sj[o] = sl < m ? k * W + a.idx[kt * C + sl] : k * W;
+        }
       }
     }
     unsigned sp = __ballot_sync(FULL, ref >= 0);
@@ -637,14 +716,19 @@ TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float*
       const int rb = __shfl_sync(FULL, ref, b);
       const int o0 = __shfl_sync(FULL, tb, b);
       const Tin* seg = a.spill_val + (size_t)rb * W;
+      // all parts of the segment first (W <= 256: at most 8 per lane)
+      float v[8];
+#pragma unroll
+      for (int part = 0; part < 8; ++part)
+        v[part] = part < W / 32 ? Elem<Tin>::scalar(seg[part * 32 + lane]) : 0.f;
       int r = 0;
-#pragma unroll 1
-      for (int part = 0; part < W / 32; ++part) {
-        const float v = Elem<Tin>::scalar(seg[part * 32 + lane]);
-        const unsigned m = __ballot_sync(FULL, v != 0.f);
+#pragma unroll
+      for (int part = 0; part < 8; ++part) {
+        if (part >= W / 32) break;
+        const unsigned m = __ballot_sync(FULL, v[part] != 0.f);
         const int o = o0 + r + __popc(m & lanemask_lt());
-        if (v != 0.f && o >= lo && o < hi) {
-          sg[o - lo] = v;
+        if (v[part] != 0.f && o >= lo && o < hi) {
+          sg[o - lo] = v[part];
           sj[o - lo] = (kb + b) * W + part * 32 + lane;
         }
         r += __popc(m);
