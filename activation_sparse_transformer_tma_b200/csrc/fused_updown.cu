@@ -561,6 +561,7 @@ struct GatherArgs {
   const int32_t* spill_ref;
   const Tin* spill_val;
   int W, C, spill_cap;  // tile width, capacity, spill entries
+  int staged;           // TwELL data and token rows are prefetched (see StageSmem)
   // hybrid entry source
   const Tin* ell_g;
   Tin* ell_u;
@@ -582,6 +583,43 @@ struct GatherArgs {
   void* out;
   int32_t* status;
   FusedWs ws;
+};
+
+// Asynchronous copies from global into shared memory; each thread waits for
+// its own copies (cp_async_wait_all) before it reads them.
+TW_DEV void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+TW_DEV void cp_async8(void* smem, const void* gmem) {
+  const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(gmem) : "memory");
+}
+TW_DEV void cp_async4(void* smem, const void* gmem) {
+  const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(gmem) : "memory");
+}
+TW_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+TW_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The next item's TwELL data and token row, copied into shared memory while
+// the current item runs (TwELL mode, when a tile's C slots are 16 bytes, the
+// token has at most kStageTiles tiles and the count array can be read in
+// aligned 4-byte words).  Lane l of a warp copies, for tile k = 32 r + l of
+// every round r, the count word into the warp's own cnt row, and for the
+// rounds the warp writes (see collect_twell) the slots, indices and spill
+// reference; and its own slices of the token row.  So every thread later
+// reads only what it copied itself.
+constexpr int kStageTiles = 64;
+template <int NCHW>
+struct StageSmem {
+  uint32_t cnt[kTeam][kStageTiles];
+  uint4 val[kStageTiles];
+  uint2 idx[kStageTiles];
+  int32_t ref[kStageTiles];
+  uint4 x[kTeam][NCHW][32];
 };
 
 // One window's entry list.
@@ -618,9 +656,12 @@ struct TeamSmem {
 // C slots are 16 bytes) with their indices and the spill reference, whether
 // or not the tile has entries.  So a list costs one dependent trip to memory
 // (two for a token with a spilled tile) instead of one per step.
-template <typename Tin>
+//
+// With `st` (see StageSmem) the round data come from this warp's copies in
+// shared memory instead.
+template <typename Tin, int NCHW = 1>
 TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float* sg, int32_t* sj,
-                         int lane, int who, int nwho) {
+                         int lane, int who, int nwho, const StageSmem<NCHW>* st = nullptr) {
   constexpr int E = Elem<Tin>::E;  // slots in 16 bytes
   const int W = a.W;
   const int K = a.F / W;
@@ -634,7 +675,15 @@ TW_DEV int collect_twell(const GatherArgs<Tin>& a, int t, int lo, int hi, float*
   auto fetch = [&](int kb) {
     Round r{0, -1, make_uint4(0, 0, 0, 0), make_uint2(0, 0)};
     const int k = kb + lane;
-    if (k < K) {
+    if (k < K && st) {
+      const size_t kt = (size_t)k * a.T + t;
+      r.n = (int)((st->cnt[who][k] >> (8 * (unsigned)(kt & 3))) & 0xFFu);
+      if (((kb >> 5) % nwho) == who) {
+        r.v = st->val[k];
+        r.ix = st->idx[k];
+        r.ref = st->ref[k];
+      }
+    } else if (k < K) {
       const size_t kt = (size_t)k * a.T + t;
       r.n = a.cnt[kt];
       if (vec && ((kb >> 5) % nwho) == who) {
@@ -816,6 +865,13 @@ TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, Entry
 template <int NCHW, int MODE>
 constexpr int teams_for() { return NCHW < 4 ? kTeams : (MODE == kModeHybBwd ? 4 : 6); }
 
+// Dynamic shared memory of a gather launch: StageSmem per team (TwELL mode
+// with staging).
+template <int NCHW, int MODE>
+constexpr size_t gather_smem_bytes() {
+  return MODE == kModeTwell ? sizeof(StageSmem<NCHW>) * teams_for<NCHW, MODE>() : 0;
+}
+
 // kFull: d is exactly the kTeam warps' slices (see load_rows2).
 template <typename Tin, int NCHW, bool kOutBf16, int MODE, bool kFull>
 __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
@@ -853,6 +909,42 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
   if (leader && lane == 0) ticket = atomicAdd(&a.ws.hdr[0], 1);
   publish(0);
   team_bar(team);
+
+  // TwELL mode: the next item's data are copied into shared memory while the
+  // current item's updates run (see StageSmem); this is the first item's.
+  // Dynamic shared memory: the teams' StageSmem (TwELL mode); see
+  // gather_smem_bytes.
+  extern __shared__ __align__(16) unsigned char stage_smem[];
+  StageSmem<NCHW>& sg = reinterpret_cast<StageSmem<NCHW>*>(stage_smem)[team];
+  const bool staged = MODE == kModeTwell && a.staged != 0;
+  auto stage = [&](int tn) {
+    const int K = a.F / a.W;
+    for (int kb = 0; kb < K; kb += 32) {
+      const int k = kb + lane;
+      if (k < K) {
+        const size_t kt = (size_t)k * a.T + tn;
+        cp_async4(&sg.cnt[tw][k], a.cnt + (kt & ~size_t(3)));
+        if (((kb >> 5) % kTeam) == tw) {
+          cp_async16(&sg.val[k], a.val + kt * a.C, true);
+          if constexpr (E == 8)
+            cp_async8(&sg.idx[k], a.idx + kt * a.C);
+          else
+            cp_async4(&sg.idx[k].x, a.idx + kt * a.C);
+          cp_async4(&sg.ref[k], a.spill_ref + kt);
+        }
+      }
+    }
+    const Tin* xn = a.xin + (size_t)tn * d;
+#pragma unroll
+    for (int c = 0; c < NCHW; ++c) {
+      const int col = c0 + c * SPAN + lane * E;
+      const bool ok = kFull || col < d;
+      cp_async16(&sg.x[tw][c][lane], ok ? xn + col : xn, ok);
+    }
+    cp_async_commit();
+  };
+  if (staged && ts.desc[0].x >= 0) stage(ts.desc[0].x);
+
   uint32_t win = 0;  // windows processed by the team: the list parity
   for (uint32_t it = 0;; ++it) {
     const int4 desc = ts.desc[it & 1];
@@ -860,15 +952,26 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
     const int t = desc.x, lo = desc.y, hi = desc.z, prow = desc.w;
     const bool to_backup = MODE == kModeHybFwd && a.row_slot[t] >= 0;
     bool published = false;
+    // after the item's last partials barrier: the next item's staged copies
+    auto stage_next = [&]() {
+      if (staged) {
+        const int4 nd = ts.desc[(it + 1) & 1];
+        if (nd.x >= 0) stage(nd.x);
+      }
+    };
 
     uint4 xr[NCHW];  // the token's row slices, kept in the input format
     float2 acc[NCHW][P];
     const Tin* xt = a.xin + (size_t)t * d;
+    if (staged) cp_async_wait_all();
 #pragma unroll
     for (int c = 0; c < NCHW; ++c) {
       const int col = c0 + c * SPAN + lane * E;
-      xr[c] = kFull || col < d ? __ldcs(reinterpret_cast<const uint4*>(xt + col))
-                               : make_uint4(0, 0, 0, 0);
+      if (staged)
+        xr[c] = sg.x[tw][c][lane];
+      else
+        xr[c] = kFull || col < d ? __ldcs(reinterpret_cast<const uint4*>(xt + col))
+                                 : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int q = 0; q < P; ++q) acc[c][q] = make_float2(0.f, 0.f);
     }
@@ -878,7 +981,8 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
       const int w1 = min(hi, w0 + kListCap);
       int n;
       if constexpr (MODE == kModeTwell) {
-        n = collect_twell(a, t, w0, w1, ls.g, ls.j, lane, tw, kTeam);
+        n = collect_twell<Tin, NCHW>(a, t, w0, w1, ls.g, ls.j, lane, tw, kTeam,
+                                     staged ? &sg : nullptr);
         team_bar(team);  // the list is written
       } else {
         if (leader) {
@@ -986,6 +1090,7 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
           continue;
         }
         team_bar(team);  // the partials (and the next descriptor) are written
+        if (w1 == hi) stage_next();
         // h of the pair's entries: u from the team's partials (added in warp
         // order), times g; 0 for a missing second entry
         static_assert(kTeam == 2, "a pair's partials are read as one float4");
@@ -1011,6 +1116,7 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
     if (!published) {  // an item without entries
       publish((it + 1) & 1);
       team_bar(team);
+      stage_next();
     }
 
     // ------------------------------------------------------------ output --
@@ -1110,11 +1216,17 @@ cudaError_t launch_nchw(GatherArgs<Tin> a, bool out_bf16, cudaStream_t stream) {
                    : (out_bf16 ? gather_kernel<Tin, NCHW, true, MODE, false>
                                : gather_kernel<Tin, NCHW, false, MODE, false>);
   constexpr int threads = 32 * kTeam * teams_for<NCHW, MODE>();
+  const size_t dyn = a.staged ? gather_smem_bytes<NCHW, MODE>() : 0;
+  cudaError_t e = cudaSuccess;
+  if (dyn > 0) {
+    e = set_smem_limit(reinterpret_cast<const void*>(kern), (int)dyn);
+    if (e != cudaSuccess) return e;
+  }
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, dyn);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  kern<<<num_sms() * per_sm, threads, 0, stream>>>(a);
+  kern<<<num_sms() * per_sm, threads, dyn, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -1288,6 +1400,10 @@ cudaError_t twell_fused_t(const void* x, const tw_twell& g, const void* Wu_t, co
   a.status = status;
   a.ws = w;
   const int T = g.T, K = g.F / g.W;
+  // prefetching the next item's TwELL data needs 16-byte slot rows, at most
+  // kStageTiles tiles and count words that stay inside the count array
+  a.staged = g.C == Elem<Tin>::E && K <= kStageTiles && T % 4 == 0 &&
+             reinterpret_cast<uintptr_t>(g.cnt) % 4 == 0;
   // A handful of tokens: one CTA per token, no plan.  Above that the planned
   // path wins, because it splits the heavy tokens of the batch over teams
   // (at T = 64 of the 2B workload: 50 us planned, 282 us one CTA per token).
