@@ -8,7 +8,7 @@
 // (d x F bf16, 33.5 MB at d = 2048, F = 8192) plus a few dozen gathered
 // weight rows per token; the separate launches of the gate and the fused
 // kernels (and their set-up) cost more than the data movement itself.  Here
-// one grid, one CTA of 16 warps per SM, runs three phases separated by grid
+// one grid, one CTA of 16 warps per SM, runs its phases separated by grid
 // barriers:
 //
 //   A  gate: work items of 16 units x 256 columns of d, spread over every
@@ -19,6 +19,8 @@
 //      tile per MMA.  x is staged in shared memory for up to 16 tokens and
 //      read through L1 for more.  The reduction over d is split into slices:
 //      each item writes fp32 partial sums zpart[slice][t][u].
+//
+// Up to 32 tokens:
 //   B  packing and dot products: each (tile k, token t) gets one or more
 //      warps.  Every one of them adds the slices in a fixed order, applies
 //      ReLU and rounds g to bf16; the first packs the tile's TwELL slots
@@ -30,7 +32,23 @@
 //   C  updates: one CTA per (token, 256-column slice of d); warp w takes the
 //      tiles k = w (mod 16) in ascending order, accumulates h Wd[j] over its
 //      columns in fp32, and the CTA adds the warps' partial rows in warp
-//      order.  y is therefore deterministic.
+//      order.
+//
+// 33 to 64 tokens, where a heavy token's tiles would hold single warps up
+// for long:
+//   B  packing only, one warp per (tile, token), as above; every non-zero's
+//      unit j and g go to its place in the tile's row of a per-token list.
+//   C  dot products: every CTA builds the same per-token prefix sums of the
+//      tile counts; the grid's warps then take the entry pairs of all tokens
+//      in turn, form u = x_t . Wu_t[j] over the whole row and store h = g u.
+//   D  updates: tasks (token, chunk of up to kChunk entries, 256-column
+//      slice), one warp each, which accumulates h Wd[j] over the chunk's
+//      entries in order, 8 columns per lane in fp32.  A token with one chunk
+//      writes y; the chunks of a longer token write partial rows.
+//   E  (only when some token was split) each split token's y is the sum of
+//      its chunks' partial rows in chunk order.
+//
+// y is deterministic in both.
 //
 #include "tw_common.cuh"
 #include "tw_internal.h"
@@ -44,8 +62,9 @@ constexpr int kThreadsD = 32 * kWarpsD;
 constexpr int kW = 128;          // TwELL tile width of this path
 constexpr int kSlice = 256;      // columns of d per gate work item
 constexpr int kSteps = kSlice / 32;
-constexpr int kMaxTokD = 64;
 constexpr int kStageTok = 16;  // x is staged in shared memory up to this many tokens
+constexpr int kChunk = 32;       // entries per phase-D task (one warp) of a token
+constexpr int kChunkRows = 512;  // partial rows in the workspace
 
 struct DecodeArgs {
   const uint16_t* x;
@@ -70,7 +89,8 @@ struct DecodeArgs {
   int32_t* bar;    // [0] arrivals, [1] departures
   float* zpart;    // [S][T][F]
   int32_t* jtile;  // [T][F]: units of the non-zeros of tile k at [k * W, k * W + cnt)
-  float* htile;    // [T][F]: their h = g u
+  float* htile;    // [T][F]: their g (phase B), then h = g u (phase C)
+  float* prow;     // [kChunkRows][d]: partial rows of the chunks of split tokens
   int32_t* status;
   unsigned long long timeout_ns;
 };
@@ -124,7 +144,10 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   extern __shared__ __align__(16) uint8_t smem[];
   const int T = a.T, d = a.d, F = a.F, K = F / kW;
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [8 * NT][d] bf16 if kStage, rows >= T zero
+  // after x: the warps' partial rows of phase C (up to 32 tokens), or the
+  // plan tables of phases C and D (more)
   float* red = reinterpret_cast<float*>(smem + (kStage ? (size_t)8 * NT * d * 2 : 0));  // [16][256]
+  int* tbl = reinterpret_cast<int*>(red);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = gridDim.x * kWarpsD;
   const int gw = blockIdx.x * kWarpsD + warp;
@@ -142,6 +165,19 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
     if (t >= T || col >= d) return make_uint4(0, 0, 0, 0);
     return kStage ? *reinterpret_cast<const uint4*>(xs + (size_t)t * d + col)
                   : __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * d + col));
+  };
+  // 8 values of y for token t at column col, in y's dtype
+  auto store_y = [&](int t, int col, const float (&v)[8]) {
+    if (a.y_bf16) {
+      uint16_t* yt = static_cast<uint16_t*>(a.y) + (size_t)t * d + col;
+      *reinterpret_cast<uint4*>(yt) =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]));
+    } else {
+      float4* yt = reinterpret_cast<float4*>(static_cast<float*>(a.y) + (size_t)t * d + col);
+      yt[0] = make_float4(v[0], v[1], v[2], v[3]);
+      yt[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
   };
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.spill_n = 0;  // before any spill (phase B)
   __syncthreads();
@@ -202,6 +238,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   }
   grid_barrier(a, 1);
 
+  if constexpr (NT < 8) {
+    // up to 32 tokens: packing with the dot products, then updates (B, C)
   // -------------------------------------- B: TwELL pack, h = g (x_t . Wu_t[j]) --
   {
     const unsigned lt = (1u << lane) - 1u;
@@ -325,7 +363,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       __syncwarp();  // the list is rewritten by the warp's next item
     }
   }
-  grid_barrier(a, 2);
+    grid_barrier(a, 2);
 
   // --------------------------------------------------- C: y_t = sum h Wd[j] --
   {
@@ -403,6 +441,320 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
     }
   }
 
+  } else {
+    // 33 to 64 tokens: packing, then dot products and updates spread evenly
+    // over the grid (B to E)
+  // ------------------------------- B: TwELL pack, and (unit, g) per entry --
+  {
+    const unsigned lt = (1u << lane) - 1u;
+    const int n_it = K * T;
+    for (int item = gw; item < n_it; item += nwarps) {
+      const int k = item / T, t = item % T;
+      uint16_t gv[4];
+      unsigned bal[4];
+      int n = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int u = k * kW + lane + 32 * i;
+        float z = 0.f;
+        for (int s2 = 0; s2 < a.S; ++s2) z += a.zpart[((size_t)s2 * T + t) * F + u];
+        const float zr = (int32_t)__float_as_uint(z) > 0 ? z : 0.0f;  // ReLU, -0 -> +0
+        gv[i] = f32_to_bf16(zr);
+        bal[i] = __ballot_sync(FULL, gv[i] != 0);
+        n += __popc(bal[i]);
+      }
+      const size_t off = (size_t)k * T + t;
+      const int C = a.C;
+      {  // the tile's TwELL slots, count, padding and spill
+        int before = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pos = before + __popc(bal[i] & lt);
+          if (gv[i] != 0 && pos < C) {
+            a.val[off * C + pos] = gv[i];
+            a.idx[off * C + pos] = (uint8_t)(lane + 32 * i);
+          }
+          before += __popc(bal[i]);
+          if (a.dump) a.dump[(size_t)t * F + k * kW + lane + 32 * i] = gv[i];
+        }
+        for (int sl = lane; sl < C; sl += 32) {
+          if (sl >= n) {
+            a.val[off * C + sl] = 0;
+            a.idx[off * C + sl] = 0;
+          }
+        }
+        if (lane == 0) a.cnt[off] = (uint8_t)n;
+        if (n > C) {  // uniform across the warp
+          int slot = 0;
+          if (lane == 0) slot = atomicAdd(a.spill_n, 1);
+          slot = __shfl_sync(FULL, slot, 0);
+          if (slot < a.spill_cap) {
+            if (lane == 0) {
+              a.spill_ref[off] = slot;
+              a.spill_tk[2 * (size_t)slot] = t;
+              a.spill_tk[2 * (size_t)slot + 1] = k;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a.spill_val[(size_t)slot * kW + lane + 32 * i] = gv[i];
+          } else if (lane == 0) {
+            a.spill_ref[off] = -1;
+            set_status(a.status, kStatusSpill);
+          }
+        }
+      }
+      // the tile's non-zeros, ascending: unit and g at [t][k * W + pos]
+      {
+        int before = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int pos = before + __popc(bal[i] & lt);
+          if (gv[i] != 0) {
+            const size_t e = (size_t)t * F + k * kW + pos;
+            a.jtile[e] = k * kW + lane + 32 * i;
+            a.htile[e] = bf16_to_f32(gv[i]);
+          }
+          before += __popc(bal[i]);
+        }
+      }
+    }
+  }
+  grid_barrier(a, 2);
+
+  // ----------------------------------------------- per-CTA plan of C and D --
+  // pre[t][k]: entries of token t in tiles before k (so E_t = pre[t][K]);
+  // every CTA builds the same tables from the counts.  Phase C takes entry
+  // pairs of each token, phase D tasks (token, chunk of kChunk entries,
+  // 256-column slice); a token with more than kChunk entries is split into
+  // chunks with partial rows (in token order while the rows last; a token
+  // past them keeps one task per slice).
+  int* pre = tbl;  // [T][K + 1]
+  int* tab = pre + (size_t)T * (K + 1);  // pair_off[T + 1], nch[T], row_off[T], task_off[T + 1]
+  int* pair_off = tab;
+  int* nch = pair_off + (T + 1);
+  int* row_off = nch + T;
+  int* task_off = row_off + T;
+  __shared__ int any_split;
+  const int nsl = (d + kSlice - 1) / kSlice;
+  // the counts [K][T] into pre[t][k + 1] with one pass of all threads, then
+  // each token's running sum over its tiles in place
+  for (int i = threadIdx.x; i < K * T; i += kThreadsD) {
+    const int k = i / T, t = i % T;
+    pre[(size_t)t * (K + 1) + k + 1] = a.cnt[i];
+  }
+  __syncthreads();
+  for (int t = warp; t < T; t += kWarpsD) {
+    int base = 0;
+    if (lane == 0) pre[(size_t)t * (K + 1)] = 0;
+    for (int kb = 0; kb < K; kb += 32) {
+      const int k = kb + lane;
+      const int n = k < K ? pre[(size_t)t * (K + 1) + k + 1] : 0;
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (k < K) pre[(size_t)t * (K + 1) + k + 1] = base + incl;
+      base += __shfl_sync(FULL, incl, 31);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int po = 0, ro = 0, to = 0, split = 0;
+    for (int t = 0; t < T; ++t) {
+      const int E = pre[(size_t)t * (K + 1) + K];
+      pair_off[t] = po;
+      po += (E + 1) / 2;
+      int c = (E + kChunk - 1) / kChunk;
+      if (c > 1 && ro + c <= kChunkRows) {
+        row_off[t] = ro;
+        ro += c;
+        split = 1;
+      } else {
+        c = 1;
+        row_off[t] = -1;
+      }
+      nch[t] = c;
+      task_off[t] = to;
+      to += c * nsl;
+    }
+    pair_off[T] = po;
+    task_off[T] = to;
+    any_split = split;
+  }
+  __syncthreads();
+  // entry e of token t: its tile k and place (largest k with pre[t][k] <= e)
+  auto locate = [&](int t, int e, int& k, int& pos) {
+    const int* pt = pre + (size_t)t * (K + 1);
+    int lo = 0, hi = K;  // pt[lo] <= e < pt[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pt[mid] <= e)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    k = lo;
+    pos = e - pt[lo];
+  };
+  // the token whose range [off[t], off[t + 1]) holds q (off[0] <= q < off[T])
+  auto owner = [&](const int* off, int q) {
+    int lo = 0, hi = T;  // off[lo] <= q < off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= q)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    return lo;
+  };
+
+  // ---------------------------------- C: h = g (x_t . Wu_t[j]) per entry --
+  {
+    const int P = pair_off[T];
+    for (int q = gw; q < P; q += nwarps) {
+      const int t = owner(pair_off, q);
+      const int E = pre[(size_t)t * (K + 1) + K];
+      const int e0 = 2 * (q - pair_off[t]);
+      const bool two = e0 + 1 < E;
+      int k0, p0, k1, p1;
+      locate(t, e0, k0, p0);
+      if (two) {
+        locate(t, e0 + 1, k1, p1);
+      } else {
+        k1 = k0;
+        p1 = p0;
+      }
+      const size_t i0 = (size_t)t * F + k0 * kW + p0, i1 = (size_t)t * F + k1 * kW + p1;
+      const int j0 = a.jtile[i0], j1 = a.jtile[i1];
+      const uint16_t* w0 = a.Wu + (size_t)j0 * d;
+      const uint16_t* w1 = a.Wu + (size_t)j1 * d;
+      float pp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
+      for (int c = lane * 8; c < d; c += 256) {
+        const uint4 xv = xrow(t, c);
+        const uint4 wa = __ldg(reinterpret_cast<const uint4*>(w0 + c));
+        const uint4 wb = __ldg(reinterpret_cast<const uint4*>(w1 + c));
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        const uint32_t aw[4] = {wa.x, wa.y, wa.z, wa.w};
+        const uint32_t bw[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          pp[0][r] = fmaf(bf16_lo(xw[r]), bf16_lo(aw[r]), pp[0][r]);
+          pp[0][r] = fmaf(bf16_hi(xw[r]), bf16_hi(aw[r]), pp[0][r]);
+          pp[1][r] = fmaf(bf16_lo(xw[r]), bf16_lo(bw[r]), pp[1][r]);
+          pp[1][r] = fmaf(bf16_hi(xw[r]), bf16_hi(bw[r]), pp[1][r]);
+        }
+      }
+      const float u0 = warp_sum((pp[0][0] + pp[0][1]) + (pp[0][2] + pp[0][3]));
+      const float u1 = warp_sum((pp[1][0] + pp[1][1]) + (pp[1][2] + pp[1][3]));
+      if (lane == 0) {
+        a.htile[i0] = a.htile[i0] * u0;  // g -> h = g u
+        if (two) a.htile[i1] = a.htile[i1] * u1;
+      }
+    }
+  }
+  grid_barrier(a, 3);
+
+  // --------------------- D: y_t (or a chunk's partial row) = sum h Wd[j] --
+  {
+    const int n_tasks = task_off[T];
+    for (int task = gw; task < n_tasks; task += nwarps) {
+      const int t = owner(task_off, task);
+      const int r = task - task_off[t];
+      const int c = r / nsl, sl = r % nsl;
+      const int E = pre[(size_t)t * (K + 1) + K];
+      const int lo = nch[t] > 1 ? c * kChunk : 0;
+      const int hi = nch[t] > 1 ? min(E, lo + kChunk) : E;
+      const int col = sl * kSlice + lane * 8;
+      const bool in = col < d;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      int k = 0, pos = 0;
+      if (lo < hi) locate(t, lo, k, pos);
+      constexpr int kB = 8;  // entries whose rows are loaded together
+      for (int e = lo; e < hi; e += kB) {
+        int jj[kB];
+        float hh[kB];
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+          // walk to entry e + b: the next non-empty tile when this one is used up
+          if (e + b < hi) {
+            while (pos >= pre[(size_t)t * (K + 1) + k + 1] - pre[(size_t)t * (K + 1) + k]) {
+              ++k;
+              pos = 0;
+            }
+            const size_t ix = (size_t)t * F + k * kW + pos;
+            jj[b] = a.jtile[ix];
+            hh[b] = a.htile[ix];
+            ++pos;
+          } else {
+            jj[b] = 0;
+            hh[b] = 0.f;
+          }
+        }
+        uint4 wv[kB];
+#pragma unroll
+        for (int b = 0; b < kB; ++b)
+          wv[b] = in && e + b < hi
+                      ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
+                      : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+          const float hb = hh[b];
+          acc[0] = fmaf(hb, bf16_lo(wv[b].x), acc[0]);
+          acc[1] = fmaf(hb, bf16_hi(wv[b].x), acc[1]);
+          acc[2] = fmaf(hb, bf16_lo(wv[b].y), acc[2]);
+          acc[3] = fmaf(hb, bf16_hi(wv[b].y), acc[3]);
+          acc[4] = fmaf(hb, bf16_lo(wv[b].z), acc[4]);
+          acc[5] = fmaf(hb, bf16_hi(wv[b].z), acc[5]);
+          acc[6] = fmaf(hb, bf16_lo(wv[b].w), acc[6]);
+          acc[7] = fmaf(hb, bf16_hi(wv[b].w), acc[7]);
+        }
+      }
+      if (in) {
+        if (nch[t] > 1) {
+          float4* pr = reinterpret_cast<float4*>(a.prow + (size_t)(row_off[t] + c) * d + col);
+          pr[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+          pr[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        } else {
+          store_y(t, col, acc);
+        }
+      }
+    }
+  }
+
+  // ------------------- E: the chunks of split tokens, added in chunk order --
+  if (any_split) {  // the same in every CTA
+    grid_barrier(a, 4);
+    for (int task = gw; task < T * nsl; task += nwarps) {
+      const int t = task / nsl, sl = task % nsl;
+      const int col = sl * kSlice + lane * 8;
+      if (nch[t] <= 1 || col >= d) continue;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      for (int c = 0; c < nch[t]; ++c) {
+        const float4* pr =
+            reinterpret_cast<const float4*>(a.prow + (size_t)(row_off[t] + c) * d + col);
+        const float4 p0 = __ldcg(pr), p1 = __ldcg(pr + 1);
+        v[0] += p0.x;
+        v[1] += p0.y;
+        v[2] += p0.z;
+        v[3] += p0.w;
+        v[4] += p1.x;
+        v[5] += p1.y;
+        v[6] += p1.z;
+        v[7] += p1.w;
+      }
+      store_y(t, col, v);
+    }
+  }
+
+  }
+
   // leave the barrier counters at zero for the next call: the last CTA to
   // depart (all CTAs have passed every barrier) resets them
   __syncthreads();
@@ -427,6 +779,7 @@ size_t decode_layout(void* base, int T, int d, int F, DecodeArgs* a) {
   const size_t o_z = take(sizeof(float) * (size_t)S * T * F);
   const size_t o_jt = take(sizeof(int32_t) * (size_t)T * F);
   const size_t o_ht = take(sizeof(float) * (size_t)T * F);
+  const size_t o_pr = take(sizeof(float) * (size_t)kChunkRows * d);
   if (base && a) {
     char* p = static_cast<char*>(base);
     a->S = S;
@@ -434,6 +787,7 @@ size_t decode_layout(void* base, int T, int d, int F, DecodeArgs* a) {
     a->zpart = reinterpret_cast<float*>(p + o_z);
     a->jtile = reinterpret_cast<int32_t*>(p + o_jt);
     a->htile = reinterpret_cast<float*>(p + o_ht);
+    a->prow = reinterpret_cast<float*>(p + o_pr);
   }
   return off;
 }
@@ -470,7 +824,10 @@ cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t
   a.timeout_ns = kWaitTimeoutNs;
   const int NT = T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : 8;
   const size_t xs_bytes = 8 * NT <= kStageTok ? (size_t)8 * NT * d * 2 : 0;
-  const size_t smem = xs_bytes + sizeof(float) * kWarpsD * kSlice;
+  const int K = F / kW;
+  const size_t smem =
+      xs_bytes + (NT < 8 ? sizeof(float) * kWarpsD * kSlice
+                         : sizeof(int) * ((size_t)T * (K + 1) + 4 * (size_t)T + 2));
   const void* kern = NT == 1 ? reinterpret_cast<const void*>(decode_step_kernel<1>)
                      : NT == 2 ? reinterpret_cast<const void*>(decode_step_kernel<2>)
                      : NT == 4 ? reinterpret_cast<const void*>(decode_step_kernel<4>)

@@ -314,7 +314,8 @@ def test_decode_sizes(T):
 
 
 # One cooperative launch for the whole small-batch FFN: gate partial sums on
-# mma.sync over every SM, TwELL packing, dot products, updates.  T crosses the
+# mma.sync over every SM, TwELL packing, dot products, updates (per chunk of
+# a token's entries, with partial rows for the long tokens).  T crosses the
 # 8-token MMA column tiles and the 16-token limit of x staged in shared
 # memory; d and F are ragged against the 256-column slices.
 SMALL_STEP = [
@@ -329,6 +330,9 @@ SMALL_STEP = [
     (17, 320, 640, 8, "dead20", 60.0),   # x read through L1 from here on
     (33, 2048, 2048, 8, "zipf", 29.0),
     (64, 512, 1280, 16, "zipf", 200.0),  # heavy tokens: many entries per tile
+    # about 6 chunks of 128 entries per token: the chunk rows of the workspace
+    # run out, and the tokens past them are added up unsplit
+    (48, 256, 2048, 8, "dead20", 700.0),
 ]
 
 
