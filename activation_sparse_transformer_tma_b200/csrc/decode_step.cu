@@ -16,9 +16,10 @@
 //      32-column steps in flight; four for more than 16 tokens) and
 //      multiplies them with the tokens' x on the tensor pipe: mma.sync
 //      m16n8k16 with the units on M and the tokens on N, one 8-token column
-//      tile per MMA.  x is staged in shared memory for up to 16 tokens and
-//      read through L1 for more.  The reduction over d is split into slices:
-//      each item writes fp32 partial sums zpart[slice][t][u].
+//      tile per MMA.  x is staged in shared memory for up to 16 tokens; for
+//      more, each CTA serves one 256-column slice of d and stages that slice
+//      of every token.  The reduction over d is split into slices: each item
+//      writes fp32 partial sums zpart[slice][t][u].
 //
 // Up to 32 tokens:
 //   B  packing and dot products: each (tile k, token t) gets one or more
@@ -63,6 +64,11 @@ constexpr int kW = 128;          // TwELL tile width of this path
 constexpr int kSlice = 256;      // columns of d per gate work item
 constexpr int kSteps = kSlice / 32;
 constexpr int kStageTok = 16;  // x is staged in shared memory up to this many tokens
+// Above that a CTA of phase A serves one 256-column slice of d and stages
+// just that slice of every token, at a row stride of kSliceRow 16-byte
+// chunks (32 used): the 64-byte pad puts the two token rows read by one
+// quarter-warp on disjoint banks.
+constexpr int kSliceRow = 36;
 constexpr int kChunk = 32;       // entries per phase-D task (one warp) of a token
 constexpr int kChunkRows = 512;  // partial rows in the workspace
 
@@ -144,9 +150,12 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   extern __shared__ __align__(16) uint8_t smem[];
   const int T = a.T, d = a.d, F = a.F, K = F / kW;
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [8 * NT][d] bf16 if kStage, rows >= T zero
+  // x slice of phase A when x is not staged whole: [8 * NT][kSliceRow]
+  uint4* xsl = reinterpret_cast<uint4*>(smem);
+  const size_t x_bytes = kStage ? (size_t)8 * NT * d * 2 : (size_t)8 * NT * kSliceRow * 16;
   // after x: the warps' partial rows of phase C (up to 32 tokens), or the
   // plan tables of phases C and D (more)
-  float* red = reinterpret_cast<float*>(smem + (kStage ? (size_t)8 * NT * d * 2 : 0));  // [16][256]
+  float* red = reinterpret_cast<float*>(smem + x_bytes);  // [16][256]
   int* tbl = reinterpret_cast<int*>(red);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = gridDim.x * kWarpsD;
@@ -185,9 +194,27 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   // ------------------------------------------------ A: gate partial sums --
   {
     const int g = lane >> 2, q = lane & 3;
-    const int n_items = (F / 16) * a.S;
-    for (int item = gw; item < n_items; item += nwarps) {
-      const int grp = item / a.S, s = item % a.S;
+    const int S = a.S;
+    // With x read through L1 (more than 16 tokens) a CTA serves one slice of
+    // d, staged in shared memory, and its warps take that slice's unit groups.
+    const int s_cta = blockIdx.x % S;
+    const int ncs = ((int)gridDim.x - s_cta + S - 1) / S;  // CTAs serving slice s_cta
+    if (!kStage) {
+      const int cs = s_cta * kSlice;
+      for (int i = threadIdx.x; i < 8 * NT * 32; i += kThreadsD) {
+        const int t = i >> 5, col = cs + (i & 31) * 8;
+        xsl[t * kSliceRow + (i & 31)] =
+            t < T && col < d ? __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * d + col))
+                             : make_uint4(0, 0, 0, 0);
+      }
+      __syncthreads();
+    }
+    const int n_items = kStage ? (F / 16) * S : F / 16;
+    const int first = kStage ? gw : (blockIdx.x / S) * kWarpsD + warp;
+    const int stride = kStage ? nwarps : ncs * kWarpsD;
+    for (int item = first; item < n_items; item += stride) {
+      const int grp = kStage ? item / S : item;
+      const int s = kStage ? item % S : s_cta;
       const int u0 = grp * 16, c0 = s * kSlice;
       const uint16_t* r_lo = a.Wg + (size_t)(u0 + g) * d;
       const uint16_t* r_hi = a.Wg + (size_t)(u0 + g + 8) * d;
@@ -214,7 +241,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
           // so the products pair Wg[u][col] with x[t][col].
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            const uint4 xb = xrow(8 * n + g, col);
+            const uint4 xb = kStage ? xrow(8 * n + g, col)
+                                    : xsl[(8 * n + g) * kSliceRow + (i0 + i) * 4 + q];
             mma16816(D[n], alo[i].x, ahi[i].x, alo[i].y, ahi[i].y, xb.x, xb.y);
             mma16816(D[n], alo[i].z, ahi[i].z, alo[i].w, ahi[i].w, xb.z, xb.w);
           }
@@ -823,7 +851,8 @@ cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t
   a.status = status;
   a.timeout_ns = kWaitTimeoutNs;
   const int NT = T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : 8;
-  const size_t xs_bytes = 8 * NT <= kStageTok ? (size_t)8 * NT * d * 2 : 0;
+  const size_t xs_bytes =
+      8 * NT <= kStageTok ? (size_t)8 * NT * d * 2 : (size_t)8 * NT * kSliceRow * 16;
   const int K = F / kW;
   const size_t smem =
       xs_bytes + (NT < 8 ? sizeof(float) * kWarpsD * kSlice
