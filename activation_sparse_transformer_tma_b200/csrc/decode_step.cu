@@ -587,28 +587,49 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int po = 0, ro = 0, to = 0, split = 0;
-    for (int t = 0; t < T; ++t) {
-      const int E = pre[(size_t)t * (K + 1) + K];
-      pair_off[t] = po;
-      po += (E + 1) / 2;
-      int c = (E + kChunk - 1) / kChunk;
-      if (c > 1 && ro + c <= kChunkRows) {
-        row_off[t] = ro;
-        ro += c;
-        split = 1;
-      } else {
-        c = 1;
-        row_off[t] = -1;
+  // warp 0, 32 tokens per round: running offsets of the pairs, the chunk
+  // rows (a token asks for its chunks' rows in token order; it is split if
+  // they fit, and once the rows asked for pass the capacity no later token
+  // is) and the tasks
+  if (warp == 0) {
+    int po = 0, ro = 0, to = 0;
+    bool split_any = false;
+    auto incl_scan = [&](int v) {
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, v, o);
+        if (lane >= o) v += u;
       }
-      nch[t] = c;
-      task_off[t] = to;
-      to += c * nsl;
+      return v;
+    };
+    for (int t0 = 0; t0 < T; t0 += 32) {
+      const int t = t0 + lane;
+      const int E = t < T ? pre[(size_t)t * (K + 1) + K] : 0;
+      const int pairs = (E + 1) / 2;
+      const int c_all = (E + kChunk - 1) / kChunk;
+      const int want = c_all > 1 ? c_all : 0;
+      const int ip = incl_scan(pairs), iw = incl_scan(want);
+      const int xw = ro + iw - want;
+      const bool split = c_all > 1 && xw + c_all <= kChunkRows;
+      const int c = split ? c_all : 1;
+      const int tasks = t < T ? c * nsl : 0;
+      const int itk = incl_scan(tasks);
+      if (t < T) {
+        pair_off[t] = po + ip - pairs;
+        row_off[t] = split ? xw : -1;
+        nch[t] = c;
+        task_off[t] = to + itk - tasks;
+      }
+      split_any = split_any || __any_sync(FULL, split);
+      po += __shfl_sync(FULL, ip, 31);
+      ro += __shfl_sync(FULL, iw, 31);
+      to += __shfl_sync(FULL, itk, 31);
     }
-    pair_off[T] = po;
-    task_off[T] = to;
-    any_split = split;
+    if (lane == 0) {
+      pair_off[T] = po;
+      task_off[T] = to;
+      any_split = split_any ? 1 : 0;
+    }
   }
   __syncthreads();
   // entry e of token t: its tile k and place (largest k with pre[t][k] <= e)
@@ -700,46 +721,43 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      int k = 0, pos = 0;
-      if (lo < hi) locate(t, lo, k, pos);
-      constexpr int kB = 8;  // entries whose rows are loaded together
-      for (int e = lo; e < hi; e += kB) {
-        int jj[kB];
-        float hh[kB];
-#pragma unroll
-        for (int b = 0; b < kB; ++b) {
-          // walk to entry e + b: the next non-empty tile when this one is used up
-          if (e + b < hi) {
-            while (pos >= pre[(size_t)t * (K + 1) + k + 1] - pre[(size_t)t * (K + 1) + k]) {
-              ++k;
-              pos = 0;
-            }
-            const size_t ix = (size_t)t * F + k * kW + pos;
-            jj[b] = a.jtile[ix];
-            hh[b] = a.htile[ix];
-            ++pos;
-          } else {
-            jj[b] = 0;
-            hh[b] = 0.f;
-          }
+      // 32 entries at a time: lane l locates entry e0 + l and loads its unit
+      // and h; the warp takes them in order by shuffles, with the Wd slices
+      // of 16 entries in flight
+      for (int e0 = lo; e0 < hi; e0 += 32) {
+        const int ne = min(32, hi - e0);
+        int jl = 0;
+        float hl = 0.f;
+        if (lane < ne) {
+          int k, pos;
+          locate(t, e0 + lane, k, pos);
+          const size_t ix = (size_t)t * F + k * kW + pos;
+          jl = a.jtile[ix];
+          hl = a.htile[ix];
         }
-        uint4 wv[kB];
+        for (int b0 = 0; b0 < ne; b0 += 16) {
+          constexpr int kB = 16;
+          uint4 wv[kB];
 #pragma unroll
-        for (int b = 0; b < kB; ++b)
-          wv[b] = in && e + b < hi
-                      ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
-                      : make_uint4(0, 0, 0, 0);
+          for (int b = 0; b < kB; ++b) {
+            const int jb = __shfl_sync(FULL, jl, (b0 + b) & 31);
+            wv[b] = in && b0 + b < ne
+                        ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jb * d + col))
+                        : make_uint4(0, 0, 0, 0);
+          }
 #pragma unroll
-        for (int b = 0; b < kB; ++b) {
-          const float hb = hh[b];
-          acc[0] = fmaf(hb, bf16_lo(wv[b].x), acc[0]);
-          acc[1] = fmaf(hb, bf16_hi(wv[b].x), acc[1]);
-          acc[2] = fmaf(hb, bf16_lo(wv[b].y), acc[2]);
-          acc[3] = fmaf(hb, bf16_hi(wv[b].y), acc[3]);
-          acc[4] = fmaf(hb, bf16_lo(wv[b].z), acc[4]);
-          acc[5] = fmaf(hb, bf16_hi(wv[b].z), acc[5]);
-          acc[6] = fmaf(hb, bf16_lo(wv[b].w), acc[6]);
-          acc[7] = fmaf(hb, bf16_hi(wv[b].w), acc[7]);
+          for (int b = 0; b < kB; ++b) {
+            const float hs = __shfl_sync(FULL, hl, (b0 + b) & 31);
+            const float hb = b0 + b < ne ? hs : 0.f;
+            acc[0] = fmaf(hb, bf16_lo(wv[b].x), acc[0]);
+            acc[1] = fmaf(hb, bf16_hi(wv[b].x), acc[1]);
+            acc[2] = fmaf(hb, bf16_lo(wv[b].y), acc[2]);
+            acc[3] = fmaf(hb, bf16_hi(wv[b].y), acc[3]);
+            acc[4] = fmaf(hb, bf16_lo(wv[b].z), acc[4]);
+            acc[5] = fmaf(hb, bf16_hi(wv[b].z), acc[5]);
+            acc[6] = fmaf(hb, bf16_lo(wv[b].w), acc[6]);
+            acc[7] = fmaf(hb, bf16_hi(wv[b].w), acc[7]);
+          }
         }
       }
       if (in) {
