@@ -74,6 +74,11 @@ SMALL = [
     (40, 512, 640, 2, "dead20", 60.0),       # small batch: x box narrower than the tile, spills
     (64, 1024, 1024, 8, "zipf", 29.0),
     (65, 256, 1024, 8, "zipf", 29.0),
+    # C = 8 with full-width rows (d is exactly a team's slices): TwELL data
+    # staged one item ahead when T % 4 == 0, read directly otherwise
+    (301, 2048, 1280, 8, "zipf", 29.0),      # direct
+    (1001, 512, 1024, 8, "dead20", 29.0),    # direct, many items
+    (300, 512, 640, 8, "dead20", 120.0),     # staged, spill-heavy
 ]
 
 
