@@ -244,6 +244,46 @@ def test_ffn_0p5b_full_size():
     check_y(f64(y), w64, rows, TOL[synth.BF16])
 
 
+def test_zipf_hot_units_in_one_tile():
+    """Zipf units without the seeded permutation of their ranks: the 128 hottest
+    units are tile 0, so nearly every token overflows that tile and most of
+    the entries come from spill segments.  TwELL on every token, y on a
+    sample of rows."""
+    w = synth.make_workload(T=4096, d=1024, F=4096, W=128, C=8, dtype=synth.BF16, kind="zipf",
+                            mean_active=29.0, seed=3, permute=False)
+    dev, g, gd, y, st = run_forward(w)
+    assert int(st.item()) == 0
+    assert int(g.spill_n.item()) > w["T"] // 2
+    g64 = f64(gd)
+    assert_twell_matches_oracle(g, g64)
+    w64 = widened(w)
+    rows = synth.subsample_rows(w["T"], 192)
+    check_gate_values(g64, w64["x"], w64["Wg_t"], rows)
+    check_y(f64(y), w64, rows, TOL[synth.BF16])
+
+
+@pytest.mark.parametrize("T", [16, 64])
+def test_small_batch_hot_units_in_one_tile(T):
+    """The single-launch small batch with every token's hottest units in tile 0
+    (one heavy tile per token): T = 16 takes the packing-with-dots path, T = 64
+    the balanced one."""
+    w = synth.make_workload(T=T, d=2048, F=8192, W=128, C=8, dtype=synth.BF16, kind="zipf",
+                            mean_active=29.0, seed=9, permute=False)
+    dev = inputs(w)
+    d, F = w["d"], w["F"]
+    g = tw.Twell(T, F, 8, dtype=torch.bfloat16, spill_cap=(F // 128) * T)
+    gd = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, y,
+                             tw.small_batch_workspace(T, d, F), gd, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, tw.status_bits(st)
+    g64 = f64(gd)
+    assert_twell_matches_oracle(g, g64)
+    check_y(f64(y), widened(w), np.arange(T, dtype=np.int32), TOL[synth.BF16])
+
+
 def test_ffn_2b_full_size():
     """The bench workload, same launch configuration: TwELL compared on every
     token (in chunks), y on a seeded sample of rows."""
