@@ -117,6 +117,16 @@ tw_status check_hybrid(const tw_hybrid* h) {
 
 extern "C" {
 
+tw_status tw_measure_row_gather(const void* mat, int32_t rows, int32_t d, int64_t n_gathers,
+                                uint32_t seed, uint32_t* checksum, cudaStream_t stream) {
+  if (rows < 1 || d < 8 || d > 2048 || d % 8 != 0 || n_gathers < 0 || !mat || !checksum)
+    return TW_ERR_INVALID_ARG;
+  if (!aligned16(mat)) return TW_ERR_ALIGNMENT;
+  if (n_gathers == 0) return TW_OK;
+  return from_cuda(
+      tw::launch_row_gather(mat, rows, d, (long long)n_gathers, seed, checksum, stream));
+}
+
 const char* tw_status_string(tw_status s) {
   switch (s) {
     case TW_OK: return "TW_OK";

@@ -111,4 +111,9 @@ cudaError_t launch_hybrid_backward(const void* x, const void* dy, const tw_hybri
                                    float* dWu_t, float* dWd, void* ws, size_t ws_bytes,
                                    int32_t* status, cudaStream_t stream);
 
+// calibrate.cu: scattered whole-row gathers of a bf16 [rows][d] matrix
+// (see tw_measure_row_gather in twell.h).
+cudaError_t launch_row_gather(const void* mat, int rows, int d, long long n, unsigned seed,
+                              uint32_t* checksum, cudaStream_t stream);
+
 }  // namespace tw

@@ -29,7 +29,8 @@ EXPORTS = ["twell_gate_gemm", "twell_fused_updown_workspace_size", "twell_fused_
            "hybrid_ffn_backward_workspace_size", "hybrid_ffn_backward", "dense_ffn_forward",
            "dense_ffn_train_workspace_size", "dense_ffn_train_saved_bytes",
            "dense_ffn_train_forward", "dense_ffn_train_backward",
-           "tw_test_withhold_next_gate_loads", "tw_status_string", "twell_version"]
+           "tw_test_withhold_next_gate_loads", "tw_measure_row_gather", "tw_status_string",
+           "twell_version"]
 
 
 class TwellError(RuntimeError):
@@ -101,6 +102,9 @@ def lib():
                                                vp, ctypes.c_size_t, vp, vp, vp, vp, vp, vp]
         L.tw_test_withhold_next_gate_loads.argtypes = [ctypes.c_uint64]
         L.tw_test_withhold_next_gate_loads.restype = None
+        L.tw_measure_row_gather.argtypes = [vp, i32, i32, ctypes.c_int64, ctypes.c_uint32, vp,
+                                            vp]
+        L.tw_measure_row_gather.restype = st
         L.tw_status_string.argtypes = [st]
         L.tw_status_string.restype = ctypes.c_char_p
         L.twell_version.restype = i32
@@ -335,3 +339,12 @@ def status_bits(dev_status) -> list:
     """Names of the device-side conditions set in a status word tensor."""
     v = int(dev_status.item())
     return [STATUS[i] for i in range(len(STATUS)) if v & (1 << i)]
+
+
+def measure_row_gather(mat, n_gathers, seed, checksum, stream=None):
+    """Measurement aid (not part of the FFN): n_gathers scattered whole rows of
+    the bf16 matrix mat [rows][d]; checksum (an int32 tensor, zeroed by the
+    caller) receives the XOR of every 32-bit word read."""
+    rows, d = mat.shape
+    _check("tw_measure_row_gather", lib().tw_measure_row_gather(
+        _ptr(mat), rows, d, int(n_gathers), int(seed) & 0xFFFFFFFF, _ptr(checksum), _stream(stream)))

@@ -342,6 +342,25 @@ def run_ours(args, rank, world, local_rank):
                   "unique_hbm_bytes": unique_bytes, "live_units": live,
                   "unique_hbm_GBps": unique_bytes / (ms_fused * 1e-3) / 1e9,
                   "unique_hbm_frac": unique_bytes / (ms_fused * 1e-3) / 1e9 / hbm}
+    # The three bounds of the fused kernel (unique HBM bytes, fp32 FMA, gathered
+    # rows through L2), the last against a live measurement of scattered
+    # whole-row gathers from an L2-resident 33.5 MB matrix (tw_measure_row_gather).
+    l2_rate = row_gather_rate(torch, tw, Wu if dt == torch.bfloat16 else None)
+    gathered = nnz * 4 * d * (2 if dt == torch.bfloat16 else 4) // 2
+    bounds_us = {"hbm_unique": unique_bytes / (hbm * 1e9) * 1e6,
+                 "fp32_fma": flops_fused / (fp32_peak * 1e12) * 1e6}
+    if l2_rate:
+        bounds_us["l2_gather"] = gathered / l2_rate * 1e6
+        roof_fused["l2_gather"] = {
+            "what": "scattered whole-row 16-byte gathers of an L2-resident 33.5 MB bf16 matrix, "
+                    "16 warps per SM, measured in this run",
+            "peak_GBps": l2_rate / 1e9, "gathered_bytes": gathered,
+            "bound_us": bounds_us["l2_gather"],
+            "frac": bounds_us["l2_gather"] / (ms_fused * 1e3)}
+    binding = max(bounds_us, key=bounds_us.get)
+    roof_fused["bounds_us"] = bounds_us
+    roof_fused["binding_bound"] = binding
+    roof_fused["frac_of_binding_bound"] = bounds_us[binding] / (ms_fused * 1e3)
     dominant = roof_fused if ms_fused >= ms_gate else roof_gate
     kernels = {"gate_twell_gemm": {"ms": ms_gate, **roof_gate},
                "fused_updown": {"ms": ms_fused, "nnz_per_token": nnz / T, **roof_fused},
@@ -520,8 +539,10 @@ def decode_leg(torch, tw, hbm):
     that buffer (a write flush would leave ~126 MB of dirty lines whose
     write-back the next kernel would pay for).  Two paths: the gate and fused
     calls (twell_gate_gemm + twell_fused_updown), and the whole FFN in one
-    cooperative launch (twell_ffn_small_batch).  The step streams
-    Wg (33.5 MB) and gathers one Wu and one Wd row per active entry."""
+    cooperative launch (twell_ffn_small_batch, also timed with a warm L2);
+    and the in-library dense FFN of the same tokens for comparison.  The
+    sparse step streams Wg (33.5 MB) and gathers one Wu and one Wd row per
+    active entry; the dense one streams all three weights (100.7 MB)."""
     flush = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device="cuda")
     sink = torch.empty((), dtype=torch.float32, device="cuda")
     # Between the flush and the start event a one-element kernel runs (L2
@@ -554,6 +575,11 @@ def decode_leg(torch, tw, hbm):
         y = torch.empty((T, d), dtype=torch.float32, device="cuda")
         ws = tw.fused_workspace(T, d)
         sws = tw.small_batch_workspace(T, d, F) if T <= 64 else None
+        if T == 1:
+            Wd_dense = dev["Wd"].t().contiguous()  # the comparator's [d][F] down weight
+        hd = torch.empty((T, F), dtype=torch.bfloat16, device="cuda")
+        yd = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+        td, tw_warm = [], []
         tg, tf, ts = [], [], []
         for it in range(25):
             cold()
@@ -569,12 +595,28 @@ def decode_leg(torch, tw, hbm):
                 e1[0].record()
                 tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, y, sws)
                 e1[1].record()
+            # the in-library dense bf16 FFN of the same tokens (streams Wg, Wu, Wd)
+            cold()
+            e2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            e2[0].record()
+            tw.dense_ffn_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], Wd_dense, hd, yd)
+            e2[1].record()
             torch.cuda.synchronize()
             if it >= 5:
                 tg.append(e[0].elapsed_time(e[1]))
                 tf.append(e[1].elapsed_time(e[2]))
                 if sws is not None:
                     ts.append(e1[0].elapsed_time(e1[1]))
+                td.append(e2[0].elapsed_time(e2[1]))
+        if sws is not None:  # warm L2: the same launch back to back
+            for it in range(25):
+                e3 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e3[0].record()
+                tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, y, sws)
+                e3[1].record()
+                torch.cuda.synchronize()
+                if it >= 5:
+                    tw_warm.append(e3[0].elapsed_time(e3[1]))
         nnz = int(g.cnt.to(torch.int64).sum().item())
         mg, mf = float(np.median(tg)), float(np.median(tf))
         wg_bytes = F * d * 2
@@ -592,9 +634,18 @@ def decode_leg(torch, tw, hbm):
             r["single_launch"] = {"step_us": ms * 1e3, "tokens_per_s": T / (ms * 1e-3),
                                   "bytes": wg_bytes + rows, "hbm_GBps": step_gbs,
                                   "hbm_frac": step_gbs / hbm, "library_launches": 1,
-                                  "speedup_vs_two_calls": (mg + mf) / ms}
+                                  "speedup_vs_two_calls": (mg + mf) / ms,
+                                  "warm_l2_step_us": float(np.median(tw_warm)) * 1e3}
+        md = float(np.median(td))
+        dense_bytes = 3 * F * d * 2
+        r["dense_comparator"] = {
+            "what": "dense_ffn_forward (tcgen05 GEMMs, bf16 h and y), cold L2",
+            "step_us": md * 1e3, "streamed_bytes": dense_bytes,
+            "hbm_GBps": dense_bytes / (md * 1e-3) / 1e9,
+            "sparse_speedup": md / (float(np.median(ts)) if ts else (mg + mf))}
         out[f"T{T}"] = r
-    del flush
+        del hd, yd
+    del flush, Wd_dense
     return out
 
 
@@ -717,6 +768,27 @@ def training_leg(torch, tw, dist=None, world=1):
     if world > 1:
         out["parallelism"] = f"dp{world}: one fp32 all-reduce of dWg, dWu, dWd ({3 * F * d * 4} B)"
     return out
+
+
+def row_gather_rate(torch, tw, mat):
+    """Bytes per second of scattered whole-row gathers from `mat` (bf16,
+    L2-resident after the first pass), or None for other dtypes."""
+    if mat is None:
+        return None
+    chk = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rows, d = mat.shape
+    n = 1 << 20  # 1 Mi rows
+    ts = []
+    for it in range(6):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        tw.measure_row_gather(mat, n, it + 1, chk)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= 1:
+            ts.append(a.elapsed_time(b))
+    return n * d * 2 / (float(np.median(ts)) * 1e-3)
 
 
 def dense_leg(torch, tw, x, Wg, Wu, Wd, T, d, F, ms_sparse, args):

@@ -326,6 +326,21 @@ TW_API tw_status dense_ffn_train_backward(const void* x, const void* dy, const v
 TW_API void tw_test_withhold_next_gate_loads(uint64_t wait_limit_ns);
 
 /* Human-readable name of a status code. */
+/* Measurement aid, not part of the FFN: the gathered-row rate of the fused
+ * up + down projection's roofline.  n_gathers rows of the bf16 matrix
+ * mat [rows][d] are read in full with 16-byte loads, gather i taking row
+ * splitmix64((seed << 32) ^ i) mod rows (splitmix64 as published by Steele,
+ * Lea and Flood, 2014), by the warps of a persistent grid (one CTA of 16
+ * warps per SM, two rows in flight per warp).
+ * checksum: device word, zeroed by the caller, receives the XOR of every
+ *           32-bit word read (so the loads happen and the result can be
+ *           checked on the host, whatever the order).
+ * Limits: rows >= 1, 8 <= d <= 2048, d % 8 == 0, n_gathers >= 0; mat
+ * 16-byte aligned.  n_gathers == 0 launches nothing. */
+TW_API tw_status tw_measure_row_gather(const void* mat, int32_t rows, int32_t d,
+                                       int64_t n_gathers, uint32_t seed, uint32_t* checksum,
+                                       cudaStream_t stream);
+
 TW_API const char* tw_status_string(tw_status s);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */

@@ -192,3 +192,20 @@ def test_dense_training_validation(L):
     args2 = list(args)
     args2[1] = FAKE + 8
     assert bwd(*args2, FAKE, None, None) == ALIGN
+
+
+def test_row_gather_validation(L):
+    """The measurement entry point rejects bad sizes and a misaligned matrix
+    before any launch, and launches nothing for zero gathers."""
+    ok = twell.STATUS.index("TW_OK")
+    bad = twell.STATUS.index("TW_ERR_INVALID_ARG")
+    align = twell.STATUS.index("TW_ERR_ALIGNMENT")
+    g = L.tw_measure_row_gather
+    assert g(FAKE, 0, 2048, 10, 1, FAKE, None) == bad       # no rows
+    assert g(FAKE, 10, 2056, 10, 1, FAKE, None) == bad      # d > 2048
+    assert g(FAKE, 10, 100, 10, 1, FAKE, None) == bad       # d % 8 != 0
+    assert g(FAKE, 10, 2048, -1, 1, FAKE, None) == bad      # negative count
+    assert g(None, 10, 2048, 10, 1, FAKE, None) == bad
+    assert g(FAKE, 10, 2048, 10, 1, None, None) == bad
+    assert g(FAKE + 8, 10, 2048, 10, 1, FAKE, None) == align
+    assert g(FAKE, 10, 2048, 0, 1, FAKE, None) == ok         # nothing to launch

@@ -523,17 +523,17 @@ def test_oracle_encoded_twell_drives_the_fused_kernel():
     assert np.max(np.abs(f64(y) - ref)) <= 1e-4 * rms(ref)
 
 
-def test_dense_comparator():
-    w = synth.make_workload(T=300, d=512, F=1024, W=128, C=8, dtype=synth.BF16, kind="dead20",
+@pytest.mark.parametrize("T", [300, 1, 8, 64])  # 1..64: the decode-sized comparator
+def test_dense_comparator(T):
+    w = synth.make_workload(T=T, d=512, F=1024, W=128, C=8, dtype=synth.BF16, kind="dead20",
                             mean_active=29.0, seed=8)
     dev = inputs(w)
     Wd_dense = dev["Wd"].t().contiguous()
-    h = torch.empty((300, 1024), dtype=torch.bfloat16, device="cuda")
-    y = torch.empty((300, 512), dtype=torch.bfloat16, device="cuda")
+    h = torch.empty((T, 1024), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, 512), dtype=torch.bfloat16, device="cuda")
     tw.dense_ffn_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], Wd_dense, h, y)
     torch.cuda.synchronize()
     w64 = widened(w)
-    rows = np.arange(300, dtype=np.int32)
     # the comparator stores h and y in bf16, as a dense bf16 FFN does
     dense = oracle.dense_ffn(w64["x"], w64["Wg_t"], w64["Wu_t"], w64["Wd"])
     hr = dense["g"] * dense["u"]
@@ -853,3 +853,31 @@ def test_training_config_full_size():
     res = run_hybrid(w, backup_cap=2048)
     got = check_hybrid_all(w, res)
     assert got["n_backup"] > 0
+
+
+def _splitmix64(x):
+    """splitmix64 (Steele, Lea and Flood, 2014) on uint64 arrays, mod 2^64."""
+    with np.errstate(over="ignore"):
+        z = x + np.uint64(0x9E3779B97F4A7C15)
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        return z ^ (z >> np.uint64(31))
+
+
+@pytest.mark.parametrize("rows,d,n", [(1000, 2048, 3001), (77, 520, 500), (5, 8, 1)])
+def test_row_gather_measurement_reads_the_rows_it_names(rows, d, n):
+    """The roofline's row-gather measurement reads row splitmix64((seed << 32)
+    ^ i) mod rows in full for every i < n: the XOR of all words read equals the
+    host's, for ragged d (chunks past the last lane round) and an odd n."""
+    rng = np.random.default_rng(rows + d)
+    bits = rng.integers(-32768, 32767, size=(rows, d), dtype=np.int16)
+    mat = torch.from_numpy(bits).cuda().view(torch.bfloat16)
+    chk = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seed = 7
+    tw.measure_row_gather(mat, n, seed, chk)
+    torch.cuda.synchronize()
+    idx = np.arange(n, dtype=np.uint64) ^ (np.uint64(seed) << np.uint64(32))
+    sel = (_splitmix64(idx) % np.uint64(rows)).astype(np.int64)
+    words = bits.view(np.uint32)[sel]
+    want = np.bitwise_xor.reduce(words.ravel()) if words.size else np.uint32(0)
+    assert int(chk.item()) & 0xFFFFFFFF == int(want)
