@@ -807,32 +807,32 @@ TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, Entry
       }
     }
   } else {
-    // dense row: 16-byte loads (V values per lane), ranks from a warp scan
-    constexpr int V = 16 / (int)sizeof(Tin);
+    // dense row, 32 * NQ * V columns per round: lane l owns NQ * V contiguous
+    // columns (NQ independent 16-byte loads), so one warp scan of the lanes'
+    // non-zero counts ranks them in column order
+    constexpr int V = 16 / (int)sizeof(Tin);  // values per 16-byte load
+    constexpr int NQ = 2;                     // loads per lane per round
+    constexpr int NV = NQ * V;                // values per lane per round (<= 32)
     const Tin* row = a.backup_g + (size_t)slot * a.F;
     int base = 0;
-    for (int c0 = 0; c0 < a.F && base < hi; c0 += 32 * V) {
-      const int cl = c0 + lane * V;
-      const uint4 raw =
-          cl < a.F ? *reinterpret_cast<const uint4*>(row + cl) : make_uint4(0, 0, 0, 0);
-      float v[V];
-      if constexpr (sizeof(Tin) == 2) {
-        float2 pr[4];
-        Elem<uint16_t>::pairs(raw, pr);
+    for (int c0 = 0; c0 < a.F && base < hi; c0 += 32 * NV) {
+      const int cl = c0 + lane * NV;  // this lane's first column
+      uint4 raw[NQ];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[2 * i] = pr[i].x;
-          v[2 * i + 1] = pr[i].y;
+      for (int q = 0; q < NQ; ++q)
+        raw[q] = cl + q * V < a.F ? *reinterpret_cast<const uint4*>(row + cl + q * V)
+                                  : make_uint4(0, 0, 0, 0);
+      unsigned mask = 0;  // bit i: column cl + i is non-zero
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const uint32_t w[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+          const bool nzv = sizeof(Tin) == 2 ? ((w[i >> 1] >> (16 * (i & 1))) & 0x7FFFu) != 0
+                                            : (w[i] & 0x7FFFFFFFu) != 0;
+          mask |= (nzv ? 1u : 0u) << (q * V + i);
         }
-      } else {
-        v[0] = __uint_as_float(raw.x);
-        v[1] = __uint_as_float(raw.y);
-        v[2] = __uint_as_float(raw.z);
-        v[3] = __uint_as_float(raw.w);
       }
-      unsigned mask = 0;
-#pragma unroll
-      for (int i = 0; i < V; ++i) mask |= (v[i] != 0.f ? 1u : 0u) << i;
       const int nz = __popc(mask);
       int incl = nz;
 #pragma unroll
@@ -840,17 +840,33 @@ TW_DEV int collect_hybrid(const GatherArgs<Tin>& a, int t, int lo, int hi, Entry
         const int u = __shfl_up_sync(FULL, incl, o);
         if (lane >= o) incl += u;
       }
-      unsigned m = mask;
-      while (m) {
-        const int i = __ffs(m) - 1;
-        m &= m - 1;
-        const int r = base + incl - nz + __popc(mask & ((1u << i) - 1u));
-        if (r >= lo && r < hi) {
-          const size_t pos = (size_t)slot * a.F + cl + i;
-          s.g[r - lo] = v[i];
-          s.j[r - lo] = cl + i;
-          s.pos[r - lo] = (int)pos;
-          if (MODE == kModeHybBwd) s.u[r - lo] = Elem<Tin>::scalar(a.backup_u[pos]);
+      const int first = base + incl - nz;  // rank of this lane's first non-zero
+      if (nz > 0 && first < hi && first + nz > lo) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          unsigned mq = (mask >> (q * V)) & ((1u << V) - 1u);
+          while (mq) {
+            const int i = __ffs(mq) - 1;
+            mq &= mq - 1;
+            const int bit = q * V + i;
+            const int r = first + __popc(mask & ((1u << bit) - 1u));
+            if (r >= lo && r < hi) {
+              const uint32_t wd = (i >> (sizeof(Tin) == 2 ? 1 : 0)) == 0   ? raw[q].x
+                                  : (i >> (sizeof(Tin) == 2 ? 1 : 0)) == 1 ? raw[q].y
+                                  : (i >> (sizeof(Tin) == 2 ? 1 : 0)) == 2 ? raw[q].z
+                                                                           : raw[q].w;
+              float v;
+              if constexpr (sizeof(Tin) == 2)
+                v = __uint_as_float((i & 1) ? (wd & 0xFFFF0000u) : (wd << 16));
+              else
+                v = __uint_as_float(wd);
+              const size_t pos = (size_t)slot * a.F + cl + bit;
+              s.g[r - lo] = v;
+              s.j[r - lo] = cl + bit;
+              s.pos[r - lo] = (int)pos;
+              if (MODE == kModeHybBwd) s.u[r - lo] = Elem<Tin>::scalar(a.backup_u[pos]);
+            }
+          }
         }
       }
       base += __shfl_sync(FULL, incl, 31);
