@@ -425,6 +425,7 @@ __global__ void __launch_bounds__(256)
 // Every pass is flat over the records, so a heavy backup row costs no one
 // thread or warp more than its share.
 constexpr int kSegSmem = 2048;  // records of a unit sorted in shared memory
+constexpr int kPaySmem = 512;   // records of a unit whose payloads are staged in shared memory
 
 __global__ void __launch_bounds__(256)
     hyb_ucount_kernel(const Payload* pay, const int32_t* e_total, int32_t* ucnt) {
@@ -513,14 +514,22 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
   }
   const int32_t* order = small ? seg : sorted + b;
+  // the payloads of a unit with few records, in summation order, fetched in
+  // one parallel pass: the summation loop then waits on the token rows only
+  __shared__ Payload pls[kPaySmem];
+  const bool staged = n <= kPaySmem;
+  if (staged) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) pls[i] = pay[order[i]];
+    __syncthreads();
+  }
   const int stride = blockDim.x * E;
   for (int col = threadIdx.x * E; col < d; col += stride) {
     float ad[E], au[E], ag[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) ad[e] = au[e] = ag[e] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
     for (int q = 0; q < n; ++q) {
-      const Payload p = pay[order[q]];
+      const Payload p = staged ? pls[q] : pay[order[q]];
       float xf[E], df[E];
       S::widen(S::load(x + (size_t)p.t * d + col), xf);
       S::widen(S::load(dy + (size_t)p.t * d + col), df);
