@@ -127,6 +127,14 @@ tw_status tw_measure_row_gather(const void* mat, int32_t rows, int32_t d, int64_
       tw::launch_row_gather(mat, rows, d, (long long)n_gathers, seed, checksum, stream));
 }
 
+tw_status tw_measure_stream_read(const void* buf, int64_t bytes, uint32_t* checksum,
+                                 cudaStream_t stream) {
+  if (bytes < 0 || bytes % 16 != 0 || !buf || !checksum) return TW_ERR_INVALID_ARG;
+  if (!aligned16(buf)) return TW_ERR_ALIGNMENT;
+  if (bytes == 0) return TW_OK;
+  return from_cuda(tw::launch_stream_read(buf, (long long)bytes, checksum, stream));
+}
+
 const char* tw_status_string(tw_status s) {
   switch (s) {
     case TW_OK: return "TW_OK";

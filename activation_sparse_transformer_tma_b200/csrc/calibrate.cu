@@ -1,9 +1,17 @@
-// calibrate.cu -- a measurement aid, not part of the FFN: the rate at which
-// the SMs pull whole rows of a bf16 matrix in scattered order with 16-byte
-// vector loads, the access pattern of the fused up + down projection ("Sparser,
-// Faster, Lighter Transformer Language Models", technical summary, section
-// 2.2: the weights of the active units only are loaded).  Timed on a matrix
-// that stays in L2, it is the gathered-row term of that kernel's roofline.
+// calibrate.cu -- measurement aids, not part of the FFN.
+//
+// Row gather: the rate at which the SMs pull whole rows of a bf16 matrix in
+// scattered order with 16-byte vector loads, the access pattern of the fused
+// up + down projection ("Sparser, Faster, Lighter Transformer Language
+// Models", technical summary, section 2.2: the weights of the active units
+// only are loaded).  Timed on a matrix that stays in L2, it is the
+// gathered-row term of that kernel's roofline.
+//
+// Stream read: one launch that reads a buffer once, front to back, with
+// 16-byte loads (eight in flight per thread, two CTAs of 512 threads per
+// SM).  Timed cold on the bytes of a small-batch step (Wg, 33.5 MB at the
+// 2B shape), it is what a launch that only streams those bytes takes, launch
+// and ramp included: the floor for the gate of a few tokens.
 //
 // Row i is splitmix64((seed << 32) ^ i) mod rows.  splitmix64 is the
 // counter-based generator of Steele, Lea and Flood ("Fast splittable
@@ -60,7 +68,48 @@ __global__ void __launch_bounds__(32 * kWarpsG, 1)
   if (lane == 0) atomicXor(checksum, acc);
 }
 
+constexpr int kStreamThreads = 512;
+constexpr int kStreamUnroll = 8;
+
+// Grid-stride over the 16-byte chunks, kStreamUnroll loads in flight per
+// thread; the XOR of every word goes to one device word, one atomic per CTA.
+__global__ void __launch_bounds__(kStreamThreads)
+    stream_read_kernel(const uint4* __restrict__ p, long long n16, uint32_t* checksum) {
+  __shared__ uint32_t wx[kStreamThreads / 32];
+  const long long stride = (long long)gridDim.x * kStreamThreads;
+  long long i = (long long)blockIdx.x * kStreamThreads + threadIdx.x;
+  uint32_t acc = 0;
+  for (; i + (kStreamUnroll - 1) * stride < n16; i += kStreamUnroll * stride) {
+    uint4 v[kStreamUnroll];
+#pragma unroll
+    for (int u = 0; u < kStreamUnroll; ++u) v[u] = __ldcs(p + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < kStreamUnroll; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 v = __ldcs(p + i);
+    acc ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if ((threadIdx.x & 31) == 0) wx[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kStreamThreads / 32; ++w) c ^= wx[w];
+    atomicXor(checksum, c);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_stream_read(const void* buf, long long bytes, uint32_t* checksum,
+                               cudaStream_t stream) {
+  stream_read_kernel<<<2 * num_sms(), kStreamThreads, 0, stream>>>(
+      static_cast<const uint4*>(buf), bytes / 16, checksum);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_row_gather(const void* mat, int rows, int d, long long n, unsigned seed,
                               uint32_t* checksum, cudaStream_t stream) {

@@ -11,15 +11,15 @@
 // one grid, one CTA of 16 warps per SM, runs its phases separated by grid
 // barriers:
 //
-//   A  gate: work items of 16 units x 256 columns of d, spread over every
-//      warp of the grid; a warp streams its 16 Wg rows (16-byte loads, eight
-//      32-column steps in flight; four for more than 16 tokens) and
-//      multiplies them with the tokens' x on the tensor pipe: mma.sync
+//   A  gate: work items of 16 units x 256 columns of d.  Each CTA serves one
+//      slice of d and stages that slice of every token's x in shared memory;
+//      its warps take the slice's unit groups, stream their 16 Wg rows
+//      (16-byte loads, all eight 32-column steps in flight up to 16 tokens,
+//      four above) and multiply them with x on the tensor pipe: mma.sync
 //      m16n8k16 with the units on M and the tokens on N, one 8-token column
-//      tile per MMA.  x is staged in shared memory for up to 16 tokens; for
-//      more, each CTA serves one 256-column slice of d and stages that slice
-//      of every token.  The reduction over d is split into slices: each item
-//      writes fp32 partial sums zpart[slice][t][u].
+//      tile per MMA.  The reduction over d is split into slices: each item
+//      writes fp32 partial sums zpart[slice][t][u], which the next phase
+//      adds in slice order.
 //
 // Up to 32 tokens:
 //   B  packing and dot products: each (tile k, token t) gets one or more
@@ -30,15 +30,19 @@
 //      split the tile's non-zeros (two at a time per warp): for an entry
 //      (j, g) a warp forms u = x_t . Wu_t[j] (fp32) and stores h = g u and j
 //      at the entry's place in the tile (stride W per tile, ascending).
+//      Each warp then asks L2 for the Wd rows of its entries, so phase C
+//      finds them there.
 //   C  updates: one CTA per (token, 256-column slice of d); warp w takes the
-//      tiles k = w (mod 16) in ascending order, accumulates h Wd[j] over its
+//      tiles k = w (mod 16) in rounds of four (one load trip for the round's
+//      counts and first eight entries per tile), accumulates h Wd[j] over its
 //      columns in fp32, and the CTA adds the warps' partial rows in warp
 //      order.
 //
 // 33 to 64 tokens, where a heavy token's tiles would hold single warps up
 // for long:
 //   B  packing only, one warp per (tile, token), as above; every non-zero's
-//      unit j and g go to its place in the tile's row of a per-token list.
+//      unit j and g go to its place in the tile's row of a per-token list,
+//      and its Wu and Wd rows are requested into L2 for phases C and D.
 //   C  dot products: every CTA builds the same per-token prefix sums of the
 //      tile counts; the grid's warps then take the entry pairs of all tokens
 //      in turn, form u = x_t . Wu_t[j] over the whole row and store h = g u.
@@ -63,9 +67,8 @@ constexpr int kThreadsD = 32 * kWarpsD;
 constexpr int kW = 128;          // TwELL tile width of this path
 constexpr int kSlice = 256;      // columns of d per gate work item
 constexpr int kSteps = kSlice / 32;
-constexpr int kStageTok = 16;  // x is staged in shared memory up to this many tokens
-// Above that a CTA of phase A serves one 256-column slice of d and stages
-// just that slice of every token, at a row stride of kSliceRow 16-byte
+// A CTA of phase A serves one 256-column slice of d and stages just that
+// slice of every token, at a row stride of kSliceRow 16-byte
 // chunks (32 used): the 64-byte pad puts the two token rows read by one
 // quarter-warp on disjoint banks.
 constexpr int kSliceRow = 36;
@@ -116,6 +119,49 @@ TW_DEV int ld_acquire(const int32_t* p) {
   return v;
 }
 
+// The bf16 g of the four units lane, lane + 32, lane + 64, lane + 96 of tile
+// k for token t: the nsl slices' fp32 partial sums added in slice order, ReLU
+// (-0 -> +0), then rounding.  The partials were written by other CTAs before
+// the grid barrier, so they are read from L2 (.cg), and a batch of slices is
+// loaded before its first add: these loads are the phase's latency.
+TW_DEV void tile_g(const DecodeArgs& a, int nsl, int t, int k, int lane, uint16_t (&gv)[4]) {
+  constexpr int kBatch = 8;  // slices loaded together (d <= 2048 is one batch)
+  const float* zp = a.zpart + (size_t)t * a.F + k * kW + lane;
+  const size_t sstride = (size_t)a.T * a.F;
+  float z[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s0 = 0; s0 < nsl; s0 += kBatch) {
+    float p[kBatch][4];
+#pragma unroll
+    for (int s = 0; s < kBatch; ++s)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        p[s][i] = s0 + s < nsl ? __ldcg(zp + (size_t)(s0 + s) * sstride + 32 * i) : 0.f;
+#pragma unroll
+    for (int s = 0; s < kBatch; ++s)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (s0 + s < nsl) z[i] += p[s][i];
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float zr = (int32_t)__float_as_uint(z[i]) > 0 ? z[i] : 0.0f;
+    gv[i] = f32_to_bf16(zr);
+  }
+}
+
+// 8 columns of token t's x from column col (zeros past T or d).
+TW_DEV uint4 xrow_g(const DecodeArgs& a, int t, int col) {
+  if (t >= a.T || col >= a.d) return make_uint4(0, 0, 0, 0);
+  return __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d + col));
+}
+
+// Asks L2 for a weight row (d bf16) ahead of its use, one 128-byte line per
+// lane and step, so that the phase after the next barrier finds it there.
+TW_DEV void prefetch_row_l2(const uint16_t* row, int d, int lane) {
+  for (int c = lane * 64; c < d; c += 32 * 64)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(row + c));
+}
+
 // Grid-wide barrier number `b` (1-based) of this launch.  Bounded: a CTA that
 // has waited longer than timeout_ns flags TW_ERR_TIMEOUT and goes on.
 TW_DEV void grid_barrier(const DecodeArgs& a, int b) {
@@ -145,36 +191,21 @@ TW_DEV void grid_barrier(const DecodeArgs& a, int b) {
 // NT: 8-token column tiles of the gate MMAs (1, 2, 4 or 8: T <= 8 * NT).
 template <int NT>
 __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeArgs a) {
-  constexpr bool kStage = 8 * NT <= kStageTok;  // x rows in shared memory
-  constexpr int kStepsA = kStage ? kSteps : kSteps / 2;  // Wg row steps in flight
   extern __shared__ __align__(16) uint8_t smem[];
   const int T = a.T, d = a.d, F = a.F, K = F / kW;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [8 * NT][d] bf16 if kStage, rows >= T zero
-  // x slice of phase A when x is not staged whole: [8 * NT][kSliceRow]
+  // x slice of phase A: [8 * NT][kSliceRow]
   uint4* xsl = reinterpret_cast<uint4*>(smem);
-  const size_t x_bytes = kStage ? (size_t)8 * NT * d * 2 : (size_t)8 * NT * kSliceRow * 16;
-  // after x: the warps' partial rows of phase C (up to 32 tokens), or the
+  const size_t x_bytes = (size_t)8 * NT * kSliceRow * 16;
+  // after it: the warps' partial rows of phase C (up to 32 tokens) or the
   // plan tables of phases C and D (more)
   float* red = reinterpret_cast<float*>(smem + x_bytes);  // [16][256]
   int* tbl = reinterpret_cast<int*>(red);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = gridDim.x * kWarpsD;
   const int gw = blockIdx.x * kWarpsD + warp;
-
-  // stage x (16-byte chunks): the token rows the MMAs read, zeros past T
-  if (kStage) {
-    for (int i = threadIdx.x; i < 8 * NT * d / 8; i += kThreadsD) {
-      const int t = i / (d / 8);
-      reinterpret_cast<uint4*>(xs)[i] =
-          t < T ? reinterpret_cast<const uint4*>(a.x)[i] : make_uint4(0, 0, 0, 0);
-    }
-  }
-  // 16 bytes of token t's x at column col (zeros past T or d)
-  auto xrow = [&](int t, int col) -> uint4 {
-    if (t >= T || col >= d) return make_uint4(0, 0, 0, 0);
-    return kStage ? *reinterpret_cast<const uint4*>(xs + (size_t)t * d + col)
-                  : __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * d + col));
-  };
+  // 16 bytes of token t's x at column col (zeros past T or d); x is a few
+  // KB per token and stays in L1 and L2
+  auto xrow = [&](int t, int col) -> uint4 { return xrow_g(a, t, col); };
   // 8 values of y for token t at column col, in y's dtype
   auto store_y = [&](int t, int col, const float (&v)[8]) {
     if (a.y_bf16) {
@@ -191,15 +222,17 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.spill_n = 0;  // before any spill (phase B)
   __syncthreads();
 
-  // ------------------------------------------------ A: gate partial sums --
+  // ------------------------------------------------------------ A: gate --
   {
+    // Work items of 16 units x 256 columns; each CTA serves one slice of d
+    // (staged for every token) and its warps take that slice's unit groups.
+    // mma.sync m16n8k16 with the units on M and the tokens on N; each item
+    // writes fp32 partial sums zpart[slice][t][u].
     const int g = lane >> 2, q = lane & 3;
     const int S = a.S;
-    // With x read through L1 (more than 16 tokens) a CTA serves one slice of
-    // d, staged in shared memory, and its warps take that slice's unit groups.
     const int s_cta = blockIdx.x % S;
     const int ncs = ((int)gridDim.x - s_cta + S - 1) / S;  // CTAs serving slice s_cta
-    if (!kStage) {
+    {
       const int cs = s_cta * kSlice;
       for (int i = threadIdx.x; i < 8 * NT * 32; i += kThreadsD) {
         const int t = i >> 5, col = cs + (i & 31) * 8;
@@ -209,13 +242,9 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       }
       __syncthreads();
     }
-    const int n_items = kStage ? (F / 16) * S : F / 16;
-    const int first = kStage ? gw : (blockIdx.x / S) * kWarpsD + warp;
-    const int stride = kStage ? nwarps : ncs * kWarpsD;
-    for (int item = first; item < n_items; item += stride) {
-      const int grp = kStage ? item / S : item;
-      const int s = kStage ? item % S : s_cta;
-      const int u0 = grp * 16, c0 = s * kSlice;
+    constexpr int kStepsA = NT <= 2 ? kSteps : kSteps / 2;  // Wg row steps in flight
+    for (int item = (blockIdx.x / S) * kWarpsD + warp; item < F / 16; item += ncs * kWarpsD) {
+      const int u0 = item * 16, c0 = s_cta * kSlice;
       const uint16_t* r_lo = a.Wg + (size_t)(u0 + g) * d;
       const uint16_t* r_hi = a.Wg + (size_t)(u0 + g + 8) * d;
       float D[NT][4];
@@ -235,21 +264,19 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
         }
 #pragma unroll
         for (int i = 0; i < kStepsA; ++i) {
-          const int col = c0 + (i0 + i) * 32 + 8 * q;
           // The 8 columns a lane loaded take the k-indices of its A fragment
           // (the same permutation of k for every unit row and token column),
           // so the products pair Wg[u][col] with x[t][col].
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            const uint4 xb = kStage ? xrow(8 * n + g, col)
-                                    : xsl[(8 * n + g) * kSliceRow + (i0 + i) * 4 + q];
+            const uint4 xb = xsl[(8 * n + g) * kSliceRow + (i0 + i) * 4 + q];
             mma16816(D[n], alo[i].x, ahi[i].x, alo[i].y, ahi[i].y, xb.x, xb.y);
             mma16816(D[n], alo[i].z, ahi[i].z, alo[i].w, ahi[i].w, xb.z, xb.w);
           }
         }
       }
       // D[m][n]: lane (g, q) holds (g, 2q), (g, 2q+1), (g+8, 2q), (g+8, 2q+1)
-      float* zp = a.zpart + (size_t)s * T * F;
+      float* zp = a.zpart + (size_t)s_cta * T * F;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         const int t0 = 8 * n + 2 * q;
@@ -278,15 +305,11 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
          item += nwarps >= n_it ? n_it : nwarps) {
       const int k = item / T, t = item % T;
       uint16_t gv[4];
+      tile_g(a, a.S, t, k, lane, gv);
       unsigned bal[4];
       int n = 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int u = k * kW + lane + 32 * i;
-        float z = 0.f;
-        for (int s2 = 0; s2 < a.S; ++s2) z += a.zpart[((size_t)s2 * T + t) * F + u];
-        const float zr = (int32_t)__float_as_uint(z) > 0 ? z : 0.0f;  // ReLU, -0 -> +0
-        gv[i] = f32_to_bf16(zr);
         bal[i] = __ballot_sync(FULL, gv[i] != 0);
         n += __popc(bal[i]);
       }
@@ -346,6 +369,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       }
       __syncwarp();
       const int nh = sub < n ? (n - sub + m - 1) / m : 0;  // entries of this warp
+      for (int r = 2; r < nh; ++r)  // the Wu rows of this warp's later pairs
+        prefetch_row_l2(a.Wu + (size_t)__float_as_int(lst[2 * r]) * d, d, lane);
       for (int r0 = 0; r0 < nh; r0 += 2) {
         const bool two = r0 + 1 < nh;
         const int j0 = __float_as_int(lst[2 * r0]);
@@ -388,6 +413,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
           }
         }
       }
+      for (int r = 0; r < nh; ++r)  // the Wd rows phase C gathers for these entries
+        prefetch_row_l2(a.Wd + (size_t)__float_as_int(lst[2 * r]) * d, d, lane);
       __syncwarp();  // the list is rewritten by the warp's next item
     }
   }
@@ -403,44 +430,87 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int k = warp; k < K; k += kWarpsD) {
-        // the count and the tile's first entries are loaded together (the
-        // entries past the count are not used)
-        const size_t e0 = (size_t)t * F + k * kW;
-        const int n = a.cnt[(size_t)k * T + t];
-        constexpr int kB = 8;  // entries whose rows are loaded together
-        int jj[kB];
-        float hh[kB];
-#pragma unroll
-        for (int b = 0; b < kB; ++b) {
-          jj[b] = a.jtile[e0 + b];
-          hh[b] = a.htile[e0 + b];
+      // acc += h Wd[j][col, col + 8)
+      auto axpy8 = [&](float h, const uint4& w) {
+        acc[0] = fmaf(h, bf16_lo(w.x), acc[0]);
+        acc[1] = fmaf(h, bf16_hi(w.x), acc[1]);
+        acc[2] = fmaf(h, bf16_lo(w.y), acc[2]);
+        acc[3] = fmaf(h, bf16_hi(w.y), acc[3]);
+        acc[4] = fmaf(h, bf16_lo(w.z), acc[4]);
+        acc[5] = fmaf(h, bf16_hi(w.z), acc[5]);
+        acc[6] = fmaf(h, bf16_lo(w.w), acc[6]);
+        acc[7] = fmaf(h, bf16_hi(w.w), acc[7]);
+      };
+      constexpr int kB = 8;  // entries whose rows are loaded together
+      // Rounds of four of the warp's tiles (k = warp + 16 i).  Lane l loads
+      // the count of tile kb + 16 (l / 8) and that tile's entry l % 8 (unit
+      // and h; past the count they are not used), so a round's lists cost one
+      // trip.  The entries are taken in tile order, kB rows in flight; the
+      // entries past the eighth of a tile follow, tile by tile, 32 to a trip.
+      for (int kb = warp; kb < K; kb += 4 * kWarpsD) {
+        const int kl = kb + kWarpsD * (lane >> 3), bl = lane & 7;
+        int nl = 0, jl = 0;
+        float hl = 0.f;
+        if (kl < K) {
+          nl = a.cnt[(size_t)kl * T + t];
+          const size_t e = (size_t)t * F + kl * kW + bl;
+          jl = a.jtile[e];
+          hl = a.htile[e];
         }
-        for (int s0 = 0; s0 < n; s0 += kB) {
-          uint4 wv[kB];
-          if (s0 > 0) {
-#pragma unroll
-            for (int b = 0; b < kB; ++b) {
-              jj[b] = s0 + b < n ? a.jtile[e0 + s0 + b] : 0;
-              hh[b] = s0 + b < n ? a.htile[e0 + s0 + b] : 0.f;
-            }
-          }
-#pragma unroll
-          for (int b = 0; b < kB; ++b)
-            wv[b] = in && s0 + b < n
-                        ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
-                        : make_uint4(0, 0, 0, 0);
+        unsigned live = __ballot_sync(FULL, bl < nl);
+        while (live != 0) {
+          int jj[kB];
+          float hh[kB];
+          bool vb[kB];
 #pragma unroll
           for (int b = 0; b < kB; ++b) {
-            const float hb = s0 + b < n ? hh[b] : 0.f;  // stale values past the count
-            acc[0] = fmaf(hb, bf16_lo(wv[b].x), acc[0]);
-            acc[1] = fmaf(hb, bf16_hi(wv[b].x), acc[1]);
-            acc[2] = fmaf(hb, bf16_lo(wv[b].y), acc[2]);
-            acc[3] = fmaf(hb, bf16_hi(wv[b].y), acc[3]);
-            acc[4] = fmaf(hb, bf16_lo(wv[b].z), acc[4]);
-            acc[5] = fmaf(hb, bf16_hi(wv[b].z), acc[5]);
-            acc[6] = fmaf(hb, bf16_lo(wv[b].w), acc[6]);
-            acc[7] = fmaf(hb, bf16_hi(wv[b].w), acc[7]);
+            vb[b] = live != 0;
+            const int src = vb[b] ? __ffs(live) - 1 : 0;
+            jj[b] = __shfl_sync(FULL, jl, src);
+            hh[b] = __shfl_sync(FULL, hl, src);
+            live &= live - 1u;
+          }
+          uint4 wv[kB];
+#pragma unroll
+          for (int b = 0; b < kB; ++b)
+            wv[b] = in && vb[b] ? __ldg(reinterpret_cast<const uint4*>(a.Wd + (size_t)jj[b] * d + col))
+                                : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int b = 0; b < kB; ++b)
+            if (vb[b]) axpy8(hh[b], wv[b]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int n = __shfl_sync(FULL, nl, 8 * i);
+          const int k = kb + kWarpsD * i;
+          if (n <= kB) continue;  // (zero past K)
+          const size_t e0 = (size_t)t * F + k * kW;
+          for (int s0 = kB; s0 < n; s0 += 32) {  // lane l loads entry s0 + l
+            const int m = min(32, n - s0);
+            int jo = 0;
+            float ho = 0.f;
+            if (lane < m) {
+              jo = a.jtile[e0 + s0 + lane];
+              ho = a.htile[e0 + s0 + lane];
+            }
+            for (int b0 = 0; b0 < m; b0 += kB) {
+              int jj[kB];
+              float hh[kB];
+#pragma unroll
+              for (int b = 0; b < kB; ++b) {
+                jj[b] = __shfl_sync(FULL, jo, (b0 + b) & 31);
+                hh[b] = __shfl_sync(FULL, ho, (b0 + b) & 31);
+              }
+              uint4 wv[kB];
+#pragma unroll
+              for (int b = 0; b < kB; ++b)
+                wv[b] = in && b0 + b < m ? __ldg(reinterpret_cast<const uint4*>(
+                                               a.Wd + (size_t)jj[b] * d + col))
+                                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+              for (int b = 0; b < kB; ++b)
+                if (b0 + b < m) axpy8(hh[b], wv[b]);
+            }
           }
         }
       }
@@ -479,15 +549,11 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
     for (int item = gw; item < n_it; item += nwarps) {
       const int k = item / T, t = item % T;
       uint16_t gv[4];
+      tile_g(a, a.S, t, k, lane, gv);
       unsigned bal[4];
       int n = 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int u = k * kW + lane + 32 * i;
-        float z = 0.f;
-        for (int s2 = 0; s2 < a.S; ++s2) z += a.zpart[((size_t)s2 * T + t) * F + u];
-        const float zr = (int32_t)__float_as_uint(z) > 0 ? z : 0.0f;  // ReLU, -0 -> +0
-        gv[i] = f32_to_bf16(zr);
         bal[i] = __ballot_sync(FULL, gv[i] != 0);
         n += __popc(bal[i]);
       }
@@ -528,6 +594,15 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
             a.spill_ref[off] = -1;
             set_status(a.status, kStatusSpill);
           }
+        }
+      }
+      // the rows phases C and D gather for the tile's non-zeros
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        for (unsigned b = bal[i]; b != 0; b &= b - 1) {
+          const int j = k * kW + 32 * i + __ffs(b) - 1;
+          prefetch_row_l2(a.Wu + (size_t)j * d, d, lane);
+          prefetch_row_l2(a.Wd + (size_t)j * d, d, lane);
         }
       }
       // the tile's non-zeros, ascending: unit and g at [t][k * W + pos]
@@ -869,8 +944,7 @@ cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t
   a.status = status;
   a.timeout_ns = kWaitTimeoutNs;
   const int NT = T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : 8;
-  const size_t xs_bytes =
-      8 * NT <= kStageTok ? (size_t)8 * NT * d * 2 : (size_t)8 * NT * kSliceRow * 16;
+  const size_t xs_bytes = (size_t)8 * NT * kSliceRow * 16;
   const int K = F / kW;
   const size_t smem =
       xs_bytes + (NT < 8 ? sizeof(float) * kWarpsD * kSlice

@@ -115,5 +115,8 @@ cudaError_t launch_hybrid_backward(const void* x, const void* dy, const tw_hybri
 // (see tw_measure_row_gather in twell.h).
 cudaError_t launch_row_gather(const void* mat, int rows, int d, long long n, unsigned seed,
                               uint32_t* checksum, cudaStream_t stream);
+// Measurement aid: one front-to-back read of `bytes` (a multiple of 16).
+cudaError_t launch_stream_read(const void* buf, long long bytes, uint32_t* checksum,
+                               cudaStream_t stream);
 
 }  // namespace tw

@@ -29,7 +29,7 @@ EXPORTS = ["twell_gate_gemm", "twell_fused_updown_workspace_size", "twell_fused_
            "hybrid_ffn_backward_workspace_size", "hybrid_ffn_backward", "dense_ffn_forward",
            "dense_ffn_train_workspace_size", "dense_ffn_train_saved_bytes",
            "dense_ffn_train_forward", "dense_ffn_train_backward",
-           "tw_test_withhold_next_gate_loads", "tw_measure_row_gather", "tw_status_string",
+           "tw_test_withhold_next_gate_loads", "tw_measure_row_gather", "tw_measure_stream_read", "tw_status_string",
            "twell_version"]
 
 
@@ -105,6 +105,8 @@ def lib():
         L.tw_measure_row_gather.argtypes = [vp, i32, i32, ctypes.c_int64, ctypes.c_uint32, vp,
                                             vp]
         L.tw_measure_row_gather.restype = st
+        L.tw_measure_stream_read.argtypes = [vp, ctypes.c_int64, vp, vp]
+        L.tw_measure_stream_read.restype = st
         L.tw_status_string.argtypes = [st]
         L.tw_status_string.restype = ctypes.c_char_p
         L.twell_version.restype = i32
@@ -348,3 +350,11 @@ def measure_row_gather(mat, n_gathers, seed, checksum, stream=None):
     rows, d = mat.shape
     _check("tw_measure_row_gather", lib().tw_measure_row_gather(
         _ptr(mat), rows, d, int(n_gathers), int(seed) & 0xFFFFFFFF, _ptr(checksum), _stream(stream)))
+
+
+def measure_stream_read(buf, checksum, stream=None):
+    """Measurement aid (not part of the FFN): one launch that reads the whole
+    device tensor buf front to back; checksum (an int32 tensor, zeroed by the
+    caller) receives the XOR of every 32-bit word read."""
+    _check("tw_measure_stream_read", lib().tw_measure_stream_read(
+        _ptr(buf), buf.numel() * buf.element_size(), _ptr(checksum), _stream(stream)))

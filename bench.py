@@ -555,17 +555,32 @@ def decode_leg(torch, tw, hbm):
         torch.sum(flush, dim=0, out=sink)
         tiny.add_(1.0)
 
-    te = []
-    for it in range(15):
-        cold()
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e[0].record()
-        tiny.add_(1.0)
-        e[1].record()
-        torch.cuda.synchronize()
-        if it >= 5:
-            te.append(e[0].elapsed_time(e[1]))
-    out = {"empty_launch_us": float(np.median(te)) * 1e3}
+    def cold_us(fn, n=15, skip=5):
+        ts = []
+        for it in range(n):
+            cold()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            e[0].record()
+            fn()
+            e[1].record()
+            torch.cuda.synchronize()
+            if it >= skip:
+                ts.append(e[0].elapsed_time(e[1]))
+        return float(np.median(ts)) * 1e3
+
+    out = {"empty_launch_us": cold_us(lambda: tiny.add_(1.0))}
+    # The floor for a launch that streams the gate's weights: one read of a
+    # 33.5 MB buffer (the bytes of Wg at the 2B shape) by the library's
+    # stream-read aid, timed the same way.
+    wg_floor = torch.empty(8192 * 2048, dtype=torch.bfloat16, device="cuda")
+    wg_floor.view(torch.int16).random_(-32768, 32767)
+    chk = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out["stream_read_floor"] = {
+        "bytes": wg_floor.numel() * 2,
+        "us": cold_us(lambda: tw.measure_stream_read(wg_floor, chk)),
+        "what": "tw_measure_stream_read of the Wg bytes, cold L2, one launch"}
+    floor_us = out["stream_read_floor"]["us"]
+    del wg_floor
     for T in (1, 8, 16, 64):
         w = synth.make_workload("decode_2b", T=T)
         d, F, C = w["d"], w["F"], w["C"]
@@ -610,7 +625,11 @@ def decode_leg(torch, tw, hbm):
                 td.append(e2[0].elapsed_time(e2[1]))
         if sws is not None:  # warm L2: the same launch back to back
             for it in range(25):
-                tiny.add_(1.0)  # queued first, as in cold(): no host latency in the interval
+                # a 50 us device-side wait queued first, so that the start
+                # event and the launch are both queued before the GPU gets
+                # to them (no host latency in the interval); it touches no
+                # memory, so L2 stays warm
+                torch.cuda._sleep(100000)
                 e3 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
                 e3[0].record()
                 tw.twell_ffn_small_batch(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], g, y, sws)
@@ -627,6 +646,7 @@ def decode_leg(torch, tw, hbm):
              "two_calls": {"gate_us": mg * 1e3, "fused_us": mf * 1e3,
                            "tokens_per_s": T / ((mg + mf) * 1e-3),
                            "gate_hbm_GBps": gate_gbs, "gate_hbm_frac": gate_gbs / hbm,
+                           "gate_frac_of_stream_floor": floor_us / (mg * 1e3),
                            "fused_gathered_GBps": rows / (mf * 1e-3) / 1e9,
                            "library_launches": 2 if T <= 16 else 5}}
         if ts:
@@ -634,7 +654,9 @@ def decode_leg(torch, tw, hbm):
             step_gbs = (wg_bytes + rows) / (ms * 1e-3) / 1e9
             r["single_launch"] = {"step_us": ms * 1e3, "tokens_per_s": T / (ms * 1e-3),
                                   "bytes": wg_bytes + rows, "hbm_GBps": step_gbs,
-                                  "hbm_frac": step_gbs / hbm, "library_launches": 1,
+                                  "hbm_frac": step_gbs / hbm,
+                                  "frac_of_stream_floor": floor_us / (ms * 1e3),
+                                  "library_launches": 1,
                                   "speedup_vs_two_calls": (mg + mf) / ms,
                                   "warm_l2_step_us": float(np.median(tw_warm)) * 1e3}
         md = float(np.median(td))

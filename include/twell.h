@@ -341,6 +341,18 @@ TW_API tw_status tw_measure_row_gather(const void* mat, int32_t rows, int32_t d,
                                        int64_t n_gathers, uint32_t seed, uint32_t* checksum,
                                        cudaStream_t stream);
 
+/* Measurement aid, not part of the FFN: the floor of a launch that streams a
+ * small-batch step's bytes.  The device buffer buf is read once, front to
+ * back, with 16-byte loads (two CTAs of 512 threads per SM, eight loads in
+ * flight per thread) by one launch.  Timed with a cold L2 on the gate's
+ * weight bytes, it is what that launch costs with nothing else to do.
+ * checksum: device word, zeroed by the caller, receives the XOR of every
+ *           32-bit word read.
+ * Limits: bytes >= 0 and a multiple of 16; buf 16-byte aligned.  bytes == 0
+ * launches nothing. */
+TW_API tw_status tw_measure_stream_read(const void* buf, int64_t bytes, uint32_t* checksum,
+                                        cudaStream_t stream);
+
 TW_API const char* tw_status_string(tw_status s);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */

@@ -195,8 +195,8 @@ def test_dense_training_validation(L):
 
 
 def test_row_gather_validation(L):
-    """The measurement entry point rejects bad sizes and a misaligned matrix
-    before any launch, and launches nothing for zero gathers."""
+    """The measurement entry points reject bad sizes and a misaligned buffer
+    before any launch, and launch nothing for zero gathers or zero bytes."""
     ok = twell.STATUS.index("TW_OK")
     bad = twell.STATUS.index("TW_ERR_INVALID_ARG")
     align = twell.STATUS.index("TW_ERR_ALIGNMENT")
@@ -209,3 +209,10 @@ def test_row_gather_validation(L):
     assert g(FAKE, 10, 2048, 10, 1, None, None) == bad
     assert g(FAKE + 8, 10, 2048, 10, 1, FAKE, None) == align
     assert g(FAKE, 10, 2048, 0, 1, FAKE, None) == ok         # nothing to launch
+    r = L.tw_measure_stream_read
+    assert r(FAKE, -16, FAKE, None) == bad                    # negative size
+    assert r(FAKE, 24, FAKE, None) == bad                     # not whole 16-byte chunks
+    assert r(None, 16, FAKE, None) == bad
+    assert r(FAKE, 16, None, None) == bad
+    assert r(FAKE + 8, 16, FAKE, None) == align
+    assert r(FAKE, 0, FAKE, None) == ok                       # nothing to launch

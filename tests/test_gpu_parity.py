@@ -361,8 +361,9 @@ def test_decode_sizes(T):
 # One cooperative launch for the whole small-batch FFN: gate partial sums on
 # mma.sync over every SM, TwELL packing, dot products, updates (per chunk of
 # a token's entries, with partial rows for the long tokens).  T crosses the
-# 8-token MMA column tiles and the 16-token limit of x staged in shared
-# memory; d and F are ragged against the 256-column slices.
+# 8-token MMA column tiles, the 16-token limit of eight column steps in
+# flight, and the 32-token switch to balanced dot products and updates; d
+# and F are ragged against the 32-column steps and 256-column slices.
 SMALL_STEP = [
     # T, d, F, C, kind, mean_active
     (1, 2048, 8192, 8, "zipf", 29.0),
@@ -372,6 +373,8 @@ SMALL_STEP = [
     (16, 2048, 4096, 8, "zipf", 29.0),
     (16, 1024, 1024, 64, "dead20", 300.0),
     (3, 64, 256, 128, "dead20", 100.0),
+    (4, 72, 384, 8, "dead20", 29.0),      # d not a multiple of 32
+    (12, 1000, 1280, 8, "zipf", 29.0),
     (17, 320, 640, 8, "dead20", 60.0),   # x read through L1 from here on
     (33, 2048, 2048, 8, "zipf", 29.0),
     (64, 512, 1280, 16, "zipf", 200.0),  # heavy tokens: many entries per tile
@@ -881,3 +884,17 @@ def test_row_gather_measurement_reads_the_rows_it_names(rows, d, n):
     words = bits.view(np.uint32)[sel]
     want = np.bitwise_xor.reduce(words.ravel()) if words.size else np.uint32(0)
     assert int(chk.item()) & 0xFFFFFFFF == int(want)
+
+
+@pytest.mark.parametrize("nbytes", [16, 4096 + 48, 33554432 + 1024 * 16 + 16])
+def test_stream_read_measurement_reads_every_word(nbytes):
+    """The stream-read floor reads every 16-byte chunk once: the XOR of all words
+    equals the host's, for sizes below one grid pass, with a ragged tail after
+    the eight-deep rounds, and at the gate's 33.5 MB plus a tail."""
+    rng = np.random.default_rng(nbytes)
+    words = rng.integers(0, 2**32, size=nbytes // 4, dtype=np.uint64).astype(np.uint32)
+    buf = torch.from_numpy(words.view(np.int32)).cuda()
+    chk = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tw.measure_stream_read(buf, chk)
+    torch.cuda.synchronize()
+    assert int(chk.item()) & 0xFFFFFFFF == int(np.bitwise_xor.reduce(words))
