@@ -14,14 +14,14 @@
 //   A  gate: work items of 16 units x 256 columns of d.  Each CTA serves one
 //      slice of d and stages that slice of every token's x in shared memory;
 //      its warps take the slice's unit groups, stream their 16 Wg rows
-//      (16-byte loads, all eight 32-column steps in flight up to 16 tokens,
-//      four above) and multiply them with x on the tensor pipe: mma.sync
+//      (16-byte loads, all eight 32-column steps in flight) and multiply
+//      them with x on the tensor pipe: mma.sync
 //      m16n8k16 with the units on M and the tokens on N, one 8-token column
 //      tile per MMA.  The reduction over d is split into slices: each item
 //      writes fp32 partial sums zpart[slice][t][u], which the next phase
 //      adds in slice order.
 //
-// Up to 32 tokens:
+// Up to 16 tokens:
 //   B  packing and dot products: each (tile k, token t) gets one or more
 //      warps.  Every one of them adds the slices in a fixed order, applies
 //      ReLU and rounds g to bf16; the first packs the tile's TwELL slots
@@ -38,14 +38,16 @@
 //      columns in fp32, and the CTA adds the warps' partial rows in warp
 //      order.
 //
-// 33 to 64 tokens, where a heavy token's tiles would hold single warps up
+// 17 to 64 tokens, where a heavy token's tiles would hold single warps up
 // for long:
 //   B  packing only, one warp per (tile, token), as above; every non-zero's
-//      unit j and g go to its place in the tile's row of a per-token list,
-//      and its Wu and Wd rows are requested into L2 for phases C and D.
+//      unit j and g go to its place in the tile's row of a per-token list.
+//      (Requesting its Wu and Wd rows into L2 here made the next grid
+//      barrier wait behind that traffic and cost more than it saved.)
 //   C  dot products: every CTA builds the same per-token prefix sums of the
 //      tile counts; the grid's warps then take the entry pairs of all tokens
-//      in turn, form u = x_t . Wu_t[j] over the whole row and store h = g u.
+//      in turn, ask L2 for the pair's Wd rows, form u = x_t . Wu_t[j] over
+//      the whole row and store h = g u.
 //   D  updates: tasks (token, chunk of up to kChunk entries, 256-column
 //      slice), one warp each, which accumulates h Wd[j] over the chunk's
 //      entries in order, 8 columns per lane in fp32.  A token with one chunk
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   // x slice of phase A: [8 * NT][kSliceRow]
   uint4* xsl = reinterpret_cast<uint4*>(smem);
   const size_t x_bytes = (size_t)8 * NT * kSliceRow * 16;
-  // after it: the warps' partial rows of phase C (up to 32 tokens) or the
+  // after it: the warps' partial rows of phase C (up to 16 tokens) or the
   // plan tables of phases C and D (more)
   float* red = reinterpret_cast<float*>(smem + x_bytes);  // [16][256]
   int* tbl = reinterpret_cast<int*>(red);
@@ -242,7 +244,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       }
       __syncthreads();
     }
-    constexpr int kStepsA = NT <= 2 ? kSteps : kSteps / 2;  // Wg row steps in flight
+    constexpr int kStepsA = kSteps;  // Wg row steps in flight: all eight
     for (int item = (blockIdx.x / S) * kWarpsD + warp; item < F / 16; item += ncs * kWarpsD) {
       const int u0 = item * 16, c0 = s_cta * kSlice;
       const uint16_t* r_lo = a.Wg + (size_t)(u0 + g) * d;
@@ -293,8 +295,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   }
   grid_barrier(a, 1);
 
-  if constexpr (NT < 8) {
-    // up to 32 tokens: packing with the dot products, then updates (B, C)
+  if constexpr (NT < 4) {
+    // up to 16 tokens: packing with the dot products, then updates (B, C)
   // -------------------------------------- B: TwELL pack, h = g (x_t . Wu_t[j]) --
   {
     const unsigned lt = (1u << lane) - 1u;
@@ -540,7 +542,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
   }
 
   } else {
-    // 33 to 64 tokens: packing, then dot products and updates spread evenly
+    // 17 to 64 tokens: packing, then dot products and updates spread evenly
     // over the grid (B to E)
   // ------------------------------- B: TwELL pack, and (unit, g) per entry --
   {
@@ -594,15 +596,6 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
             a.spill_ref[off] = -1;
             set_status(a.status, kStatusSpill);
           }
-        }
-      }
-      // the rows phases C and D gather for the tile's non-zeros
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        for (unsigned b = bal[i]; b != 0; b &= b - 1) {
-          const int j = k * kW + 32 * i + __ffs(b) - 1;
-          prefetch_row_l2(a.Wu + (size_t)j * d, d, lane);
-          prefetch_row_l2(a.Wd + (size_t)j * d, d, lane);
         }
       }
       // the tile's non-zeros, ascending: unit and g at [t][k * W + pos]
@@ -752,6 +745,12 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       }
       const size_t i0 = (size_t)t * F + k0 * kW + p0, i1 = (size_t)t * F + k1 * kW + p1;
       const int j0 = a.jtile[i0], j1 = a.jtile[i1];
+      // the pair's Wd rows, which phase D gathers, are requested into L2
+      // first: their DRAM reads overlap these dot products, and the next
+      // grid barrier (whose release waits for them) comes after the Wu rows
+      // anyway
+      prefetch_row_l2(a.Wd + (size_t)j0 * d, d, lane);
+      if (two) prefetch_row_l2(a.Wd + (size_t)j1 * d, d, lane);
       const uint16_t* w0 = a.Wu + (size_t)j0 * d;
       const uint16_t* w1 = a.Wu + (size_t)j1 * d;
       float pp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -798,7 +797,7 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
       // 32 entries at a time: lane l locates entry e0 + l and loads its unit
       // and h; the warp takes them in order by shuffles, with the Wd slices
-      // of 16 entries in flight
+      // of 8 entries in flight
       for (int e0 = lo; e0 < hi; e0 += 32) {
         const int ne = min(32, hi - e0);
         int jl = 0;
@@ -810,8 +809,8 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
           jl = a.jtile[ix];
           hl = a.htile[ix];
         }
-        for (int b0 = 0; b0 < ne; b0 += 16) {
-          constexpr int kB = 16;
+        for (int b0 = 0; b0 < ne; b0 += 8) {
+          constexpr int kB = 8;  // (16 in flight per lane measured slower)
           uint4 wv[kB];
 #pragma unroll
           for (int b = 0; b < kB; ++b) {
@@ -857,18 +856,31 @@ __global__ void __launch_bounds__(kThreadsD, 1) decode_step_kernel(const DecodeA
       float v[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = 0.f;
-      for (int c = 0; c < nch[t]; ++c) {
-        const float4* pr =
-            reinterpret_cast<const float4*>(a.prow + (size_t)(row_off[t] + c) * d + col);
-        const float4 p0 = __ldcg(pr), p1 = __ldcg(pr + 1);
-        v[0] += p0.x;
-        v[1] += p0.y;
-        v[2] += p0.z;
-        v[3] += p0.w;
-        v[4] += p1.x;
-        v[5] += p1.y;
-        v[6] += p1.z;
-        v[7] += p1.w;
+      // eight chunks' rows loaded before they are added, in chunk order
+      constexpr int kCB = 8;
+      const int nc = nch[t];
+      for (int c0 = 0; c0 < nc; c0 += kCB) {
+        float4 p[kCB][2];
+#pragma unroll
+        for (int c = 0; c < kCB; ++c) {
+          const float4* pr =
+              reinterpret_cast<const float4*>(a.prow + (size_t)(row_off[t] + c0 + c) * d + col);
+          p[c][0] = c0 + c < nc ? __ldcg(pr) : make_float4(0.f, 0.f, 0.f, 0.f);
+          p[c][1] = c0 + c < nc ? __ldcg(pr + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int c = 0; c < kCB; ++c) {
+          if (c0 + c < nc) {
+            v[0] += p[c][0].x;
+            v[1] += p[c][0].y;
+            v[2] += p[c][0].z;
+            v[3] += p[c][0].w;
+            v[4] += p[c][1].x;
+            v[5] += p[c][1].y;
+            v[6] += p[c][1].z;
+            v[7] += p[c][1].w;
+          }
+        }
       }
       store_y(t, col, v);
     }
@@ -947,7 +959,7 @@ cudaError_t launch_decode_step(const void* x, const void* Wg_t, const void* Wu_t
   const size_t xs_bytes = (size_t)8 * NT * kSliceRow * 16;
   const int K = F / kW;
   const size_t smem =
-      xs_bytes + (NT < 8 ? sizeof(float) * kWarpsD * kSlice
+      xs_bytes + (NT < 4 ? sizeof(float) * kWarpsD * kSlice
                          : sizeof(int) * ((size_t)T * (K + 1) + 4 * (size_t)T + 2));
   const void* kern = NT == 1 ? reinterpret_cast<const void*>(decode_step_kernel<1>)
                      : NT == 2 ? reinterpret_cast<const void*>(decode_step_kernel<2>)

@@ -361,9 +361,9 @@ def test_decode_sizes(T):
 # One cooperative launch for the whole small-batch FFN: gate partial sums on
 # mma.sync over every SM, TwELL packing, dot products, updates (per chunk of
 # a token's entries, with partial rows for the long tokens).  T crosses the
-# 8-token MMA column tiles, the 16-token limit of eight column steps in
-# flight, and the 32-token switch to balanced dot products and updates; d
-# and F are ragged against the 32-column steps and 256-column slices.
+# 8-token MMA column tiles and the 16-token switch to balanced dot products
+# and updates; d and F are ragged against the 32-column steps and 256-column
+# slices.
 SMALL_STEP = [
     # T, d, F, C, kind, mean_active
     (1, 2048, 8192, 8, "zipf", 29.0),
@@ -375,7 +375,8 @@ SMALL_STEP = [
     (3, 64, 256, 128, "dead20", 100.0),
     (4, 72, 384, 8, "dead20", 29.0),      # d not a multiple of 32
     (12, 1000, 1280, 8, "zipf", 29.0),
-    (17, 320, 640, 8, "dead20", 60.0),   # x read through L1 from here on
+    (17, 320, 640, 8, "dead20", 60.0),   # balanced dot products and updates from here on
+    (32, 512, 1024, 8, "zipf", 100.0),
     (33, 2048, 2048, 8, "zipf", 29.0),
     (64, 512, 1280, 16, "zipf", 200.0),  # heavy tokens: many entries per tile
     # about 6 chunks of 128 entries per token: the chunk rows of the workspace
