@@ -522,30 +522,36 @@ __global__ void __launch_bounds__(256)
     for (int i = threadIdx.x; i < n; i += blockDim.x) pls[i] = pay[order[i]];
     __syncthreads();
   }
+  // column pairs on the paired fp32 FMA (each half is one fma.rn.f32, so
+  // the sums are those of scalar FMAs in the same order)
+  constexpr int E2 = E / 2;
   const int stride = blockDim.x * E;
   for (int col = threadIdx.x * E; col < d; col += stride) {
-    float ad[E], au[E], ag[E];
+    float2 ad[E2], au[E2], ag[E2];
 #pragma unroll
-    for (int e = 0; e < E; ++e) ad[e] = au[e] = ag[e] = 0.f;
+    for (int e = 0; e < E2; ++e) ad[e] = au[e] = ag[e] = make_float2(0.f, 0.f);
 #pragma unroll 8
     for (int q = 0; q < n; ++q) {
       const Payload p = staged ? pls[q] : pay[order[q]];
       float xf[E], df[E];
       S::widen(S::load(x + (size_t)p.t * d + col), xf);
       S::widen(S::load(dy + (size_t)p.t * d + col), df);
+      const float2 h2 = make_float2(p.h, p.h), du2 = make_float2(p.du, p.du),
+                   dz2 = make_float2(p.dz, p.dz);
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        ad[e] = fmaf(p.h, df[e], ad[e]);
-        au[e] = fmaf(p.du, xf[e], au[e]);
-        ag[e] = fmaf(p.dz, xf[e], ag[e]);
+      for (int e = 0; e < E2; ++e) {
+        const float2 x2 = make_float2(xf[2 * e], xf[2 * e + 1]);
+        ad[e] = __ffma2_rn(h2, make_float2(df[2 * e], df[2 * e + 1]), ad[e]);
+        au[e] = __ffma2_rn(du2, x2, au[e]);
+        ag[e] = __ffma2_rn(dz2, x2, ag[e]);
       }
     }
     const size_t o = (size_t)j * d + col;
 #pragma unroll
-    for (int e = 0; e < E; e += 4) {
-      *reinterpret_cast<float4*>(dWd + o + e) = make_float4(ad[e], ad[e + 1], ad[e + 2], ad[e + 3]);
-      *reinterpret_cast<float4*>(dWu_t + o + e) = make_float4(au[e], au[e + 1], au[e + 2], au[e + 3]);
-      *reinterpret_cast<float4*>(dWg_t + o + e) = make_float4(ag[e], ag[e + 1], ag[e + 2], ag[e + 3]);
+    for (int e = 0; e < E2; e += 2) {
+      *reinterpret_cast<float4*>(dWd + o + 2 * e) = make_float4(ad[e].x, ad[e].y, ad[e + 1].x, ad[e + 1].y);
+      *reinterpret_cast<float4*>(dWu_t + o + 2 * e) = make_float4(au[e].x, au[e].y, au[e + 1].x, au[e + 1].y);
+      *reinterpret_cast<float4*>(dWg_t + o + 2 * e) = make_float4(ag[e].x, ag[e].y, ag[e + 1].x, ag[e + 1].y);
     }
   }
 }
