@@ -28,6 +28,10 @@
 //   3. gather_kernel       persistent teams take work items from a ticket
 //                          counter (the next ticket is fetched while the
 //                          current item runs).
+// The launches are programmatic dependent launches: each kernel's start-up
+// overlaps the previous kernel's tail, and waits for its results before its
+// first global access.  The planner clears the ticket and the arrival
+// counters, so a call needs no memset.
 // A split token's parts are added up a binary tree over the part index
 // through fp32 partial rows in the workspace (one arrival counter per tree
 // node); the tree's shape is fixed by the number of parts, so the output is
@@ -57,6 +61,7 @@
 // Arithmetic.  bf16 dot products use the mixed-precision FMA (bf16 operands,
 // fp32 accumulator); the scaled-row updates widen bf16 pairs exactly and use
 // packed fp32x2 FMA.
+#include "pdl.cuh"
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -88,8 +93,7 @@ struct FusedWs {
                        // with the largest part size; the planner's fast path scans them
   float* partial;      // [parts_cap][d]
   int parts_cap, max_items;
-  size_t bytes;
-  size_t zero_bytes;   // prefix (hdr, done) cleared before every call
+  size_t bytes;        // hdr[0] and done are cleared by the planner (plan_scan_kernel)
 };
 
 size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -104,7 +108,6 @@ FusedWs layout(void* base, int T, int d, int cap) {
   auto take = [&](size_t b) { size_t o = off; off = al256(off + b); return o; };
   const size_t o_hdr = take(4 * sizeof(int32_t));
   const size_t o_done = take(sizeof(int32_t) * (size_t)(cap > 0 ? cap : 1));
-  w.zero_bytes = off;
   const size_t o_nnz = take(sizeof(int32_t) * (size_t)T);
   const size_t o_slot = take(sizeof(int32_t) * (size_t)T);
   const size_t o_desc = take(sizeof(int4) * (size_t)w.max_items);
@@ -173,6 +176,8 @@ TW_DEV void count_block_partials(int n, bool valid, int4* bpart) {
 __global__ void __launch_bounds__(kCountBlock)
     plan_count_twell_kernel(int T, int K, const uint8_t* __restrict__ cnt, int32_t* nnz,
                             int4* bpart) {
+  pdl_wait();  // the counts come from the gate
+  pdl_launch_next();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   int s = 0;
   if (t < T) {
@@ -188,6 +193,8 @@ __global__ void __launch_bounds__(kCountBlock)
     plan_count_hybrid_kernel(int T, const int32_t* __restrict__ row_nnz,
                              const int32_t* __restrict__ row_slot, int cap, int32_t* nnz,
                              int4* bpart) {
+  pdl_wait();
+  pdl_launch_next();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   int s = 0;
   if (t < T) {
@@ -248,10 +255,16 @@ size_t plan_scan_smem(int T) {
 __global__ void __launch_bounds__(kScanThreads)
     plan_scan_kernel(int T, const int32_t* __restrict__ nnz, int parts_cap, int max_items,
                      int n_teams, int32_t* slot_off, int4* item_desc, int32_t* hdr, int4* bpart,
-                     int nb) {
+                     int nb, int32_t* done) {
   __shared__ int warp_sums[32];
   __shared__ int part_sh;
   extern __shared__ int32_t staged[];
+  pdl_wait();
+  pdl_launch_next();
+  // the engine's item ticket and the arrival counters of split tokens' sum
+  // trees start at zero (the gather kernel, two launches on, uses them)
+  if (threadIdx.x == 0) hdr[0] = 0;
+  for (int i = threadIdx.x; i < parts_cap; i += kScanThreads) done[i] = 0;
   // Fast path, from the count kernels' per-block partials: when there is
   // enough work for the largest part size and every split token fits the
   // partial rows, the plan below would use part = kPart and split every token
@@ -375,6 +388,8 @@ __global__ void __launch_bounds__(kCountBlock)
     plan_write_kernel(int T, const int32_t* __restrict__ nnz, int max_items, int32_t* slot_off,
                       int4* item_desc, const int32_t* hdr, const int4* bpart) {
   __shared__ int warp_sums[32];
+  pdl_wait();
+  pdl_launch_next();
   if (hdr[3] == 0) return;  // uniform
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   const int n = t < T ? nnz[t] : 0;
@@ -907,6 +922,8 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
   const int c0 = tw * COLS;    // first column of this warp
   const int my_cols = d - c0 < COLS ? (d - c0 > 0 ? d - c0 : 0) : COLS;
   TeamSmem& ts = team_smem[team];
+  pdl_wait();  // the plan comes from the previous launch
+  pdl_launch_next();
   const int n_items = a.ws.hdr[1];
   const bool leader = tw == 0;
   const uint64_t pol = policy_evict_last();
@@ -1242,8 +1259,7 @@ cudaError_t launch_nchw(GatherArgs<Tin> a, bool out_bf16, cudaStream_t stream) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, dyn);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  kern<<<num_sms() * per_sm, threads, dyn, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(num_sms() * per_sm), dim3(threads), dyn, stream, a);
 }
 
 // Small batches (T <= kDecodeMaxT, decoding): one CTA per token, no work
@@ -1368,15 +1384,15 @@ cudaError_t launch_mode(const GatherArgs<Tin>& a, bool out_bf16, cudaStream_t st
   return cudaErrorInvalidValue;  // d beyond the validated maximum
 }
 
-// Clear the workspace prefix, plan the items from the counts in w.nnz (filled
-// by `count`), run the engine.
+// Plan the items from the counts in w.nnz (filled by `count`, which launches
+// the count kernel and returns its launch status), run the engine.  The four
+// launches are programmatic dependent launches (launch_pdl).
 template <typename Tin, int MODE, class CountFn>
 cudaError_t run_engine(GatherArgs<Tin> a, bool out_bf16, void* base, CountFn count,
                        cudaStream_t stream) {
   const int n_teams = num_sms() * kTeams;  // workers taking items
-  cudaError_t e = cudaMemsetAsync(base, 0, a.ws.zero_bytes, stream);
+  cudaError_t e = count();
   if (e != cudaSuccess) return e;
-  count();
   const size_t scan_smem = plan_scan_smem(a.T);
   if (scan_smem > 48 * 1024) {
     e = set_smem_limit(reinterpret_cast<const void*>(plan_scan_kernel),
@@ -1384,12 +1400,14 @@ cudaError_t run_engine(GatherArgs<Tin> a, bool out_bf16, void* base, CountFn cou
     if (e != cudaSuccess) return e;
   }
   const int nb = (a.T + kCountBlock - 1) / kCountBlock;
-  plan_scan_kernel<<<1, kScanThreads, scan_smem, stream>>>(a.T, a.ws.nnz, a.ws.parts_cap,
-                                                   a.ws.max_items, n_teams,
-                                                   a.ws.slot_off, a.ws.item_desc, a.ws.hdr,
-                                                   a.ws.bpart, nb);
-  plan_write_kernel<<<nb, kCountBlock, 0, stream>>>(a.T, a.ws.nnz, a.ws.max_items, a.ws.slot_off,
-                                                    a.ws.item_desc, a.ws.hdr, a.ws.bpart);
+  e = launch_pdl(plan_scan_kernel, dim3(1), dim3(kScanThreads), scan_smem, stream, a.T,
+                 (const int32_t*)a.ws.nnz, a.ws.parts_cap, a.ws.max_items, n_teams, a.ws.slot_off,
+                 a.ws.item_desc, a.ws.hdr, a.ws.bpart, nb, a.ws.done);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(plan_write_kernel, dim3(nb), dim3(kCountBlock), 0, stream, a.T,
+                 (const int32_t*)a.ws.nnz, a.ws.max_items, a.ws.slot_off, a.ws.item_desc,
+                 (const int32_t*)a.ws.hdr, (const int4*)a.ws.bpart);
+  if (e != cudaSuccess) return e;
   return launch_mode<Tin, MODE>(a, out_bf16, stream);
 }
 
@@ -1431,8 +1449,9 @@ cudaError_t twell_fused_t(const void* x, const tw_twell& g, const void* Wu_t, co
   return run_engine<Tin, kModeTwell>(
       a, y_dtype == TW_BF16, base,
       [&] {
-        plan_count_twell_kernel<<<(T + kCountBlock - 1) / kCountBlock, kCountBlock, 0, stream>>>(
-            T, K, g.cnt, w.nnz, w.bpart);
+        return launch_pdl(plan_count_twell_kernel, dim3((T + kCountBlock - 1) / kCountBlock),
+                          dim3(kCountBlock), 0, stream, T, K, (const uint8_t*)g.cnt, w.nnz,
+                          w.bpart);
       },
       stream);
 }
@@ -1477,9 +1496,9 @@ cudaError_t hybrid_t(const void* xin, const tw_hybrid& h, const void* rdot, cons
   return run_engine<Tin, MODE>(
       a, out_dtype == TW_BF16, base,
       [&] {
-        plan_count_hybrid_kernel<<<(T + kCountBlock - 1) / kCountBlock, kCountBlock, 0,
-                                   stream>>>(T, h.row_nnz, h.row_slot, h.backup_cap, w.nnz,
-                                             w.bpart);
+        return launch_pdl(plan_count_hybrid_kernel, dim3((T + kCountBlock - 1) / kCountBlock),
+                          dim3(kCountBlock), 0, stream, T, (const int32_t*)h.row_nnz,
+                          (const int32_t*)h.row_slot, h.backup_cap, w.nnz, w.bpart);
       },
       stream);
 }

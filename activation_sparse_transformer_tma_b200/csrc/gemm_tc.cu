@@ -15,10 +15,12 @@
 //   warps 2..5  epilogue: tcgen05.ld one TMEM lane (= one token row) per
 //               thread, so the TwELL packing of a row is thread-local.
 // The epilogue of tile i overlaps the main loop of tile i+1 (double-buffered
-// accumulator).  Every wait is bounded: on timeout the CTA raises an abort
+// accumulator).  The launch is a programmatic dependent launch: barrier and
+// TMEM set-up overlap the previous kernel's tail.  Every wait is bounded: on timeout the CTA raises an abort
 // flag, flags TW_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees its
 // TMEM and returns.
 #include "tmap.h"
+#include "pdl.cuh"
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -466,6 +468,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = sm->tmem_base;
   volatile int* abort = &sm->abort;
+  // set-up above overlaps the previous kernel's tail (programmatic dependent
+  // launch); its results are visible from here on
+  pdl_wait();
+  pdl_launch_next();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -624,10 +630,10 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   const int num_tiles = n_tiles_m * n_tiles_n;
   if (num_tiles == 0) return cudaSuccess;
   const int grid = num_tiles < num_sms() ? num_tiles : num_sms();
-  gemm_tc_kernel<Epi, BN><<<grid, NUM_THREADS, smem_bytes<BN>(), stream>>>(
-      a, b0, b1, a1 ? *a1 : a, Kdim, n_tiles_n, num_tiles, a_bytes, epi, status,
-      withheld_wait_ns ? withheld_wait_ns : kWaitTimeoutNs, withheld_wait_ns ? 1 : 0);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<Epi, BN>, dim3(grid), dim3(NUM_THREADS), smem_bytes<BN>(),
+                    stream, a, b0, b1, a1 ? *a1 : a, Kdim, n_tiles_n, num_tiles, a_bytes, epi,
+                    status, withheld_wait_ns ? withheld_wait_ns : kWaitTimeoutNs,
+                    withheld_wait_ns ? 1 : 0);
 }
 
 }  // namespace

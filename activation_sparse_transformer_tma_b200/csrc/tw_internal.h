@@ -17,6 +17,26 @@ int num_sms();
 // on each of them.
 cudaError_t set_smem_limit(const void* func, int bytes);
 
+// Launch with the programmatic stream-serialization attribute: the kernel's
+// CTAs may be scheduled while the previous kernel on the stream finishes, so
+// its launch overlaps that kernel's tail.  Every kernel launched this way
+// calls pdl_wait() (tw_common.cuh) before its first global memory access.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Host-side argument checks shared by the entry points (abi.cu).
 bool row_d_ok(int d, tw_dtype t);
 bool aligned16(const void* p);

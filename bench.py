@@ -329,14 +329,14 @@ def run_ours(args, rank, world, local_rank):
                  "peak_source": f"{src} bf16 burst (the timed region is well under a second)",
                  "frac_of_sustained_peak": tflops_gate / tf_sust,
                  "traffic": profiled_traffic("gate_twell_gemm_ffn_2b.md",
-                                             src_sha("gemm_tc.cu", "tw_common.cuh")),
+                                             src_sha("gemm_tc.cu", "pdl.cuh", "tw_common.cuh")),
                  "algorithmic": f"2*T*d*F = {flops_gate:.4g} FLOP per launch"}
     roof_fused = {"kernel": "twell_fused_updown (gather dot + axpy on CUDA cores)", "bound": "alu",
                   "achieved": tflops_fused, "peak": fp32_peak, "unit": "TFLOP/s",
                   "frac": tflops_fused / fp32_peak,
                   "peak_source": f"derived: {n_sm} SMs x 128 fp32 FMA lanes x 2 x {sm_max_mhz():.0f} MHz",
                   "traffic": profiled_traffic("fused_updown_ffn_2b.md",
-                                              src_sha("fused_updown.cu", "tw_common.cuh")),
+                                              src_sha("fused_updown.cu", "pdl.cuh", "tw_common.cuh")),
                   "algorithmic": f"4*d*nnz = {flops_fused:.4g} FLOP per launch (nnz = {nnz})",
                   "gathered_GBps": nnz * 4 * d / (ms_fused * 1e-3) / 1e9,
                   "unique_hbm_bytes": unique_bytes, "live_units": live,
