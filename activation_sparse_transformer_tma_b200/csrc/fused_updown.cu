@@ -1527,17 +1527,47 @@ cudaError_t launch_fused_updown_in_scratch(const void* x, const tw_twell& g, con
   return twell_fused(x, g, Wu_t, Wd, d, y, y_dtype, scratch, w, status, stream);
 }
 
+namespace {
+
+// u is +0 off the pattern: clears ell_u and the stored rows of backup_u (the
+// first min(*n_backup, cap), the rows a backup slot holds), 16 bytes per
+// store with a byte tail, before the engine writes the pattern's entries.
+__global__ void __launch_bounds__(256)
+    hyb_zero_u_kernel(uint8_t* ell_u, size_t ell_bytes, uint8_t* backup_u, size_t row_bytes,
+                      const int32_t* n_backup, int cap) {
+  pdl_wait();
+  pdl_launch_next();
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t i0 = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  auto clear = [&](uint8_t* p, size_t bytes) {
+    const size_t n16 = bytes / 16;
+    for (size_t i = i0; i < n16; i += stride) reinterpret_cast<uint4*>(p)[i] = make_uint4(0, 0, 0, 0);
+    for (size_t b = n16 * 16 + i0; b < bytes; b += stride) p[b] = 0;
+  };
+  if (ell_u != nullptr) clear(ell_u, ell_bytes);
+  if (backup_u != nullptr) {
+    const int nb = min(*n_backup, cap);
+    clear(backup_u, (size_t)(nb > 0 ? nb : 0) * row_bytes);
+  }
+}
+
+}  // namespace
+
 cudaError_t launch_hybrid_gather_forward(const void* x, const tw_hybrid& gu, const void* Wu_t,
                                          const void* Wd, int d, void* y, tw_dtype y_dtype,
                                          void* ws, int32_t* status, cudaStream_t stream) {
   // u is defined as +0 off the pattern: clear both u arrays, the engine then
   // writes the pattern's entries
-  cudaError_t e = cudaSuccess;
   const size_t esz = gu.dtype == TW_BF16 ? 2 : 4;
-  if (gu.C_h > 0) e = cudaMemsetAsync(gu.ell_u, 0, esz * (size_t)gu.T * gu.C_h, stream);
-  if (e == cudaSuccess && gu.backup_cap > 0)
-    e = cudaMemsetAsync(gu.backup_u, 0, esz * (size_t)gu.backup_cap * gu.F, stream);
-  if (e != cudaSuccess) return e;
+  if (gu.C_h > 0 || gu.backup_cap > 0) {
+    cudaError_t e = launch_pdl(
+        hyb_zero_u_kernel, dim3(num_sms() * 4), dim3(256), 0, stream,
+        gu.C_h > 0 ? static_cast<uint8_t*>(gu.ell_u) : (uint8_t*)nullptr,
+        esz * (size_t)gu.T * gu.C_h,
+        gu.backup_cap > 0 ? static_cast<uint8_t*>(gu.backup_u) : (uint8_t*)nullptr,
+        esz * (size_t)gu.F, (const int32_t*)gu.n_backup, gu.backup_cap);
+    if (e != cudaSuccess) return e;
+  }
   return gu.dtype == TW_BF16
              ? hybrid_t<uint16_t, kModeHybFwd>(x, gu, Wu_t, Wd, nullptr, d, 0.f, nullptr, nullptr,
                                                y, y_dtype, ws, status, stream)

@@ -9,6 +9,7 @@
 //   * the weight gradients are summed per unit from the backward's per-entry
 //     records after a deterministic, token-ordered transposition (stable
 //     counting sort by unit; no float atomics).
+#include "pdl.cuh"
 #include "tw_common.cuh"
 #include "tw_internal.h"
 
@@ -168,6 +169,8 @@ __global__ void __launch_bounds__(256)
     hyb_rows_kernel(int Tn, int F, int W, int C, const uint8_t* cnt, const T* val, const uint8_t* idx,
                     const int32_t* spill_ref, int spill_cap, const T* spill_val, int C_h,
                     T* ell_g, uint16_t* ell_idx, int32_t* row_nnz, int32_t* status) {
+  pdl_wait();
+  pdl_launch_next();
   const int lane = threadIdx.x & 31;
   const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   if (t >= Tn) return;
@@ -280,10 +283,14 @@ __global__ void __launch_bounds__(256)
 constexpr int SCAN_THREADS = 1024;
 __global__ void __launch_bounds__(SCAN_THREADS)
     scan_kernel(int mode, int n, const int32_t* in, int thr, int32_t* out, int32_t* aux, int cap,
-                int32_t* total, int32_t* status) {
+                int32_t* total, int32_t* status, int32_t* zero, int nzero) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
+  pdl_wait();
+  pdl_launch_next();
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  // a counter array of a later kernel, cleared here instead of by a memset
+  for (int i = tid; i < nzero; i += SCAN_THREADS) zero[i] = 0;
   if (tid == 0) carry = 0;
   __syncthreads();
   for (int base = 0; base < n; base += SCAN_THREADS) {
@@ -342,6 +349,8 @@ __global__ void __launch_bounds__(256)
                       const int32_t* spill_ref, int spill_cap, const T* spill_val,
                       const int32_t* backup_rows, const int32_t* n_backup, int backup_cap,
                       T* backup_g) {
+  pdl_wait();
+  pdl_launch_next();
   const int lane = threadIdx.x & 31;
   const int slot = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int nb = min(*n_backup, backup_cap);
@@ -429,6 +438,8 @@ constexpr int kPaySmem = 512;   // records of a unit whose payloads are staged i
 
 __global__ void __launch_bounds__(256)
     hyb_ucount_kernel(const Payload* pay, const int32_t* e_total, int32_t* ucnt) {
+  pdl_wait();
+  pdl_launch_next();
   const int n = *e_total;
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x)
     atomicAdd(&ucnt[pay[e].j], 1);
@@ -437,6 +448,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     hyb_place_kernel(const Payload* pay, const int32_t* e_total, const int32_t* unit_off,
                      int32_t* cursor, int32_t* list) {
+  pdl_wait();
+  pdl_launch_next();
   const int n = *e_total;
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
     const int j = pay[e].j;
@@ -473,6 +486,8 @@ __global__ void __launch_bounds__(256)
   using S = Slice<T>;
   constexpr int E = S::E;
   __shared__ int32_t seg[kSegSmem];
+  pdl_wait();
+  pdl_launch_next();
   const int j = blockIdx.x;
   const int b = unit_off[j], n = unit_off[j + 1] - b;
   const bool small = n <= kSegSmem;
@@ -621,21 +636,26 @@ unsigned warp_blocks(int n) { return (unsigned)(((size_t)n + 7) / 8); }
 template <typename T>
 cudaError_t to_hybrid_t(const tw_twell& g, const tw_hybrid& o, int32_t* status, cudaStream_t s) {
   if (g.T == 0) return cudaSuccess;
-  hyb_rows_kernel<T><<<warp_blocks(g.T), 256, 0, s>>>(
-      g.T, g.F, g.W, g.C, g.cnt, static_cast<const T*>(g.val), g.idx, g.spill_ref, g.spill_cap,
-      static_cast<const T*>(g.spill_val), o.C_h, static_cast<T*>(o.ell_g), o.ell_idx, o.row_nnz,
-      status);
-  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(0, g.T, o.row_nnz, o.C_h, o.row_slot, o.backup_rows,
-                                         o.backup_cap, o.n_backup, status);
+  cudaError_t e = launch_pdl(
+      hyb_rows_kernel<T>, dim3(warp_blocks(g.T)), dim3(256), 0, s, g.T, g.F, g.W, g.C,
+      (const uint8_t*)g.cnt, static_cast<const T*>(g.val), (const uint8_t*)g.idx,
+      (const int32_t*)g.spill_ref, g.spill_cap, static_cast<const T*>(g.spill_val), o.C_h,
+      static_cast<T*>(o.ell_g), o.ell_idx, o.row_nnz, status);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(scan_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, 0, g.T, (const int32_t*)o.row_nnz,
+                 o.C_h, o.row_slot, o.backup_rows, o.backup_cap, o.n_backup, status,
+                 (int32_t*)nullptr, 0);
+  if (e != cudaSuccess) return e;
   if (o.backup_cap > 0) {
     auto kern = g.W == 64 ? hyb_backup_kernel<T, 64>
                           : (g.W == 256 ? hyb_backup_kernel<T, 256> : hyb_backup_kernel<T, 128>);
-    kern<<<warp_blocks(o.backup_cap), 256, 0, s>>>(
-        g.T, g.F, g.C, g.cnt, static_cast<const T*>(g.val), g.idx, g.spill_ref, g.spill_cap,
-        static_cast<const T*>(g.spill_val), o.backup_rows, o.n_backup, o.backup_cap,
-        static_cast<T*>(o.backup_g));
+    e = launch_pdl(kern, dim3(warp_blocks(o.backup_cap)), dim3(256), 0, s, g.T, g.F, g.C,
+                   (const uint8_t*)g.cnt, static_cast<const T*>(g.val), (const uint8_t*)g.idx,
+                   (const int32_t*)g.spill_ref, g.spill_cap, static_cast<const T*>(g.spill_val),
+                   (const int32_t*)o.backup_rows, (const int32_t*)o.n_backup, o.backup_cap,
+                   static_cast<T*>(o.backup_g));
   }
-  return cudaGetLastError();
+  return e;
 }
 
 template <typename T>
@@ -645,26 +665,33 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
                        int32_t* status, cudaStream_t s) {
   const BwdWs w = carve(ws, gu.T, gu.F, gu.C_h, gu.backup_cap);
   void* engine_ws = static_cast<char*>(ws) + w.bytes;
-  // entry offsets of every token (token-major order)
-  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(2, gu.T, gu.row_nnz, 0, w.e0, gu.row_slot,
-                                         gu.backup_cap, nullptr, status);
+  // entry offsets of every token (token-major order); the per-unit record
+  // counts and placement cursors of the weight-gradient pass are cleared here
+  cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, 2, gu.T,
+                             (const int32_t*)gu.row_nnz, 0, w.e0, gu.row_slot, gu.backup_cap,
+                             (int32_t*)nullptr, status, w.ucnt, 2 * gu.F);
+  if (e != cudaSuccess) return e;
   // per-token pass: dh, du, dz, dx and one record per entry
-  cudaError_t e = launch_hybrid_gather_backward(dy, gu, Wg_t, Wu_t, Wd, d, lam, w.e0, w.pay, dx,
-                                                dx_dtype, engine_ws, status, s);
+  e = launch_hybrid_gather_backward(dy, gu, Wg_t, Wu_t, Wd, d, lam, w.e0, w.pay, dx, dx_dtype,
+                                    engine_ws, status, s);
   if (e != cudaSuccess) return e;
   // weight gradients: records grouped by unit, then each unit sorted and summed
-  e = cudaMemsetAsync(w.ucnt, 0, sizeof(int32_t) * 2 * (size_t)gu.F, s);
-  if (e != cudaSuccess) return e;
   const int grid = num_sms() * 8;
   const int32_t* e_total = w.e0 + gu.T;
-  hyb_ucount_kernel<<<grid, 256, 0, s>>>(w.pay, e_total, w.ucnt);
-  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(1, gu.F, w.ucnt, 0, w.unit_off, nullptr, 0, nullptr,
-                                         status);
-  hyb_place_kernel<<<grid, 256, 0, s>>>(w.pay, e_total, w.unit_off, w.cursor, w.list);
-  hyb_wgrad_kernel<T><<<gu.F, 256, 0, s>>>(gu.F, d, static_cast<const T*>(x),
-                                           static_cast<const T*>(dy), w.unit_off, w.list,
-                                           w.sorted, w.pay, dWg_t, dWu_t, dWd);
-  return cudaGetLastError();
+  e = launch_pdl(hyb_ucount_kernel, dim3(grid), dim3(256), 0, s, (const Payload*)w.pay, e_total,
+                 w.ucnt);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(scan_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, 1, gu.F, (const int32_t*)w.ucnt,
+                 0, w.unit_off, (int32_t*)nullptr, 0, (int32_t*)nullptr, status,
+                 (int32_t*)nullptr, 0);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(hyb_place_kernel, dim3(grid), dim3(256), 0, s, (const Payload*)w.pay, e_total,
+                 (const int32_t*)w.unit_off, w.cursor, w.list);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(hyb_wgrad_kernel<T>, dim3(gu.F), dim3(256), 0, s, gu.F, d,
+                    static_cast<const T*>(x), static_cast<const T*>(dy),
+                    (const int32_t*)w.unit_off, w.list, w.sorted, (const Payload*)w.pay, dWg_t,
+                    dWu_t, dWd);
 }
 
 }  // namespace

@@ -717,7 +717,21 @@ def training_leg(torch, tw, dist=None, world=1):
             for i, n in enumerate(names):
                 times[n].append(e[i].elapsed_time(e[i + 1]))
     ms = {n: float(np.median(v)) for n, v in times.items()}
-    step = sum(ms.values())
+    phases_sum = sum(ms.values())
+
+    # The step itself: whole steps back to back between two events, as the
+    # inference step is timed (the phase times above carry an event and, for
+    # the first phase, the host's launch latency at each boundary).
+    def sparse_step():
+        tw.twell_gate_gemm(dev["x"], dev["Wg_t"], g, None, st)
+        tw.twell_to_hybrid(g, hy, st)
+        tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], y, fws, st)
+        tw.hybrid_ffn_backward(dev["x"], dev["dy"], hy, dev["Wg_t"], dev["Wu_t"], dev["Wd"],
+                               w["lam"], dx, grads.dWg_t, grads.dWu_t, grads.dWd, ws, st)
+        if world > 1:
+            grads.allreduce()
+
+    step = back_to_back_ms(torch, sparse_step)
     n_backup = int(hy.n_backup.item())
     st_sparse = int(st.item())
     # bytes of the hybrid step: activations kept from the forward for the
@@ -754,7 +768,13 @@ def training_leg(torch, tw, dist=None, world=1):
             dn["dense_forward"].append(e[0].elapsed_time(e[1]))
             dn["dense_backward"].append(e[1].elapsed_time(e[2]))
     dms = {n: float(np.median(v)) for n, v in dn.items()}
-    dense_step = sum(dms.values())
+
+    def dense_step_fn():
+        tw.dense_ffn_train_forward(dev["x"], dev["Wg_t"], dev["Wu_t"], dev["Wd"], dws, y, dst)
+        tw.dense_ffn_train_backward(dev["x"], dev["dy"], dev["Wg_t"], dev["Wu_t"], dev["Wd"],
+                                    w["lam"], dws, dx, grads.dWg_t, grads.dWu_t, grads.dWd, dst)
+
+    dense_step = back_to_back_ms(torch, dense_step_fn)
     dense_saved = tw.dense_ffn_train_saved_bytes(T, F)
     dense_ws = tw.dense_ffn_train_workspace_size(T, F)
     del dws
@@ -764,8 +784,11 @@ def training_leg(torch, tw, dist=None, world=1):
         step = float(tt.item())
     out = {"workload": "train_2b", "T": T, "d": d, "F": F, "C": C, "C_h": C_h,
            "ms": ms, "ms_per_step": step, "tokens_per_s": world * T / (step * 1e-3),
+           "timing": "ms_per_step: 10 whole steps back to back between two CUDA events, median "
+                     "of 3 such runs; ms: each phase between events, median of 5 steps",
+           "phases_sum_ms": phases_sum,
            "n_backup": n_backup, "backup_cap": cap, "device_status": st_sparse,
-           "dense": {"ms": dms, "ms_per_step": dense_step,
+           "dense": {"ms": dms, "ms_per_step": dense_step, "phases_sum_ms": sum(dms.values()),
                      "tokens_per_s": T / (dense_step * 1e-3),
                      "flops_per_step": 9 * 2.0 * T * d * F,
                      "tflops": 9 * 2.0 * T * d * F / (dense_step * 1e-3) / 1e12,
@@ -791,6 +814,26 @@ def training_leg(torch, tw, dist=None, world=1):
     if world > 1:
         out["parallelism"] = f"dp{world}: one fp32 all-reduce of dWg, dWu, dWd ({3 * F * d * 4} B)"
     return out
+
+
+def back_to_back_ms(torch, fn, steps=10, runs=3):
+    """Milliseconds per call of fn, from `steps` calls back to back between two
+    CUDA events on the current stream (a device-side wait queued first, so the
+    host's launch latency is not in the interval); median of `runs`."""
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    res = []
+    for _ in range(runs):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda._sleep(200000)
+        e[0].record()
+        for _ in range(steps):
+            fn()
+        e[1].record()
+        torch.cuda.synchronize()
+        res.append(e[0].elapsed_time(e[1]) / steps)
+    return float(np.median(res))
 
 
 def row_gather_rate(torch, tw, mat):

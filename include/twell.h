@@ -118,7 +118,9 @@ typedef struct {
  *                backup rows needed (rows past backup_cap are dropped and
  *                TW_ERR_BACKUP_CAPACITY is flagged).
  * ell_u / backup_u hold the up activation u = x Wu on the same pattern (+0
- * elsewhere); hybrid_ffn_forward fills them and the backward reads them.
+ * elsewhere in ell_u and in the stored backup rows, the first
+ * min(*n_backup, backup_cap); rows past those are not written);
+ * hybrid_ffn_forward fills them and the backward reads them.
  * Shapes: ell_g, ell_u [T][C_h] (dtype); ell_idx [T][C_h] uint16; row_nnz,
  * row_slot [T] int32; backup_rows [backup_cap] int32; backup_g, backup_u
  * [backup_cap][F] (dtype); n_backup one int32.
