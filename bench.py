@@ -794,6 +794,7 @@ def training_leg(torch, tw, dist=None, world=1):
                      "tflops": 9 * 2.0 * T * d * F / (dense_step * 1e-3) / 1e12,
                      "device_status": int(dst.item())},
            "sparse_speedup_vs_dense": dense_step / step,
+           "sparse_speedup_vs_dense_phases": sum(dms.values()) / phases_sum,
            "memory_bytes": {
                "what": "FFN-layer activation bytes per GPU, excluding x, dy, the weights and "
                        "their gradients (the same for both paths)",
