@@ -258,58 +258,66 @@ def run_ours(args, rank, world, local_rank):
     # and the copy-out of step k-1 overlap the kernels of step k.
     xh = torch.empty((T, d), dtype=dt, pin_memory=True)
     xh.copy_(x.cpu())
-    yh = torch.empty((T, d), dtype=torch.float32, pin_memory=True)
     E = max(3, min(K, 30))
-    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    xd = [torch.empty_like(x) for _ in range(2)]
-    yd = [torch.empty_like(y) for _ in range(2)]
-    ev = {n: [torch.cuda.Event() for _ in range(2)]
-          for n in ("x_ready", "x_free", "y_ready", "y_free")}
-    for b in range(2):  # every buffer starts free
-        ev["x_free"][b].record(s_cmp)
-        ev["y_free"][b].record(s_out)
 
-    def e2e_step(k):
-        b = k & 1
-        s_in.wait_event(ev["x_free"][b])
-        with torch.cuda.stream(s_in):
-            xd[b].copy_(xh, non_blocking=True)
-        ev["x_ready"][b].record(s_in)
-        s_cmp.wait_event(ev["x_ready"][b])
-        s_cmp.wait_event(ev["y_free"][b])
-        tw.twell_gate_gemm(xd[b], Wg, g, None, status, stream=s_cmp)
-        tw.twell_fused_updown(xd[b], g, Wu, Wd, yd[b], ws, status, stream=s_cmp)
-        ev["x_free"][b].record(s_cmp)
-        ev["y_ready"][b].record(s_cmp)
-        s_out.wait_event(ev["y_ready"][b])
-        with torch.cuda.stream(s_out):
-            yh.copy_(yd[b], non_blocking=True)
-        ev["y_free"][b].record(s_out)
+    def e2e_rate(y_dtype):
+        yh = torch.empty((T, d), dtype=y_dtype, pin_memory=True)
+        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        xd = [torch.empty_like(x) for _ in range(2)]
+        yd = [torch.empty((T, d), dtype=y_dtype, device="cuda") for _ in range(2)]
+        ev = {n: [torch.cuda.Event() for _ in range(2)]
+              for n in ("x_ready", "x_free", "y_ready", "y_free")}
+        for b in range(2):  # every buffer starts free
+            ev["x_free"][b].record(s_cmp)
+            ev["y_free"][b].record(s_out)
 
-    for k in range(3):
-        e2e_step(k)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    s_cmp.wait_event(e0)
-    s_out.wait_event(e0)
-    for k in range(E):
-        e2e_step(k)
-    e1.record(s_out)
-    torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if dist:
-        tt = torch.tensor([ms_e2e], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = float(tt.item())
-    e2e = {"value": world * T * E / (ms_e2e / 1e3), "unit": UNIT,
-           "h2d_bytes_per_step": xh.numel() * xh.element_size(),
-           "d2h_bytes_per_step": yh.numel() * yh.element_size(),
-           "pipeline": "3 streams (copy-in, kernels, copy-out), double-buffered x and y"}
-    del xd, yd
+        def e2e_step(k):
+            b = k & 1
+            s_in.wait_event(ev["x_free"][b])
+            with torch.cuda.stream(s_in):
+                xd[b].copy_(xh, non_blocking=True)
+            ev["x_ready"][b].record(s_in)
+            s_cmp.wait_event(ev["x_ready"][b])
+            s_cmp.wait_event(ev["y_free"][b])
+            tw.twell_gate_gemm(xd[b], Wg, g, None, status, stream=s_cmp)
+            tw.twell_fused_updown(xd[b], g, Wu, Wd, yd[b], ws, status, stream=s_cmp)
+            ev["x_free"][b].record(s_cmp)
+            ev["y_ready"][b].record(s_cmp)
+            s_out.wait_event(ev["y_ready"][b])
+            with torch.cuda.stream(s_out):
+                yh.copy_(yd[b], non_blocking=True)
+            ev["y_free"][b].record(s_out)
+
+        for k in range(3):
+            e2e_step(k)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s_in)
+        s_cmp.wait_event(e0)
+        s_out.wait_event(e0)
+        for k in range(E):
+            e2e_step(k)
+        e1.record(s_out)
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1)
+        if dist:
+            tt = torch.tensor([ms_e2e], device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms_e2e = float(tt.item())
+        return {"value": world * T * E / (ms_e2e / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+                "d2h_bytes_per_step": yh.numel() * yh.element_size(),
+                "pipeline": "3 streams (copy-in, kernels, copy-out), double-buffered x and y"}
+
+    # y in fp32, the accumulator's precision (the headline); then the same
+    # path writing y rounded once to bf16, which halves the read-back that
+    # bounds this pipeline
+    e2e = e2e_rate(torch.float32)
+    e2e_bf16 = e2e_rate(torch.bfloat16)
+    e2e_bf16["what"] = "as e2e, with y returned in bf16 (the fp32 sums rounded once)"
 
     hbm, tf_burst, tf_sust, src = peaks()
     n_sm = torch.cuda.get_device_properties(0).multi_processor_count
@@ -372,6 +380,7 @@ def run_ours(args, rank, world, local_rank):
             "data": "synthetic (seeded generator: Zipf(1.1) units, lognormal token skew, "
                     "mean 29 active units per token)",
             "config": config_of(w, args), "roofline": dominant, "e2e": e2e,
+            "e2e_bf16_y": e2e_bf16,
             "gpu_launches": KERNELS_PER_STEP * K, "clocks": clk, "kernels": kernels,
             "device_status": st}
 
@@ -386,7 +395,7 @@ def run_ours(args, rank, world, local_rank):
         if rank == 0 and "energy" in legs:
             line["energy"] = energy_leg(torch, tw, x, Wg, Wu, Wd, g, y, ws, status, T, d, F,
                                         local_rank)
-        del x, Wg, Wu, Wd, g, y, ws, xh, yh
+        del x, Wg, Wu, Wd, g, y, ws, xh
         torch.cuda.empty_cache()
         if rank == 0 and "decode" in legs:
             line["decode"] = decode_leg(torch, tw, hbm)
