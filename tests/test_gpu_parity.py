@@ -300,6 +300,40 @@ def test_ffn_2b_full_size():
     check_y(f64(y), w64, rows, TOL[synth.BF16])
 
 
+def test_back_to_back_calls_share_one_workspace():
+    """Gate and fused calls of two different batches queued back to back on one
+    stream, sharing the TwELL buffers and the fused workspace, with no host
+    synchronisation between them: each launch waits for the previous one's
+    results (programmatic dependent launches) and the planner clears the
+    engine's counters itself.  Both outputs equal those of separate,
+    synchronised calls, bit for bit."""
+    T, d, F = 3000, 1024, 2048
+    wa = synth.make_workload(T=T, d=d, F=F, W=128, C=8, dtype=synth.BF16, kind="zipf",
+                             mean_active=29.0, seed=101)
+    wb = synth.make_workload(T=T, d=d, F=F, W=128, C=8, dtype=synth.BF16, kind="zipf",
+                             mean_active=60.0, seed=202)
+    da, db = inputs(wa), inputs(wb)
+    g = tw.Twell(T, F, 8, dtype=torch.bfloat16, spill_cap=(F // 128) * T)
+    ws = tw.fused_workspace(T, d)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    refs = []
+    for dv in (da, db):  # separate calls, synchronised
+        y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+        tw.twell_gate_gemm(dv["x"], dv["Wg_t"], g, None, st)
+        tw.twell_fused_updown(dv["x"], g, dv["Wu_t"], dv["Wd"], y, ws, st)
+        torch.cuda.synchronize()
+        refs.append(y)
+    ys = [torch.empty((T, d), dtype=torch.float32, device="cuda") for _ in range(4)]
+    for i, dv in enumerate((da, db, da, db)):  # queued back to back
+        tw.twell_gate_gemm(dv["x"], dv["Wg_t"], g, None, st)
+        tw.twell_fused_updown(dv["x"], g, dv["Wu_t"], dv["Wd"], ys[i], ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, tw.status_bits(st)
+    for i in range(4):
+        assert torch.equal(ys[i], refs[i % 2]), i
+    check_y(f64(refs[1]), widened(wb), synth.subsample_rows(T, 48), TOL[synth.BF16])
+
+
 # Small batches (T <= 64) take the cluster split-K gate; the cases cover
 # cluster sizes 8, 8 with uneven k-block shares (d = 520), 2 (partials of
 # 48 tokens), 1 (more tiles than SMs), C = 0 and the largest C.  The last
@@ -691,6 +725,52 @@ def run_hybrid(w, backup_cap=None):
                            w["lam"], dx, dW[0], dW[1], dW[2], ws, st)
     torch.cuda.synchronize()
     return dev, g, gd, y, st, hy, yh, dx, dW
+
+
+def test_hybrid_steps_back_to_back():
+    """Whole training steps of two batches (gate, TwELL -> hybrid, forward,
+    backward) queued back to back on one stream with shared buffers and
+    workspaces: every output equals that of separate, synchronised steps, bit
+    for bit (the launches wait for their predecessors' results, and the
+    counters and u arrays are cleared by the library's own kernels)."""
+    ws_ = [synth.make_workload(T=900, d=256, F=1024, W=128, C=8, C_h=16, dtype=synth.BF16,
+                               kind="pareto", lam=2e-5, seed=s_, mean_active=14.0)
+           for s_ in (31, 32)]
+    T, d, F, C_h = 900, 256, 1024, 16
+    devs = [inputs(w) for w in ws_]
+    g = tw.Twell(T, F, 8, dtype=torch.bfloat16, spill_cap=(F // 128) * T)
+    hy = tw.Hybrid(T, F, C_h, dtype=torch.bfloat16, backup_cap=T)
+    bws = torch.empty(tw.hybrid_ffn_backward_workspace_size(T, d, F, C_h, T), dtype=torch.uint8,
+                      device="cuda")
+    fws = torch.empty(tw.hybrid_ffn_forward_workspace_size(T, d), dtype=torch.uint8,
+                      device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(dv, w, outs):
+        tw.twell_gate_gemm(dv["x"], dv["Wg_t"], g, None, st)
+        tw.twell_to_hybrid(g, hy, st)
+        tw.hybrid_ffn_forward(dv["x"], hy, dv["Wu_t"], dv["Wd"], outs[0], fws, st)
+        tw.hybrid_ffn_backward(dv["x"], dv["dy"], hy, dv["Wg_t"], dv["Wu_t"], dv["Wd"], w["lam"],
+                               outs[1], outs[2], outs[3], outs[4], bws, st)
+
+    def fresh():
+        return [torch.empty((T, d), dtype=torch.float32, device="cuda") for _ in range(2)] + \
+               [torch.empty((F, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+
+    refs = []
+    for dv, w in zip(devs, ws_):  # separate, synchronised steps
+        outs = fresh()
+        step(dv, w, outs)
+        torch.cuda.synchronize()
+        refs.append(outs)
+    runs = [fresh() for _ in range(4)]
+    for i in range(4):  # queued back to back
+        step(devs[i % 2], ws_[i % 2], runs[i])
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, tw.status_bits(st)
+    for i in range(4):
+        for a, b in zip(runs[i], refs[i % 2]):
+            assert torch.equal(a, b), i
 
 
 def hybrid_to_np(hy):
