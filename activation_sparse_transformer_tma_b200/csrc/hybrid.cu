@@ -427,10 +427,11 @@ __global__ void __launch_bounds__(256)
 //   2. scan_kernel        exclusive prefix of the counts -> unit_off;
 //   3. hyb_place_kernel   each record's index at its unit's next place (the
 //                         order inside a unit is arbitrary here);
-//   4. hyb_wgrad_kernel   one CTA per unit sorts its segment (bitonic, in
-//                         shared memory up to kSegSmem records; longer
-//                         segments as sorted runs merged by rank into a
-//                         scratch list) and sums in that order.
+//   4. hyb_wgrad_kernel   one CTA per unit sorts its segment (bitonic: in one
+//                         warp's registers up to 64 records, in shared
+//                         memory up to kSegSmem; longer segments as sorted
+//                         runs merged by rank into a scratch list) and sums
+//                         in that order.
 // Every pass is flat over the records, so a heavy backup row costs no one
 // thread or warp more than its share.
 constexpr int kSegSmem = 2048;  // records of a unit sorted in shared memory
@@ -477,6 +478,28 @@ TW_DEV void block_bitonic(int32_t* v, int P) {
   }
 }
 
+// Ascending bitonic sort of 64 values held by one warp, two per lane: a at
+// position lane, b at position lane + 32.  All in registers and shuffles.
+TW_DEV void warp_bitonic64(int32_t& a, int32_t& b, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {  // partners in the same lane; k == 64, ascending everywhere
+        const int32_t lo = min(a, b), hi = max(a, b);
+        a = lo;
+        b = hi;
+      } else {
+        const int32_t pa = __shfl_xor_sync(FULL, a, j), pb = __shfl_xor_sync(FULL, b, j);
+        const bool lower = (lane & j) == 0;
+        const bool asc_a = (lane & k) == 0, asc_b = ((lane + 32) & k) == 0;
+        a = (asc_a == lower) ? min(a, pa) : max(a, pa);
+        b = (asc_b == lower) ? min(b, pb) : max(b, pb);
+      }
+    }
+  }
+}
+
 // Weight gradients of one unit per CTA, records summed in token order.
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -491,7 +514,17 @@ __global__ void __launch_bounds__(256)
   const int j = blockIdx.x;
   const int b = unit_off[j], n = unit_off[j + 1] - b;
   const bool small = n <= kSegSmem;
-  if (small) {
+  if (n <= 64) {  // most units: one warp sorts in registers
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      int32_t va = lane < n ? list[b + lane] : INT32_MAX;
+      int32_t vb = lane + 32 < n ? list[b + lane + 32] : INT32_MAX;
+      warp_bitonic64(va, vb, lane);
+      seg[lane] = va;
+      seg[lane + 32] = vb;
+    }
+    __syncthreads();
+  } else if (small) {
     int P = 1;
     while (P < n) P <<= 1;
     for (int i = threadIdx.x; i < P; i += blockDim.x) seg[i] = i < n ? list[b + i] : INT32_MAX;
