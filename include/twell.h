@@ -166,8 +166,9 @@ TW_API size_t twell_fused_updown_workspace_size(int32_t T, int32_t d);
  * x, Wu_t and Wd have g->dtype.  y [T][d].
  * ws: device workspace of at least twell_fused_updown_workspace_size(T, d)
  * bytes (a work plan, and fp32 partial rows for tokens whose active units are
- * split over several warps).  Its first bytes are cleared on `stream` by the
- * call; calls that share one workspace must not overlap on the device.  y is
+ * split over several warps).  Its counters are cleared on `stream` by the
+ * call's own kernels; calls that share one workspace must not overlap on the
+ * device (calls queued one after another on one stream do not).  y is
  * deterministic: partial rows are summed in a fixed order.
  */
 TW_API tw_status twell_fused_updown(const void* x, const tw_twell* g, const void* Wu_t,
