@@ -595,7 +595,6 @@ struct GatherArgs {
   float lam;
   const int32_t* e0;
   Payload* pay;
-  int32_t* ucnt;  // backward: records per unit (one atomic per record)
   void* out;
   int32_t* status;
   FusedWs ws;
@@ -1106,7 +1105,6 @@ __global__ void __launch_bounds__(32 * kTeam * teams_for<NCHW, MODE>(), 1)
               pl.du = du;
               pl.dz = dz;
               a.pay[a.e0[t] + w0 + e] = pl;
-              atomicAdd(&a.ucnt[pl.j], 1);
             }
           };
           auto upd2 = [&](uint4 (&RU)[2][NCHW], uint4 (&RG)[2][NCHW], int pp) {
@@ -1469,7 +1467,7 @@ cudaError_t twell_fused(const void* x, const tw_twell& g, const void* Wu_t, cons
 template <typename Tin, int MODE>
 cudaError_t hybrid_t(const void* xin, const tw_hybrid& h, const void* rdot, const void* rax1,
                      const void* rax2, int d, float lam, const int32_t* e0, Payload* pay,
-                     int32_t* ucnt, void* out, tw_dtype out_dtype, void* base, int32_t* status,
+                     void* out, tw_dtype out_dtype, void* base, int32_t* status,
                      cudaStream_t stream) {
   const FusedWs w = carve(base, h.T, d);
   GatherArgs<Tin> a{};
@@ -1491,7 +1489,6 @@ cudaError_t hybrid_t(const void* xin, const tw_hybrid& h, const void* rdot, cons
   a.lam = lam;
   a.e0 = e0;
   a.pay = pay;
-  a.ucnt = ucnt;
   a.out = out;
   a.status = status;
   a.ws = w;
@@ -1573,21 +1570,21 @@ cudaError_t launch_hybrid_gather_forward(const void* x, const tw_hybrid& gu, con
   }
   return gu.dtype == TW_BF16
              ? hybrid_t<uint16_t, kModeHybFwd>(x, gu, Wu_t, Wd, nullptr, d, 0.f, nullptr, nullptr,
-                                               nullptr, y, y_dtype, ws, status, stream)
-             : hybrid_t<float, kModeHybFwd>(x, gu, Wu_t, Wd, nullptr, d, 0.f, nullptr, nullptr,
-                                            nullptr, y, y_dtype, ws, status, stream);
+                                               y, y_dtype, ws, status, stream)
+             : hybrid_t<float, kModeHybFwd>(x, gu, Wu_t, Wd, nullptr, d, 0.f, nullptr, nullptr, y,
+                                            y_dtype, ws, status, stream);
 }
 
 cudaError_t launch_hybrid_gather_backward(const void* dy, const tw_hybrid& gu, const void* Wg_t,
                                           const void* Wu_t, const void* Wd, int d, float lam,
-                                          const int32_t* e0, Payload* pay, int32_t* ucnt,
-                                          void* dx, tw_dtype dx_dtype, void* ws,
-                                          int32_t* status, cudaStream_t stream) {
+                                          const int32_t* e0, Payload* pay, void* dx,
+                                          tw_dtype dx_dtype, void* ws, int32_t* status,
+                                          cudaStream_t stream) {
   return gu.dtype == TW_BF16
-             ? hybrid_t<uint16_t, kModeHybBwd>(dy, gu, Wd, Wu_t, Wg_t, d, lam, e0, pay, ucnt, dx,
+             ? hybrid_t<uint16_t, kModeHybBwd>(dy, gu, Wd, Wu_t, Wg_t, d, lam, e0, pay, dx,
                                                dx_dtype, ws, status, stream)
-             : hybrid_t<float, kModeHybBwd>(dy, gu, Wd, Wu_t, Wg_t, d, lam, e0, pay, ucnt, dx,
-                                            dx_dtype, ws, status, stream);
+             : hybrid_t<float, kModeHybBwd>(dy, gu, Wd, Wu_t, Wg_t, d, lam, e0, pay, dx, dx_dtype,
+                                            ws, status, stream);
 }
 
 }  // namespace tw

@@ -423,8 +423,7 @@ __global__ void __launch_bounds__(256)
 // and each carries its unit.  The weight gradients sum them per unit in
 // ascending token order, i.e. ascending record index, so each unit's records
 // are gathered into a unit-major list and sorted there:
-//   1. the backward gather counts the records of each unit as it writes
-//      them (one atomic per record);
+//   1. hyb_ucount_kernel  records per unit (one atomic per record);
 //   2. scan_kernel        exclusive prefix of the counts -> unit_off;
 //   3. hyb_place_kernel   each record's index at its unit's next place (the
 //                         order inside a unit is arbitrary here);
@@ -437,6 +436,15 @@ __global__ void __launch_bounds__(256)
 // thread or warp more than its share.
 constexpr int kSegSmem = 2048;  // records of a unit sorted in shared memory
 constexpr int kPaySmem = 512;   // records of a unit whose payloads are staged in shared memory
+
+__global__ void __launch_bounds__(256)
+    hyb_ucount_kernel(const Payload* pay, const int32_t* e_total, int32_t* ucnt) {
+  pdl_wait();
+  pdl_launch_next();
+  const int n = *e_total;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x)
+    atomicAdd(&ucnt[pay[e].j], 1);
+}
 
 __global__ void __launch_bounds__(256)
     hyb_place_kernel(const Payload* pay, const int32_t* e_total, const int32_t* unit_off,
@@ -697,13 +705,15 @@ cudaError_t backward_t(const void* x, const void* dy, const tw_hybrid& gu, const
                              (int32_t*)nullptr, status, w.ucnt, 2 * gu.F);
   if (e != cudaSuccess) return e;
   // per-token pass: dh, du, dz, dx and one record per entry
-  // (it also counts each unit's records into w.ucnt)
-  e = launch_hybrid_gather_backward(dy, gu, Wg_t, Wu_t, Wd, d, lam, w.e0, w.pay, w.ucnt, dx,
-                                    dx_dtype, engine_ws, status, s);
+  e = launch_hybrid_gather_backward(dy, gu, Wg_t, Wu_t, Wd, d, lam, w.e0, w.pay, dx, dx_dtype,
+                                    engine_ws, status, s);
   if (e != cudaSuccess) return e;
   // weight gradients: records grouped by unit, then each unit sorted and summed
   const int grid = num_sms() * 8;
   const int32_t* e_total = w.e0 + gu.T;
+  e = launch_pdl(hyb_ucount_kernel, dim3(grid), dim3(256), 0, s, (const Payload*)w.pay, e_total,
+                 w.ucnt);
+  if (e != cudaSuccess) return e;
   e = launch_pdl(scan_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, 1, gu.F, (const int32_t*)w.ucnt,
                  0, w.unit_off, (int32_t*)nullptr, 0, (int32_t*)nullptr, status,
                  (int32_t*)nullptr, 0);

@@ -111,13 +111,11 @@ struct Payload {
 cudaError_t launch_hybrid_gather_forward(const void* x, const tw_hybrid& gu, const void* Wu_t,
                                          const void* Wd, int d, void* y, tw_dtype y_dtype,
                                          void* ws, int32_t* status, cudaStream_t stream);
-// Writes one record per entry at pay[e0[t] + rank] and counts the records
-// of each unit into ucnt[j] (zeroed by the caller).
 cudaError_t launch_hybrid_gather_backward(const void* dy, const tw_hybrid& gu, const void* Wg_t,
                                           const void* Wu_t, const void* Wd, int d, float lam,
-                                          const int32_t* e0, Payload* pay, int32_t* ucnt,
-                                          void* dx, tw_dtype dx_dtype, void* ws,
-                                          int32_t* status, cudaStream_t stream);
+                                          const int32_t* e0, Payload* pay, void* dx,
+                                          tw_dtype dx_dtype, void* ws, int32_t* status,
+                                          cudaStream_t stream);
 
 // Hybrid (training) kernels.
 cudaError_t launch_twell_to_hybrid(const tw_twell& g, const tw_hybrid& out, int32_t* status,
