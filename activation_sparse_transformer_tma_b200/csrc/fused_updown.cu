@@ -1271,8 +1271,12 @@ cudaError_t launch_nchw(GatherArgs<Tin> a, bool out_bf16, cudaStream_t stream) {
 //   each thread then accumulates its own columns of y over all entries of
 //     the window, eight rows of Wd in flight.
 // Entries are summed in their (tile-major) order, so y is deterministic.
+// One CTA per token leaves a token with hundreds of entries (heavy-tailed
+// activity) to a single CTA: at 16 tokens of the 2B decoding workload, with
+// a 425-entry token, that took 120 us, so the planned path (which splits
+// heavy tokens) takes over above 8 tokens.
 constexpr int kDecWarps = 8;
-constexpr int kDecodeMaxT = 16;
+constexpr int kDecodeMaxT = 8;
 
 template <typename Tin, bool kOutBf16>
 __global__ void __launch_bounds__(32 * kDecWarps) decode_kernel(const GatherArgs<Tin> a) {

@@ -657,7 +657,7 @@ def decode_leg(torch, tw, hbm):
                            "gate_hbm_GBps": gate_gbs, "gate_hbm_frac": gate_gbs / hbm,
                            "gate_frac_of_stream_floor": floor_us / (mg * 1e3),
                            "fused_gathered_GBps": rows / (mf * 1e-3) / 1e9,
-                           "library_launches": 2 if T <= 16 else 5}}
+                           "library_launches": 2 if T <= 8 else 5}}
         if ts:
             ms = float(np.median(ts))
             step_gbs = (wg_bytes + rows) / (ms * 1e-3) / 1e9

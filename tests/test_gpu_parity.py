@@ -96,9 +96,9 @@ def test_bf16_gate_and_fused_small(T, d, F, C, kind, ma):
     check_y(f64(y), w64, rows, TOL[synth.BF16])
 
 
-# planned gather engine with both slice widths, and the one-CTA-per-token
-# small-batch kernel (T <= 16)
-@pytest.mark.parametrize("d,T", [(320, 300), (256, 300), (256, 12)])
+# planned gather engine with both slice widths (and 12 tokens), and the
+# one-CTA-per-token small-batch kernel (T <= 8)
+@pytest.mark.parametrize("d,T", [(320, 300), (256, 300), (256, 12), (256, 6)])
 def test_bf16_output_y(d, T):
     w = synth.make_workload(T=T, d=d, F=640, W=128, C=8, dtype=synth.BF16, kind="dead20",
                             mean_active=29.0, seed=620)
