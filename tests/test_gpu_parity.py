@@ -930,6 +930,15 @@ def test_hybrid_backup_capacity_overflow_is_flagged():
     torch.cuda.synchronize()
     assert int(hy.n_backup.item()) > 3
     assert "TW_ERR_BACKUP_CAPACITY" in tw.status_bits(st)
+    # the forward still runs on what was stored: u is cleared in the 3 stored
+    # backup rows (and no further) and is +0 wherever g is
+    hy.backup_u.view(torch.int16).fill_(0x3F80)  # bf16 1.0 everywhere beforehand
+    yh = torch.empty((256, 128), dtype=torch.float32, device="cuda")
+    tw.hybrid_ffn_forward(dev["x"], hy, dev["Wu_t"], dev["Wd"], yh, dev_status=st)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(yh).all())
+    bg, bu = f64(hy.backup_g), f64(hy.backup_u)
+    assert np.all(bu[:3][bg[:3] == 0] == 0)
 
 
 def test_training_config_full_size():
